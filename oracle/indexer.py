@@ -1,0 +1,83 @@
+"""Lightning Indexer scores, causal visibility and exact top-k selection.
+
+What the pages fix:
+* The indexer gives every query a cheap relevance score against all
+  compressed entries, then only the top-k go on to the main attention
+  ([SW] §六 funnel; [TR] §4.2 LightningIndexer: scores = relu(q_idx k_idx^T)).
+* Each head's score goes through ReLU before the heads are summed, so one
+  strongly positive head is not cancelled by a negative one: heads (8, -7)
+  give 8, not 1 ([SW] §七).
+* It runs at low precision, FP8 or even FP4 ([SW] §六.1; [TR] §4.2).
+* k = 1024 at full scale ([AM]).
+* A query reads only compressed blocks that lie strictly before it and are
+  complete: token 98 may not read block 24 (tokens 96..99) ([SW] §十).
+
+Readings taken where the pages leave the form open:
+* Score of entry i for a query with heads h = 0..Hi-1:
+      s_i = sum_h w_h * ReLU(sq_h * sk_i * <q_h, k_i>)
+  with per-(query, head) scales sq_h and per-entry scales sk_i of the FP8
+  codes (1 when the indexer is stored unscaled) and head weights w_h
+  (default 1; the pages sum the heads without weights).
+* Entry i (ratio m) is visible to position p iff m*(i+1) <= p+1, i.e. the
+  query sees entries 0 .. floor((p+1)/m) - 1.
+* Top-k keeps min(k, visible) entries: the largest scores, ties going to the
+  lower entry index.  The selected set is returned in ascending index order
+  and padded with -1 to length k.
+
+Parity: pinned (worked (8, -7) example, block-24 causal example, brute-force
+enumeration of k-subsets on tiny inputs, ties).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+
+def visible_entries(p: int, ratio: int) -> int:
+    """Number of complete blocks strictly before or ending at position p."""
+    return (int(p) + 1) // int(ratio)
+
+
+def entry_visible(i: int, p: int, ratio: int) -> bool:
+    """Entry i (tokens ratio*i .. ratio*i+ratio-1) is complete at position p."""
+    return ratio * (int(i) + 1) <= int(p) + 1
+
+
+def index_scores(q_idx, k_idx, q_scale=None, k_scale=None, head_w=None) -> np.ndarray:
+    """Scores [V] of V entries for one query.
+
+    q_idx [Hi, di] and k_idx [V, di] are decoded float64 values; q_scale [Hi],
+    k_scale [V] and head_w [Hi] are optional (1 when absent).
+    """
+    q = np.asarray(q_idx, dtype=np.float64)
+    k = np.asarray(k_idx, dtype=np.float64)
+    Hi = q.shape[0]
+    V = k.shape[0]
+    sq = np.ones(Hi) if q_scale is None else np.asarray(q_scale, dtype=np.float64)
+    sk = np.ones(V) if k_scale is None else np.asarray(k_scale, dtype=np.float64)
+    w = np.ones(Hi) if head_w is None else np.asarray(head_w, dtype=np.float64)
+    dots = k @ q.T                                   # [V, Hi]: <q_h, k_i>
+    per_head = sq[None, :] * sk[:, None] * dots      # scaled head scores
+    return np.sum(w[None, :] * np.maximum(per_head, 0.0), axis=1)
+
+
+def topk_order(scores: np.ndarray) -> np.ndarray:
+    """Entry indices ordered by score descending, ties by index ascending."""
+    s = np.asarray(scores, dtype=np.float64)
+    return np.lexsort((np.arange(len(s)), -s))
+
+
+def topk_select(scores: np.ndarray, k: int) -> np.ndarray:
+    """The min(k, V) best entries, in ascending index order, padded with -1."""
+    order = topk_order(scores)[: min(int(k), len(scores))]
+    out = np.full(int(k), -1, dtype=np.int64)
+    out[: len(order)] = np.sort(order)
+    return out
+
+
+def kth_score(scores: np.ndarray, k: int) -> float:
+    """Score of the last entry that top-k keeps (-inf when nothing is kept)."""
+    kk = min(int(k), len(scores))
+    if kk == 0:
+        return -np.inf
+    return float(np.asarray(scores, dtype=np.float64)[topk_order(scores)[kk - 1]])

@@ -1,0 +1,66 @@
+"""Pins of the oracle's storage codecs (bf16, OCP E4M3) against the format
+specification's printed values and against torch's own conversions."""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import codecs
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_e4m3_known_values_from_spec():
+    g = json.load(open(os.path.join(GOLD, "e4m3_values.json")))
+    for code, val in g["codes"].items():
+        got = codecs.e4m3_decode(np.array([int(code, 16)], np.uint8))[0]
+        assert got == val and np.signbit(got) == np.signbit(val), code
+    for code in g["nan_codes"]:
+        assert np.isnan(codecs.e4m3_decode(np.array([int(code, 16)], np.uint8))[0])
+
+
+def test_e4m3_all_codes_match_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = codecs.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(ours[ok], ref[ok])
+
+
+def test_bf16_decode_matches_torch_all_codes():
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = codecs.bf16_decode(codes)
+    ref = torch.from_numpy(codes.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(ours[ok], ref[ok])
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_bf16_encode_matches_torch_rne(seed):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal(200000) * np.exp(rng.uniform(-30, 30, 200000))).astype(np.float32)
+    # exact halfway points between neighbouring bf16 values (ties go to even)
+    # finite values only: the top 16 bits stay below the all-ones exponent
+    base = rng.integers(0, 0x7F7F, 5000).astype(np.uint32) << np.uint32(16)
+    half = (base | np.uint32(0x8000)).view(np.float32)
+    # fp32 subnormals and values next to the overflow threshold
+    sub = (rng.integers(1, 1 << 23, 2000).astype(np.uint32)).view(np.float32)
+    big = np.array([3.3895314e38, 3.3961776e38, 3.4e38, -3.39e38, np.inf, -np.inf, 0.0, -0.0], np.float32)
+    allx = np.concatenate([x, half, -half, sub, big])
+    ours = codecs.bf16_encode(allx.astype(np.float64))
+    ref = torch.from_numpy(allx).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_bf16_encode_rounds_doubles_once():
+    # 1 + 2^-8 + 2^-30 lies just above the midpoint of 1 and 1 + 2^-7: it must round up,
+    # while a detour through float32 (which drops the 2^-30) would tie to even and round down.
+    x = np.array([1.0 + 2.0 ** -8 + 2.0 ** -30, 1.0 + 2.0 ** -8])
+    got = codecs.bf16_decode(codecs.bf16_encode(x))
+    assert got[0] == 1.0 + 2.0 ** -7
+    assert got[1] == 1.0
