@@ -1,0 +1,116 @@
+"""Torch-tensor front end of the cskv C ABI: argument marshalling only.
+
+Every function here turns tensors into pointers, sizes and dtype codes and
+calls the C entry point of the same name on the current CUDA stream (or the
+one given).  All computation happens in the CUDA library.
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _lib
+from ._lib import BF16, CSA, F32, FP8E4M3, HCA  # noqa: F401
+
+_DT = {torch.float32: F32, torch.bfloat16: BF16, torch.uint8: FP8E4M3, torch.float8_e4m3fn: FP8E4M3}
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("cskv expects contiguous tensors")
+    return t.data_ptr()
+
+
+def _dt(t) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise ValueError(f"unsupported dtype {t.dtype}") from None
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def csa_compress(x_a, z_a, x_b, z_b, tok_off, ent_off, out, *, max_blocks, bias_a=None, bias_b=None, tok0=None,
+                 first_block=None, num_blocks=None, dev_status=None, stream=None):
+    lib = _lib.load()
+    st = lib.csa_compress(_ptr(x_a), _ptr(z_a), _ptr(x_b), _ptr(z_b), _ptr(bias_a), _ptr(bias_b), _ptr(tok_off),
+                          _ptr(tok0), tok_off.numel() - 1, _ptr(ent_off), _ptr(first_block), _ptr(num_blocks),
+                          int(max_blocks), _dt(x_a), _dt(out), _ptr(out), _ptr(dev_status), _stream(stream))
+    _lib.check("csa_compress", st)
+    return out
+
+
+def hca_compress(x, z, tok_off, ent_off, out, *, max_blocks, bias=None, tok0=None, first_block=None,
+                 num_blocks=None, dev_status=None, stream=None):
+    lib = _lib.load()
+    st = lib.hca_compress(_ptr(x), _ptr(z), _ptr(bias), _ptr(tok_off), _ptr(tok0), tok_off.numel() - 1,
+                          _ptr(ent_off), _ptr(first_block), _ptr(num_blocks), int(max_blocks), _dt(x), _dt(out),
+                          _ptr(out), _ptr(dev_status), _stream(stream))
+    _lib.check("hca_compress", st)
+    return out
+
+
+def lindex_workspace_size(T: int, k: int, max_entries: int) -> int:
+    return int(_lib.load().lindex_workspace_size(int(T), int(k), int(max_entries)))
+
+
+def lindex_workspace(T: int, k: int, max_entries: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace; calls hand it back zero-filled."""
+    return torch.zeros(max(16, lindex_workspace_size(T, k, max_entries)), dtype=torch.uint8, device=device)
+
+
+def lindex_score_topk(q_idx, k_idx, q_seq, q_pos, ent_off, out_idx, workspace, *, max_entries, q_scale=None,
+                      k_scale=None, head_w=None, out_score=None, dev_status=None, stream=None):
+    T, Hi, Di = q_idx.shape
+    lib = _lib.load()
+    st = lib.lindex_score_topk(_ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(head_w), _ptr(q_seq),
+                               _ptr(q_pos), _ptr(ent_off), ent_off.numel() - 1, T, Hi, Di, out_idx.shape[1],
+                               _dt(q_idx), int(max_entries), _ptr(out_idx), _ptr(out_score), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream))
+    _lib.check("lindex_score_topk", st)
+    return out_idx
+
+
+def lindex_topk_from_scores(scores, n_valid, out_idx, workspace, *, max_entries, out_score=None, dev_status=None,
+                            stream=None):
+    T, ld = scores.shape
+    lib = _lib.load()
+    st = lib.lindex_topk_from_scores(_ptr(scores), ld, _ptr(n_valid), T, out_idx.shape[1], int(max_entries),
+                                     _ptr(out_idx), _ptr(out_score), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                     _stream(stream))
+    _lib.check("lindex_topk_from_scores", st)
+    return out_idx
+
+
+def attn_workspace_size(mode: int, T: int, H: int, k: int, window: int, max_entries: int) -> int:
+    return int(_lib.load().hybrid_attn_workspace_size(int(mode), int(T), int(H), 128, int(k), int(window),
+                                                      int(max_entries)))
+
+
+def attn_workspace(mode, T, H, k, window, max_entries, device="cuda") -> torch.Tensor:
+    n = attn_workspace_size(mode, T, H, k, window, max_entries)
+    return torch.empty(max(16, n), dtype=torch.uint8, device=device)
+
+
+def hybrid_decode_attn(mode, q, kv_cmp, cmp_off, kv_raw, raw_off, q_seq, q_pos, out, workspace, *, window,
+                       idx=None, raw_tok0=None, sink=None, scale=None, lse=None, max_entries=0, dev_status=None,
+                       stream=None):
+    T, H, d = q.shape
+    k = idx.shape[1] if idx is not None else 0
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    lib = _lib.load()
+    st = lib.hybrid_decode_attn(int(mode), _ptr(q), _ptr(kv_cmp), _ptr(cmp_off), _ptr(idx), k, _ptr(kv_raw),
+                                _ptr(raw_off), _ptr(raw_tok0), int(window), _ptr(sink), scale, _ptr(q_seq),
+                                _ptr(q_pos), cmp_off.numel() - 1, T, H, d, _dt(q), int(max_entries), _ptr(out),
+                                _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _ptr(dev_status), _stream(stream))
+    _lib.check("hybrid_decode_attn", st)
+    return out

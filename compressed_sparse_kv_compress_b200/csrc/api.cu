@@ -1,0 +1,216 @@
+// C ABI of the cskv library: host-side validation, then dispatch to the launchers.
+// Every check here runs before any launch, so an error return means nothing ran.
+#include <stdio.h>
+
+#include "launch.cuh"
+
+using namespace cskv;
+
+static thread_local char g_cuda_err[256] = "no error";
+
+static int launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return CSKV_OK;
+  snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return CSKV_ERR_LAUNCH;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static int device_sms(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+  return launch_status(e);
+}
+
+extern "C" {
+
+const char* cskv_status_string(int status) {
+  switch (status) {
+    case CSKV_OK: return "CSKV_OK";
+    case CSKV_ERR_INVALID_ARG: return "CSKV_ERR_INVALID_ARG: null pointer, bad size, misaligned pointer or bad enum";
+    case CSKV_ERR_UNSUPPORTED: return "CSKV_ERR_UNSUPPORTED: combination of dtype / head dim / heads not implemented";
+    case CSKV_ERR_WORKSPACE: return "CSKV_ERR_WORKSPACE: workspace missing or too small";
+    case CSKV_ERR_LAUNCH: return "CSKV_ERR_LAUNCH: the CUDA runtime refused a launch or query";
+    default: return "unknown cskv status";
+  }
+}
+
+const char* cskv_last_cuda_error(void) { return g_cuda_err; }
+
+int cskv_version(void) { return 100; }
+
+static int check_compress_common(const void* x, const void* z, const int64_t* tok_off, int batch,
+                                 const int64_t* ent_off, int64_t max_blocks, int in_dtype, int out_dtype,
+                                 const void* out) {
+  if (!x || !z || !tok_off || !ent_off || !out) return CSKV_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || max_blocks < 0 || max_blocks > (1LL << 31) - 1) return CSKV_ERR_INVALID_ARG;
+  if ((in_dtype != CSKV_F32 && in_dtype != CSKV_BF16) || (out_dtype != CSKV_F32 && out_dtype != CSKV_BF16))
+    return in_dtype == CSKV_FP8E4M3 || out_dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(z) || !aligned16(out)) return CSKV_ERR_INVALID_ARG;
+  return CSKV_OK;
+}
+
+int csa_compress(const void* x_a, const void* z_a, const void* x_b, const void* z_b, const float* bias_a,
+                 const float* bias_b, const int64_t* tok_off, const int64_t* tok0, int batch,
+                 const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
+                 int64_t max_blocks, int in_dtype, int out_dtype, void* out, int* dev_status,
+                 cskv_stream_t stream) {
+  int rc = check_compress_common(x_a, z_a, tok_off, batch, ent_off, max_blocks, in_dtype, out_dtype, out);
+  if (rc) return rc;
+  if ((x_b == nullptr) != (z_b == nullptr)) return CSKV_ERR_INVALID_ARG;
+  if (x_b && (!aligned16(x_b) || !aligned16(z_b))) return CSKV_ERR_INVALID_ARG;
+  if ((bias_a && !aligned16(bias_a)) || (bias_b && !aligned16(bias_b))) return CSKV_ERR_INVALID_ARG;
+  if (max_blocks == 0) return CSKV_OK;
+  return launch_status(launch_csa_compress(x_a, z_a, x_b, z_b, bias_a, bias_b, tok_off, tok0, batch, ent_off,
+                                           first_block, num_blocks, max_blocks, in_dtype, out_dtype, out,
+                                           dev_status, (cudaStream_t)stream));
+}
+
+int hca_compress(const void* x, const void* z, const float* bias, const int64_t* tok_off, const int64_t* tok0,
+                 int batch, const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
+                 int64_t max_blocks, int in_dtype, int out_dtype, void* out, int* dev_status,
+                 cskv_stream_t stream) {
+  int rc = check_compress_common(x, z, tok_off, batch, ent_off, max_blocks, in_dtype, out_dtype, out);
+  if (rc) return rc;
+  if (bias && !aligned16(bias)) return CSKV_ERR_INVALID_ARG;
+  if (max_blocks == 0) return CSKV_OK;
+  return launch_status(launch_hca_compress(x, z, bias, tok_off, tok0, batch, ent_off, first_block, num_blocks,
+                                           max_blocks, in_dtype, out_dtype, out, dev_status,
+                                           (cudaStream_t)stream));
+}
+
+size_t lindex_workspace_size(int T, int k, int64_t max_entries) {
+  (void)k;
+  if (T < 1) return 0;
+  return lindex_ws_bytes(T, max_entries);
+}
+
+static int check_topk_common(int T, int k, int64_t max_entries, const int32_t* out_idx, const void* ws,
+                             size_t ws_bytes) {
+  if (T < 0 || k < 1 || k > (1 << 24) || max_entries < 0 || max_entries >= (1LL << 31)) return CSKV_ERR_INVALID_ARG;
+  if (T > 0 && !out_idx) return CSKV_ERR_INVALID_ARG;
+  if (T > 0 && !lindex_capacity_ok(max_entries, T)) return CSKV_ERR_UNSUPPORTED;
+  if (T > 0 && (!ws || ws_bytes < lindex_ws_bytes(T, max_entries) || !aligned16(ws))) return CSKV_ERR_WORKSPACE;
+  return CSKV_OK;
+}
+
+int lindex_score_topk(const void* q_idx, const float* q_scale, const void* k_idx, const float* k_scale,
+                      const float* head_w, const int32_t* q_seq, const int64_t* q_pos, const int64_t* ent_off,
+                      int batch, int T, int Hi, int Di, int k, int dtype, int64_t max_entries, int32_t* out_idx,
+                      float* out_score, void* workspace, size_t ws_bytes, int* dev_status,
+                      cskv_stream_t stream) {
+  if (dtype != CSKV_F32 && dtype != CSKV_FP8E4M3 && dtype != CSKV_BF16) return CSKV_ERR_INVALID_ARG;
+  if (!lindex_shape_supported(dtype, Hi, Di)) return CSKV_ERR_UNSUPPORTED;
+  if (T > 0 && (!q_idx || !k_idx || !q_seq || !q_pos || !ent_off || batch < 1)) return CSKV_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx)) return CSKV_ERR_INVALID_ARG;
+  int rc = check_topk_common(T, k, max_entries, out_idx, workspace, ws_bytes);
+  if (rc || T == 0) return rc;
+  IdxParams p = {};
+  p.q_idx = (const uint8_t*)q_idx;
+  p.q_scale = q_scale;
+  p.k_idx = (const uint8_t*)k_idx;
+  p.k_scale = k_scale;
+  p.head_w = head_w;
+  p.q_seq = q_seq;
+  p.q_pos = q_pos;
+  p.ent_off = ent_off;
+  p.batch = batch;
+  p.Hi = Hi;
+  p.Di = Di;
+  p.k = k;
+  p.max_entries = max_entries;
+  p.out_idx = out_idx;
+  p.out_score = out_score;
+  p.ws = (QueryWS*)workspace;
+  p.st = dev_status;
+  return launch_status(launch_lindex(p, dtype, T, (cudaStream_t)stream));
+}
+
+int lindex_topk_from_scores(const float* scores, int64_t ld_scores, const int64_t* n_valid, int T, int k,
+                            int64_t max_entries, int32_t* out_idx, float* out_score, void* workspace,
+                            size_t ws_bytes, int* dev_status, cskv_stream_t stream) {
+  if (T > 0 && (!scores || !n_valid)) return CSKV_ERR_INVALID_ARG;
+  if (ld_scores < max_entries || ld_scores < 0) return CSKV_ERR_INVALID_ARG;
+  int rc = check_topk_common(T, k, max_entries, out_idx, workspace, ws_bytes);
+  if (rc || T == 0) return rc;
+  IdxParams p = {};
+  p.scores = scores;
+  p.ld_scores = ld_scores;
+  p.n_valid = n_valid;
+  p.Hi = 1;
+  p.Di = 64;
+  p.k = k;
+  p.max_entries = max_entries;
+  p.out_idx = out_idx;
+  p.out_score = out_score;
+  p.ws = (QueryWS*)workspace;
+  p.st = dev_status;
+  return launch_status(launch_lindex(p, CSKV_F32, T, (cudaStream_t)stream));
+}
+
+static int attn_plan(int mode, int T, int k, int window, int64_t max_entries, int* R, int* S) {
+  int sms = 0;
+  int rc = device_sms(&sms);
+  if (rc) return rc;
+  *R = attn_rows_per_split(mode, T, k, window, max_entries, sms);
+  *S = attn_max_splits(mode, k, window, max_entries, *R);
+  return CSKV_OK;
+}
+
+size_t hybrid_attn_workspace_size(int mode, int T, int H, int d, int k, int window, int64_t max_entries) {
+  if (T < 1 || H < 1 || d != kHeadDim || window < 0) return 0;
+  int R = 0, S = 0;
+  if (attn_plan(mode, T, k, window, max_entries, &R, &S)) return 0;
+  return (size_t)T * S * H * (kHeadDim + 2) * sizeof(float);
+}
+
+int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off, const int32_t* idx,
+                       int k, const void* kv_raw, const int64_t* raw_off, const int64_t* raw_tok0, int window,
+                       const float* sink, float scale, const int32_t* q_seq, const int64_t* q_pos, int batch,
+                       int T, int H, int d, int dtype, int64_t max_entries, float* out, float* lse,
+                       void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream) {
+  if (mode != CSKV_CSA && mode != CSKV_HCA) return CSKV_ERR_INVALID_ARG;
+  if (dtype != CSKV_F32 && dtype != CSKV_BF16) return dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+  if (d != kHeadDim) return CSKV_ERR_UNSUPPORTED;
+  if (H < 1 || H > 128 || T < 0 || window < 0 || window > (1 << 20) || batch < 1) return CSKV_ERR_INVALID_ARG;
+  if (mode == CSKV_CSA && (k < 1 || k > (1 << 20) || !idx)) return CSKV_ERR_INVALID_ARG;
+  if (mode == CSKV_HCA && (max_entries < 0 || max_entries > (1LL << 30))) return CSKV_ERR_INVALID_ARG;
+  if (T == 0) return CSKV_OK;
+  if (!q || !kv_cmp || !cmp_off || !kv_raw || !raw_off || !q_seq || !q_pos || !out) return CSKV_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_cmp) || !aligned16(kv_raw)) return CSKV_ERR_INVALID_ARG;
+  if (!(scale == scale)) return CSKV_ERR_INVALID_ARG;
+  int R = 0, S = 0;
+  int rc = attn_plan(mode, T, mode == CSKV_CSA ? k : 0, window, max_entries, &R, &S);
+  if (rc) return rc;
+  const size_t need = (size_t)T * S * H * (kHeadDim + 2) * sizeof(float);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSKV_ERR_WORKSPACE;
+  AttnParams p = {};
+  p.mode = mode;
+  p.q = q;
+  p.kv_cmp = kv_cmp;
+  p.cmp_off = cmp_off;
+  p.idx = idx;
+  p.k = mode == CSKV_CSA ? k : 0;
+  p.kv_raw = kv_raw;
+  p.raw_off = raw_off;
+  p.raw_tok0 = raw_tok0;
+  p.window = window;
+  p.sink = sink;
+  p.scale_log2 = scale * kLog2e;
+  p.q_seq = q_seq;
+  p.q_pos = q_pos;
+  p.batch = batch;
+  p.T = T;
+  p.H = H;
+  p.rows_per_split = R;
+  p.max_splits = S;
+  p.part_acc = (float*)workspace;
+  p.part_ml = p.part_acc + (size_t)T * S * H * kHeadDim;
+  p.out = out;
+  p.lse = lse;
+  p.st = dev_status;
+  return launch_status(launch_attn_generic(p, dtype, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,309 @@
+// Hybrid decode attention on CUDA cores: split-KV partials + merge with the sink.
+//
+// [SW] = shareware.cn/news/167317 (DeepSeek V4 Hybrid Attention essay): §三.1 / §十
+// (raw 128-token window, which also covers the query's incomplete block), §六 (main
+// attention over the indexer's top-k), §八 (HCA: dense over every entry), §十一 (MQA: all
+// query heads share one KV), §十二 (attention sink).  [TR] = trdm.cn/news/516303: §2.2
+// (QK^T / sqrt(d_k)), §3.1 (online softmax: running max and sum reproduce the full
+// softmax exactly), §4.3 (compressed rows and window rows concatenated; HCA keeps the
+// token-granularity window).
+//
+// Rows of query t (position p, sequence b) form one virtual list:
+//   [0, n_cmp)       CSA: idx[t, r] (skipped when < 0);  HCA: entry r (r < floor((p+1)/128))
+//   [n_cmp, +W)      window token p - W + 1 + (r - n_cmp) (skipped when < 0)
+// CTA (split s, query t) runs an online softmax over rows [s*R, (s+1)*R) in tiles of 32
+// and writes (m, l, acc) in the log2 domain; attn_combine merges the splits of a query
+// and folds the sink logit in once.  This generic kernel serves fp32 and any head count;
+// bf16 with many heads goes to the tensor-core kernel.
+#include "launch.cuh"
+
+namespace cskv {
+
+
+struct QueryRows {
+  int s;          // sequence (-1: invalid query)
+  int64_t pos;    // position
+  int64_t n_cmp;  // compressed slots
+  int64_t vis_c;  // visible CSA entries (index check)
+  int64_t cmp0, cmp_cap, raw0, raw_rows, tok0;
+  int64_t n_rows;
+};
+
+__device__ __forceinline__ QueryRows query_rows(const AttnParams& p, int t) {
+  QueryRows q;
+  q.s = __ldg(p.q_seq + t);
+  if (q.s < 0 || q.s >= p.batch) {
+    q.s = -1;
+    q.n_rows = 0;
+    return q;
+  }
+  q.pos = __ldg(p.q_pos + t);
+  q.cmp0 = __ldg(p.cmp_off + q.s);
+  q.cmp_cap = __ldg(p.cmp_off + q.s + 1) - q.cmp0;
+  q.raw0 = __ldg(p.raw_off + q.s);
+  q.raw_rows = __ldg(p.raw_off + q.s + 1) - q.raw0;
+  q.tok0 = p.raw_tok0 ? __ldg(p.raw_tok0 + q.s) : 0;
+  const int64_t ratio = p.mode == CSKV_CSA ? 4 : 128;
+  const int64_t vis = q.pos >= 0 ? (q.pos + 1) / ratio : 0;
+  q.vis_c = vis < q.cmp_cap ? vis : q.cmp_cap;
+  q.n_cmp = p.mode == CSKV_CSA ? p.k : q.vis_c;
+  q.n_rows = q.n_cmp + p.window;
+  return q;
+}
+
+// Row pointer (element offset into kv_cmp or kv_raw) of virtual row r, or -1 when the
+// row is skipped.  *raw tells which array.
+__device__ __forceinline__ int64_t resolve_row(const AttnParams& p, const QueryRows& q, int t, int64_t r,
+                                               bool* raw) {
+  if (r < q.n_cmp) {
+    *raw = false;
+    int64_t e = r;
+    if (p.mode == CSKV_CSA) {
+      e = __ldg(p.idx + (size_t)t * p.k + r);
+      if (e < 0) return -1;
+      if (e >= q.vis_c) {
+        flag(p.st, CSKV_DEV_BAD_INDEX);
+        return -1;
+      }
+    }
+    return (q.cmp0 + e) * kRow;
+  }
+  *raw = true;
+  const int64_t tok = q.pos - p.window + 1 + (r - q.n_cmp);
+  if (tok < 0) return -1;
+  const int64_t row = tok - q.tok0;
+  if (row < 0) {
+    flag(p.st, CSKV_DEV_TAIL_MISSING);
+    return -1;
+  }
+  if (row >= q.raw_rows) {
+    flag(p.st, CSKV_DEV_BAD_INDEX);
+    return -1;
+  }
+  return (q.raw0 + row) * kRow;
+}
+
+constexpr int kAttnThreads = 256;
+constexpr int kAttnTile = 32;
+constexpr int kPsStride = kAttnTile + 1;  // padded row of the probability tile
+
+template <typename T, int HP>
+__global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) {
+  constexpr int d = kHeadDim;
+  constexpr int TPH = kAttnThreads / HP;  // threads per head in the PV update
+  constexpr int ACC = d / TPH;            // accumulators per thread
+  extern __shared__ __align__(16) float smf[];
+  float* qs = smf;                               // [HP][d]
+  float* ks = qs + HP * d;                       // [tile][d + 1]
+  float* vs = ks + kAttnTile * (d + 1);          // [tile][d]
+  float* ps = vs + kAttnTile * d;                // [HP][tile + 1]
+  float* m_run = ps + HP * kPsStride;            // [HP]
+  float* l_run = m_run + HP;                     // [HP]
+  float* alpha = l_run + HP;                     // [HP]
+  __shared__ int valid[kAttnTile];
+
+  const int t = blockIdx.y, split = blockIdx.x, tid = threadIdx.x;
+  const QueryRows q = query_rows(p, t);
+  if (q.s < 0) {
+    if (split == 0 && tid == 0) flag(p.st, CSKV_DEV_BAD_INDEX);
+    return;
+  }
+  const int64_t r0 = (int64_t)split * p.rows_per_split;
+  if (r0 >= q.n_rows) return;
+  const int64_t r1 = min(q.n_rows, r0 + p.rows_per_split);
+  const int H = p.H;
+  const T* qg = reinterpret_cast<const T*>(p.q) + (size_t)t * H * d;
+  for (int i = tid; i < HP * d; i += kAttnThreads) qs[i] = (i < H * d) ? to_f(qg[i]) : 0.f;
+  for (int h = tid; h < HP; h += kAttnThreads) {
+    m_run[h] = -INFINITY;
+    l_run[h] = 0.f;
+  }
+  const int hh = tid / TPH, jj = tid % TPH;
+  float acc[ACC];
+#pragma unroll
+  for (int i = 0; i < ACC; ++i) acc[i] = 0.f;
+  const T* cmp = reinterpret_cast<const T*>(p.kv_cmp);
+  const T* raw = reinterpret_cast<const T*>(p.kv_raw);
+  __syncthreads();
+
+  for (int64_t a = r0; a < r1; a += kAttnTile) {
+    // ---- load up to 32 rows: thread -> (row tid/8, 32-value part tid%8)
+    {
+      const int rr = tid >> 3, part = tid & 7;
+      const int64_t r = a + rr;
+      int64_t off = -1;
+      bool is_raw = false;
+      if (r < r1) off = resolve_row(p, q, t, r, &is_raw);
+      if (part == 0) valid[rr] = off >= 0;
+      if (off >= 0) {
+        const T* src = (is_raw ? raw : cmp) + off + part * 32;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          float f[8];
+          Vec8<T>::load(src + 8 * v, f);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int col = part * 32 + 8 * v + u;
+            if (col < d)
+              ks[rr * (d + 1) + col] = f[u];
+            else
+              vs[rr * d + col - d] = f[u];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // ---- logits (log2 units)
+    for (int i = tid; i < H * kAttnTile; i += kAttnThreads) {
+      const int h = i / kAttnTile, rr = i % kAttnTile;
+      float s = -INFINITY;
+      if (valid[rr]) {
+        const float* qh = qs + h * d;
+        const float* kr = ks + rr * (d + 1);
+        float dot = 0.f;
+#pragma unroll 8
+        for (int c = 0; c < d; ++c) dot = fmaf(qh[c], kr[c], dot);
+        s = dot * p.scale_log2;
+      }
+      ps[h * kPsStride + rr] = s;
+    }
+    __syncthreads();
+    // ---- online softmax per head
+    for (int h = tid; h < H; h += kAttnThreads) {
+      float mt = -INFINITY;
+      for (int rr = 0; rr < kAttnTile; ++rr) mt = fmaxf(mt, ps[h * kPsStride + rr]);
+      const float m_old = m_run[h];
+      const float m_new = fmaxf(m_old, mt);
+      float al = 1.f, sum = 0.f;
+      if (m_new != -INFINITY) {
+        al = exp2f(m_old - m_new);
+        for (int rr = 0; rr < kAttnTile; ++rr) {
+          const float e = exp2f(ps[h * kPsStride + rr] - m_new);
+          ps[h * kPsStride + rr] = e;
+          sum += e;
+        }
+      } else {
+        for (int rr = 0; rr < kAttnTile; ++rr) ps[h * kPsStride + rr] = 0.f;
+      }
+      m_run[h] = m_new;
+      l_run[h] = l_run[h] * al + sum;
+      alpha[h] = al;
+    }
+    __syncthreads();
+    // ---- acc = acc * alpha + P V
+    if (hh < H) {
+      const float al = alpha[hh];
+#pragma unroll
+      for (int i = 0; i < ACC; ++i) acc[i] *= al;
+      for (int rr = 0; rr < kAttnTile; ++rr) {
+        if (!valid[rr]) continue;
+        const float pr = ps[hh * kPsStride + rr];
+        const float* vr = vs + rr * d;
+#pragma unroll
+        for (int i = 0; i < ACC; ++i) acc[i] = fmaf(pr, vr[jj + TPH * i], acc[i]);
+      }
+    }
+    __syncthreads();
+  }
+  // ---- partial out
+  const size_t pbase = ((size_t)t * p.max_splits + split) * H;
+  if (hh < H) {
+    float* dst = p.part_acc + (pbase + hh) * d;
+#pragma unroll
+    for (int i = 0; i < ACC; ++i) dst[jj + TPH * i] = acc[i];
+  }
+  for (int h = tid; h < H; h += kAttnThreads) {
+    p.part_ml[(pbase + h) * 2] = m_run[h];
+    p.part_ml[(pbase + h) * 2 + 1] = l_run[h];
+  }
+}
+
+// Merge the splits of each query ([TR] §3.1), the sink once ([SW] §十二):
+//   M = max(max_s m_s, sink), L = sum_s 2^{m_s - M} l_s + 2^{sink - M},
+//   o = sum_s 2^{m_s - M} acc_s / L,   lse = ln 2 * (M + log2 L).
+__global__ void __launch_bounds__(256) attn_combine_kernel(AttnParams p) {
+  const int t = blockIdx.x;
+  const QueryRows q = query_rows(p, t);
+  const int H = p.H;
+  int S = q.s < 0 ? 0 : (int)((q.n_rows + p.rows_per_split - 1) / p.rows_per_split);
+  if (S > p.max_splits) {
+    if (threadIdx.x == 0) flag(p.st, CSKV_DEV_CAPACITY);
+    S = p.max_splits;
+  }
+  for (int i = threadIdx.x; i < H * kHeadDim; i += blockDim.x) {
+    const int h = i / kHeadDim, j = i % kHeadDim;
+    const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+    const float* ml = p.part_ml + ((size_t)t * p.max_splits * H + h) * 2;
+    float M = sk;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, ml[(size_t)s * H * 2]);
+    float L = 0.f, o = 0.f;
+    if (M != -INFINITY) {
+      if (p.sink) L = exp2f(sk - M);
+      const float* acc = p.part_acc + ((size_t)t * p.max_splits * H + h) * kHeadDim + j;
+      for (int s = 0; s < S; ++s) {
+        const float ms = ml[(size_t)s * H * 2];
+        if (ms == -INFINITY) continue;
+        const float f = exp2f(ms - M);
+        L = fmaf(ml[(size_t)s * H * 2 + 1], f, L);
+        o = fmaf(acc[(size_t)s * H * kHeadDim], f, o);
+      }
+    }
+    p.out[((size_t)t * H + h) * kHeadDim + j] = L > 0.f ? o / L : 0.f;
+    if (j == 0 && p.lse) p.lse[(size_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  }
+}
+
+// ------------------------------------------------------------------ host side
+static int attn_hp(int H) { return H <= 16 ? 16 : H <= 32 ? 32 : H <= 64 ? 64 : 128; }
+
+static size_t attn_smem(int HP) {
+  const int d = kHeadDim;
+  return sizeof(float) * ((size_t)HP * d + kAttnTile * (d + 1) + kAttnTile * d + HP * kPsStride + 3 * HP);
+}
+
+int attn_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms) {
+  const int64_t rows_max = (mode == CSKV_CSA ? (int64_t)k : max_entries) + window;
+  int64_t R = (rows_max * (int64_t)T + 2 * sms - 1) / (2 * (int64_t)sms);
+  R = (R + kAttnTile - 1) / kAttnTile * kAttnTile;
+  if (R < kAttnTile) R = kAttnTile;
+  if (R > 4096) R = 4096;
+  return (int)R;
+}
+
+int attn_max_splits(int mode, int k, int window, int64_t max_entries, int R) {
+  const int64_t rows_max = (mode == CSKV_CSA ? (int64_t)k : max_entries) + window;
+  const int64_t s = (rows_max + R - 1) / R;
+  return (int)(s > 0 ? s : 1);
+}
+
+template <typename T, int HP>
+static cudaError_t launch_split(const AttnParams& p, cudaStream_t stream) {
+  const size_t smem = attn_smem(HP);
+  auto kern = attn_split_kernel<T, HP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.max_splits, p.T);
+  kern<<<grid, kAttnThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t stream) {
+  const int hp = attn_hp(p.H);
+  cudaError_t e;
+  if (dtype == CSKV_F32) {
+    e = hp == 16 ? launch_split<float, 16>(p, stream)
+        : hp == 32 ? launch_split<float, 32>(p, stream)
+        : hp == 64 ? launch_split<float, 64>(p, stream)
+                   : launch_split<float, 128>(p, stream);
+  } else {
+    e = hp == 16 ? launch_split<__nv_bfloat16, 16>(p, stream)
+        : hp == 32 ? launch_split<__nv_bfloat16, 32>(p, stream)
+        : hp == 64 ? launch_split<__nv_bfloat16, 64>(p, stream)
+                   : launch_split<__nv_bfloat16, 128>(p, stream);
+  }
+  if (e != cudaSuccess) return e;
+  attn_combine_kernel<<<p.T, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace cskv

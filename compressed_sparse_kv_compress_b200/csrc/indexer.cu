@@ -1,0 +1,800 @@
+// Lightning Indexer scan fused with an exact top-k.
+//
+// [SW] = shareware.cn/news/167317 (DeepSeek V4 Hybrid Attention essay): §六 (cheap
+// scoring of every compressed entry, then top-k, then the main attention; low
+// precision), §七 (ReLU per head before the heads are summed), §十 (a query sees
+// complete blocks only).  [TR] = trdm.cn/news/516303, §4.2 (LightningIndexer:
+// scores = relu(q_idx k_idx^T), FP8).  [AM] = aimodeling.com DeepSeek V4 news (k = 1024).
+//
+// Query t sees CSA entries i < V_t = floor((p_t + 1) / 4) and scores
+//     s_i = sum_h w_h * ReLU(sq_h * sk_i * <q_h, k_i>).
+// The min(k, V_t) best entries are kept (equal scores: lower index first) and written
+// in ascending index order, padded with -1.
+//
+// Work decomposition.  A query's entries are cut into contiguous segments, one per
+// CTA; the CTAs of one query form a group.
+//  * split mode (few queries, decode): one round, every CTA of a cooperative grid
+//    gets one segment, groups sized in proportion to V_t;
+//  * row mode (many queries, prefill): every CTA owns whole queries (group of one)
+//    and loops over them.
+// A segment's scores never leave shared memory.  Selection is a most-significant-digit
+// radix select on the 64-bit key (order-preserving score bits << 32 | ~index), so the
+// selected set is "key >= threshold" and ties resolve to the lower index exactly:
+//  pass 0: 12-bit digit histogram of the group (shared atomics, then global atomics
+//          and one group barrier when the group has several CTAs);
+//  then, if the threshold bin holds <= kCandMax entries, they are compacted to global
+//  memory (second barrier) and every CTA finishes the selection on that small set in
+//  shared memory; otherwise further 10-bit global passes run (rare: massive ties).
+//  Output positions come from per-CTA counts, so the result needs no sort.
+//
+// Scan of E4M3 keys: a producer warp streams 128-entry tiles (8 KiB) of k_idx into a
+// shared-memory ring with TMA bulk copies; eight consumer warps each take 16 entries of
+// a tile and run m16n8k32 E4M3 MMAs (entries x dims) x (dims x 8 heads) with fp32
+// accumulation -- the head dimension fills N = 8 exactly -- then apply scales, ReLU and
+// the head sum in registers.
+#include "launch.cuh"
+#include "sm100.cuh"
+
+namespace cskv {
+
+constexpr int kIdxConsumerWarps = 8;
+constexpr int kIdxThreads = 32 * (kIdxConsumerWarps + 1);  // + one producer warp
+constexpr int kIdxTile = 16 * kIdxConsumerWarps;          // entries per ring stage
+constexpr int kBins0 = 4096;                              // first digit: 12 bits
+constexpr int kBinsP = 1024;                              // later digits: 10 bits
+constexpr int kMaxPasses = 7;                             // 12 + 5 * 10 + 2 = 64 bits
+constexpr int kCandMax = 4096;
+constexpr int kMaxGroup = 1024;
+constexpr int kMinSeg = 256;
+constexpr int kMaxSplitQueries = 128;
+constexpr int kIdxMaxHeads = 16;
+constexpr int kIdxMaxDim = 128;
+
+enum IdxSrc { kSrcFp8 = 0, kSrcF32 = 1, kSrcScores = 2 };
+
+struct alignas(16) QueryWS {
+  unsigned bar_count, bar_gen, done, cand_count;
+  unsigned hist0[kBins0];
+  unsigned histp[kMaxPasses - 1][kBinsP];
+  unsigned above[kMaxGroup];
+  unsigned long long cand[kCandMax];
+};
+
+
+// TMA ring depth: 48 KiB of k_idx tiles in flight per CTA whatever Di is.
+__host__ __device__ constexpr int idx_stages(int Di) { return 6 * 64 / Di; }
+
+// Bytes of the shared region used first as the TMA ring, then for histograms and
+// candidates (48 KiB either way).
+__host__ __device__ constexpr size_t idx_union_bytes(int Di) {
+  return (size_t)idx_stages(Di) * kIdxTile * Di > (size_t)kBins0 * 4 + (size_t)kCandMax * 8
+             ? (size_t)idx_stages(Di) * kIdxTile * Di
+             : (size_t)kBins0 * 4 + (size_t)kCandMax * 8;
+}
+
+// ------------------------------------------------------------------ keys
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t u = __float_as_uint(s);
+  if (u == 0x80000000u) u = 0u;  // -0 ranks with +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ uint64_t comp_key(float s, int64_t e) {
+  return ((uint64_t)score_key(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
+}
+__device__ __forceinline__ bool key_selected(uint64_t c, uint64_t P, int nb) {
+  return (c >> (64 - nb)) >= P;
+}
+
+// ------------------------------------------------------------------ block helpers
+// Exclusive prefix sum over threads in thread order; *total receives the sum.
+__device__ unsigned block_excl_scan(unsigned v, unsigned* red, unsigned* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  unsigned x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    unsigned y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned w = lane < nw ? red[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      unsigned y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) red[lane] = w;  // inclusive warp-total prefix
+  }
+  __syncthreads();
+  const unsigned before = (warp ? red[warp - 1] : 0u) + x - v;
+  if (total) *total = red[nw - 1];
+  __syncthreads();
+  return before;
+}
+
+struct Crossing {
+  unsigned bin, above, cnt;
+};
+
+// hist[nbins] in shared memory; finds the bin where the count accumulated from the
+// highest bin downwards first reaches r (1 <= r <= sum of hist).
+__device__ Crossing find_crossing(const unsigned* hist, int nbins, unsigned r, unsigned* red, Crossing* out) {
+  const int per = nbins >= 256 ? nbins / 256 : 1;
+  const int nthr = nbins / per;
+  const int tid = threadIdx.x;
+  if (tid == 0) {  // safe default if a corrupted histogram never reaches r
+    out->bin = 0;
+    out->above = 0;
+    out->cnt = r;
+  }
+  unsigned local = 0;
+  int hi = 0, lo = 0;
+  if (tid < nthr) {
+    hi = nbins - tid * per;  // exclusive
+    lo = hi - per;
+    for (int b = hi - 1; b >= lo; --b) local += hist[b];
+  }
+  const unsigned excl = block_excl_scan(local, red, nullptr);
+  if (tid < nthr && local > 0 && excl < r && r <= excl + local) {
+    unsigned cum = excl;
+    for (int b = hi - 1; b >= lo; --b) {
+      const unsigned h = hist[b];
+      if (cum + h >= r) {
+        out->bin = (unsigned)b;
+        out->above = cum;
+        out->cnt = h;
+        break;
+      }
+      cum += h;
+    }
+  }
+  __syncthreads();
+  Crossing c = *out;
+  __syncthreads();
+  return c;
+}
+
+// Barrier over the G CTAs of one query group (all co-resident: cooperative launch).
+// Bounded: gives up after ~1 s and reports CSKV_DEV_TIMEOUT.
+__device__ bool group_barrier(QueryWS* ws, unsigned G, int* st, int* sm_flag) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool ok = true;
+    const unsigned g0 = ld_acquire_gpu(&ws->bar_gen);
+    const unsigned arrived = atomicAdd(&ws->bar_count, 1u);
+    if (arrived == G - 1) {
+      atomicExch(&ws->bar_count, 0u);
+      __threadfence();
+      atomicAdd(&ws->bar_gen, 1u);
+    } else {
+      long it = 0;
+      while (ld_acquire_gpu(&ws->bar_gen) == g0) {
+        if (++it > (1L << 24)) {
+          ok = false;
+          flag(st, CSKV_DEV_TIMEOUT);
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    *sm_flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  __threadfence();
+  return *sm_flag != 0;
+}
+
+// ------------------------------------------------------------------ shared state
+struct IdxShared {
+  uint64_t full[8];
+  uint64_t empty[8];
+  unsigned red[32];
+  Crossing cross;
+  int flag;
+  unsigned ubuf[4];
+  int plan_t, plan_j, plan_G;
+  long long plan_V[kMaxSplitQueries];
+  float q_f32[kIdxMaxHeads * kIdxMaxDim];
+};
+
+// ------------------------------------------------------------------ scan: E4M3 via TMA + MMA
+template <int KS, int NTILE>
+__device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, int64_t len,
+                         float* sc, uint8_t* ring, IdxShared& S) {
+  constexpr int Di = KS * 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int stages = p.stages;
+  const int64_t ntiles = (len + kIdxTile - 1) / kIdxTile;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], kIdxConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  // generic-proxy writes to the ring region (histograms of a previous segment) must be
+  // ordered before the TMA unit writes it
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
+  if (warp == kIdxConsumerWarps) {
+    if (lane == 0) {
+      for (int64_t it = 0; it < ntiles; ++it) {
+        const int s = (int)(it % stages);
+        const unsigned ph = (unsigned)((it / stages) & 1);
+        if (it >= stages && !mbar_wait_bounded(&S.empty[s], ph ^ 1u)) {
+          flag(p.st, CSKV_DEV_TIMEOUT);
+          break;
+        }
+        const int64_t rows = min((int64_t)kIdxTile, len - it * kIdxTile);
+        const unsigned bytes = (unsigned)(rows * Di);
+        mbar_arrive_expect_tx(&S.full[s], bytes);
+        tma_bulk_g2s(ring + (size_t)s * kIdxTile * Di, kbase + it * kIdxTile * Di, bytes, &S.full[s]);
+      }
+    }
+  } else {
+    const int g = lane >> 2, tq = lane & 3;
+    // B fragments (the query's heads) and per-head scale / weight, loaded once.
+    uint32_t bq[NTILE][KS][2];
+    float sq[NTILE][2], wh[NTILE][2];
+    const uint8_t* qrow = p.q_idx + (size_t)t * p.Hi * Di;
+#pragma unroll
+    for (int nt = 0; nt < NTILE; ++nt) {
+      const int h = nt * 8 + g;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int chunk = tq + 4 * (ks >> 1), wp = (ks & 1) * 2;
+        if (h < p.Hi) {
+          const uint32_t* src = reinterpret_cast<const uint32_t*>(qrow + (size_t)h * Di + chunk * 16);
+          bq[nt][ks][0] = __ldg(src + wp);
+          bq[nt][ks][1] = __ldg(src + wp + 1);
+        } else {
+          bq[nt][ks][0] = bq[nt][ks][1] = 0u;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int h = nt * 8 + 2 * tq + c;
+        const bool ok = h < p.Hi;
+        sq[nt][c] = ok ? (p.q_scale ? __ldg(p.q_scale + (size_t)t * p.Hi + h) : 1.f) : 0.f;
+        wh[nt][c] = ok ? (p.head_w ? __ldg(p.head_w + h) : 1.f) : 0.f;
+      }
+    }
+    bool alive = true;
+    for (int64_t it = 0; it < ntiles && alive; ++it) {
+      const int s = (int)(it % stages);
+      const unsigned ph = (unsigned)((it / stages) & 1);
+      if (!mbar_wait_bounded(&S.full[s], ph)) {
+        flag(p.st, CSKV_DEV_TIMEOUT);
+        alive = false;
+        break;
+      }
+      const int64_t rows = min((int64_t)kIdxTile, len - it * kIdxTile);
+      const int r0 = warp * 16;
+      if (r0 < rows) {
+        const uint8_t* tile = ring + (size_t)s * kIdxTile * Di;
+        uint4 ra[KS / 2], rb[KS / 2];
+#pragma unroll
+        for (int c = 0; c < KS / 2; ++c) {
+          ra[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g) * Di + (tq + 4 * c) * 16);
+          rb[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g + 8) * Di + (tq + 4 * c) * 16);
+        }
+        float acc[NTILE][4];
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt) {
+          acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const uint4& A = ra[ks >> 1];
+            const uint4& B = rb[ks >> 1];
+            const bool hiw = ks & 1;
+            mma_e4m3_16832(acc[nt], hiw ? A.z : A.x, hiw ? B.z : B.x, hiw ? A.w : A.y, hiw ? B.w : B.y,
+                           bq[nt][ks][0], bq[nt][ks][1]);
+          }
+        }
+        const int64_t e_g = it * kIdxTile + r0 + g, e_g8 = e_g + 8;
+        const float skg = (e_g < len) ? (kscale ? __ldg(kscale + e_g) : 1.f) : 0.f;
+        const float skg8 = (e_g8 < len) ? (kscale ? __ldg(kscale + e_g8) : 1.f) : 0.f;
+        float vg = 0.f, vg8 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            vg = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * skg) * acc[nt][c]), vg);
+            vg8 = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * skg8) * acc[nt][2 + c]), vg8);
+          }
+        vg += __shfl_xor_sync(0xffffffffu, vg, 1);
+        vg += __shfl_xor_sync(0xffffffffu, vg, 2);
+        vg8 += __shfl_xor_sync(0xffffffffu, vg8, 1);
+        vg8 += __shfl_xor_sync(0xffffffffu, vg8, 2);
+        if (tq == 0 && e_g < len) sc[e_g] = vg;
+        if (tq == 1 && e_g8 < len) sc[e_g8] = vg8;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[s]);
+    }
+  }
+  __syncthreads();
+  // Every copy issued has completed (each full barrier was waited on), so the ring can be
+  // reused and the barriers retired.
+  if (threadIdx.x == 0)
+    for (int s = 0; s < stages; ++s) {
+      asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(&S.full[s])) : "memory");
+      asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(&S.empty[s])) : "memory");
+    }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ scan: fp32 (CUDA cores)
+__device__ void scan_f32(const IdxParams& p, int t, const float* kbase, const float* kscale, int64_t len,
+                         float* sc, IdxShared& S) {
+  const int Hi = p.Hi, Di = p.Di;
+  for (int i = threadIdx.x; i < Hi * Di; i += blockDim.x)
+    S.q_f32[i] = reinterpret_cast<const float*>(p.q_idx)[(size_t)t * Hi * Di + i];
+  __syncthreads();
+  float sq[kIdxMaxHeads], wh[kIdxMaxHeads];
+#pragma unroll
+  for (int h = 0; h < kIdxMaxHeads; ++h) {
+    sq[h] = (h < Hi) ? (p.q_scale ? __ldg(p.q_scale + (size_t)t * Hi + h) : 1.f) : 0.f;
+    wh[h] = (h < Hi) ? (p.head_w ? __ldg(p.head_w + h) : 1.f) : 0.f;
+  }
+  for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
+    float acc[kIdxMaxHeads];
+#pragma unroll
+    for (int h = 0; h < kIdxMaxHeads; ++h) acc[h] = 0.f;
+    const float4* kr = reinterpret_cast<const float4*>(kbase + (size_t)e * Di);
+    for (int d4 = 0; d4 < Di / 4; ++d4) {
+      const float4 kv = __ldg(kr + d4);
+#pragma unroll
+      for (int h = 0; h < kIdxMaxHeads; ++h)
+        if (h < Hi) {
+          const float* q = S.q_f32 + h * Di + 4 * d4;
+          acc[h] = fmaf(q[0], kv.x, acc[h]);
+          acc[h] = fmaf(q[1], kv.y, acc[h]);
+          acc[h] = fmaf(q[2], kv.z, acc[h]);
+          acc[h] = fmaf(q[3], kv.w, acc[h]);
+        }
+    }
+    const float sk = kscale ? __ldg(kscale + e) : 1.f;
+    float v = 0.f;
+#pragma unroll
+    for (int h = 0; h < kIdxMaxHeads; ++h)
+      if (h < Hi) v = fmaf(wh[h], fmaxf(0.f, (sq[h] * sk) * acc[h]), v);
+    sc[e] = v;
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ selection helpers
+// One local radix pass over `n` keys produced by get(i), restricted to keys whose top
+// nb bits equal P.  Updates (P, nb, r); returns true when the threshold is final.
+template <typename Get>
+__device__ bool local_pass(Get get, int64_t n, uint64_t& P, int& nb, unsigned& r, unsigned* hist,
+                           IdxShared& S) {
+  const int w = min(10, 64 - nb);
+  const int nbins = 1 << w;
+  for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint64_t c = get(i);
+    if ((c >> (64 - nb)) == P) atomicAdd(&hist[(unsigned)((c >> (64 - nb - w)) & (uint64_t)(nbins - 1))], 1u);
+  }
+  __syncthreads();
+  const Crossing x = find_crossing(hist, nbins, r, S.red, &S.cross);
+  P = (P << w) | x.bin;
+  nb += w;
+  r -= x.above;
+  return x.cnt == r || nb == 64;
+}
+
+// Writes the selected entries of this segment in ascending order at out[base ...].
+// Positions are bounded by k, so even an inconsistent threshold (after a timed-out
+// group barrier) cannot write outside the output row.
+__device__ void emit(const float* sc, int64_t len, int64_t lo, bool all, uint64_t P, int nb, int64_t base,
+                     int64_t k, int32_t* oi, float* os, IdxShared& S) {
+  const int64_t per = (len + blockDim.x - 1) / blockDim.x;
+  const int64_t a = min(len, (int64_t)threadIdx.x * per), b = min(len, a + per);
+  unsigned c = 0;
+  for (int64_t e = a; e < b; ++e) c += (all || key_selected(comp_key(sc[e], lo + e), P, nb)) ? 1u : 0u;
+  int64_t pos = base + block_excl_scan(c, S.red, nullptr);
+  for (int64_t e = a; e < b; ++e)
+    if (all || key_selected(comp_key(sc[e], lo + e), P, nb)) {
+      if (pos >= 0 && pos < k) {
+        oi[pos] = (int32_t)(lo + e);
+        if (os) os[pos] = sc[e];
+      }
+      ++pos;
+    }
+}
+
+__device__ unsigned count_selected(const float* sc, int64_t len, int64_t lo, uint64_t P, int nb, IdxShared& S) {
+  unsigned c = 0;
+  for (int64_t e = threadIdx.x; e < len; e += blockDim.x) c += key_selected(comp_key(sc[e], lo + e), P, nb);
+  unsigned tot;
+  block_excl_scan(c, S.red, &tot);
+  return tot;
+}
+
+// ------------------------------------------------------------------ one segment
+template <int SRC, int KS, int NTILE>
+__device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t V, int64_t ebase, QueryWS* ws,
+                                float* sc, uint8_t* un, IdxShared& S) {
+  const int64_t lo = (int64_t)j * V / G, hi = (int64_t)(j + 1) * V / G;
+  int64_t len = hi - lo;
+  const size_t tq = (size_t)t;
+  int32_t* oi = p.out_idx + tq * p.k;
+  float* os = p.out_score ? p.out_score + tq * p.k : nullptr;
+  const int64_t keff = min((int64_t)p.k, V);
+  if (j == 0)
+    for (int64_t i = keff + threadIdx.x; i < p.k; i += blockDim.x) {
+      oi[i] = -1;
+      if (os) os[i] = 0.f;
+    }
+  if (keff == 0) return;
+  if (len > p.seg_cap) {
+    if (threadIdx.x == 0) flag(p.st, CSKV_DEV_CAPACITY);
+    len = p.seg_cap;
+  }
+  // ---- scores of this segment into shared memory
+  if constexpr (SRC == kSrcFp8) {
+    const uint8_t* kb = p.k_idx + (size_t)(ebase + lo) * (KS * 32);
+    const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
+    scan_fp8<KS, NTILE>(p, t, kb, ks, len, sc, un, S);
+  } else if constexpr (SRC == kSrcF32) {
+    const float* kb = reinterpret_cast<const float*>(p.k_idx) + (size_t)(ebase + lo) * p.Di;
+    const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
+    scan_f32(p, t, kb, ks, len, sc, S);
+  } else {
+    const float* src = p.scores + tq * p.ld_scores + lo;
+    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) sc[e] = __ldg(src + e);
+    __syncthreads();
+  }
+  // ---- everything kept: output position of entry e is e
+  if (keff == V) {
+    emit(sc, len, lo, true, 0, 0, lo, keff, oi, os, S);
+    return;
+  }
+  unsigned* hist = reinterpret_cast<unsigned*>(un);
+  unsigned long long* cands = reinterpret_cast<unsigned long long*>(un + kBins0 * 4);
+  // ---- pass 0: 12-bit digit
+  for (int i = threadIdx.x; i < kBins0; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for (int64_t e = threadIdx.x; e < len; e += blockDim.x) atomicAdd(&hist[score_key(sc[e]) >> 20], 1u);
+  __syncthreads();
+  bool ok = true;
+  if (G > 1) {
+    for (int i = threadIdx.x; i < kBins0; i += blockDim.x)
+      if (hist[i]) atomicAdd(&ws->hist0[i], hist[i]);
+    ok = group_barrier(ws, G, p.st, &S.flag);
+    for (int i = threadIdx.x; i < kBins0; i += blockDim.x) hist[i] = __ldcg(&ws->hist0[i]);
+    __syncthreads();
+  }
+  unsigned r = (unsigned)keff;
+  Crossing x = find_crossing(hist, kBins0, r, S.red, &S.cross);
+  uint64_t P = x.bin;
+  int nb = 12;
+  r -= x.above;
+  bool done = (x.cnt == r);
+  int used_passes = 0;
+  int64_t base = 0;
+  bool have_base = (G == 1);
+  if (!done && G == 1) {
+    while (!done) done = local_pass([&](int64_t i) { return comp_key(sc[i], lo + i); }, len, P, nb, r, hist, S);
+  } else if (!done && x.cnt <= kCandMax) {
+    // compaction of the threshold bin's entries into the group's candidate list
+    const unsigned b0 = x.bin;
+    unsigned above = 0, mine = 0;
+    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
+      const unsigned d = score_key(sc[e]) >> 20;
+      above += d > b0;
+    }
+    const int64_t per = (len + blockDim.x - 1) / blockDim.x;
+    const int64_t a = min(len, (int64_t)threadIdx.x * per), b = min(len, a + per);
+    for (int64_t e = a; e < b; ++e) mine += (score_key(sc[e]) >> 20) == b0;
+    unsigned tot_above, tot_mine;
+    block_excl_scan(above, S.red, &tot_above);
+    const unsigned off = block_excl_scan(mine, S.red, &tot_mine);
+    if (threadIdx.x == 0) {
+      S.ubuf[0] = tot_mine ? atomicAdd(&ws->cand_count, tot_mine) : 0u;
+      ws->above[j] = tot_above;
+    }
+    __syncthreads();
+    unsigned slot = S.ubuf[0] + off;
+    for (int64_t e = a; e < b; ++e)
+      if ((score_key(sc[e]) >> 20) == b0) {
+        if (slot < (unsigned)kCandMax) ws->cand[slot] = comp_key(sc[e], lo + e);
+        ++slot;
+      }
+    ok = group_barrier(ws, G, p.st, &S.flag) && ok;
+    const unsigned n_c = min(__ldcg(&ws->cand_count), (unsigned)kCandMax);
+    for (unsigned i = threadIdx.x; i < n_c; i += blockDim.x) cands[i] = __ldcg(&ws->cand[i]);
+    __syncthreads();
+    while (!done) done = local_pass([&](int64_t i) { return (uint64_t)cands[i]; }, n_c, P, nb, r, hist, S);
+    // output base = selected entries of lower segments
+    unsigned c = 0;
+    for (unsigned i = threadIdx.x; i < n_c; i += blockDim.x) {
+      const uint64_t ck = cands[i];
+      const int64_t e = (int64_t)(0xFFFFFFFFu - (uint32_t)(ck & 0xFFFFFFFFull));
+      c += (e < lo && key_selected(ck, P, nb)) ? 1u : 0u;
+    }
+    for (int i = threadIdx.x; i < j; i += blockDim.x) c += __ldcg(&ws->above[i]);
+    unsigned tot;
+    block_excl_scan(c, S.red, &tot);
+    base = tot;
+    have_base = true;
+  } else if (!done) {
+    // massive ties: further digits through the group's global histograms
+    while (!done && ok) {
+      const int w = min(10, 64 - nb);
+      const int nbins = 1 << w;
+      for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0u;
+      __syncthreads();
+      for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
+        const uint64_t c = comp_key(sc[e], lo + e);
+        if ((c >> (64 - nb)) == P) atomicAdd(&hist[(unsigned)((c >> (64 - nb - w)) & (uint64_t)(nbins - 1))], 1u);
+      }
+      __syncthreads();
+      unsigned* gh = ws->histp[used_passes];
+      for (int i = threadIdx.x; i < nbins; i += blockDim.x)
+        if (hist[i]) atomicAdd(&gh[i], hist[i]);
+      ++used_passes;
+      ok = group_barrier(ws, G, p.st, &S.flag) && ok;
+      for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = __ldcg(&gh[i]);
+      __syncthreads();
+      const Crossing y = find_crossing(hist, nbins, r, S.red, &S.cross);
+      P = (P << w) | y.bin;
+      nb += w;
+      r -= y.above;
+      done = (y.cnt == r) || nb == 64;
+    }
+  }
+  if (!have_base) {
+    // per-segment selected counts -> output offsets
+    const unsigned mine = count_selected(sc, len, lo, P, nb, S);
+    if (threadIdx.x == 0) ws->above[j] = mine;
+    ok = group_barrier(ws, G, p.st, &S.flag) && ok;
+    unsigned c = 0;
+    for (int i = threadIdx.x; i < j; i += blockDim.x) c += __ldcg(&ws->above[i]);
+    unsigned tot;
+    block_excl_scan(c, S.red, &tot);
+    base = tot;
+  }
+  emit(sc, len, lo, false, P, nb, base, keff, oi, os, S);
+  if (G > 1) {
+    // the last CTA of the group to finish returns the group's workspace to zero
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) S.flag = (atomicAdd(&ws->done, 1u) == (unsigned)(G - 1));
+    __syncthreads();
+    if (S.flag) {
+      __threadfence();
+      for (int i = threadIdx.x; i < kBins0; i += blockDim.x) ws->hist0[i] = 0u;
+      for (int q = 0; q < used_passes; ++q)
+        for (int i = threadIdx.x; i < kBinsP; i += blockDim.x) ws->histp[q][i] = 0u;
+      if (threadIdx.x == 0) {
+        ws->cand_count = 0u;
+        ws->done = 0u;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__device__ __forceinline__ int64_t visible_of(const IdxParams& p, int t, int64_t* ebase) {
+  if (p.scores) {
+    *ebase = 0;
+    int64_t v = __ldg(p.n_valid + t);
+    if (v < 0 || v > p.ld_scores) {
+      flag(p.st, CSKV_DEV_BAD_INDEX);
+      v = v < 0 ? 0 : p.ld_scores;
+    }
+    return v;
+  }
+  const int s = __ldg(p.q_seq + t);
+  if (s < 0 || s >= p.batch) {
+    flag(p.st, CSKV_DEV_BAD_INDEX);
+    *ebase = 0;
+    return 0;
+  }
+  const int64_t e0 = __ldg(p.ent_off + s), e1 = __ldg(p.ent_off + s + 1);
+  *ebase = e0;
+  const int64_t pos = __ldg(p.q_pos + t);
+  int64_t v = pos >= 0 ? (pos + 1) / 4 : 0;
+  if (v > e1 - e0) {
+    flag(p.st, CSKV_DEV_BAD_INDEX);
+    v = e1 - e0;
+  }
+  return v;
+}
+
+template <int SRC, int KS, int NTILE>
+__global__ void __launch_bounds__(kIdxThreads, 1) lindex_topk_kernel(IdxParams p) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ IdxShared S;
+  uint8_t* un = dsm;                                              // ring / histogram / candidates
+  float* sc = reinterpret_cast<float*>(dsm + idx_union_bytes(KS * 32));  // segment scores
+  if (p.split) {
+    for (int i = threadIdx.x; i < p.T; i += blockDim.x) {
+      int64_t eb;
+      S.plan_V[i] = visible_of(p, p.t_begin + i, &eb);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const int T = p.T, P = gridDim.x;
+      int64_t total = 0;
+      for (int i = 0; i < T; ++i) total += S.plan_V[i];
+      const int64_t avail = P - T;
+      int start = 0;
+      S.plan_t = -1;
+      for (int i = 0; i < T; ++i) {
+        const int64_t v = S.plan_V[i];
+        int64_t s = 1 + (total > 0 ? (v * avail) / total : 0);
+        const int64_t smax = v > kMinSeg ? (v + kMinSeg - 1) / kMinSeg : 1;
+        s = min(s, smax);
+        s = min(s, (int64_t)kMaxGroup);
+        if ((int)blockIdx.x >= start && (int)blockIdx.x < start + s) {
+          S.plan_t = i;
+          S.plan_j = (int)blockIdx.x - start;
+          S.plan_G = (int)s;
+        }
+        start += (int)s;
+      }
+    }
+    __syncthreads();
+    const int i = S.plan_t;
+    if (i < 0) return;
+    const int t = p.t_begin + i;
+    int64_t eb;
+    const int64_t V = visible_of(p, t, &eb);
+    const int j = S.plan_j, G = S.plan_G;
+    process_segment<SRC, KS, NTILE>(p, t, j, G, V, eb, p.ws + i, sc, un, S);
+  } else {
+    for (int i = blockIdx.x; i < p.T; i += gridDim.x) {
+      const int t = p.t_begin + i;
+      int64_t eb;
+      const int64_t V = visible_of(p, t, &eb);
+      process_segment<SRC, KS, NTILE>(p, t, 0, 1, V, eb, nullptr, sc, un, S);
+      __syncthreads();
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+struct DevInfo {
+  int sms;
+  int smem_optin;
+};
+
+// SM count and opt-in shared memory of the current device ({0, 0} without a device).
+static DevInfo dev_info() {
+  static thread_local int cached_dev = -1;
+  static thread_local DevInfo info;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return DevInfo{0, 0};
+  }
+  if (dev != cached_dev) {
+    DevInfo d{0, 0};
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return DevInfo{0, 0};
+    }
+    info = d;
+    cached_dev = dev;
+  }
+  return info;
+}
+
+static size_t idx_dyn_smem(int Di, int64_t seg_cap) { return idx_union_bytes(Di) + (size_t)seg_cap * 4; }
+
+static size_t idx_smem_budget() {
+  const DevInfo d = dev_info();
+  const size_t reserve = sizeof(IdxShared) + 1024;
+  return (size_t)d.smem_optin > reserve ? (size_t)d.smem_optin - reserve : 0;
+}
+
+// Largest number of queries per split-mode launch for which a segment fits in shared memory.
+static int split_queries_per_launch(int T, int64_t max_entries, int Di, int P, int64_t* seg_cap) {
+  const size_t budget = idx_smem_budget();
+  int Tb = min(T, min(P / 2, kMaxSplitQueries));
+  while (Tb >= 1) {
+    int64_t cap = (int64_t)Tb * max_entries / (P - Tb) + 1;
+    cap = max(cap, (int64_t)2 * kMinSeg);
+    cap = min(cap, max_entries);
+    if (idx_dyn_smem(Di, cap) <= budget) {
+      *seg_cap = cap;
+      return Tb;
+    }
+    Tb /= 2;
+  }
+  return 0;
+}
+
+// Workspace of one launch: one QueryWS per query handled in split mode (0 without a device).
+size_t lindex_ws_bytes(int T, int64_t max_entries) {
+  (void)max_entries;
+  const DevInfo d = dev_info();
+  if (d.sms == 0) return 0;
+  const int slots = min(T, min(d.sms / 2, kMaxSplitQueries));
+  return (size_t)(slots > 0 ? slots : 1) * sizeof(QueryWS);
+}
+
+template <int SRC, int KS, int NTILE>
+static cudaError_t launch_one(const IdxParams& p, int grid, bool coop, size_t smem, cudaStream_t stream) {
+  auto kern = lindex_topk_kernel<SRC, KS, NTILE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kIdxThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = coop ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int SRC, int KS, int NTILE>
+static cudaError_t run_topk(IdxParams p, int T, cudaStream_t stream) {
+  const DevInfo d = dev_info();
+  const int P = d.sms;
+  const int Di = SRC == kSrcFp8 ? KS * 32 : 64;
+  int64_t seg_cap = 0;
+  const int Tb = split_queries_per_launch(T, p.max_entries, Di, P, &seg_cap);
+  const bool row_fits = idx_dyn_smem(Di, p.max_entries) <= idx_smem_budget();
+  p.stages = idx_stages(Di);
+  if (Tb >= 1 && (Tb == T || !row_fits)) {
+    p.split = 1;
+    p.seg_cap = seg_cap;
+    for (int t0 = 0; t0 < T; t0 += Tb) {
+      p.t_begin = t0;
+      p.T = min(Tb, T - t0);
+      cudaError_t e = launch_one<SRC, KS, NTILE>(p, P, true, idx_dyn_smem(Di, seg_cap), stream);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  if (!row_fits) return cudaErrorInvalidValue;
+  p.split = 0;
+  p.seg_cap = max(p.max_entries, (int64_t)1);
+  p.t_begin = 0;
+  p.T = T;
+  return launch_one<SRC, KS, NTILE>(p, min(T, P), false, idx_dyn_smem(Di, p.seg_cap), stream);
+}
+
+bool lindex_shape_supported(int dtype, int Hi, int Di) {
+  if (Hi < 1 || Hi > kIdxMaxHeads) return false;
+  if (dtype == CSKV_FP8E4M3) return Di == 64 || Di == 128;
+  if (dtype == CSKV_F32) return Di >= 4 && Di <= kIdxMaxDim && Di % 4 == 0;
+  return false;
+}
+
+bool lindex_capacity_ok(int64_t max_entries, int T) {
+  const DevInfo d = dev_info();
+  if (d.sms < 2) return false;
+  int64_t cap;
+  const bool split = split_queries_per_launch(T, max_entries, 128, d.sms, &cap) >= 1;
+  const bool row = idx_dyn_smem(128, max_entries) <= idx_smem_budget();
+  return split || row;
+}
+
+cudaError_t launch_lindex(const IdxParams& p0, int dtype, int T, cudaStream_t stream) {
+  IdxParams p = p0;
+  if (p.scores) return run_topk<kSrcScores, 2, 1>(p, T, stream);
+  if (dtype == CSKV_F32) return run_topk<kSrcF32, 2, 1>(p, T, stream);
+  const int ks = p.Di / 32;
+  const int nt = p.Hi > 8 ? 2 : 1;
+  if (ks == 2 && nt == 1) return run_topk<kSrcFp8, 2, 1>(p, T, stream);
+  if (ks == 2 && nt == 2) return run_topk<kSrcFp8, 2, 2>(p, T, stream);
+  if (ks == 4 && nt == 1) return run_topk<kSrcFp8, 4, 1>(p, T, stream);
+  return run_topk<kSrcFp8, 4, 2>(p, T, stream);
+}
+
+}  // namespace cskv

@@ -1,0 +1,79 @@
+// Parameter blocks and host launchers shared by the kernel files and the C ABI.
+#pragma once
+
+#include "common.cuh"
+
+namespace cskv {
+
+struct QueryWS;
+
+// compress.cu
+cudaError_t launch_csa_compress(const void* xa, const void* za, const void* xb, const void* zb,
+                                const float* ba, const float* bb, const int64_t* tok_off,
+                                const int64_t* tok0, int batch, const int64_t* ent_off,
+                                const int64_t* first, const int64_t* num, int64_t max_blocks,
+                                int in_dt, int out_dt, void* out, int* st, cudaStream_t stream);
+cudaError_t launch_hca_compress(const void* x, const void* z, const float* bias, const int64_t* tok_off,
+                                const int64_t* tok0, int batch, const int64_t* ent_off,
+                                const int64_t* first, const int64_t* num, int64_t max_blocks,
+                                int in_dt, int out_dt, void* out, int* st, cudaStream_t stream);
+
+// indexer.cu
+struct IdxParams {
+  const uint8_t* q_idx;
+  const float* q_scale;
+  const uint8_t* k_idx;
+  const float* k_scale;
+  const float* head_w;
+  const float* scores;
+  int64_t ld_scores;
+  const int64_t* n_valid;
+  const int32_t* q_seq;
+  const int64_t* q_pos;
+  const int64_t* ent_off;
+  int batch;
+  int t_begin, T;
+  int Hi, Di, k;
+  int64_t max_entries;
+  int64_t seg_cap;
+  int split;
+  int stages;
+  int32_t* out_idx;
+  float* out_score;
+  QueryWS* ws;
+  int* st;
+};
+cudaError_t launch_lindex(const IdxParams& p, int dtype, int T, cudaStream_t stream);
+size_t lindex_ws_bytes(int T, int64_t max_entries);
+bool lindex_shape_supported(int dtype, int Hi, int Di);
+bool lindex_capacity_ok(int64_t max_entries, int T);
+
+// attention.cu
+struct AttnParams {
+  int mode;
+  const void* q;
+  const void* kv_cmp;
+  const int64_t* cmp_off;
+  const int32_t* idx;
+  int k;
+  const void* kv_raw;
+  const int64_t* raw_off;
+  const int64_t* raw_tok0;
+  int window;
+  const float* sink;
+  float scale_log2;
+  const int32_t* q_seq;
+  const int64_t* q_pos;
+  int batch, T, H;
+  int rows_per_split;
+  int max_splits;
+  float* part_acc;
+  float* part_ml;
+  float* out;
+  float* lse;
+  int* st;
+};
+cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t stream);
+int attn_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms);
+int attn_max_splits(int mode, int k, int window, int64_t max_entries, int R);
+}  // namespace cskv

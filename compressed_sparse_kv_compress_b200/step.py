@@ -1,0 +1,121 @@
+"""One hybrid decode step through the C ABI: compress, index + top-k, attend.
+
+``DecodeStep`` holds the caller's device tensors (caches, tails, queries) and
+the workspaces, and issues, in the pages' order ([SW] §三-§十二, [TR] §4.2-4.3
+as cited in the C header):
+
+  CSA layer: csa_compress (the entries the new tokens complete)
+             -> lindex_score_topk -> hybrid_decode_attn(CSA)
+  HCA layer: hca_compress -> hybrid_decode_attn(HCA)
+
+The HCA layer does not depend on the indexer, so with ``two_streams`` it runs
+on a second stream that forks from and joins the caller's stream.  The whole
+step can be captured into a CUDA graph and replayed.
+
+Tensor names (all device tensors, int64 offsets unless noted):
+  CSA rows  x_a z_a x_b z_b [rows, 256], csa_x_off [B+1], csa_t0 [B],
+            bias_a bias_b [4, 256] fp32 or None, csa_first csa_num [B]
+  HCA rows  x_h z_h, hca_x_off, hca_t0, bias_h [128, 256] or None, hca_first hca_num
+  caches    cmp_c [sum ceil(n/4), 256] + csa_off [B+1]; cmp_h + hca_off
+  indexer   k_idx [entries, Di] (+ k_scale), q_idx [T, Hi, Di] (+ q_scale), head_w
+  window    raw_c raw_h [rows, 256], raw_off [B+1], raw_t0 [B]
+  queries   q_c q_h [T, H, 128], sink_c sink_h [H] or None, q_seq [T] int32, q_pos [T]
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import api
+
+
+class DecodeStep:
+    def __init__(self, t: dict, *, k: int, window: int, scale: float, max_csa_blocks: int, max_hca_blocks: int,
+                 max_csa_visible: int, max_hca_visible: int, two_streams: bool = False):
+        self.t = t
+        self.k, self.W, self.scale = int(k), int(window), float(scale)
+        self.max_csa_blocks, self.max_hca_blocks = int(max_csa_blocks), int(max_hca_blocks)
+        self.max_csa_visible, self.max_hca_visible = int(max_csa_visible), int(max_hca_visible)
+        dev = t["q_c"].device
+        T, H, _ = t["q_c"].shape
+        self.T, self.H = T, H
+        self.idx = torch.empty(T, self.k, dtype=torch.int32, device=dev)
+        self.score = torch.empty(T, self.k, dtype=torch.float32, device=dev)
+        self.o_c = torch.empty(T, H, 128, dtype=torch.float32, device=dev)
+        self.o_h = torch.empty_like(self.o_c)
+        self.lse_c = torch.empty(T, H, dtype=torch.float32, device=dev)
+        self.lse_h = torch.empty_like(self.lse_c)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.ws_idx = api.lindex_workspace(T, self.k, self.max_csa_visible, dev)
+        self.ws_c = api.attn_workspace(api.CSA, T, H, self.k, self.W, 0, dev)
+        self.ws_h = api.attn_workspace(api.HCA, T, H, 0, self.W, self.max_hca_visible, dev)
+        self.two_streams = two_streams
+        self.side = torch.cuda.Stream(device=dev) if two_streams else None
+        self.graph = None
+
+    # ------------------------------------------------------------------
+    def bulk_compress(self, max_csa_entries: int, max_hca_entries: int, stream=None):
+        """Compress every entry of both caches from the rows provided (a cache built from scratch).
+
+        max_*_entries bound ceil(n/4) and ceil(n/128) over the sequences."""
+        t = self.t
+        api.csa_compress(t["x_a"], t["z_a"], t["x_b"], t["z_b"], t["csa_x_off"], t["csa_off"], t["cmp_c"],
+                         max_blocks=max_csa_entries, bias_a=t.get("bias_a"), bias_b=t.get("bias_b"),
+                         tok0=t["csa_t0"], dev_status=self.status, stream=stream)
+        api.hca_compress(t["x_h"], t["z_h"], t["hca_x_off"], t["hca_off"], t["cmp_h"],
+                         max_blocks=max_hca_entries, bias=t.get("bias_h"), tok0=t["hca_t0"],
+                         dev_status=self.status, stream=stream)
+
+    def csa_layer(self, stream=None):
+        t = self.t
+        api.csa_compress(t["x_a"], t["z_a"], t["x_b"], t["z_b"], t["csa_x_off"], t["csa_off"], t["cmp_c"],
+                         max_blocks=self.max_csa_blocks, bias_a=t.get("bias_a"), bias_b=t.get("bias_b"),
+                         tok0=t["csa_t0"], first_block=t["csa_first"], num_blocks=t["csa_num"],
+                         dev_status=self.status, stream=stream)
+        api.lindex_score_topk(t["q_idx"], t["k_idx"], t["q_seq"], t["q_pos"], t["csa_off"], self.idx, self.ws_idx,
+                              max_entries=self.max_csa_visible, q_scale=t.get("q_scale"), k_scale=t.get("k_scale"),
+                              head_w=t.get("head_w"), out_score=self.score, dev_status=self.status, stream=stream)
+        api.hybrid_decode_attn(api.CSA, t["q_c"], t["cmp_c"], t["csa_off"], t["raw_c"], t["raw_off"], t["q_seq"],
+                               t["q_pos"], self.o_c, self.ws_c, window=self.W, idx=self.idx, raw_tok0=t["raw_t0"],
+                               sink=t.get("sink_c"), scale=self.scale, lse=self.lse_c, dev_status=self.status,
+                               stream=stream)
+
+    def hca_layer(self, stream=None):
+        t = self.t
+        api.hca_compress(t["x_h"], t["z_h"], t["hca_x_off"], t["hca_off"], t["cmp_h"],
+                         max_blocks=self.max_hca_blocks, bias=t.get("bias_h"), tok0=t["hca_t0"],
+                         first_block=t["hca_first"], num_blocks=t["hca_num"], dev_status=self.status,
+                         stream=stream)
+        api.hybrid_decode_attn(api.HCA, t["q_h"], t["cmp_h"], t["hca_off"], t["raw_h"], t["raw_off"], t["q_seq"],
+                               t["q_pos"], self.o_h, self.ws_h, window=self.W, raw_tok0=t["raw_t0"],
+                               sink=t.get("sink_h"), scale=self.scale, lse=self.lse_h,
+                               max_entries=self.max_hca_visible, dev_status=self.status, stream=stream)
+
+    def run(self, stream=None):
+        """Issue the whole step on `stream` (default: the current stream)."""
+        main = stream if stream is not None else torch.cuda.current_stream()
+        if not self.two_streams:
+            self.csa_layer(main)
+            self.hca_layer(main)
+            return
+        self.side.wait_stream(main)
+        self.hca_layer(self.side)
+        self.csa_layer(main)
+        main.wait_stream(self.side)
+
+    # ------------------------------------------------------------------
+    def capture(self):
+        """Capture run() into a CUDA graph (replay with replay())."""
+        s = torch.cuda.Stream(device=self.o_c.device)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.run(s)  # warm-up outside capture (sets kernel attributes)
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run()
+        self.graph = g
+        return g
+
+    def replay(self):
+        self.graph.replay()

@@ -1,0 +1,202 @@
+/*
+ * cskv -- hybrid compressed sparse KV attention (DeepSeek V4 CSA / HCA) for
+ * NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * Source pages of the method (cited by page and section):
+ *   [SW] shareware.cn/news/167317 -- essay on DeepSeek V4 Hybrid Attention.
+ *   [TR] trdm.cn/news/516303 -- "从 MLA 到 CSA，聊聊大模型 Attention 的瘦身与闪送".
+ *   [AM] aimodeling.com news "DeepSeek V4 混合注意力架构解析：如何在1M上下文下
+ *        将计算量降至原来的27%？".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument is a DEVICE pointer unless its comment says host.
+ *   The caller owns all memory; the library allocates nothing.
+ * - Every call is asynchronous on `stream` (NULL = the legacy default stream)
+ *   and may be captured into a CUDA graph.
+ * - A KV row is packed K||V: D = 2*d values, K in columns 0..d-1, V in d..2d-1.
+ *   d (head dim) must be 128.  Rows are contiguous, row-major.
+ * - Sequences are concatenated; int64 CSR offsets give each sequence's rows:
+ *   rows of sequence b are [off[b], off[b+1]).
+ * - Return value: CSKV_OK, or an error code.  Arguments are validated on the
+ *   host before anything is launched, so an error return means nothing ran.
+ *   CSKV_ERR_LAUNCH carries a CUDA error; cskv_last_cuda_error() names it.
+ * - `dev_status` (optional, may be NULL): device int that kernels OR the
+ *   CSKV_DEV_* bits into when a device-side check fails (an index out of
+ *   range, a row the caller did not provide, a bounded wait that gave up).
+ *   The offending element is skipped; the call still completes.  The caller
+ *   zeroes it and reads it back when it wants to know.
+ * - Alignment: every row array must start on a 16-byte boundary.
+ */
+#ifndef CSKV_H
+#define CSKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cskv_stream_t; /* same type as cudaStream_t */
+
+#if defined(__GNUC__)
+#define CSKV_API __attribute__((visibility("default")))
+#else
+#define CSKV_API
+#endif
+
+enum cskv_status {
+  CSKV_OK = 0,
+  CSKV_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, bad enum */
+  CSKV_ERR_UNSUPPORTED = 2, /* valid but not implemented combination (dtype, d, Di, Hi) */
+  CSKV_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the *_workspace_size() figure */
+  CSKV_ERR_LAUNCH = 4,      /* the CUDA runtime refused a launch or a device query */
+};
+
+enum cskv_dtype { CSKV_F32 = 0, CSKV_BF16 = 1, CSKV_FP8E4M3 = 2 };
+enum cskv_mode { CSKV_CSA = 0, CSKV_HCA = 1 };
+
+/* Bits OR-ed into *dev_status by device-side checks. */
+enum cskv_dev_status {
+  CSKV_DEV_BAD_INDEX = 1,    /* an index or offset pointed outside its array; element skipped */
+  CSKV_DEV_TAIL_MISSING = 2, /* a token row needed lies before the provided tail; element skipped */
+  CSKV_DEV_CAPACITY = 4,     /* a size exceeded the host-side bound given to the call */
+  CSKV_DEV_TIMEOUT = 8,      /* a bounded cross-block wait gave up; outputs of that call are invalid */
+};
+
+CSKV_API const char* cskv_status_string(int status);
+CSKV_API const char* cskv_last_cuda_error(void); /* text of the CUDA error behind the last CSKV_ERR_LAUNCH */
+CSKV_API int cskv_version(void);
+
+/* ------------------------------------------------------------------------
+ * csa_compress -- CSA token-dimension compression, 4 tokens -> 1 entry.
+ *
+ * [SW] §二/§四/§五, [TR] §4.3 改进一/改进二: entry i of a sequence mixes, for
+ * every dimension j separately, the tokens of block i through path A
+ * (value x_a[t,j], logit z_a[t,j] + bias_a[t-4i, j]) and the tokens of block
+ * i-1 through path B (value x_b[t,j], logit z_b[t,j] + bias_b[t-4(i-1), j]):
+ *     w = softmax over the candidates of the logits;  out[i,j] = sum w * value.
+ * Entry 0 has no path-B candidates; a partial last block uses the tokens it has.
+ *
+ * x_a, z_a, x_b, z_b : [rows, 256] in_dtype (CSKV_F32 or CSKV_BF16).  x_b and
+ *                      z_b may both be NULL: path A alone.
+ * bias_a, bias_b     : [4, 256] fp32, or NULL for zero biases.
+ * tok_off            : [batch+1] int64, rows of sequence b are tok_off[b]..tok_off[b+1]-1.
+ * tok0               : [batch] int64 or NULL (all 0): the token position of
+ *                      sequence b's first provided row.  Its length is
+ *                      n_b = tok0[b] + tok_off[b+1] - tok_off[b]; only the tail
+ *                      from tok0[b] need be provided.
+ * ent_off            : [batch+1] int64, entry i of sequence b is written to row
+ *                      ent_off[b] + i of `out` (needs ceil(n_b/4) rows).
+ * first_block, num_blocks : [batch] int64 or NULL: entries first..first+num-1
+ *                      are computed (NULL: first 0, num ceil(n_b/4) - first).
+ * max_blocks         : host, >= every num_blocks[b]; entries beyond it are
+ *                      skipped and flagged CSKV_DEV_CAPACITY.
+ * out                : [*, 256] out_dtype (CSKV_F32 or CSKV_BF16; bf16 rounds to
+ *                      nearest even).  fp32 arithmetic inside.
+ * ------------------------------------------------------------------------ */
+CSKV_API int csa_compress(const void* x_a, const void* z_a, const void* x_b, const void* z_b,
+                 const float* bias_a, const float* bias_b,
+                 const int64_t* tok_off, const int64_t* tok0, int batch,
+                 const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
+                 int64_t max_blocks, int in_dtype, int out_dtype, void* out,
+                 int* dev_status, cskv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * hca_compress -- HCA compression, 128 tokens -> 1 entry, one stream.
+ *
+ * [SW] §三.3, [TR] §4.3 (HCA, no dual stream): entry i mixes the tokens of
+ * block i (value x[t,j], logit z[t,j] + bias[t-128i, j]) with one softmax per
+ * dimension.  Arguments as csa_compress; bias is [128, 256] fp32 or NULL.
+ * ------------------------------------------------------------------------ */
+CSKV_API int hca_compress(const void* x, const void* z, const float* bias,
+                 const int64_t* tok_off, const int64_t* tok0, int batch,
+                 const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
+                 int64_t max_blocks, int in_dtype, int out_dtype, void* out,
+                 int* dev_status, cskv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * lindex_score_topk -- Lightning Indexer scan fused with exact top-k.
+ *
+ * [SW] §六/§七/§十, [TR] §4.2, [AM]: query t (sequence q_seq[t], position
+ * q_pos[t]) sees CSA entries i < V_t = floor((q_pos[t]+1)/4); entry i scores
+ *     s_i = sum_h head_w[h] * ReLU(q_scale[t,h] * k_scale[i] * <q_idx[t,h,:], k_idx[i,:]>)
+ * (fp32 arithmetic; scales and weights default to 1 when NULL).  The
+ * min(k, V_t) best entries are kept, equal scores going to the lower index.
+ *
+ * q_idx   : [T, Hi, Di] dtype;  q_scale: [T, Hi] fp32 or NULL.
+ * k_idx   : [sum entries, Di] dtype;  k_scale: [sum entries] fp32 or NULL.
+ *           dtype CSKV_FP8E4M3 (OCP E4M3 codes; Hi <= 16, Di in {64, 128}) or
+ *           CSKV_F32 (Hi <= 16, Di <= 128, Di % 4 == 0).
+ * head_w  : [Hi] fp32 or NULL.
+ * q_seq   : [T] int32 sequence of each query; q_pos: [T] int64.
+ * ent_off : [batch+1] int64, entries of sequence b are rows ent_off[b].. of k_idx.
+ * max_entries : host, >= every V_t (visible entries); sizes the plan.
+ * out_idx : [T, k] int32: the kept entries (indices within the sequence) in
+ *           ascending index order, then -1 padding.
+ * out_score : [T, k] fp32 or NULL: the score of each kept entry (0 on padding).
+ * workspace : lindex_workspace_size(T, k, max_entries) bytes, zero-filled before
+ *           its first use; every call leaves it zero-filled again unless it
+ *           flagged CSKV_DEV_TIMEOUT.  Calls sharing a workspace must be
+ *           ordered on one stream.
+ * ------------------------------------------------------------------------ */
+CSKV_API int lindex_score_topk(const void* q_idx, const float* q_scale, const void* k_idx, const float* k_scale,
+                      const float* head_w, const int32_t* q_seq, const int64_t* q_pos,
+                      const int64_t* ent_off, int batch, int T, int Hi, int Di, int k, int dtype,
+                      int64_t max_entries, int32_t* out_idx, float* out_score,
+                      void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * lindex_topk_from_scores -- the selection half of lindex_score_topk alone.
+ *
+ * Keeps, for every row t, the min(k, n_valid[t]) largest of scores[t, 0..n_valid[t]-1]
+ * (ties to the lower index), with the same output format and workspace rules.
+ * scores : [T, ld_scores] fp32; n_valid : [T] int64 (<= max_entries <= ld_scores).
+ * ------------------------------------------------------------------------ */
+CSKV_API int lindex_topk_from_scores(const float* scores, int64_t ld_scores, const int64_t* n_valid,
+                            int T, int k, int64_t max_entries, int32_t* out_idx, float* out_score,
+                            void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream);
+
+CSKV_API size_t lindex_workspace_size(int T, int k, int64_t max_entries);
+
+/* ------------------------------------------------------------------------
+ * hybrid_decode_attn -- MQA attention over compressed entries + raw window + sink.
+ *
+ * [SW] §三.1/§六/§八/§十/§十一/§十二, [TR] §2.2/§3.1/§4.3: for query t at
+ * position p in sequence b, the rows are
+ *   mode CSKV_CSA: the compressed entries idx[t, 0..k-1] (entries < 0 skipped;
+ *                  entries not visible at p, i.e. >= floor((p+1)/4), flagged
+ *                  CSKV_DEV_BAD_INDEX and skipped),
+ *   mode CSKV_HCA: every visible HCA entry i < floor((p+1)/128) (idx unused),
+ * followed by the raw window tokens max(0, p-window+1) .. p.  With logits
+ * l = scale * <q_h, K_row> and the sink logit sink[h] in the denominator:
+ *   o[t,h,:] = sum_rows softmax(l ∪ {sink})_row * V_row,
+ *   lse[t,h] = log(sum_rows exp(l) + exp(sink[h])).
+ * Split-KV partials are merged on device ([TR] §3.1 online softmax).
+ *
+ * q       : [T, H, d] dtype (CSKV_F32 or CSKV_BF16), H <= 128, d == 128.
+ * kv_cmp  : [sum entries, 2d] dtype; cmp_off: [batch+1] int64 entry offsets.
+ * idx     : [T, k] int32 (mode CSA), NULL for HCA.
+ * kv_raw  : [rows, 2d] dtype raw window rows; raw_off: [batch+1] int64;
+ *           raw_tok0: [batch] int64 or NULL (0): token of sequence b's first row.
+ * sink    : [H] fp32 or NULL (no sink).  scale: host float (1/sqrt(d) typical).
+ * q_seq   : [T] int32; q_pos: [T] int64.
+ * max_entries : host; mode HCA: >= every visible HCA entry count; mode CSA: unused.
+ * out     : [T, H, d] fp32;  lse: [T, H] fp32 or NULL.
+ * workspace : hybrid_attn_workspace_size(...) bytes (no zero-fill needed).
+ * ------------------------------------------------------------------------ */
+CSKV_API int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off,
+                       const int32_t* idx, int k, const void* kv_raw, const int64_t* raw_off,
+                       const int64_t* raw_tok0, int window, const float* sink, float scale,
+                       const int32_t* q_seq, const int64_t* q_pos, int batch, int T, int H, int d,
+                       int dtype, int64_t max_entries, float* out, float* lse,
+                       void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream);
+
+CSKV_API size_t hybrid_attn_workspace_size(int mode, int T, int H, int d, int k, int window, int64_t max_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSKV_H */

@@ -1,0 +1,114 @@
+"""The C-ABI library builds, loads and exports every symbol its header declares;
+argument validation rejects bad calls before touching the GPU (no compute here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_sparse_kv_compress_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _declared():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"CSKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return names
+
+
+def test_header_declares_the_four_operations():
+    names = _declared()
+    for op in ("csa_compress", "hca_compress", "lindex_score_topk", "hybrid_decode_attn"):
+        assert op in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_library_is_sm100a_and_in_tree(lib):
+    assert os.path.dirname(_lib.LIB_PATH) == os.path.join(ROOT, "compressed_sparse_kv_compress_b200")
+    assert lib.cskv_version() >= 100
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.cskv_status_string(s)
+    assert b"INVALID" in lib.cskv_status_string(_lib.ERR_INVALID_ARG)
+
+
+def _p(v=0x1000):
+    return ctypes.c_void_p(v)
+
+
+def test_compress_validation(lib):
+    nul = None
+    # null rows
+    assert lib.csa_compress(nul, _p(), nul, nul, nul, nul, _p(), nul, 1, _p(), nul, nul, 4, 1, 1, _p(), nul,
+                            nul) == _lib.ERR_INVALID_ARG
+    # x_b without z_b
+    assert lib.csa_compress(_p(), _p(), _p(), nul, nul, nul, _p(), nul, 1, _p(), nul, nul, 4, 1, 1, _p(), nul,
+                            nul) == _lib.ERR_INVALID_ARG
+    # misaligned output
+    assert lib.csa_compress(_p(), _p(), nul, nul, nul, nul, _p(), nul, 1, _p(), nul, nul, 4, 1, 1, _p(0x1004), nul,
+                            nul) == _lib.ERR_INVALID_ARG
+    # fp8 rows are not a compression input
+    assert lib.hca_compress(_p(), _p(), nul, _p(), nul, 1, _p(), nul, nul, 4, 2, 1, _p(), nul,
+                            nul) == _lib.ERR_UNSUPPORTED
+    # bad batch / bad enum
+    assert lib.hca_compress(_p(), _p(), nul, _p(), nul, 0, _p(), nul, nul, 4, 1, 1, _p(), nul,
+                            nul) == _lib.ERR_INVALID_ARG
+    assert lib.hca_compress(_p(), _p(), nul, _p(), nul, 1, _p(), nul, nul, 4, 7, 1, _p(), nul,
+                            nul) == _lib.ERR_INVALID_ARG
+    # nothing to do
+    assert lib.hca_compress(_p(), _p(), nul, _p(), nul, 1, _p(), nul, nul, 0, 1, 1, _p(), nul, nul) == _lib.OK
+
+
+def test_indexer_validation(lib):
+    nul = None
+    args = dict(Hi=8, Di=64, k=16, dtype=_lib.FP8E4M3)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return lib.lindex_score_topk(_p(), nul, _p(), nul, nul, _p(), _p(), _p(), 1, kw.get("T", 1), a["Hi"], a["Di"],
+                                     a["k"], a["dtype"], 100, _p(), nul, _p(), 1 << 20, nul, nul)
+
+    assert call(dtype=9) == _lib.ERR_INVALID_ARG
+    assert call(dtype=_lib.BF16) == _lib.ERR_UNSUPPORTED
+    assert call(Di=96) == _lib.ERR_UNSUPPORTED
+    assert call(Hi=17) == _lib.ERR_UNSUPPORTED
+    assert call(k=0) == _lib.ERR_INVALID_ARG
+    assert call(T=0) == _lib.OK
+    assert lib.lindex_topk_from_scores(nul, 10, _p(), 1, 4, 10, _p(), nul, _p(), 1 << 20, nul,
+                                       nul) == _lib.ERR_INVALID_ARG
+    assert lib.lindex_topk_from_scores(_p(), 5, _p(), 1, 4, 10, _p(), nul, _p(), 1 << 20, nul,
+                                       nul) == _lib.ERR_INVALID_ARG
+
+
+def test_attention_validation(lib):
+    nul = None
+
+    def call(mode=0, d=128, H=16, dtype=1, idx=_p(), k=8, T=1):
+        return lib.hybrid_decode_attn(mode, _p(), _p(), _p(), idx, k, _p(), _p(), nul, 128, nul, 0.1, _p(), _p(), 1,
+                                      T, H, d, dtype, 0, _p(), nul, _p(), 1 << 20, nul, nul)
+
+    assert call(mode=5) == _lib.ERR_INVALID_ARG
+    assert call(d=64) == _lib.ERR_UNSUPPORTED
+    assert call(dtype=_lib.FP8E4M3) == _lib.ERR_UNSUPPORTED
+    assert call(H=0) == _lib.ERR_INVALID_ARG
+    assert call(H=129) == _lib.ERR_INVALID_ARG
+    assert call(idx=nul) == _lib.ERR_INVALID_ARG
+    assert call(T=0) == _lib.OK

@@ -1,0 +1,103 @@
+"""End-to-end GPU decode step (compress -> index/top-k -> CSA and HCA attention)
+against the oracle's step on the same seeded inputs, at small sizes and at the
+full workload sizes (sampled queries), eager, two-stream and graph-replayed."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as oatt
+from oracle import indexer
+from oracle import step as ostep
+from synth import Workload, spec_by_name
+
+from helpers import bulk_bounds, check_attention, check_selection, compress_tol_check, decode_step, dtypes, \
+    np_arrays, storage_rows, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_gpu(w, two_streams=False, graph=False):
+    step, dev = decode_step(w, two_streams=two_streams)
+    if w.spec.cache == "compress":
+        step.bulk_compress(*bulk_bounds(w))
+    if graph:
+        step.capture()
+        step.replay()
+    else:
+        step.run()
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0, f"device status {int(step.status.item())}"
+    return step, dev
+
+
+def _check(w, step, dev, queries, extra_rel=None):
+    m, a = w.meta, np_arrays(w)
+    res = ostep.run_step(m, a, dtypes(w), queries=queries, bulk=(w.spec.cache == "compress"))
+    # caches: the step's recompressed entries
+    for b in range(m["B"]):
+        for layer, key, off in (("csa", "cmp_c", "csa_off"), ("hca", "cmp_h", "hca_off")):
+            ents, ref = res["new"][(layer, b)]
+            got = storage_rows(dev[key][m[off][b] + ents[0]: m[off][b] + ents[-1] + 1])
+            compress_tol_check(got, ref, w.spec.dtype, f"{layer} seq{b}")
+    idx = step.idx.cpu().numpy()
+    o_c, o_h = to_f64(step.o_c), to_f64(step.o_h)
+    lse_c = to_f64(step.lse_c)
+    arrays_after = {**a, "cmp_c": res["cmp_c"], "cmp_h": res["cmp_h"]}
+    n_diff = 0
+    for j, t in enumerate(queries):
+        n_diff += check_selection(idx[t], res["scores"][j], m["k"], f"query {t}")
+        sel = idx[t][idx[t] >= 0]
+        if np.array_equal(sel, res["idx"][j][res["idx"][j] >= 0]):
+            ref_c = res["o_c"][j]
+            np.testing.assert_allclose(lse_c[t], res["lse_c"][j], rtol=1e-5, atol=1e-5)
+        else:  # an allowed near-tie swap: attend over the GPU's selection
+            ref_c = ostep.query_attention(m, arrays_after, dtypes(w), res["cmp_c"], t, "c", sel)[0]
+        check_attention(o_c[t], ref_c, extra_rel, f"CSA query {t}")
+        check_attention(o_h[t], res["o_h"][j], extra_rel, f"HCA query {t}")
+    return res, n_diff
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_bias"])
+def test_tiny_fp32(name):
+    w = Workload(spec_by_name(name))
+    step, dev = _run_gpu(w)
+    _check(w, step, dev, [0], extra_rel=1e-4)
+
+
+def test_small_bf16_two_streams_graph_equal_eager():
+    spec = spec_by_name("ragged_b64").replace(batch=6, len_range=(3000, 40000), heads=64)
+    w = Workload(spec)
+    s1, d1 = _run_gpu(w)
+    _check(w, s1, d1, list(range(6)))
+    w2 = Workload(spec)
+    s2, _ = _run_gpu(w2, two_streams=True, graph=True)
+    assert torch.equal(s1.idx, s2.idx)
+    assert torch.equal(s1.o_c, s2.o_c) and torch.equal(s1.o_h, s2.o_h)
+
+
+def test_b8_ctx64k_full():
+    w = Workload(spec_by_name("b8_ctx64k"))
+    step, dev = _run_gpu(w, two_streams=True)
+    _check(w, step, dev, list(range(8)))
+
+
+def test_b1_ctx1m_full_with_needles():
+    w = Workload(spec_by_name("b1_ctx1m"))
+    step, dev = _run_gpu(w, two_streams=True, graph=True)
+    assert set(w.needles) <= set(step.idx[0].cpu().tolist())
+    _check(w, step, dev, [0])
+
+
+def test_ragged_b64_full_sampled():
+    w = Workload(spec_by_name("ragged_b64"))
+    step, dev = _run_gpu(w, two_streams=True)
+    n = w.meta["n"]
+    queries = sorted({0, 63, int(np.argmax(n)), int(np.argmin(n)), 17, 40})
+    _check(w, step, dev, queries)
+
+
+def test_prefill_chunk_full_sampled():
+    w = Workload(spec_by_name("prefill_4k_at_128k"))
+    step, dev = _run_gpu(w)
+    _check(w, step, dev, [0, 1, 2, 3, 1001, 2048, 4094, 4095])
