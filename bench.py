@@ -1,0 +1,375 @@
+"""Benchmark of one hybrid CSA/HCA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl cskv|reference]
+
+A step = every row of the hot path on one batch of synthetic input: CSA
+compression of the entries the new tokens complete, the Lightning Indexer
+scan + exact top-k, CSA attention (top-k + window + sink), HCA compression,
+HCA dense attention (+ window + sink), split merges.  Inputs are resident in
+HBM; the step is replayed from a CUDA graph; L2 is flushed (a 256 MiB write)
+before every timed step, outside its events.  Prints one JSON line on rank 0.
+
+--impl reference times the CPU oracle (plain fp64 numpy) on the machine's host
+cores on a bounded sample of the same workload.
+Multi-GPU (torchrun, N > 1): every rank runs an independent replica of the
+workload (weak scaling); the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import Workload, spec_by_name  # noqa: E402
+
+METRIC = "hybrid decode attention query-tokens/s at 1M ctx"
+UNIT = "query-tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------- byte model
+def step_bytes(w: Workload) -> dict:
+    """Algorithmic HBM bytes of one step (what the method must move), per kernel family."""
+    m = w.meta
+    s = w.spec
+    kvb = 2 if s.dtype == "bf16" else 4
+    ib = 1 if s.idx_dtype == "fp8" else 4
+    row = 256 * kvb
+    T, H, Hi, di, k, W = m["T"], m["H"], m["Hi"], m["di"], m["k"], m["W"]
+    vis_c = [(p + 1) // 4 for p in m["q_pos"]]
+    vis_h = [(p + 1) // 128 for p in m["q_pos"]]
+    key = di * ib + (4 if s.idx_dtype == "fp8" else 0)
+    idx = sum(v * key for v in vis_c) + T * Hi * key + T * k * 8
+    q = H * 128 * kvb
+    o = H * 128 * 4 + H * 4
+    csa_attn = sum(min(k, v) * row + min(W, p + 1) * row + q + o + k * 4 for v, p in zip(vis_c, m["q_pos"]))
+    hca_attn = sum(v * row + min(W, p + 1) * row + q + o for v, p in zip(vis_h, m["q_pos"]))
+    comp = 0
+    for b in range(m["B"]):
+        n = m["n"][b]
+        for i in range(m["csa_first"][b], m["csa_first"][b] + m["csa_num"][b]):
+            a_tok = min(4, n - 4 * i)
+            comp += (a_tok + (4 if i >= 1 else 0)) * 2 * row + row
+        for i in range(m["hca_first"][b], m["hca_first"][b] + m["hca_num"][b]):
+            comp += min(128, n - 128 * i) * 2 * row + row
+    return dict(indexer=idx, csa_attn=csa_attn, hca_attn=hca_attn, compress=comp,
+                total=idx + csa_attn + hca_attn + comp)
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------- oracle timing
+def oracle_sample(w: Workload, budget_s: float = 12.0, max_queries: int = 64):
+    """Times the CPU oracle on whole queries of the workload until the budget is spent."""
+    from oracle import step as ostep
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    a = {k: w.numpy(k) for k in w.arrays}
+    dt = {"kv": w.spec.dtype, "idx": w.spec.idx_dtype}
+    t0 = time.perf_counter()
+    done = 0
+    for t in range(min(w.meta["T"], max_queries)):
+        ostep.run_step(w.meta, a, dt, queries=[t])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    el = time.perf_counter() - t0
+    return {"value": done / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} whole query step(s) of {w.spec.name} (each: compress of the step's entries, "
+                      f"full indexer scan + top-k, CSA and HCA attention), {el:.1f} s"}
+
+
+# ---------------------------------------------------------------------- distributed
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def reduce_max(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------- arms
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return
+    w = Workload(spec_by_name(args.workload))
+    vals = []
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state
+    t0 = time.perf_counter()
+    per = []
+    for _ in range(args.steps):
+        r = oracle_sample(w, budget_s=args.ref_budget, max_queries=1)
+        per.append(1.0 / r["value"])
+        vals.append(r)
+    el = time.perf_counter() - t0
+    value = len(per) / sum(per)
+    cb = dict(vals[-1])
+    cb["value"] = value
+    cb["sample"] = f"{len(per)} step(s) of one whole query of {args.workload} each, {el:.1f} s"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(per),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload}, "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_cskv(args, ws, rank, local):
+    from compressed_sparse_kv_compress_b200 import _lib, api
+    from compressed_sparse_kv_compress_b200.step import DecodeStep
+
+    lib = _lib.load()
+    spec = spec_by_name(args.workload)
+    spec = spec.replace(seed=spec.seed + rank)
+    w = Workload(spec)
+    m = w.meta
+    dev = w.device("cuda")
+    bd = dict(max_csa_blocks=max(m["csa_num"]), max_hca_blocks=max(m["hca_num"]),
+              max_csa_visible=max((p + 1) // 4 for p in m["q_pos"]),
+              max_hca_visible=max((p + 1) // 128 for p in m["q_pos"]))
+    step = DecodeStep(dev, k=m["k"], window=m["W"], scale=m["scale"], two_streams=not args.one_stream, **bd)
+    if spec.cache == "compress":
+        step.bulk_compress(max(m["ncsa"]), max(m["nhca"]))
+    torch.cuda.synchronize()
+    n0 = lib.cskv_launch_count()
+    step.capture()
+    launches_per_step = (lib.cskv_launch_count() - n0) // 2  # capture() runs the step once eagerly, once captured
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step.replay()
+    torch.cuda.synchronize()
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} during warm-up")
+
+    # ---- timed region: K graph replays, each after an L2 flush outside its events
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_((i + 1) & 0xFF)
+        evs[i][0].record(stream)
+        step.replay()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms_steps = [a.elapsed_time(b) for a, b in evs]
+    ms_local = statistics.mean(ms_steps)
+
+    # ---- dominant kernel alone (indexer scan + top-k), same stream, same flush discipline
+    t = step.t
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_((i + 7) & 0xFF)
+        kev[i][0].record(stream)
+        api.lindex_score_topk(t["q_idx"], t["k_idx"], t["q_seq"], t["q_pos"], t["csa_off"], step.idx, step.ws_idx,
+                              max_entries=step.max_csa_visible, q_scale=t.get("q_scale"), k_scale=t.get("k_scale"),
+                              head_w=t.get("head_w"), out_score=step.score, dev_status=step.status)
+        kev[i][1].record(stream)
+    torch.cuda.synchronize()
+    idx_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in kev)
+
+    # ---- end to end through the public API with host buffers
+    pairs = []  # (pinned host tensor, device destination view)
+
+    def add(dst):
+        h = torch.empty(dst.shape, dtype=dst.dtype, pin_memory=True)
+        h.copy_(dst.cpu())
+        pairs.append((h, dst))
+
+    for name in ("q_c", "q_h", "q_idx", "q_scale"):
+        if t.get(name) is not None:
+            add(t[name])
+    for b in range(m["B"]):  # the newest token's rows of every per-token array
+        for name, off in (("x_a", "csa_x_off"), ("z_a", "csa_x_off"), ("x_b", "csa_x_off"), ("z_b", "csa_x_off"),
+                          ("x_h", "hca_x_off"), ("z_h", "hca_x_off"), ("raw_c", "raw_off"), ("raw_h", "raw_off")):
+            r = m[off][b + 1] - 1
+            add(t[name][r:r + 1])
+        e = m["ncsa"][b] - 1 + m["csa_off"][b]  # the indexer key of the newest entry
+        add(t["k_idx"][e:e + 1])
+        if t.get("k_scale") is not None:
+            add(t["k_scale"][e:e + 1])
+    outs = [(step.o_c, torch.empty(step.o_c.shape, dtype=step.o_c.dtype, pin_memory=True)),
+            (step.o_h, torch.empty(step.o_h.shape, dtype=step.o_h.dtype, pin_memory=True))]
+    h2d = sum(h.numel() * h.element_size() for h, _ in pairs)
+    d2h = sum(h.numel() * h.element_size() for _, h in outs)
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_((i + 3) & 0xFF)
+        eev[i][0].record(stream)
+        for h, d in pairs:
+            d.copy_(h, non_blocking=True)
+        step.replay()
+        for d, h in outs:
+            h.copy_(d, non_blocking=True)
+        eev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = statistics.mean(a.elapsed_time(b) for a, b in eev)
+    clk = clocks.stop()
+
+    ms = reduce_max(ms_local, ws)
+    ms_e2e = reduce_max(ms_e2e, ws)
+    T = m["T"]
+    value = T * ws / (ms / 1e3)
+    by = step_bytes(w)
+    hbm, hbm_src = peaks()
+    achieved = by["indexer"] / (idx_us * 1e-6) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if
+        spec.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": m["B"], "context": max(m["n"]), "query_tokens_per_step": T,
+                   "heads": m["H"], "topk": m["k"], "window": m["W"], "indexer": f"{m['Hi']}x{m['di']} "
+                   f"{spec.idx_dtype}", "l2": "flushed (256 MiB write) before every timed step",
+                   "replay": "cuda graph", "streams": 1 if args.one_stream else 2},
+        "step_hbm_bytes": by["total"], "step_gbs": by["total"] / (ms * 1e-3) / 1e9,
+        "step_frac_of_measured_hbm": by["total"] / (ms * 1e-3) / 1e9 / hbm,
+        "roofline": {"kernel": "lindex_topk_kernel (indexer scan + top-k)", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "peak_source": hbm_src,
+                     "bytes_per_launch": by["indexer"], "us_per_launch": idx_us, "traffic": None},
+        "e2e": {"value": T * ws / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches_per_step) * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(w, budget_s=args.ref_budget, max_queries=4)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del step
+    torch.cuda.synchronize()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="b1_ctx1m")
+    ap.add_argument("--impl", default="cskv", choices=["cskv", "reference"])
+    ap.add_argument("--one-stream", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    ws, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank)
+        else:
+            run_cskv(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -4,7 +4,12 @@
 
 #include "launch.cuh"
 
+#include <atomic>
+
 using namespace cskv;
+
+static std::atomic<unsigned long long> g_launches{0};
+void cskv::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 static thread_local char g_cuda_err[256] = "no error";
 
@@ -39,6 +44,8 @@ const char* cskv_status_string(int status) {
 const char* cskv_last_cuda_error(void) { return g_cuda_err; }
 
 int cskv_version(void) { return 100; }
+
+unsigned long long cskv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 static int check_compress_common(const void* x, const void* z, const int64_t* tok_off, int batch,
                                  const int64_t* ent_off, int64_t max_blocks, int in_dtype, int out_dtype,

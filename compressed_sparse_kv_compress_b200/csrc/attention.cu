@@ -284,6 +284,7 @@ static cudaError_t launch_split(const AttnParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   dim3 grid(p.max_splits, p.T);
   kern<<<grid, kAttnThreads, smem, stream>>>(p);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -303,6 +304,7 @@ cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t str
   }
   if (e != cudaSuccess) return e;
   attn_combine_kernel<<<p.T, 256, 0, stream>>>(p);
+  note_launch();
   return cudaGetLastError();
 }
 

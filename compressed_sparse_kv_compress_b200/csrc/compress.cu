@@ -268,6 +268,7 @@ static cudaError_t launch_csa_t(const void* xa, const void* za, const void* xb, 
     csa_compress_kernel<TI, TO, false><<<grid, 256, 0, stream>>>(
         (const TI*)xa, (const TI*)za, nullptr, nullptr, ba, bb, tok_off, tok0, ent_off, first, num,
         max_blocks, (TO*)out, st);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -297,6 +298,7 @@ static cudaError_t launch_hca_t(const void* x, const void* z, const float* bias,
   dim3 grid((unsigned)max_blocks, (unsigned)batch);
   hca_compress_kernel<TI, TO><<<grid, 512, 0, stream>>>((const TI*)x, (const TI*)z, bias, tok_off, tok0,
                                                        ent_off, first, num, max_blocks, (TO*)out, st);
+  note_launch();
   return cudaGetLastError();
 }
 

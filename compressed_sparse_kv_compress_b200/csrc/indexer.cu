@@ -478,6 +478,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   r -= x.above;
   bool done = (x.cnt == r);
   int used_passes = 0;
+  unsigned cands_used = 0;
   int64_t base = 0;
   bool have_base = (G == 1);
   if (!done && G == 1) {
@@ -509,6 +510,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       }
     ok = group_barrier(ws, G, p.st, &S.flag) && ok;
     const unsigned n_c = min(__ldcg(&ws->cand_count), (unsigned)kCandMax);
+    cands_used = n_c;
     for (unsigned i = threadIdx.x; i < n_c; i += blockDim.x) cands[i] = __ldcg(&ws->cand[i]);
     __syncthreads();
     while (!done) done = local_pass([&](int64_t i) { return (uint64_t)cands[i]; }, n_c, P, nb, r, hist, S);
@@ -573,7 +575,11 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       for (int i = threadIdx.x; i < kBins0; i += blockDim.x) ws->hist0[i] = 0u;
       for (int q = 0; q < used_passes; ++q)
         for (int i = threadIdx.x; i < kBinsP; i += blockDim.x) ws->histp[q][i] = 0u;
+      for (int i = threadIdx.x; i < G; i += blockDim.x) ws->above[i] = 0u;
+      for (unsigned i = threadIdx.x; i < cands_used; i += blockDim.x) ws->cand[i] = 0ull;
       if (threadIdx.x == 0) {
+        // every CTA of the group is past its last barrier, so the generation can restart
+        ws->bar_gen = 0u;
         ws->cand_count = 0u;
         ws->done = 0u;
       }
@@ -738,7 +744,9 @@ static cudaError_t launch_one(const IdxParams& p, int grid, bool coop, size_t sm
   attr[0].val.cooperative = coop ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e == cudaSuccess) note_launch();
+  return e;
 }
 
 template <int SRC, int KS, int NTILE>

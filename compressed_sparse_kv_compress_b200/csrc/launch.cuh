@@ -7,6 +7,9 @@ namespace cskv {
 
 struct QueryWS;
 
+// Host-side count of kernels this library has launched (api.cu).
+void note_launch();
+
 // compress.cu
 cudaError_t launch_csa_compress(const void* xa, const void* za, const void* xb, const void* zb,
                                 const float* ba, const float* bb, const int64_t* tok_off,

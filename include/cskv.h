@@ -68,6 +68,9 @@ enum cskv_dev_status {
 CSKV_API const char* cskv_status_string(int status);
 CSKV_API const char* cskv_last_cuda_error(void); /* text of the CUDA error behind the last CSKV_ERR_LAUNCH */
 CSKV_API int cskv_version(void);
+/* Number of kernels this library has launched in this process (host-side count;
+ * a captured CUDA graph replays its kernels without adding to it). */
+CSKV_API unsigned long long cskv_launch_count(void);
 
 /* ------------------------------------------------------------------------
  * csa_compress -- CSA token-dimension compression, 4 tokens -> 1 entry.
