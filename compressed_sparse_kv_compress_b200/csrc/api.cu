@@ -5,11 +5,32 @@
 #include "launch.cuh"
 
 #include <atomic>
+#include <mutex>
+#include <vector>
 
 using namespace cskv;
 
 static std::atomic<unsigned long long> g_launches{0};
 void cskv::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+cudaError_t cskv::ensure_smem_raw(const void* kern, size_t bytes) {
+  struct Entry {
+    const void* kern;
+    int dev;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& x : done)
+    if (x.kern == kern && x.dev == dev && x.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.push_back(Entry{kern, dev, bytes});
+  return e;
+}
 
 static thread_local char g_cuda_err[256] = "no error";
 
@@ -156,20 +177,28 @@ int lindex_topk_from_scores(const float* scores, int64_t ld_scores, const int64_
   return launch_status(launch_lindex(p, CSKV_F32, T, (cudaStream_t)stream));
 }
 
-static int attn_plan(int mode, int T, int k, int window, int64_t max_entries, int* R, int* S) {
+// Split plan of hybrid_decode_attn: rows per split R and the split count S for the
+// tensor-core kernel (bf16) or the CUDA-core kernel (fp32).
+static int attn_plan(int mode, int T, int k, int window, int64_t max_entries, bool tc, int* R, int* S) {
   int sms = 0;
   int rc = device_sms(&sms);
   if (rc) return rc;
-  *R = attn_rows_per_split(mode, T, k, window, max_entries, sms);
+  *R = tc ? attn_tc_rows_per_split(mode, T, k, window, max_entries, sms)
+          : attn_rows_per_split(mode, T, k, window, max_entries, sms);
   *S = attn_max_splits(mode, k, window, max_entries, *R);
   return CSKV_OK;
 }
 
 size_t hybrid_attn_workspace_size(int mode, int T, int H, int d, int k, int window, int64_t max_entries) {
   if (T < 1 || H < 1 || d != kHeadDim || window < 0) return 0;
-  int R = 0, S = 0;
-  if (attn_plan(mode, T, k, window, max_entries, &R, &S)) return 0;
-  return (size_t)T * S * H * (kHeadDim + 2) * sizeof(float);
+  size_t best = 0;
+  for (int tc = 0; tc < 2; ++tc) {
+    int R = 0, S = 0;
+    if (attn_plan(mode, T, k, window, max_entries, tc != 0, &R, &S)) return 0;
+    const size_t need = (size_t)T * S * H * (kHeadDim + 2) * sizeof(float);
+    if (need > best) best = need;
+  }
+  return best;
 }
 
 int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off, const int32_t* idx,
@@ -187,8 +216,9 @@ int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_
   if (!q || !kv_cmp || !cmp_off || !kv_raw || !raw_off || !q_seq || !q_pos || !out) return CSKV_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(kv_cmp) || !aligned16(kv_raw)) return CSKV_ERR_INVALID_ARG;
   if (!(scale == scale)) return CSKV_ERR_INVALID_ARG;
+  const bool tc = dtype == CSKV_BF16;
   int R = 0, S = 0;
-  int rc = attn_plan(mode, T, mode == CSKV_CSA ? k : 0, window, max_entries, &R, &S);
+  int rc = attn_plan(mode, T, mode == CSKV_CSA ? k : 0, window, max_entries, tc, &R, &S);
   if (rc) return rc;
   const size_t need = (size_t)T * S * H * (kHeadDim + 2) * sizeof(float);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSKV_ERR_WORKSPACE;
@@ -217,6 +247,7 @@ int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_
   p.out = out;
   p.lse = lse;
   p.st = dev_status;
+  if (tc) return launch_status(launch_attn_tc(p, (cudaStream_t)stream));
   return launch_status(launch_attn_generic(p, dtype, (cudaStream_t)stream));
 }
 

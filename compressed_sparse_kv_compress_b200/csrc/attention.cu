@@ -15,73 +15,10 @@
 // and writes (m, l, acc) in the log2 domain; attn_combine merges the splits of a query
 // and folds the sink logit in once.  This generic kernel serves fp32 and any head count;
 // bf16 with many heads goes to the tensor-core kernel.
-#include "launch.cuh"
+#include "attn_rows.cuh"
 
 namespace cskv {
 
-
-struct QueryRows {
-  int s;          // sequence (-1: invalid query)
-  int64_t pos;    // position
-  int64_t n_cmp;  // compressed slots
-  int64_t vis_c;  // visible CSA entries (index check)
-  int64_t cmp0, cmp_cap, raw0, raw_rows, tok0;
-  int64_t n_rows;
-};
-
-__device__ __forceinline__ QueryRows query_rows(const AttnParams& p, int t) {
-  QueryRows q;
-  q.s = __ldg(p.q_seq + t);
-  if (q.s < 0 || q.s >= p.batch) {
-    q.s = -1;
-    q.n_rows = 0;
-    return q;
-  }
-  q.pos = __ldg(p.q_pos + t);
-  q.cmp0 = __ldg(p.cmp_off + q.s);
-  q.cmp_cap = __ldg(p.cmp_off + q.s + 1) - q.cmp0;
-  q.raw0 = __ldg(p.raw_off + q.s);
-  q.raw_rows = __ldg(p.raw_off + q.s + 1) - q.raw0;
-  q.tok0 = p.raw_tok0 ? __ldg(p.raw_tok0 + q.s) : 0;
-  const int64_t ratio = p.mode == CSKV_CSA ? 4 : 128;
-  const int64_t vis = q.pos >= 0 ? (q.pos + 1) / ratio : 0;
-  q.vis_c = vis < q.cmp_cap ? vis : q.cmp_cap;
-  q.n_cmp = p.mode == CSKV_CSA ? p.k : q.vis_c;
-  q.n_rows = q.n_cmp + p.window;
-  return q;
-}
-
-// Row pointer (element offset into kv_cmp or kv_raw) of virtual row r, or -1 when the
-// row is skipped.  *raw tells which array.
-__device__ __forceinline__ int64_t resolve_row(const AttnParams& p, const QueryRows& q, int t, int64_t r,
-                                               bool* raw) {
-  if (r < q.n_cmp) {
-    *raw = false;
-    int64_t e = r;
-    if (p.mode == CSKV_CSA) {
-      e = __ldg(p.idx + (size_t)t * p.k + r);
-      if (e < 0) return -1;
-      if (e >= q.vis_c) {
-        flag(p.st, CSKV_DEV_BAD_INDEX);
-        return -1;
-      }
-    }
-    return (q.cmp0 + e) * kRow;
-  }
-  *raw = true;
-  const int64_t tok = q.pos - p.window + 1 + (r - q.n_cmp);
-  if (tok < 0) return -1;
-  const int64_t row = tok - q.tok0;
-  if (row < 0) {
-    flag(p.st, CSKV_DEV_TAIL_MISSING);
-    return -1;
-  }
-  if (row >= q.raw_rows) {
-    flag(p.st, CSKV_DEV_BAD_INDEX);
-    return -1;
-  }
-  return (q.raw0 + row) * kRow;
-}
 
 constexpr int kAttnThreads = 256;
 constexpr int kAttnTile = 32;
@@ -221,36 +158,34 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) 
 // Merge the splits of each query ([TR] §3.1), the sink once ([SW] §十二):
 //   M = max(max_s m_s, sink), L = sum_s 2^{m_s - M} l_s + 2^{sink - M},
 //   o = sum_s 2^{m_s - M} acc_s / L,   lse = ln 2 * (M + log2 L).
-__global__ void __launch_bounds__(256) attn_combine_kernel(AttnParams p) {
-  const int t = blockIdx.x;
+// One CTA per (query, head), one thread per output dimension.
+__global__ void __launch_bounds__(kHeadDim) attn_combine_kernel(AttnParams p) {
+  const int t = blockIdx.y, h = blockIdx.x, j = threadIdx.x;
   const QueryRows q = query_rows(p, t);
   const int H = p.H;
   int S = q.s < 0 ? 0 : (int)((q.n_rows + p.rows_per_split - 1) / p.rows_per_split);
   if (S > p.max_splits) {
-    if (threadIdx.x == 0) flag(p.st, CSKV_DEV_CAPACITY);
+    if (j == 0 && h == 0) flag(p.st, CSKV_DEV_CAPACITY);
     S = p.max_splits;
   }
-  for (int i = threadIdx.x; i < H * kHeadDim; i += blockDim.x) {
-    const int h = i / kHeadDim, j = i % kHeadDim;
-    const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
-    const float* ml = p.part_ml + ((size_t)t * p.max_splits * H + h) * 2;
-    float M = sk;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, ml[(size_t)s * H * 2]);
-    float L = 0.f, o = 0.f;
-    if (M != -INFINITY) {
-      if (p.sink) L = exp2f(sk - M);
-      const float* acc = p.part_acc + ((size_t)t * p.max_splits * H + h) * kHeadDim + j;
-      for (int s = 0; s < S; ++s) {
-        const float ms = ml[(size_t)s * H * 2];
-        if (ms == -INFINITY) continue;
-        const float f = exp2f(ms - M);
-        L = fmaf(ml[(size_t)s * H * 2 + 1], f, L);
-        o = fmaf(acc[(size_t)s * H * kHeadDim], f, o);
-      }
+  const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+  const float* ml = p.part_ml + ((size_t)t * p.max_splits * H + h) * 2;
+  float M = sk;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, __ldg(ml + (size_t)s * H * 2));
+  float L = 0.f, o = 0.f;
+  if (M != -INFINITY) {
+    if (p.sink) L = exp2f(sk - M);
+    const float* acc = p.part_acc + ((size_t)t * p.max_splits * H + h) * kHeadDim + j;
+    for (int s = 0; s < S; ++s) {
+      const float ms = __ldg(ml + (size_t)s * H * 2);
+      if (ms == -INFINITY) continue;
+      const float f = exp2f(ms - M);
+      L = fmaf(__ldg(ml + (size_t)s * H * 2 + 1), f, L);
+      o = fmaf(__ldg(acc + (size_t)s * H * kHeadDim), f, o);
     }
-    p.out[((size_t)t * H + h) * kHeadDim + j] = L > 0.f ? o / L : 0.f;
-    if (j == 0 && p.lse) p.lse[(size_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
+  p.out[((size_t)t * H + h) * kHeadDim + j] = L > 0.f ? o / L : 0.f;
+  if (j == 0 && p.lse) p.lse[(size_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 // ------------------------------------------------------------------ host side
@@ -270,6 +205,17 @@ int attn_rows_per_split(int mode, int T, int k, int window, int64_t max_entries,
   return (int)R;
 }
 
+// Tensor-core kernel: a split is a whole number of 128-row chunks, sized so that the
+// queries' splits about fill one wave of the SMs (at most 8 chunks per split).
+int attn_tc_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms) {
+  const int64_t rows_max = (mode == CSKV_CSA ? (int64_t)k : max_entries) + window;
+  int64_t R = (rows_max * (int64_t)T + sms - 1) / sms;
+  R = (R + 127) / 128 * 128;
+  if (R < 128) R = 128;
+  if (R > 1024) R = 1024;
+  return (int)R;
+}
+
 int attn_max_splits(int mode, int k, int window, int64_t max_entries, int R) {
   const int64_t rows_max = (mode == CSKV_CSA ? (int64_t)k : max_entries) + window;
   const int64_t s = (rows_max + R - 1) / R;
@@ -280,7 +226,7 @@ template <typename T, int HP>
 static cudaError_t launch_split(const AttnParams& p, cudaStream_t stream) {
   const size_t smem = attn_smem(HP);
   auto kern = attn_split_kernel<T, HP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.max_splits, p.T);
   kern<<<grid, kAttnThreads, smem, stream>>>(p);
@@ -303,7 +249,7 @@ cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t str
                    : launch_split<__nv_bfloat16, 128>(p, stream);
   }
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<<<p.T, 256, 0, stream>>>(p);
+  attn_combine_kernel<<<dim3(p.H, p.T), kHeadDim, 0, stream>>>(p);
   note_launch();
   return cudaGetLastError();
 }

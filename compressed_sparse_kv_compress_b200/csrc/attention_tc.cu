@@ -1,0 +1,246 @@
+// Hybrid decode attention on the 5th-generation tensor cores (tcgen05, TMEM accumulators).
+//
+// [SW] = shareware.cn/news/167317 (DeepSeek V4 Hybrid Attention essay), §八: after 128:1
+// compression a dense pass over every entry is the cheaper, regular kernel; §十一: MQA, all
+// query heads read one shared KV.  [TR] = trdm.cn/news/516303, §3.1: the online softmax
+// (running max and sum) equals the full softmax exactly.
+//
+// With MQA every gathered K||V row is shared by all H query heads, so one split of rows is a
+// real dense contraction: S = Q K^T is [H x rows] x [rows x 128] and O = P V the same size.
+// One CTA (4 warps) takes a split of the query's virtual row list (attn_rows.cuh) in chunks
+// of up to 128 rows:
+//   1. cp.async gathers the chunk's K and V halves (16-byte pieces) into shared memory in
+//      the no-swizzle core-matrix layout (8 rows x 16 bytes per core matrix);
+//   2. one thread issues tcgen05.mma: S[128 x nc] (fp32, TMEM) = Q[128 x 128] K^T (bf16);
+//   3. thread h (TMEM lane h) owns head h's row: masks skipped rows, updates the running
+//      max / sum (log2 units), rescales its O row in TMEM when the max grew, and writes
+//      P = 2^(s - m) as bf16 into shared memory;
+//   4. one thread issues O[128 x 128] (+)= P[128 x nc] V[nc x 128] (V read MN-major).
+// The split's (m, l, O) go to the workspace; attn_combine_kernel merges the splits and the
+// sink.  Heads beyond H are zero rows of Q (M is always 128).
+#include "attn_rows.cuh"
+#include "sm100.cuh"
+
+namespace cskv {
+
+constexpr int kTcThreads = 128;
+constexpr int kTcChunk = 128;                      // rows per chunk (MMA N of S, K of PV)
+constexpr uint32_t kTileBytes = 128 * 128 * 2;     // one 128 x 128 bf16 operand tile
+constexpr uint32_t kCoreStride = 128;              // bytes between neighbouring core matrices (rows)
+constexpr uint32_t kColStride = 16 * kCoreStride;  // bytes between neighbouring 16-byte column groups
+constexpr size_t kTcSmem = 4 * (size_t)kTileBytes + 1024;
+
+// Byte offset of element group (row r, 16-byte column group c) in a 128-row core-matrix tile.
+__device__ __forceinline__ uint32_t core_off(int r, int c) {
+  return (uint32_t)c * kColStride + (uint32_t)(r >> 3) * kCoreStride + (uint32_t)(r & 7) * 16;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smraw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* Qs = sm;                   // A of S = Q K^T   [128 heads x 128 d], K-major
+  uint8_t* Ks = sm + kTileBytes;      // B of S           [128 rows x 128 d], K-major
+  uint8_t* Vs = sm + 2 * kTileBytes;  // B of O = P V     [128 rows (K) x 128 d (N)], MN-major
+  uint8_t* Ps = sm + 3 * kTileBytes;  // A of O = P V     [128 heads x 128 rows], K-major
+  __shared__ uint64_t bar_s, bar_o;
+  __shared__ uint32_t tmem_base;
+  __shared__ int64_t row_src[kTcChunk];  // element offset of each chunk row, -1 = skipped
+  __shared__ uint8_t row_raw[kTcChunk];
+
+  const int t = blockIdx.y, split = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const QueryRows q = query_rows(p, t);
+  if (q.s < 0) {
+    if (split == 0 && tid == 0) flag(p.st, CSKV_DEV_BAD_INDEX);
+    return;
+  }
+  const int64_t r0 = (int64_t)split * p.rows_per_split;
+  if (r0 >= q.n_rows) return;
+  const int64_t r1 = min(q.n_rows, r0 + p.rows_per_split);
+  const int H = p.H;
+  const __nv_bfloat16* cmp = reinterpret_cast<const __nv_bfloat16*>(p.kv_cmp);
+  const __nv_bfloat16* raw = reinterpret_cast<const __nv_bfloat16*>(p.kv_raw);
+  const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(p.q) + (size_t)t * H * kHeadDim;
+
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, 256);  // S: columns 0..127, O: columns 128..255
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_s, 1);
+    mbar_init(&bar_o, 1);
+    fence_mbar_init();
+  }
+  // Q tile: thread h copies head h (zero rows beyond H)
+  for (int c = 0; c < 16; ++c)
+    cp_async16(Qs + core_off(tid, c), tid < H ? (const void*)(qg + (size_t)tid * kHeadDim + 8 * c) : (const void*)qg,
+               tid < H ? 16u : 0u);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tS = tmem_base, tO = tmem_base + 128;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+
+  const uint32_t qs_a = smem_u32(Qs), ks_a = smem_u32(Ks), vs_a = smem_u32(Vs), ps_a = smem_u32(Ps);
+  float m_run = -INFINITY, l_run = 0.f;
+  bool alive = true;
+  int c = 0;
+  for (int64_t a = r0; a < r1 && alive; a += kTcChunk, ++c) {
+    const int rows = (int)min((int64_t)kTcChunk, r1 - a);
+    const int nc = (rows + 31) & ~31;  // MMA N / K of this chunk (multiple of 32)
+    // ---- resolve the chunk's rows
+    {
+      int64_t off = -1;
+      bool is_raw = false;
+      if (tid < rows) off = resolve_row(p, q, t, a + tid, &is_raw);
+      row_src[tid] = off;
+      row_raw[tid] = is_raw;
+    }
+    __syncthreads();
+    // ---- gather K and V halves: per warp instruction 8 rows x 4 column groups, so every
+    //      quarter-warp fills one 128-byte core matrix and reads 64 contiguous bytes per row
+    for (int u = warp; u < (nc / 8) * 8; u += 4) {
+      const int rg = u >> 3, cg = u & 7;
+      const int r = rg * 8 + (lane & 7);
+      const int col = cg * 4 + (lane >> 3);  // 16-byte column group of the 512-byte row, 0..31
+      const int64_t off = row_src[r];
+      const __nv_bfloat16* src = off >= 0 ? (row_raw[r] ? raw : cmp) + off + 8 * col : qg;
+      uint8_t* dst = col < 16 ? Ks + core_off(r, col) : Vs + core_off(r, col - 16);
+      cp_async16(dst, src, off >= 0 ? 16u : 0u);
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- S = Q K^T
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(128, nc, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc_mma_f16(tS, smem_desc_noswz(qs_a + 2 * kk * kColStride, kColStride, kCoreStride),
+                   smem_desc_noswz(ks_a + 2 * kk * kColStride, kColStride, kCoreStride), idesc, kk > 0);
+      tc_commit(&bar_s);
+    }
+    if (!mbar_wait_bounded(&bar_s, c & 1)) flag(p.st, CSKV_DEV_TIMEOUT);
+    tc_fence_after();
+    // ---- online softmax of row tid over the nc columns (log2 units)
+    float mx = -INFINITY;
+    for (int cc = 0; cc < nc; cc += 32) {
+      uint32_t v[32];
+      tmem_ld32(tS + lane_base + cc, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (row_src[cc + i] >= 0) mx = fmaxf(mx, __uint_as_float(v[i]) * p.scale_log2);
+    }
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+    float lsum = 0.f;
+    for (int cc = 0; cc < nc; cc += 32) {
+      uint32_t v[32];
+      tmem_ld32(tS + lane_base + cc, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float pr[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = cc + g * 8 + i * 2 + e;
+            const float s = __uint_as_float(v[g * 8 + i * 2 + e]) * p.scale_log2;
+            pr[e] = (row_src[col] >= 0 && m_new != -INFINITY) ? exp2f(s - m_new) : 0.f;
+            lsum += pr[e];
+          }
+          w4[i] = pack_bf16(pr[0], pr[1]);
+        }
+        *reinterpret_cast<uint4*>(Ps + core_off(tid, (cc >> 3) + g)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    }
+    // O of the previous chunks is complete (its MMA was waited on).  TMEM loads and stores are
+    // warp-collective, so a warp rescales when any of its rows needs it (alpha = 1 elsewhere).
+    if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      for (int cc = 0; cc < 128; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(tO + lane_base + cc, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+        tmem_st32(tO + lane_base + cc, v);
+      }
+      tmem_st_wait();
+    }
+    l_run = l_run * alpha + lsum;
+    m_run = m_new;
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- O (+)= P V
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
+      // V tile read MN-major: the leading byte offset steps along K (row groups, 128 B apart),
+      // the stride byte offset along N (16-byte d groups, kColStride apart)
+      const uint32_t v_lbo = kCoreStride;
+      const uint32_t v_sbo = kColStride;
+      for (int kk = 0; kk < nc / 16; ++kk)
+        tc_mma_f16(tO, smem_desc_noswz(ps_a + 2 * kk * kColStride, kColStride, kCoreStride),
+                   smem_desc_noswz(vs_a + 2 * kk * kCoreStride, v_lbo, v_sbo), idesc, (c > 0 || kk > 0));
+      tc_commit(&bar_o);
+    }
+    const bool timed_out = !mbar_wait_bounded(&bar_o, c & 1);
+    if (timed_out) flag(p.st, CSKV_DEV_TIMEOUT);
+    alive = !__syncthreads_or(timed_out);  // block-uniform, so every thread leaves the loop together
+    tc_fence_after();
+  }
+  // ---- partial of this split: O row (unnormalised, relative to m_run), m_run, l_run.
+  //      Every lane takes part in the warp-collective TMEM loads; only real heads store.
+  if (c > 0) {
+    const size_t pb = ((size_t)t * p.max_splits + split) * H + tid;
+    float* dst = p.part_acc + pb * kHeadDim;
+    for (int cc = 0; cc < 128; cc += 32) {
+      uint32_t v[32];
+      tmem_ld32(tO + lane_base + cc, v);
+      tmem_ld_wait();
+      if (tid < H) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dst + cc + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                                                 __uint_as_float(v[i + 2]),
+                                                                 __uint_as_float(v[i + 3]));
+      }
+    }
+    if (tid < H) {
+      p.part_ml[pb * 2] = m_run;
+      p.part_ml[pb * 2 + 1] = l_run;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 256);
+  }
+}
+
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
+  auto kern = attn_tc_kernel;
+  cudaError_t e = ensure_smem(kern, kTcSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.max_splits, p.T);
+  kern<<<grid, kTcThreads, kTcSmem, stream>>>(p);
+  note_launch();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_combine_kernel<<<dim3(p.H, p.T), kHeadDim, 0, stream>>>(p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace cskv

@@ -203,7 +203,7 @@ struct IdxShared {
 // ------------------------------------------------------------------ scan: E4M3 via TMA + MMA
 template <int KS, int NTILE>
 __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, int64_t len,
-                         float* sc, uint8_t* ring, IdxShared& S) {
+                         float* sc, float* ssk, uint8_t* ring, IdxShared& S) {
   constexpr int Di = KS * 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int stages = p.stages;
@@ -235,6 +235,9 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
       }
     }
   } else {
+    // the segment's entry scales, fetched once while the first tiles stream in
+    for (int64_t e = threadIdx.x; e < len; e += 32 * kIdxConsumerWarps) ssk[e] = kscale ? __ldg(kscale + e) : 1.f;
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kIdxConsumerWarps) : "memory");  // consumer warps only
     const int g = lane >> 2, tq = lane & 3;
     // B fragments (the query's heads) and per-head scale / weight, loaded once.
     uint32_t bq[NTILE][KS][2];
@@ -295,8 +298,8 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
           }
         }
         const int64_t e_g = it * kIdxTile + r0 + g, e_g8 = e_g + 8;
-        const float skg = (e_g < len) ? (kscale ? __ldg(kscale + e_g) : 1.f) : 0.f;
-        const float skg8 = (e_g8 < len) ? (kscale ? __ldg(kscale + e_g8) : 1.f) : 0.f;
+        const float skg = (e_g < len) ? ssk[e_g] : 0.f;
+        const float skg8 = (e_g8 < len) ? ssk[e_g8] : 0.f;
         float vg = 0.f, vg8 = 0.f;
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt)
@@ -441,7 +444,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   if constexpr (SRC == kSrcFp8) {
     const uint8_t* kb = p.k_idx + (size_t)(ebase + lo) * (KS * 32);
     const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
-    scan_fp8<KS, NTILE>(p, t, kb, ks, len, sc, un, S);
+    scan_fp8<KS, NTILE>(p, t, kb, ks, len, sc, sc + p.seg_cap, un, S);
   } else if constexpr (SRC == kSrcF32) {
     const float* kb = reinterpret_cast<const float*>(p.k_idx) + (size_t)(ebase + lo) * p.Di;
     const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
@@ -695,7 +698,8 @@ static DevInfo dev_info() {
   return info;
 }
 
-static size_t idx_dyn_smem(int Di, int64_t seg_cap) { return idx_union_bytes(Di) + (size_t)seg_cap * 4; }
+// ring/histogram region + the segment's scores + its entry scales
+static size_t idx_dyn_smem(int Di, int64_t seg_cap) { return idx_union_bytes(Di) + (size_t)seg_cap * 8; }
 
 static size_t idx_smem_budget() {
   const DevInfo d = dev_info();
@@ -732,7 +736,7 @@ size_t lindex_ws_bytes(int T, int64_t max_entries) {
 template <int SRC, int KS, int NTILE>
 static cudaError_t launch_one(const IdxParams& p, int grid, bool coop, size_t smem, cudaStream_t stream) {
   auto kern = lindex_topk_kernel<SRC, KS, NTILE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

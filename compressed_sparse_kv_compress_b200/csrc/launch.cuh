@@ -10,6 +10,14 @@ struct QueryWS;
 // Host-side count of kernels this library has launched (api.cu).
 void note_launch();
 
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device):
+// cudaFuncSetAttribute is a host round trip that repeated launches skip (api.cu).
+cudaError_t ensure_smem_raw(const void* kern, size_t bytes);
+template <typename K>
+cudaError_t ensure_smem(K kern, size_t bytes) {
+  return ensure_smem_raw(reinterpret_cast<const void*>(kern), bytes);
+}
+
 // compress.cu
 cudaError_t launch_csa_compress(const void* xa, const void* za, const void* xb, const void* zb,
                                 const float* ba, const float* bb, const int64_t* tok_off,
@@ -77,6 +85,9 @@ struct AttnParams {
   int* st;
 };
 cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t stream);
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream);
+int attn_tc_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms);
+__global__ void attn_combine_kernel(AttnParams p);
 int attn_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms);
 int attn_max_splits(int mode, int k, int window, int64_t max_entries, int R);
 }  // namespace cskv
