@@ -142,50 +142,67 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) 
     }
     __syncthreads();
   }
-  // ---- partial out
-  const size_t pbase = ((size_t)t * p.max_splits + split) * H;
+  // ---- partial out, dimension-major: acc[split][j][h], (m, l)[split][2][h]
+  const size_t sb = (size_t)t * p.max_splits + split;
   if (hh < H) {
-    float* dst = p.part_acc + (pbase + hh) * d;
+    float* dst = p.part_acc + sb * d * H + hh;
 #pragma unroll
-    for (int i = 0; i < ACC; ++i) dst[jj + TPH * i] = acc[i];
+    for (int i = 0; i < ACC; ++i) dst[(size_t)(jj + TPH * i) * H] = acc[i];
   }
   for (int h = tid; h < H; h += kAttnThreads) {
-    p.part_ml[(pbase + h) * 2] = m_run[h];
-    p.part_ml[(pbase + h) * 2 + 1] = l_run[h];
+    p.part_ml[sb * 2 * H + h] = m_run[h];
+    p.part_ml[(sb * 2 + 1) * H + h] = l_run[h];
   }
 }
 
 // Merge the splits of each query ([TR] §3.1), the sink once ([SW] §十二):
 //   M = max(max_s m_s, sink), L = sum_s 2^{m_s - M} l_s + 2^{sink - M},
 //   o = sum_s 2^{m_s - M} acc_s / L,   lse = ln 2 * (M + log2 L).
-// One CTA per (query, head), one thread per output dimension.
-__global__ void __launch_bounds__(kHeadDim) attn_combine_kernel(AttnParams p) {
-  const int t = blockIdx.y, h = blockIdx.x, j = threadIdx.x;
-  const QueryRows q = query_rows(p, t);
+// CTA (dimension block, query), thread h = head: kCombineDims output dimensions per CTA,
+// so a query's partials are read by d / kCombineDims CTAs with coalesced loads.
+constexpr int kCombineDims = 4;
+
+__global__ void __launch_bounds__(128) attn_combine_kernel(AttnParams p) {
+  const int t = blockIdx.y, j0 = blockIdx.x * kCombineDims, h = threadIdx.x;
   const int H = p.H;
+  if (h >= H) return;
+  const QueryRows q = query_rows(p, t);
   int S = q.s < 0 ? 0 : (int)((q.n_rows + p.rows_per_split - 1) / p.rows_per_split);
   if (S > p.max_splits) {
-    if (j == 0 && h == 0) flag(p.st, CSKV_DEV_CAPACITY);
+    if (h == 0 && j0 == 0) flag(p.st, CSKV_DEV_CAPACITY);
     S = p.max_splits;
   }
+  const size_t sb0 = (size_t)t * p.max_splits;
+  const float* mrow = p.part_ml + sb0 * 2 * H + h;  // m of split s at mrow[s * 2H], l at mrow[s * 2H + H]
   const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
-  const float* ml = p.part_ml + ((size_t)t * p.max_splits * H + h) * 2;
   float M = sk;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, __ldg(ml + (size_t)s * H * 2));
-  float L = 0.f, o = 0.f;
+#pragma unroll 8
+  for (int s = 0; s < S; ++s) M = fmaxf(M, __ldg(mrow + (size_t)s * 2 * H));
+  float L = 0.f, o[kCombineDims] = {};
   if (M != -INFINITY) {
     if (p.sink) L = exp2f(sk - M);
-    const float* acc = p.part_acc + ((size_t)t * p.max_splits * H + h) * kHeadDim + j;
+    const float* acc = p.part_acc + sb0 * kHeadDim * H + (size_t)j0 * H + h;
+#pragma unroll 4
     for (int s = 0; s < S; ++s) {
-      const float ms = __ldg(ml + (size_t)s * H * 2);
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      L = fmaf(__ldg(ml + (size_t)s * H * 2 + 1), f, L);
-      o = fmaf(__ldg(acc + (size_t)s * H * kHeadDim), f, o);
+      const float ms = __ldg(mrow + (size_t)s * 2 * H);
+      const float f = ms == -INFINITY ? 0.f : exp2f(ms - M);
+      L = fmaf(__ldg(mrow + (size_t)s * 2 * H + H), f, L);
+#pragma unroll
+      for (int jj = 0; jj < kCombineDims; ++jj)
+        o[jj] = fmaf(__ldg(acc + (size_t)s * kHeadDim * H + (size_t)jj * H), f, o[jj]);
     }
   }
-  p.out[((size_t)t * H + h) * kHeadDim + j] = L > 0.f ? o / L : 0.f;
-  if (j == 0 && p.lse) p.lse[(size_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  float* dst = p.out + ((size_t)t * H + h) * kHeadDim + j0;
+#pragma unroll
+  for (int jj = 0; jj < kCombineDims; ++jj) dst[jj] = o[jj] * inv;
+  if (j0 == 0 && p.lse) p.lse[(size_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream) {
+  attn_combine_kernel<<<dim3(kHeadDim / kCombineDims, p.T), 128, 0, stream>>>(p);
+  note_launch();
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ host side
@@ -249,9 +266,7 @@ cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t str
                    : launch_split<__nv_bfloat16, 128>(p, stream);
   }
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<<<dim3(p.H, p.T), kHeadDim, 0, stream>>>(p);
-  note_launch();
-  return cudaGetLastError();
+  return launch_attn_combine(p, stream);
 }
 
 }  // namespace cskv

@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   __shared__ uint32_t tmem_base;
   __shared__ int64_t row_src[kTcChunk];  // element offset of each chunk row, -1 = skipped
   __shared__ uint8_t row_raw[kTcChunk];
+  __shared__ uint32_t row_mask[kTcChunk / 32];  // bit r: chunk row r is attended
 
   const int t = blockIdx.y, split = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const QueryRows q = query_rows(p, t);
@@ -75,14 +76,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     mbar_init(&bar_o, 1);
     fence_mbar_init();
   }
-  // Q tile: thread h copies head h (zero rows beyond H)
+  // Q tile: thread h copies head h (zero rows beyond H); the copies complete together with the
+  // first chunk's gather, and the barriers of that chunk publish the TMEM address.
   for (int c = 0; c < 16; ++c)
     cp_async16(Qs + core_off(tid, c), tid < H ? (const void*)(qg + (size_t)tid * kHeadDim + 8 * c) : (const void*)qg,
                tid < H ? 16u : 0u);
   tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tS = tmem_base, tO = tmem_base + 128;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
   const uint32_t qs_a = smem_u32(Qs), ks_a = smem_u32(Ks), vs_a = smem_u32(Vs), ps_a = smem_u32(Ps);
@@ -99,6 +98,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
       if (tid < rows) off = resolve_row(p, q, t, a + tid, &is_raw);
       row_src[tid] = off;
       row_raw[tid] = is_raw;
+      const uint32_t bal = __ballot_sync(0xffffffffu, off >= 0);
+      if (lane == 0) row_mask[warp] = bal;
     }
     __syncthreads();
     // ---- gather K and V halves: per warp instruction 8 rows x 4 column groups, so every
@@ -116,9 +117,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tS = tmem_base, tO = tmem_base + 128;
     // ---- S = Q K^T
     if (tid == 0) {
-      tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(128, nc, false, false);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
@@ -129,19 +131,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     if (!mbar_wait_bounded(&bar_s, c & 1)) flag(p.st, CSKV_DEV_TIMEOUT);
     tc_fence_after();
     // ---- online softmax of row tid over the nc columns (log2 units)
+    const float sl2 = p.scale_log2;
     float mx = -INFINITY;
     for (int cc = 0; cc < nc; cc += 32) {
+      const uint32_t vm = row_mask[cc >> 5];
       uint32_t v[32];
       tmem_ld32(tS + lane_base + cc, v);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i)
-        if (row_src[cc + i] >= 0) mx = fmaxf(mx, __uint_as_float(v[i]) * p.scale_log2);
+        if ((vm >> i) & 1u) mx = fmaxf(mx, __uint_as_float(v[i]) * sl2);
     }
     const float m_new = fmaxf(m_run, mx);
-    const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+    const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
+    const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
     float lsum = 0.f;
     for (int cc = 0; cc < nc; cc += 32) {
+      const uint32_t vm = row_mask[cc >> 5];
       uint32_t v[32];
       tmem_ld32(tS + lane_base + cc, v);
       tmem_ld_wait();
@@ -153,9 +159,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
           float pr[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int col = cc + g * 8 + i * 2 + e;
-            const float s = __uint_as_float(v[g * 8 + i * 2 + e]) * p.scale_log2;
-            pr[e] = (row_src[col] >= 0 && m_new != -INFINITY) ? exp2f(s - m_new) : 0.f;
+            const int col = g * 8 + i * 2 + e;
+            pr[e] = ((vm >> col) & 1u) ? fast_exp2(__uint_as_float(v[col]) * sl2 - m_use) : 0.f;
             lsum += pr[e];
           }
           w4[i] = pack_bf16(pr[0], pr[1]);
@@ -201,24 +206,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   }
   // ---- partial of this split: O row (unnormalised, relative to m_run), m_run, l_run.
   //      Every lane takes part in the warp-collective TMEM loads; only real heads store.
+  //      Partials are stored dimension-major ([split][j][h]), so a warp's stores are contiguous.
   if (c > 0) {
-    const size_t pb = ((size_t)t * p.max_splits + split) * H + tid;
-    float* dst = p.part_acc + pb * kHeadDim;
+    const uint32_t tO = tmem_base + 128;
+    const size_t sb = (size_t)t * p.max_splits + split;
+    float* dst = p.part_acc + sb * kHeadDim * H + tid;
     for (int cc = 0; cc < 128; cc += 32) {
       uint32_t v[32];
       tmem_ld32(tO + lane_base + cc, v);
       tmem_ld_wait();
       if (tid < H) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(dst + cc + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                                                                 __uint_as_float(v[i + 2]),
-                                                                 __uint_as_float(v[i + 3]));
+        for (int i = 0; i < 32; ++i) dst[(size_t)(cc + i) * H] = __uint_as_float(v[i]);
       }
     }
     if (tid < H) {
-      p.part_ml[pb * 2] = m_run;
-      p.part_ml[pb * 2 + 1] = l_run;
+      p.part_ml[sb * 2 * H + tid] = m_run;
+      p.part_ml[(sb * 2 + 1) * H + tid] = l_run;
     }
   }
   tc_fence_before();
@@ -238,9 +242,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
   note_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<<<dim3(p.H, p.T), kHeadDim, 0, stream>>>(p);
-  note_launch();
-  return cudaGetLastError();
+  return launch_attn_combine(p, stream);
 }
 
 }  // namespace cskv

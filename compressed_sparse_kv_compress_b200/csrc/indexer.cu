@@ -43,7 +43,7 @@ constexpr int kIdxTile = 16 * kIdxConsumerWarps;          // entries per ring st
 constexpr int kBins0 = 4096;                              // first digit: 12 bits
 constexpr int kBinsP = 1024;                              // later digits: 10 bits
 constexpr int kMaxPasses = 7;                             // 12 + 5 * 10 + 2 = 64 bits
-constexpr int kCandMax = 4096;
+constexpr int kCandMax = 8192;  // candidates exchanged per query group (global and shared)
 constexpr int kMaxGroup = 1024;
 constexpr int kMinSeg = 256;
 constexpr int kMaxSplitQueries = 128;
@@ -57,15 +57,16 @@ struct alignas(16) QueryWS {
   unsigned hist0[kBins0];
   unsigned histp[kMaxPasses - 1][kBinsP];
   unsigned above[kMaxGroup];
+  unsigned long long cut[kMaxGroup];  // speculative path: each CTA's local cutoff key
   unsigned long long cand[kCandMax];
 };
 
 
-// TMA ring depth: 48 KiB of k_idx tiles in flight per CTA whatever Di is.
-__host__ __device__ constexpr int idx_stages(int Di) { return 6 * 64 / Di; }
+// TMA ring depth: 96 KiB of k_idx tiles in flight per CTA whatever Di is.
+__host__ __device__ constexpr int idx_stages(int Di) { return 12 * 64 / Di; }
 
-// Bytes of the shared region used first as the TMA ring, then for histograms and
-// candidates (48 KiB either way).
+// Bytes of the shared region used first as the TMA ring, then for the histogram and the
+// candidate keys.
 __host__ __device__ constexpr size_t idx_union_bytes(int Di) {
   return (size_t)idx_stages(Di) * kIdxTile * Di > (size_t)kBins0 * 4 + (size_t)kCandMax * 8
              ? (size_t)idx_stages(Di) * kIdxTile * Di
@@ -86,32 +87,52 @@ __device__ __forceinline__ bool key_selected(uint64_t c, uint64_t P, int nb) {
 }
 
 // ------------------------------------------------------------------ block helpers
-// Exclusive prefix sum over threads in thread order; *total receives the sum.
+// Copies n values global -> shared with 8 loads in flight per thread (a loop that stores
+// each value before loading the next would pay one memory round trip per iteration).
+template <bool kCG, typename T>
+__device__ __forceinline__ void copy_to_smem(T* dst, const T* src, int64_t n, int tid, int nthr) {
+  constexpr int U = 8;
+  for (int64_t b = tid; b < n; b += (int64_t)nthr * U) {
+    T v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = b + (int64_t)u * nthr;
+      if (i < n) v[u] = kCG ? __ldcg(src + i) : __ldg(src + i);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = b + (int64_t)u * nthr;
+      if (i < n) dst[i] = v[u];
+    }
+  }
+}
+
+// Exclusive prefix sum over threads in thread order; *total receives the sum.  Two block
+// barriers: the warp totals are published once, and `red` is free again on return.
 __device__ unsigned block_excl_scan(unsigned v, unsigned* red, unsigned* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   unsigned x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    unsigned y = __shfl_up_sync(0xffffffffu, x, o);
+    const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  __syncthreads();
   if (lane == 31) red[warp] = x;
   __syncthreads();
-  if (warp == 0) {
-    unsigned w = lane < nw ? red[lane] : 0u;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      unsigned y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    if (lane < nw) red[lane] = w;  // inclusive warp-total prefix
+  unsigned before = x - v, tot = 0;
+  for (int w = 0; w < nw; ++w) {
+    const unsigned r = red[w];
+    before += w < warp ? r : 0u;
+    tot += r;
   }
-  __syncthreads();
-  const unsigned before = (warp ? red[warp - 1] : 0u) + x - v;
-  if (total) *total = red[nw - 1];
+  if (total) *total = tot;
   __syncthreads();
   return before;
+}
+
+// Shared-memory histogram increment (called warp-uniformly).
+__device__ __forceinline__ void hist_add(unsigned* hist, unsigned bin, bool active) {
+  if (active) atomicAdd(&hist[bin], 1u);
 }
 
 struct Crossing {
@@ -119,16 +140,12 @@ struct Crossing {
 };
 
 // hist[nbins] in shared memory; finds the bin where the count accumulated from the
-// highest bin downwards first reaches r (1 <= r <= sum of hist).
+// highest bin downwards first reaches r (1 <= r <= sum of hist).  Two block barriers;
+// `red` (>= 9 words) must not be used by anything else until the next barrier after return.
 __device__ Crossing find_crossing(const unsigned* hist, int nbins, unsigned r, unsigned* red, Crossing* out) {
   const int per = nbins >= 256 ? nbins / 256 : 1;
   const int nthr = nbins / per;
-  const int tid = threadIdx.x;
-  if (tid == 0) {  // safe default if a corrupted histogram never reaches r
-    out->bin = 0;
-    out->above = 0;
-    out->cnt = r;
-  }
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned local = 0;
   int hi = 0, lo = 0;
   if (tid < nthr) {
@@ -136,7 +153,21 @@ __device__ Crossing find_crossing(const unsigned* hist, int nbins, unsigned r, u
     lo = hi - per;
     for (int b = hi - 1; b >= lo; --b) local += hist[b];
   }
-  const unsigned excl = block_excl_scan(local, red, nullptr);
+  unsigned x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  if (tid == 0) {  // safe default if a corrupted histogram never reaches r
+    out->bin = 0;
+    out->above = 0;
+    out->cnt = r;
+  }
+  __syncthreads();
+  unsigned excl = x - local;
+  for (int w = 0; w < warp; ++w) excl += red[w];
   if (tid < nthr && local > 0 && excl < r && r <= excl + local) {
     unsigned cum = excl;
     for (int b = hi - 1; b >= lo; --b) {
@@ -151,9 +182,7 @@ __device__ Crossing find_crossing(const unsigned* hist, int nbins, unsigned r, u
     }
   }
   __syncthreads();
-  Crossing c = *out;
-  __syncthreads();
-  return c;
+  return *out;
 }
 
 // Barrier over the G CTAs of one query group (all co-resident: cooperative launch).
@@ -189,8 +218,8 @@ __device__ bool group_barrier(QueryWS* ws, unsigned G, int* st, int* sm_flag) {
 
 // ------------------------------------------------------------------ shared state
 struct IdxShared {
-  uint64_t full[8];
-  uint64_t empty[8];
+  uint64_t full[12];
+  uint64_t empty[12];
   unsigned red[32];
   Crossing cross;
   int flag;
@@ -236,7 +265,10 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
     }
   } else {
     // the segment's entry scales, fetched once while the first tiles stream in
-    for (int64_t e = threadIdx.x; e < len; e += 32 * kIdxConsumerWarps) ssk[e] = kscale ? __ldg(kscale + e) : 1.f;
+    if (kscale)
+      copy_to_smem<false>(ssk, kscale, len, threadIdx.x, 32 * kIdxConsumerWarps);
+    else
+      for (int64_t e = threadIdx.x; e < len; e += 32 * kIdxConsumerWarps) ssk[e] = 1.f;
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kIdxConsumerWarps) : "memory");  // consumer warps only
     const int g = lane >> 2, tq = lane & 3;
     // B fragments (the query's heads) and per-head scale / weight, loaded once.
@@ -334,8 +366,8 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
 __device__ void scan_f32(const IdxParams& p, int t, const float* kbase, const float* kscale, int64_t len,
                          float* sc, IdxShared& S) {
   const int Hi = p.Hi, Di = p.Di;
-  for (int i = threadIdx.x; i < Hi * Di; i += blockDim.x)
-    S.q_f32[i] = reinterpret_cast<const float*>(p.q_idx)[(size_t)t * Hi * Di + i];
+  copy_to_smem<false>(S.q_f32, reinterpret_cast<const float*>(p.q_idx) + (size_t)t * Hi * Di, Hi * Di, threadIdx.x,
+                      blockDim.x);
   __syncthreads();
   float sq[kIdxMaxHeads], wh[kIdxMaxHeads];
 #pragma unroll
@@ -371,18 +403,23 @@ __device__ void scan_f32(const IdxParams& p, int t, const float* kbase, const fl
 }
 
 // ------------------------------------------------------------------ selection helpers
-// One local radix pass over `n` keys produced by get(i), restricted to keys whose top
-// nb bits equal P.  Updates (P, nb, r); returns true when the threshold is final.
+// One local radix pass over `n` keys produced by get(i), restricted to keys whose top nb
+// bits equal P (all keys when nb == 0).  The first digit has 12 bits, later ones 10.
+// Updates (P, nb, r); returns true when "top nb bits >= P" keeps exactly the r best keys.
 template <typename Get>
 __device__ bool local_pass(Get get, int64_t n, uint64_t& P, int& nb, unsigned& r, unsigned* hist,
                            IdxShared& S) {
-  const int w = min(10, 64 - nb);
+  const int w = nb == 0 ? 12 : min(10, 64 - nb);
   const int nbins = 1 << w;
   for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0u;
   __syncthreads();
-  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-    const uint64_t c = get(i);
-    if ((c >> (64 - nb)) == P) atomicAdd(&hist[(unsigned)((c >> (64 - nb - w)) & (uint64_t)(nbins - 1))], 1u);
+  const int lane = threadIdx.x & 31;
+  for (int64_t b0 = threadIdx.x - lane; b0 < n; b0 += blockDim.x) {  // warp-uniform trip count
+    const int64_t i = b0 + lane;
+    uint64_t c = 0;
+    if (i < n) c = get(i);
+    hist_add(hist, (unsigned)((c >> (64 - nb - w)) & (uint64_t)(nbins - 1)),
+             i < n && (nb == 0 || (c >> (64 - nb)) == P));
   }
   __syncthreads();
   const Crossing x = find_crossing(hist, nbins, r, S.red, &S.cross);
@@ -390,6 +427,16 @@ __device__ bool local_pass(Get get, int64_t n, uint64_t& P, int& nb, unsigned& r
   nb += w;
   r -= x.above;
   return x.cnt == r || nb == 64;
+}
+
+// Exact top-r of n local keys: returns (P, nb) such that exactly r keys satisfy
+// "top nb bits >= P".
+template <typename Get>
+__device__ void local_select(Get get, int64_t n, unsigned r, uint64_t& P, int& nb, unsigned* hist, IdxShared& S) {
+  P = 0;
+  nb = 0;
+  bool done = false;
+  while (!done) done = local_pass(get, n, P, nb, r, hist, S);
 }
 
 // Writes the selected entries of this segment in ascending order at out[base ...].
@@ -418,6 +465,39 @@ __device__ unsigned count_selected(const float* sc, int64_t len, int64_t lo, uin
   unsigned tot;
   block_excl_scan(c, S.red, &tot);
   return tot;
+}
+
+// Candidates a segment proposes in the speculative exchange: 1.5x its expected share of
+// the top-k, plus 16, at most its length.
+__device__ __forceinline__ int64_t spec_quota(int64_t len, int64_t keff, int64_t V) {
+  const int64_t q = (3 * keff * len + 2 * V - 1) / (2 * V) + 16;
+  return q < len ? q : len;
+}
+
+// Returns the group's workspace to zero; run by the last CTA of the group to finish.
+__device__ void group_cleanup(QueryWS* ws, int G, int used_passes, unsigned cands_used, IdxShared& S) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) S.flag = (atomicAdd(&ws->done, 1u) == (unsigned)(G - 1));
+  __syncthreads();
+  if (S.flag) {
+    __threadfence();
+    for (int i = threadIdx.x; i < kBins0; i += blockDim.x) ws->hist0[i] = 0u;
+    for (int q = 0; q < used_passes; ++q)
+      for (int i = threadIdx.x; i < kBinsP; i += blockDim.x) ws->histp[q][i] = 0u;
+    for (int i = threadIdx.x; i < G; i += blockDim.x) {
+      ws->above[i] = 0u;
+      ws->cut[i] = 0ull;
+    }
+    for (unsigned i = threadIdx.x; i < cands_used; i += blockDim.x) ws->cand[i] = 0ull;
+    if (threadIdx.x == 0) {
+      // every CTA of the group is past its last barrier, so the generation can restart
+      ws->bar_gen = 0u;
+      ws->cand_count = 0u;
+      ws->done = 0u;
+    }
+  }
+  __syncthreads();
 }
 
 // ------------------------------------------------------------------ one segment
@@ -451,7 +531,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     scan_f32(p, t, kb, ks, len, sc, S);
   } else {
     const float* src = p.scores + tq * p.ld_scores + lo;
-    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) sc[e] = __ldg(src + e);
+    copy_to_smem<false>(sc, src, len, threadIdx.x, blockDim.x);
     __syncthreads();
   }
   // ---- everything kept: output position of entry e is e
@@ -461,39 +541,102 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   }
   unsigned* hist = reinterpret_cast<unsigned*>(un);
   unsigned long long* cands = reinterpret_cast<unsigned long long*>(un + kBins0 * 4);
-  // ---- pass 0: 12-bit digit
+  auto own_key = [&](int64_t i) { return comp_key(sc[i], lo + i); };
+  uint64_t P = 0;
+  int nb = 0;
+  // ---- a single CTA owns the query: exact selection in shared memory
+  if (G == 1) {
+    local_select(own_key, len, (unsigned)keff, P, nb, hist, S);
+    emit(sc, len, lo, false, P, nb, 0, keff, oi, os, S);
+    return;
+  }
+  bool ok = true;
+  // ---- speculative exchange (one group barrier): every CTA proposes its best `quota` keys
+  //      and its cutoff; all CTAs resolve the exact top-k among the proposals and accept it
+  //      when no CTA can hold an unproposed key above the resulting threshold.
+  {
+    const int64_t myq = spec_quota(len, keff, V);
+    unsigned qv = 0;
+    if ((int)threadIdx.x < G) {
+      const int jj = threadIdx.x;
+      const int64_t l2 = (int64_t)(jj + 1) * V / G - (int64_t)jj * V / G;
+      qv = (unsigned)spec_quota(l2, keff, V);
+    }
+    unsigned total;
+    const unsigned excl = block_excl_scan(qv, S.red, &total);
+    if ((int)threadIdx.x == j) S.ubuf[1] = excl;
+    __syncthreads();
+    const unsigned my_off = S.ubuf[1];
+    if (G <= (int)blockDim.x && total <= (unsigned)kCandMax && total >= (unsigned)keff) {
+      uint64_t Pq;
+      int nbq;
+      local_select(own_key, len, (unsigned)myq, Pq, nbq, hist, S);
+      // proposals in index order at cand[my_off ...] (exactly myq of them)
+      {
+        const int64_t per = (len + blockDim.x - 1) / blockDim.x;
+        const int64_t a = min(len, (int64_t)threadIdx.x * per), b = min(len, a + per);
+        unsigned c = 0;
+        for (int64_t e = a; e < b; ++e) c += key_selected(own_key(e), Pq, nbq);
+        unsigned pos = my_off + block_excl_scan(c, S.red, nullptr);
+        for (int64_t e = a; e < b; ++e) {
+          const uint64_t ck = own_key(e);
+          if (key_selected(ck, Pq, nbq)) {
+            if (pos < (unsigned)kCandMax) ws->cand[pos] = ck;
+            ++pos;
+          }
+        }
+      }
+      if (threadIdx.x == 0) ws->cut[j] = (myq == len) ? 0ull : (Pq << (64 - nbq));
+      ok = group_barrier(ws, G, p.st, &S.flag);
+      copy_to_smem<true>(cands, ws->cand, total, threadIdx.x, blockDim.x);
+      __syncthreads();
+      local_select([&](int64_t i) { return (uint64_t)cands[i]; }, total, (unsigned)keff, P, nb, hist, S);
+      const uint64_t Tstar = P << (64 - nb);
+      unsigned bad = 0;
+      for (int i = threadIdx.x; i < G; i += blockDim.x) bad += __ldcg(&ws->cut[i]) > Tstar;
+      unsigned nbad;
+      block_excl_scan(bad, S.red, &nbad);
+      if (nbad == 0) {
+        unsigned c = 0;
+        for (unsigned i = threadIdx.x; i < my_off; i += blockDim.x) c += cands[i] >= Tstar;
+        unsigned base;
+        block_excl_scan(c, S.red, &base);
+        emit(sc, len, lo, false, P, nb, base, keff, oi, os, S);
+        group_cleanup(ws, G, 0, total, S);
+        return;
+      }
+      // some CTA may hold keys above the threshold that it did not propose: exact path
+      // (the next barrier orders every read of the proposals before the slots are reused)
+    }
+  }
+  // ---- exact path: 12-bit digit histogram of the whole group
   for (int i = threadIdx.x; i < kBins0; i += blockDim.x) hist[i] = 0u;
   __syncthreads();
-  for (int64_t e = threadIdx.x; e < len; e += blockDim.x) atomicAdd(&hist[score_key(sc[e]) >> 20], 1u);
-  __syncthreads();
-  bool ok = true;
-  if (G > 1) {
-    for (int i = threadIdx.x; i < kBins0; i += blockDim.x)
-      if (hist[i]) atomicAdd(&ws->hist0[i], hist[i]);
-    ok = group_barrier(ws, G, p.st, &S.flag);
-    for (int i = threadIdx.x; i < kBins0; i += blockDim.x) hist[i] = __ldcg(&ws->hist0[i]);
-    __syncthreads();
+  for (int64_t b0 = threadIdx.x - (threadIdx.x & 31); b0 < len; b0 += blockDim.x) {
+    const int64_t e = b0 + (threadIdx.x & 31);
+    hist_add(hist, e < len ? score_key(sc[e]) >> 20 : 0u, e < len);
   }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBins0; i += blockDim.x)
+    if (hist[i]) atomicAdd(&ws->hist0[i], hist[i]);
+  ok = group_barrier(ws, G, p.st, &S.flag) && ok;
+  copy_to_smem<true>(hist, ws->hist0, kBins0, threadIdx.x, blockDim.x);
+  __syncthreads();
   unsigned r = (unsigned)keff;
   Crossing x = find_crossing(hist, kBins0, r, S.red, &S.cross);
-  uint64_t P = x.bin;
-  int nb = 12;
+  P = x.bin;
+  nb = 12;
   r -= x.above;
   bool done = (x.cnt == r);
   int used_passes = 0;
   unsigned cands_used = 0;
   int64_t base = 0;
-  bool have_base = (G == 1);
-  if (!done && G == 1) {
-    while (!done) done = local_pass([&](int64_t i) { return comp_key(sc[i], lo + i); }, len, P, nb, r, hist, S);
-  } else if (!done && x.cnt <= kCandMax) {
+  bool have_base = false;
+  if (!done && x.cnt <= kCandMax) {
     // compaction of the threshold bin's entries into the group's candidate list
     const unsigned b0 = x.bin;
     unsigned above = 0, mine = 0;
-    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
-      const unsigned d = score_key(sc[e]) >> 20;
-      above += d > b0;
-    }
+    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) above += (score_key(sc[e]) >> 20) > b0;
     const int64_t per = (len + blockDim.x - 1) / blockDim.x;
     const int64_t a = min(len, (int64_t)threadIdx.x * per), b = min(len, a + per);
     for (int64_t e = a; e < b; ++e) mine += (score_key(sc[e]) >> 20) == b0;
@@ -508,13 +651,13 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     unsigned slot = S.ubuf[0] + off;
     for (int64_t e = a; e < b; ++e)
       if ((score_key(sc[e]) >> 20) == b0) {
-        if (slot < (unsigned)kCandMax) ws->cand[slot] = comp_key(sc[e], lo + e);
+        if (slot < (unsigned)kCandMax) ws->cand[slot] = own_key(e);
         ++slot;
       }
     ok = group_barrier(ws, G, p.st, &S.flag) && ok;
     const unsigned n_c = min(__ldcg(&ws->cand_count), (unsigned)kCandMax);
     cands_used = n_c;
-    for (unsigned i = threadIdx.x; i < n_c; i += blockDim.x) cands[i] = __ldcg(&ws->cand[i]);
+    copy_to_smem<true>(cands, ws->cand, n_c, threadIdx.x, blockDim.x);
     __syncthreads();
     while (!done) done = local_pass([&](int64_t i) { return (uint64_t)cands[i]; }, n_c, P, nb, r, hist, S);
     // output base = selected entries of lower segments
@@ -536,9 +679,10 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       const int nbins = 1 << w;
       for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0u;
       __syncthreads();
-      for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
-        const uint64_t c = comp_key(sc[e], lo + e);
-        if ((c >> (64 - nb)) == P) atomicAdd(&hist[(unsigned)((c >> (64 - nb - w)) & (uint64_t)(nbins - 1))], 1u);
+      for (int64_t b0 = threadIdx.x - (threadIdx.x & 31); b0 < len; b0 += blockDim.x) {
+        const int64_t e = b0 + (threadIdx.x & 31);
+        const uint64_t c = e < len ? own_key(e) : 0ull;
+        hist_add(hist, (unsigned)((c >> (64 - nb - w)) & (uint64_t)(nbins - 1)), e < len && (c >> (64 - nb)) == P);
       }
       __syncthreads();
       unsigned* gh = ws->histp[used_passes];
@@ -546,7 +690,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
         if (hist[i]) atomicAdd(&gh[i], hist[i]);
       ++used_passes;
       ok = group_barrier(ws, G, p.st, &S.flag) && ok;
-      for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = __ldcg(&gh[i]);
+      copy_to_smem<true>(hist, gh, nbins, threadIdx.x, blockDim.x);
       __syncthreads();
       const Crossing y = find_crossing(hist, nbins, r, S.red, &S.cross);
       P = (P << w) | y.bin;
@@ -567,28 +711,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     base = tot;
   }
   emit(sc, len, lo, false, P, nb, base, keff, oi, os, S);
-  if (G > 1) {
-    // the last CTA of the group to finish returns the group's workspace to zero
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) S.flag = (atomicAdd(&ws->done, 1u) == (unsigned)(G - 1));
-    __syncthreads();
-    if (S.flag) {
-      __threadfence();
-      for (int i = threadIdx.x; i < kBins0; i += blockDim.x) ws->hist0[i] = 0u;
-      for (int q = 0; q < used_passes; ++q)
-        for (int i = threadIdx.x; i < kBinsP; i += blockDim.x) ws->histp[q][i] = 0u;
-      for (int i = threadIdx.x; i < G; i += blockDim.x) ws->above[i] = 0u;
-      for (unsigned i = threadIdx.x; i < cands_used; i += blockDim.x) ws->cand[i] = 0ull;
-      if (threadIdx.x == 0) {
-        // every CTA of the group is past its last barrier, so the generation can restart
-        ws->bar_gen = 0u;
-        ws->cand_count = 0u;
-        ws->done = 0u;
-      }
-    }
-    __syncthreads();
-  }
+  group_cleanup(ws, G, used_passes, max(cands_used, (unsigned)kCandMax), S);
 }
 
 __device__ __forceinline__ int64_t visible_of(const IdxParams& p, int t, int64_t* ebase) {
@@ -625,31 +748,29 @@ __global__ void __launch_bounds__(kIdxThreads, 1) lindex_topk_kernel(IdxParams p
   uint8_t* un = dsm;                                              // ring / histogram / candidates
   float* sc = reinterpret_cast<float*>(dsm + idx_union_bytes(KS * 32));  // segment scores
   if (p.split) {
-    for (int i = threadIdx.x; i < p.T; i += blockDim.x) {
+    // plan, in parallel over queries: visible counts, group sizes (one round), CTA ranges
+    if (threadIdx.x == 0) S.plan_t = -1;
+    int64_t v = 0;
+    if ((int)threadIdx.x < p.T) {
       int64_t eb;
-      S.plan_V[i] = visible_of(p, p.t_begin + i, &eb);
+      v = visible_of(p, p.t_begin + threadIdx.x, &eb);
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const int T = p.T, P = gridDim.x;
-      int64_t total = 0;
-      for (int i = 0; i < T; ++i) total += S.plan_V[i];
-      const int64_t avail = P - T;
-      int start = 0;
-      S.plan_t = -1;
-      for (int i = 0; i < T; ++i) {
-        const int64_t v = S.plan_V[i];
-        int64_t s = 1 + (total > 0 ? (v * avail) / total : 0);
-        const int64_t smax = v > kMinSeg ? (v + kMinSeg - 1) / kMinSeg : 1;
-        s = min(s, smax);
-        s = min(s, (int64_t)kMaxGroup);
-        if ((int)blockIdx.x >= start && (int)blockIdx.x < start + s) {
-          S.plan_t = i;
-          S.plan_j = (int)blockIdx.x - start;
-          S.plan_G = (int)s;
-        }
-        start += (int)s;
-      }
+    unsigned vt;  // totals fit: the host bounds T * max_entries below 2^31 per launch
+    block_excl_scan((unsigned)v, S.red, &vt);
+    const int64_t total = vt, avail = (int64_t)gridDim.x - p.T;
+    unsigned sz = 0;
+    if ((int)threadIdx.x < p.T) {
+      int64_t sv = 1 + (total > 0 ? (v * avail) / total : 0);
+      const int64_t smax = v > kMinSeg ? (v + kMinSeg - 1) / kMinSeg : 1;
+      sv = min(sv, smax);
+      sv = min(sv, (int64_t)kMaxGroup);
+      sz = (unsigned)sv;
+    }
+    const unsigned start = block_excl_scan(sz, S.red, nullptr);
+    if ((int)threadIdx.x < p.T && blockIdx.x >= start && blockIdx.x < start + sz) {
+      S.plan_t = threadIdx.x;
+      S.plan_j = (int)(blockIdx.x - start);
+      S.plan_G = (int)sz;
     }
     __syncthreads();
     const int i = S.plan_t;
@@ -711,6 +832,7 @@ static size_t idx_smem_budget() {
 static int split_queries_per_launch(int T, int64_t max_entries, int Di, int P, int64_t* seg_cap) {
   const size_t budget = idx_smem_budget();
   int Tb = min(T, min(P / 2, kMaxSplitQueries));
+  while (Tb >= 1 && (int64_t)Tb * max_entries >= (1LL << 31)) Tb /= 2;  // the plan sums V in 32 bits
   while (Tb >= 1) {
     int64_t cap = (int64_t)Tb * max_entries / (P - Tb) + 1;
     cap = max(cap, (int64_t)2 * kMinSeg);

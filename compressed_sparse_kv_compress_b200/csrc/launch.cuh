@@ -87,7 +87,7 @@ struct AttnParams {
 cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t stream);
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream);
 int attn_tc_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms);
-__global__ void attn_combine_kernel(AttnParams p);
+cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
 int attn_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms);
 int attn_max_splits(int mode, int k, int window, int64_t max_entries, int R);
 }  // namespace cskv

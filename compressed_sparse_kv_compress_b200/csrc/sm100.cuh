@@ -163,4 +163,11 @@ __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src, unsi
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// 2^x with the hardware approximation (relative error ~2^-22; flushes subnormal results to 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 }  // namespace cskv

@@ -97,3 +97,13 @@ def test_repeated_calls_reuse_workspace():
     rng = np.random.default_rng(5)
     for i in range(3):
         _check([rng.standard_normal(100000).astype(np.float32), rng.standard_normal(50000).astype(np.float32)], 1024)
+
+
+def test_winners_concentrated_in_one_segment():
+    # ascending scores put the whole top-k in the last segment of the group, so the
+    # speculative proposals cannot cover it and the exact path must take over
+    _check([np.arange(262144, dtype=np.float32)], 1024)
+    s = np.random.default_rng(6).random(100000).astype(np.float32)
+    s[40000:41500] += 10.0
+    _check([s], 1024)
+    _check([s[::-1].copy()], 1500)
