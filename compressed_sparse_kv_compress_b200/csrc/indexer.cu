@@ -57,7 +57,8 @@ struct alignas(16) QueryWS {
   unsigned hist0[kBins0];
   unsigned histp[kMaxPasses - 1][kBinsP];
   unsigned above[kMaxGroup];
-  unsigned long long cut[kMaxGroup];  // speculative path: each CTA's local cutoff key
+  unsigned prop[kMaxGroup];            // speculative path: proposals of each CTA
+  unsigned long long unp[kMaxGroup];   // speculative path: best key each CTA did not propose
   unsigned long long cand[kCandMax];
 };
 
@@ -81,6 +82,11 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 }
 __device__ __forceinline__ uint64_t comp_key(float s, int64_t e) {
   return ((uint64_t)score_key(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
+}
+// Score of a composite key (inverse of score_key on the top 32 bits).
+__device__ __forceinline__ float key_score(uint64_t c) {
+  const uint32_t k = (uint32_t)(c >> 32);
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 __device__ __forceinline__ bool key_selected(uint64_t c, uint64_t P, int nb) {
   return (c >> (64 - nb)) >= P;
@@ -221,6 +227,11 @@ struct IdxShared {
   uint64_t full[12];
   uint64_t empty[12];
   unsigned red[32];
+  float fred[32];
+  unsigned long long ured[16];
+  unsigned long long tstar;
+  unsigned poff[kIdxThreads];
+  unsigned pcnt[kIdxThreads];
   Crossing cross;
   int flag;
   unsigned ubuf[4];
@@ -467,11 +478,51 @@ __device__ unsigned count_selected(const float* sc, int64_t len, int64_t lo, uin
   return tot;
 }
 
-// Candidates a segment proposes in the speculative exchange: 1.5x its expected share of
-// the top-k, plus 16, at most its length.
-__device__ __forceinline__ int64_t spec_quota(int64_t len, int64_t keff, int64_t V) {
-  const int64_t q = (3 * keff * len + 2 * V - 1) / (2 * V) + 16;
-  return q < len ? q : len;
+// ---- speculative exchange helpers
+constexpr int kLinBins = 1024;  // linear score bins (<= kBins0, shares the histogram buffer)
+
+// Block-wide min and max of one float per thread.
+__device__ void block_minmax(float mn, float mx, IdxShared& S, float& gmn, float& gmx) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    S.fred[warp] = mn;
+    S.fred[16 + warp] = mx;
+  }
+  __syncthreads();
+  gmn = INFINITY;
+  gmx = -INFINITY;
+  for (int w = 0; w < nw; ++w) {
+    gmn = fminf(gmn, S.fred[w]);
+    gmx = fmaxf(gmx, S.fred[16 + w]);
+  }
+  __syncthreads();
+}
+
+// Block-wide max of one 64-bit key per thread.
+__device__ uint64_t block_max_u64(uint64_t v, IdxShared& S) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t y = __shfl_xor_sync(0xffffffffu, v, o);
+    v = y > v ? y : v;
+  }
+  if (lane == 0) S.ured[warp] = v;
+  __syncthreads();
+  uint64_t m = 0;
+  for (int w = 0; w < nw; ++w) m = S.ured[w] > m ? S.ured[w] : m;
+  __syncthreads();
+  return m;
+}
+
+// Linear bin of a score inside [lo, lo + 1024/scl]; monotone in s.
+__device__ __forceinline__ unsigned lin_bin(float s, float lo, float scl) {
+  const float f = (s - lo) * scl;
+  return f <= 0.f ? 0u : (f >= (float)(kLinBins - 1) ? (unsigned)(kLinBins - 1) : (unsigned)f);
 }
 
 // Returns the group's workspace to zero; run by the last CTA of the group to finish.
@@ -487,7 +538,8 @@ __device__ void group_cleanup(QueryWS* ws, int G, int used_passes, unsigned cand
       for (int i = threadIdx.x; i < kBinsP; i += blockDim.x) ws->histp[q][i] = 0u;
     for (int i = threadIdx.x; i < G; i += blockDim.x) {
       ws->above[i] = 0u;
-      ws->cut[i] = 0ull;
+      ws->prop[i] = 0u;
+      ws->unp[i] = 0ull;
     }
     for (unsigned i = threadIdx.x; i < cands_used; i += blockDim.x) ws->cand[i] = 0ull;
     if (threadIdx.x == 0) {
@@ -551,63 +603,197 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     return;
   }
   bool ok = true;
-  // ---- speculative exchange (one group barrier): every CTA proposes its best `quota` keys
-  //      and its cutoff; all CTAs resolve the exact top-k among the proposals and accept it
-  //      when no CTA can hold an unproposed key above the resulting threshold.
-  {
-    const int64_t myq = spec_quota(len, keff, V);
-    unsigned qv = 0;
-    if ((int)threadIdx.x < G) {
-      const int jj = threadIdx.x;
-      const int64_t l2 = (int64_t)(jj + 1) * V / G - (int64_t)jj * V / G;
-      qv = (unsigned)spec_quota(l2, keff, V);
+  // ---- speculative exchange (one group barrier).  Every CTA proposes its best entries
+  //      (those in the top bins of a linear histogram over its own score range, at most
+  //      `cap`) and reports the best key it did NOT propose.  After the barrier every CTA
+  //      finds the exact k-th best proposal T*; when no CTA holds an unproposed key >= T*,
+  //      the selection is exactly {key >= T*} and no second exchange is needed.  Otherwise
+  //      (winners crowded into one segment, massive ties) the exact path below runs.
+  // slot capacity per CTA: group-uniform (every CTA lays out and reads the slots alike)
+  const int cap = (int)min((int64_t)(kCandMax / G), (V + G - 1) / G);
+  if (G <= (int)blockDim.x && cap >= 1 && (int64_t)cap * G >= keff) {
+    // -- local range and histogram
+    float mn = INFINITY, mx = -INFINITY;
+    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
+      mn = fminf(mn, sc[e]);
+      mx = fmaxf(mx, sc[e]);
     }
-    unsigned total;
-    const unsigned excl = block_excl_scan(qv, S.red, &total);
-    if ((int)threadIdx.x == j) S.ubuf[1] = excl;
+    for (int i = threadIdx.x; i < kLinBins; i += blockDim.x) hist[i] = 0u;
+    float gmn, gmx;
+    block_minmax(mn, mx, S, gmn, gmx);
+    const float scl = gmx > gmn ? (float)kLinBins / (gmx - gmn) : 0.f;
+    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) atomicAdd(&hist[lin_bin(sc[e], gmn, scl)], 1u);
     __syncthreads();
-    const unsigned my_off = S.ubuf[1];
-    if (G <= (int)blockDim.x && total <= (unsigned)kCandMax && total >= (unsigned)keff) {
-      uint64_t Pq;
-      int nbq;
-      local_select(own_key, len, (unsigned)myq, Pq, nbq, hist, S);
-      // proposals in index order at cand[my_off ...] (exactly myq of them)
-      {
-        const int64_t per = (len + blockDim.x - 1) / blockDim.x;
-        const int64_t a = min(len, (int64_t)threadIdx.x * per), b = min(len, a + per);
-        unsigned c = 0;
-        for (int64_t e = a; e < b; ++e) c += key_selected(own_key(e), Pq, nbq);
-        unsigned pos = my_off + block_excl_scan(c, S.red, nullptr);
-        for (int64_t e = a; e < b; ++e) {
-          const uint64_t ck = own_key(e);
-          if (key_selected(ck, Pq, nbq)) {
-            if (pos < (unsigned)kCandMax) ws->cand[pos] = ck;
-            ++pos;
-          }
+    // -- warp 0: lowest bin b whose suffix count stays within the per-CTA limit
+    const unsigned limit = (unsigned)min((int64_t)cap, (3 * keff * len + 2 * V - 1) / (2 * V) + 16);
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      constexpr int per = kLinBins / 32;
+      const int bhi = kLinBins - lane * per;  // lane 0 owns the highest bins
+      unsigned loc = 0;
+      for (int bb = bhi - 1; bb >= bhi - per; --bb) loc += hist[bb];
+      unsigned inc = loc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      // suffix count before this lane's bins = inc - loc; walk down while within limit
+      unsigned cum = inc - loc;
+      int best = kLinBins;
+      unsigned bestc = 0;
+      if (cum <= limit) {
+        for (int bb = bhi - 1; bb >= bhi - per; --bb) {
+          if (cum + hist[bb] > limit) break;
+          cum += hist[bb];
+          best = bb;
+          bestc = cum;
         }
       }
-      if (threadIdx.x == 0) ws->cut[j] = (myq == len) ? 0ull : (Pq << (64 - nbq));
-      ok = group_barrier(ws, G, p.st, &S.flag);
-      copy_to_smem<true>(cands, ws->cand, total, threadIdx.x, blockDim.x);
+      // the lowest admissible bin over all lanes (suffix counts grow downwards)
+      int cand_b = best;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cand_b = min(cand_b, __shfl_xor_sync(0xffffffffu, cand_b, o));
+      if (best == cand_b && best < kLinBins) {
+        S.ubuf[2] = (unsigned)best;
+        S.ubuf[3] = bestc;
+      }
+      if (lane == 0 && cand_b == kLinBins) {
+        S.ubuf[2] = kLinBins;
+        S.ubuf[3] = 0u;
+      }
+    }
+    if (threadIdx.x == 0) S.ubuf[0] = 0u;  // proposal slot counter
+    __syncthreads();
+    const unsigned pb = S.ubuf[2];
+    // -- proposals into this CTA's slots; best unproposed key
+    uint64_t unp = 0;
+    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
+      const uint64_t ck = own_key(e);
+      if (lin_bin(sc[e], gmn, scl) >= pb) {
+        const unsigned slot = atomicAdd(&S.ubuf[0], 1u);
+        if (slot < (unsigned)cap) ws->cand[(size_t)j * cap + slot] = ck;
+      } else {
+        unp = ck > unp ? ck : unp;
+      }
+    }
+    unp = block_max_u64(unp, S);
+    if (threadIdx.x == 0) {
+      ws->prop[j] = min(S.ubuf[0], (unsigned)cap);
+      ws->unp[j] = unp;
+    }
+    ok = group_barrier(ws, G, p.st, &S.flag);
+    // -- gather every proposal (compact order = CTA order)
+    unsigned np = 0;
+    uint64_t u = 0;
+    if ((int)threadIdx.x < G) {
+      np = __ldcg(&ws->prop[threadIdx.x]);
+      u = __ldcg(&ws->unp[threadIdx.x]);
+    }
+    unsigned total;
+    const unsigned off = block_excl_scan(np, S.red, &total);
+    if ((int)threadIdx.x < G) {
+      S.poff[threadIdx.x] = off;
+      S.pcnt[threadIdx.x] = np;
+    }
+    __syncthreads();
+    if (total >= (unsigned)keff && total <= (unsigned)kCandMax) {
+      // flat copy with 8 loads in flight per thread: compact index -> (owner CTA, slot)
+      for (unsigned b0 = threadIdx.x; b0 < total; b0 += blockDim.x * 8) {
+        unsigned long long v[8];
+#pragma unroll
+        for (int uu = 0; uu < 8; ++uu) {
+          const unsigned c = b0 + uu * blockDim.x;
+          if (c < total) {
+            int lo_i = 0, hi_i = G - 1;  // last CTA whose block starts at or before c
+            while (lo_i < hi_i) {
+              const int mid = (lo_i + hi_i + 1) >> 1;
+              if (S.poff[mid] <= c) lo_i = mid; else hi_i = mid - 1;
+            }
+            v[uu] = __ldcg(ws->cand + (size_t)lo_i * cap + (c - S.poff[lo_i]));
+          }
+        }
+#pragma unroll
+        for (int uu = 0; uu < 8; ++uu) {
+          const unsigned c = b0 + uu * blockDim.x;
+          if (c < total) cands[c] = v[uu];
+        }
+      }
       __syncthreads();
-      local_select([&](int64_t i) { return (uint64_t)cands[i]; }, total, (unsigned)keff, P, nb, hist, S);
-      const uint64_t Tstar = P << (64 - nb);
-      unsigned bad = 0;
-      for (int i = threadIdx.x; i < G; i += blockDim.x) bad += __ldcg(&ws->cut[i]) > Tstar;
+      // -- exact k-th best proposal: linear histogram, then rank inside the threshold bin
+      float cmn = INFINITY, cmx = -INFINITY;
+      for (unsigned i = threadIdx.x; i < total; i += blockDim.x) {
+        const float sv = key_score(cands[i]);
+        cmn = fminf(cmn, sv);
+        cmx = fmaxf(cmx, sv);
+      }
+      for (int i = threadIdx.x; i < kLinBins; i += blockDim.x) hist[i] = 0u;
+      float qmn, qmx;
+      block_minmax(cmn, cmx, S, qmn, qmx);
+      const float qscl = qmx > qmn ? (float)kLinBins / (qmx - qmn) : 0.f;
+      for (unsigned i = threadIdx.x; i < total; i += blockDim.x)
+        atomicAdd(&hist[lin_bin(key_score(cands[i]), qmn, qscl)], 1u);
+      __syncthreads();
+      const Crossing x = find_crossing(hist, kLinBins, (unsigned)keff, S.red, &S.cross);
+      const unsigned rr = (unsigned)keff - x.above;  // rank wanted inside bin x.bin (1-based)
+      const bool bin_fits = x.cnt <= (unsigned)kCandMax - total;
+      // collect the threshold bin's keys
+      if (threadIdx.x == 0) S.ubuf[1] = 0u;
+      __syncthreads();
+      unsigned long long* bin_keys = cands + total;  // scratch after the proposals
+      const unsigned bin_cap = (unsigned)kCandMax - total;
+      for (unsigned i = threadIdx.x; i < total; i += blockDim.x)
+        if (lin_bin(key_score(cands[i]), qmn, qscl) == x.bin) {
+          const unsigned sl = atomicAdd(&S.ubuf[1], 1u);
+          if (sl < bin_cap) bin_keys[sl] = cands[i];
+        }
+      __syncthreads();
+      const unsigned nbk = min(S.ubuf[1], bin_cap);
+      uint64_t Tstar = ~0ull;
+      if (!bin_fits) {
+        // the threshold bin does not fit the scratch: leave T* at "select nothing", which the
+        // check below rejects (every CTA has an unproposed or proposed key below it)
+      } else if (nbk <= 32) {
+        if (threadIdx.x < 32) {
+          const uint64_t mine = threadIdx.x < nbk ? (uint64_t)bin_keys[threadIdx.x] : 0ull;
+          unsigned rank = 0;  // keys strictly better than mine
+          for (unsigned m = 0; m < nbk; ++m) rank += (uint64_t)bin_keys[m] > mine;
+          if (threadIdx.x < nbk && rank + 1 == rr) S.tstar = mine;
+        }
+        __syncthreads();  // (every key is distinct, so exactly one lane matches)
+        Tstar = S.tstar;
+      } else {
+        // radix select inside the bin, then T* = the smallest selected key exactly (a bare
+        // prefix threshold could also admit keys of lower linear bins)
+        uint64_t P2;
+        int nb2;
+        local_select([&](int64_t i) { return (uint64_t)bin_keys[i]; }, nbk, rr, P2, nb2, hist, S);
+        uint64_t mnk = ~0ull;
+        for (unsigned i = threadIdx.x; i < nbk; i += blockDim.x) {
+          const uint64_t kk = bin_keys[i];
+          if (key_selected(kk, P2, nb2) && kk < mnk) mnk = kk;
+        }
+        Tstar = ~block_max_u64(~mnk, S);
+      }
+      // -- accepted when no CTA kept back a key >= T*
+      unsigned bad = bin_fits ? 0u : 1u;
+      if ((int)threadIdx.x < G) bad += u >= Tstar;
       unsigned nbad;
       block_excl_scan(bad, S.red, &nbad);
-      if (nbad == 0) {
+      if (nbad == 0 && ok) {
+        const unsigned my_off = S.poff[j];
         unsigned c = 0;
         for (unsigned i = threadIdx.x; i < my_off; i += blockDim.x) c += cands[i] >= Tstar;
         unsigned base;
         block_excl_scan(c, S.red, &base);
-        emit(sc, len, lo, false, P, nb, base, keff, oi, os, S);
-        group_cleanup(ws, G, 0, total, S);
+        // emit keys >= T*: the rule "top 64 bits >= T*"
+        emit(sc, len, lo, false, Tstar, 64, base, keff, oi, os, S);
+        group_cleanup(ws, G, 0, (unsigned)G * cap, S);
         return;
       }
-      // some CTA may hold keys above the threshold that it did not propose: exact path
-      // (the next barrier orders every read of the proposals before the slots are reused)
     }
+    // fall through: the next group barrier orders every read of the proposals before the
+    // candidate slots are reused
   }
   // ---- exact path: 12-bit digit histogram of the whole group
   for (int i = threadIdx.x; i < kBins0; i += blockDim.x) hist[i] = 0u;
