@@ -16,6 +16,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_LAUNCH = 0, 1, 2, 3, 4
 F32, BF16, FP8E4M3 = 0, 1, 2
 CSA, HCA = 0, 1
 DEV_BAD_INDEX, DEV_TAIL_MISSING, DEV_CAPACITY, DEV_TIMEOUT = 1, 2, 4, 8
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _p = ctypes.c_void_p
 _i32 = ctypes.c_int
@@ -37,6 +38,8 @@ SIGNATURES = {
     "hybrid_decode_attn": (_i32, [_i32, _p, _p, _p, _p, _i32, _p, _p, _p, _i32, _p, _f, _p, _p, _i32, _i32,
                                   _i32, _i32, _i32, _i64, _p, _p, _p, _sz, _p, _p]),
     "hybrid_attn_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i64]),
+    "hybrid_decode_attn_noalloc": (_i32, [_i32, _p, _p, _p, _p, _i32, _p, _p, _p, _i32, _p, _f, _p, _p, _i32,
+                                          _i32, _i32, _i32, _i32, _i64, _p, _p, _p, _p]),
 }
 
 _lib = None

@@ -198,6 +198,33 @@ CSKV_API int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, con
 
 CSKV_API size_t hybrid_attn_workspace_size(int mode, int T, int H, int d, int k, int window, int64_t max_entries);
 
+/* ------------------------------------------------------------------------
+ * hybrid_decode_attn_noalloc -- hybrid_decode_attn for callers that cannot allocate.
+ *
+ * The source pages have no counterpart: this is a library convenience.  Some callers
+ * cannot allocate device memory when they run attention (a memory pool that owns all
+ * device memory, a plugin host that forbids allocations after start-up, a hot path that
+ * must never synchronise, as cudaMalloc/cudaFree can).  This variant takes the same
+ * arguments as hybrid_decode_attn minus the workspace, and keeps its split-KV partials
+ * in one array of CSKV_NOALLOC_SCRATCH_BYTES that the library declares in device memory.
+ * It allocates nothing.
+ * - A call whose hybrid_attn_workspace_size() exceeds CSKV_NOALLOC_SCRATCH_BYTES returns
+ *   CSKV_ERR_WORKSPACE and launches nothing.
+ * - Every GPU that loads the library holds the array until the process exits.
+ * - All calls share the array, which keeps the last call's contents.  Nothing in it needs
+ *   clearing (every partial is written before it is read), but calls that overlap on the
+ *   GPU (unordered streams) race on it.
+ * - The first call on a device looks up the array's address with that device current;
+ *   make that first call before any stream capture.
+ * ------------------------------------------------------------------------ */
+#define CSKV_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+CSKV_API int hybrid_decode_attn_noalloc(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off,
+                       const int32_t* idx, int k, const void* kv_raw, const int64_t* raw_off,
+                       const int64_t* raw_tok0, int window, const float* sink, float scale,
+                       const int32_t* q_seq, const int64_t* q_pos, int batch, int T, int H, int d,
+                       int dtype, int64_t max_entries, float* out, float* lse,
+                       int* dev_status, cskv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
