@@ -37,7 +37,7 @@
 
 namespace cskv {
 
-constexpr int kIdxConsumerWarps = 8;
+constexpr int kIdxConsumerWarps = 16;
 constexpr int kIdxThreads = 32 * (kIdxConsumerWarps + 1);  // + one producer warp
 constexpr int kIdxTile = 16 * kIdxConsumerWarps;          // entries per ring stage
 constexpr int kBins0 = 4096;                              // first digit: 12 bits
@@ -59,12 +59,13 @@ struct alignas(16) QueryWS {
   unsigned above[kMaxGroup];
   unsigned prop[kMaxGroup];            // speculative path: proposals of each CTA
   unsigned long long unp[kMaxGroup];   // speculative path: best key each CTA did not propose
+  float plo[kMaxGroup], phi[kMaxGroup];  // speculative path: score range of each CTA's proposals
   unsigned long long cand[kCandMax];
 };
 
 
 // TMA ring depth: 96 KiB of k_idx tiles in flight per CTA whatever Di is.
-__host__ __device__ constexpr int idx_stages(int Di) { return 12 * 64 / Di; }
+__host__ __device__ constexpr int idx_stages(int Di) { return (96 * 1024) / (kIdxTile * Di); }
 
 // Bytes of the shared region used first as the TMA ring, then for the histogram and the
 // candidate keys.
@@ -96,18 +97,18 @@ __device__ __forceinline__ bool key_selected(uint64_t c, uint64_t P, int nb) {
 // Copies n values global -> shared with 8 loads in flight per thread (a loop that stores
 // each value before loading the next would pay one memory round trip per iteration).
 template <bool kCG, typename T>
-__device__ __forceinline__ void copy_to_smem(T* dst, const T* src, int64_t n, int tid, int nthr) {
+__device__ __forceinline__ void copy_to_smem(T* dst, const T* src, int n, int tid, int nthr) {
   constexpr int U = 8;
-  for (int64_t b = tid; b < n; b += (int64_t)nthr * U) {
+  for (int b = tid; b < n; b += nthr * U) {
     T v[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t i = b + (int64_t)u * nthr;
+      const int i = b + u * nthr;
       if (i < n) v[u] = kCG ? __ldcg(src + i) : __ldg(src + i);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t i = b + (int64_t)u * nthr;
+      const int i = b + u * nthr;
       if (i < n) dst[i] = v[u];
     }
   }
@@ -116,7 +117,8 @@ __device__ __forceinline__ void copy_to_smem(T* dst, const T* src, int64_t n, in
 // Exclusive prefix sum over threads in thread order; *total receives the sum.  Two block
 // barriers: the warp totals are published once, and `red` is free again on return.
 __device__ unsigned block_excl_scan(unsigned v, unsigned* red, unsigned* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int nw = kIdxThreads / 32;
   unsigned x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -191,34 +193,30 @@ __device__ Crossing find_crossing(const unsigned* hist, int nbins, unsigned r, u
   return *out;
 }
 
-// Barrier over the G CTAs of one query group (all co-resident: cooperative launch).
-// Bounded: gives up after ~1 s and reports CSKV_DEV_TIMEOUT.
+// Barrier over the G CTAs of one query group (all co-resident: cooperative launch).  The
+// arrival counter only grows during a call: arrival number a belongs to the barrier that
+// completes when the counter reaches the next multiple of G.  Thread 0 publishes the CTA's
+// prior writes with a release fence (cumulative over the block barrier before it) and
+// acquires the others' after the wait.  Bounded: gives up after ~1 s (CSKV_DEV_TIMEOUT).
 __device__ bool group_barrier(QueryWS* ws, unsigned G, int* st, int* sm_flag) {
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     bool ok = true;
-    const unsigned g0 = ld_acquire_gpu(&ws->bar_gen);
-    const unsigned arrived = atomicAdd(&ws->bar_count, 1u);
-    if (arrived == G - 1) {
-      atomicExch(&ws->bar_count, 0u);
-      __threadfence();
-      atomicAdd(&ws->bar_gen, 1u);
-    } else {
-      long it = 0;
-      while (ld_acquire_gpu(&ws->bar_gen) == g0) {
-        if (++it > (1L << 24)) {
-          ok = false;
-          flag(st, CSKV_DEV_TIMEOUT);
-          break;
-        }
-        __nanosleep(64);
+    __threadfence();
+    const unsigned arrived = atomicAdd(&ws->bar_count, 1u) + 1u;
+    const unsigned target = (arrived + G - 1) / G * G;
+    long it = 0;
+    while (ld_acquire_gpu(&ws->bar_count) < target) {
+      if (++it > (1L << 24)) {
+        ok = false;
+        flag(st, CSKV_DEV_TIMEOUT);
+        break;
       }
+      __nanosleep(32);
     }
     *sm_flag = ok ? 1 : 0;
   }
   __syncthreads();
-  __threadfence();
   return *sm_flag != 0;
 }
 
@@ -227,8 +225,10 @@ struct IdxShared {
   uint64_t full[12];
   uint64_t empty[12];
   unsigned red[32];
-  float fred[32];
-  unsigned long long ured[16];
+  float fred[64];
+  unsigned long long ured[32];
+  float pmin[kIdxThreads], pmax[kIdxThreads];
+  unsigned short owner[kCandMax];
   unsigned long long tstar;
   unsigned poff[kIdxThreads];
   unsigned pcnt[kIdxThreads];
@@ -242,12 +242,12 @@ struct IdxShared {
 
 // ------------------------------------------------------------------ scan: E4M3 via TMA + MMA
 template <int KS, int NTILE>
-__device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, int64_t len,
+__device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, int len,
                          float* sc, float* ssk, uint8_t* ring, IdxShared& S) {
   constexpr int Di = KS * 32;
+  constexpr int stages = idx_stages(Di);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int stages = p.stages;
-  const int64_t ntiles = (len + kIdxTile - 1) / kIdxTile;
+  const int ntiles = (len + kIdxTile - 1) / kIdxTile;
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&S.full[s], 1);
@@ -260,27 +260,26 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
   if (warp == kIdxConsumerWarps) {
+    asm volatile("bar.sync 2, %0;" ::"n"(kIdxThreads) : "memory");  // consumers' scale loads issued
     if (lane == 0) {
-      for (int64_t it = 0; it < ntiles; ++it) {
-        const int s = (int)(it % stages);
-        const unsigned ph = (unsigned)((it / stages) & 1);
+      int s = 0;
+      unsigned ph = 0;
+      for (int it = 0; it < ntiles; ++it) {
         if (it >= stages && !mbar_wait_bounded(&S.empty[s], ph ^ 1u)) {
           flag(p.st, CSKV_DEV_TIMEOUT);
           break;
         }
-        const int64_t rows = min((int64_t)kIdxTile, len - it * kIdxTile);
+        const int rows = min(kIdxTile, len - it * kIdxTile);
         const unsigned bytes = (unsigned)(rows * Di);
         mbar_arrive_expect_tx(&S.full[s], bytes);
-        tma_bulk_g2s(ring + (size_t)s * kIdxTile * Di, kbase + it * kIdxTile * Di, bytes, &S.full[s]);
+        tma_bulk_g2s(ring + (size_t)s * kIdxTile * Di, kbase + (size_t)it * kIdxTile * Di, bytes, &S.full[s]);
+        if (++s == stages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
     }
   } else {
-    // the segment's entry scales, fetched once while the first tiles stream in
-    if (kscale)
-      copy_to_smem<false>(ssk, kscale, len, threadIdx.x, 32 * kIdxConsumerWarps);
-    else
-      for (int64_t e = threadIdx.x; e < len; e += 32 * kIdxConsumerWarps) ssk[e] = 1.f;
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * kIdxConsumerWarps) : "memory");  // consumer warps only
     const int g = lane >> 2, tq = lane & 3;
     // B fragments (the query's heads) and per-head scale / weight, loaded once.
     uint32_t bq[NTILE][KS][2];
@@ -308,17 +307,40 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
         wh[nt][c] = ok ? (p.head_w ? __ldg(p.head_w + h) : 1.f) : 0.f;
       }
     }
+    // Entry scales of this warp's rows for the next kScalePF tiles, held in registers and
+    // shifted along; the first batch is requested before the producer starts streaming, so
+    // these small loads are not queued behind the tile traffic.
+    constexpr int kScalePF = 8;
+    const int r0 = warp * 16;
+    float ska[kScalePF], skb[kScalePF];
+#pragma unroll
+    for (int i = 0; i < kScalePF; ++i) {
+      const int e = i * kIdxTile + r0 + g;
+      ska[i] = e < len ? (kscale ? __ldg(kscale + e) : 1.f) : 0.f;
+      skb[i] = e + 8 < len ? (kscale ? __ldg(kscale + e + 8) : 1.f) : 0.f;
+    }
+    asm volatile("bar.arrive 2, %0;" ::"n"(kIdxThreads) : "memory");
     bool alive = true;
-    for (int64_t it = 0; it < ntiles && alive; ++it) {
-      const int s = (int)(it % stages);
-      const unsigned ph = (unsigned)((it / stages) & 1);
+    int s = 0;
+    unsigned ph = 0;
+    for (int it = 0; it < ntiles && alive; ++it) {
       if (!mbar_wait_bounded(&S.full[s], ph)) {
         flag(p.st, CSKV_DEV_TIMEOUT);
         alive = false;
         break;
       }
-      const int64_t rows = min((int64_t)kIdxTile, len - it * kIdxTile);
-      const int r0 = warp * 16;
+      const int rows = min(kIdxTile, len - it * kIdxTile);
+      const float skg = ska[0], skg8 = skb[0];
+#pragma unroll
+      for (int i = 0; i + 1 < kScalePF; ++i) {
+        ska[i] = ska[i + 1];
+        skb[i] = skb[i + 1];
+      }
+      {
+        const int e = (it + kScalePF) * kIdxTile + r0 + g;
+        ska[kScalePF - 1] = e < len ? (kscale ? __ldg(kscale + e) : 1.f) : 0.f;
+        skb[kScalePF - 1] = e + 8 < len ? (kscale ? __ldg(kscale + e + 8) : 1.f) : 0.f;
+      }
       if (r0 < rows) {
         const uint8_t* tile = ring + (size_t)s * kIdxTile * Di;
         uint4 ra[KS / 2], rb[KS / 2];
@@ -340,9 +362,7 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
                            bq[nt][ks][0], bq[nt][ks][1]);
           }
         }
-        const int64_t e_g = it * kIdxTile + r0 + g, e_g8 = e_g + 8;
-        const float skg = (e_g < len) ? ssk[e_g] : 0.f;
-        const float skg8 = (e_g8 < len) ? ssk[e_g8] : 0.f;
+        const int e_g = it * kIdxTile + r0 + g, e_g8 = e_g + 8;
         float vg = 0.f, vg8 = 0.f;
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt)
@@ -360,6 +380,10 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.empty[s]);
+      if (++s == stages) {
+        s = 0;
+        ph ^= 1u;
+      }
     }
   }
   __syncthreads();
@@ -374,11 +398,11 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
 }
 
 // ------------------------------------------------------------------ scan: fp32 (CUDA cores)
-__device__ void scan_f32(const IdxParams& p, int t, const float* kbase, const float* kscale, int64_t len,
+__device__ void scan_f32(const IdxParams& p, int t, const float* kbase, const float* kscale, int len,
                          float* sc, IdxShared& S) {
   const int Hi = p.Hi, Di = p.Di;
   copy_to_smem<false>(S.q_f32, reinterpret_cast<const float*>(p.q_idx) + (size_t)t * Hi * Di, Hi * Di, threadIdx.x,
-                      blockDim.x);
+                      kIdxThreads);
   __syncthreads();
   float sq[kIdxMaxHeads], wh[kIdxMaxHeads];
 #pragma unroll
@@ -386,7 +410,7 @@ __device__ void scan_f32(const IdxParams& p, int t, const float* kbase, const fl
     sq[h] = (h < Hi) ? (p.q_scale ? __ldg(p.q_scale + (size_t)t * Hi + h) : 1.f) : 0.f;
     wh[h] = (h < Hi) ? (p.head_w ? __ldg(p.head_w + h) : 1.f) : 0.f;
   }
-  for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
+  for (int e = threadIdx.x; e < len; e += kIdxThreads) {
     float acc[kIdxMaxHeads];
 #pragma unroll
     for (int h = 0; h < kIdxMaxHeads; ++h) acc[h] = 0.f;
@@ -418,15 +442,15 @@ __device__ void scan_f32(const IdxParams& p, int t, const float* kbase, const fl
 // bits equal P (all keys when nb == 0).  The first digit has 12 bits, later ones 10.
 // Updates (P, nb, r); returns true when "top nb bits >= P" keeps exactly the r best keys.
 template <typename Get>
-__device__ bool local_pass(Get get, int64_t n, uint64_t& P, int& nb, unsigned& r, unsigned* hist,
+__device__ bool local_pass(Get get, int n, uint64_t& P, int& nb, unsigned& r, unsigned* hist,
                            IdxShared& S) {
   const int w = nb == 0 ? 12 : min(10, 64 - nb);
   const int nbins = 1 << w;
-  for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0u;
+  for (int i = threadIdx.x; i < nbins; i += kIdxThreads) hist[i] = 0u;
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  for (int64_t b0 = threadIdx.x - lane; b0 < n; b0 += blockDim.x) {  // warp-uniform trip count
-    const int64_t i = b0 + lane;
+  for (int b0 = threadIdx.x - lane; b0 < n; b0 += kIdxThreads) {  // warp-uniform trip count
+    const int i = b0 + lane;
     uint64_t c = 0;
     if (i < n) c = get(i);
     hist_add(hist, (unsigned)((c >> (64 - nb - w)) & (uint64_t)(nbins - 1)),
@@ -443,7 +467,7 @@ __device__ bool local_pass(Get get, int64_t n, uint64_t& P, int& nb, unsigned& r
 // Exact top-r of n local keys: returns (P, nb) such that exactly r keys satisfy
 // "top nb bits >= P".
 template <typename Get>
-__device__ void local_select(Get get, int64_t n, unsigned r, uint64_t& P, int& nb, unsigned* hist, IdxShared& S) {
+__device__ void local_select(Get get, int n, unsigned r, uint64_t& P, int& nb, unsigned* hist, IdxShared& S) {
   P = 0;
   nb = 0;
   bool done = false;
@@ -453,14 +477,14 @@ __device__ void local_select(Get get, int64_t n, unsigned r, uint64_t& P, int& n
 // Writes the selected entries of this segment in ascending order at out[base ...].
 // Positions are bounded by k, so even an inconsistent threshold (after a timed-out
 // group barrier) cannot write outside the output row.
-__device__ void emit(const float* sc, int64_t len, int64_t lo, bool all, uint64_t P, int nb, int64_t base,
+__device__ void emit(const float* sc, int len, int64_t lo, bool all, uint64_t P, int nb, int64_t base,
                      int64_t k, int32_t* oi, float* os, IdxShared& S) {
-  const int64_t per = (len + blockDim.x - 1) / blockDim.x;
-  const int64_t a = min(len, (int64_t)threadIdx.x * per), b = min(len, a + per);
+  const int per = (len + kIdxThreads - 1) / kIdxThreads;
+  const int a = min(len, (int)threadIdx.x * per), b = min(len, a + per);
   unsigned c = 0;
-  for (int64_t e = a; e < b; ++e) c += (all || key_selected(comp_key(sc[e], lo + e), P, nb)) ? 1u : 0u;
+  for (int e = a; e < b; ++e) c += (all || key_selected(comp_key(sc[e], lo + e), P, nb)) ? 1u : 0u;
   int64_t pos = base + block_excl_scan(c, S.red, nullptr);
-  for (int64_t e = a; e < b; ++e)
+  for (int e = a; e < b; ++e)
     if (all || key_selected(comp_key(sc[e], lo + e), P, nb)) {
       if (pos >= 0 && pos < k) {
         oi[pos] = (int32_t)(lo + e);
@@ -470,9 +494,9 @@ __device__ void emit(const float* sc, int64_t len, int64_t lo, bool all, uint64_
     }
 }
 
-__device__ unsigned count_selected(const float* sc, int64_t len, int64_t lo, uint64_t P, int nb, IdxShared& S) {
+__device__ unsigned count_selected(const float* sc, int len, int64_t lo, uint64_t P, int nb, IdxShared& S) {
   unsigned c = 0;
-  for (int64_t e = threadIdx.x; e < len; e += blockDim.x) c += key_selected(comp_key(sc[e], lo + e), P, nb);
+  for (int e = threadIdx.x; e < len; e += kIdxThreads) c += key_selected(comp_key(sc[e], lo + e), P, nb);
   unsigned tot;
   block_excl_scan(c, S.red, &tot);
   return tot;
@@ -483,7 +507,8 @@ constexpr int kLinBins = 1024;  // linear score bins (<= kBins0, shares the hist
 
 // Block-wide min and max of one float per thread.
 __device__ void block_minmax(float mn, float mx, IdxShared& S, float& gmn, float& gmx) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int nw = kIdxThreads / 32;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -491,21 +516,22 @@ __device__ void block_minmax(float mn, float mx, IdxShared& S, float& gmn, float
   }
   if (lane == 0) {
     S.fred[warp] = mn;
-    S.fred[16 + warp] = mx;
+    S.fred[32 + warp] = mx;
   }
   __syncthreads();
   gmn = INFINITY;
   gmx = -INFINITY;
   for (int w = 0; w < nw; ++w) {
     gmn = fminf(gmn, S.fred[w]);
-    gmx = fmaxf(gmx, S.fred[16 + w]);
+    gmx = fmaxf(gmx, S.fred[32 + w]);
   }
   __syncthreads();
 }
 
 // Block-wide max of one 64-bit key per thread.
 __device__ uint64_t block_max_u64(uint64_t v, IdxShared& S) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int nw = kIdxThreads / 32;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const uint64_t y = __shfl_xor_sync(0xffffffffu, v, o);
@@ -519,31 +545,37 @@ __device__ uint64_t block_max_u64(uint64_t v, IdxShared& S) {
   return m;
 }
 
+// Linear bin (of kBins0) of a score inside [lo, lo + kBins0/scl]; monotone in s.
+__device__ __forceinline__ unsigned lin_bin4k(float s, float lo, float scl) {
+  const float f = (s - lo) * scl;
+  return f <= 0.f ? 0u : (f >= (float)(kBins0 - 1) ? (unsigned)(kBins0 - 1) : (unsigned)f);
+}
+
 // Linear bin of a score inside [lo, lo + 1024/scl]; monotone in s.
 __device__ __forceinline__ unsigned lin_bin(float s, float lo, float scl) {
   const float f = (s - lo) * scl;
   return f <= 0.f ? 0u : (f >= (float)(kLinBins - 1) ? (unsigned)(kLinBins - 1) : (unsigned)f);
 }
 
-// Returns the group's workspace to zero; run by the last CTA of the group to finish.
-__device__ void group_cleanup(QueryWS* ws, int G, int used_passes, unsigned cands_used, IdxShared& S) {
-  __threadfence();
+// Returns the group's synchronisation state (and any global histogram it used) to zero;
+// run by the last CTA of the group to finish.  Candidate slots and per-CTA fields are
+// scratch: every call writes them before reading them.
+__device__ void group_cleanup(QueryWS* ws, int G, bool used_hist0, int used_passes, IdxShared& S) {
   __syncthreads();
-  if (threadIdx.x == 0) S.flag = (atomicAdd(&ws->done, 1u) == (unsigned)(G - 1));
+  if (threadIdx.x == 0) {
+    __threadfence();
+    S.flag = (atomicAdd(&ws->done, 1u) == (unsigned)(G - 1));
+  }
   __syncthreads();
   if (S.flag) {
     __threadfence();
-    for (int i = threadIdx.x; i < kBins0; i += blockDim.x) ws->hist0[i] = 0u;
+    if (used_hist0)
+      for (int i = threadIdx.x; i < kBins0; i += kIdxThreads) ws->hist0[i] = 0u;
     for (int q = 0; q < used_passes; ++q)
-      for (int i = threadIdx.x; i < kBinsP; i += blockDim.x) ws->histp[q][i] = 0u;
-    for (int i = threadIdx.x; i < G; i += blockDim.x) {
-      ws->above[i] = 0u;
-      ws->prop[i] = 0u;
-      ws->unp[i] = 0ull;
-    }
-    for (unsigned i = threadIdx.x; i < cands_used; i += blockDim.x) ws->cand[i] = 0ull;
+      for (int i = threadIdx.x; i < kBinsP; i += kIdxThreads) ws->histp[q][i] = 0u;
     if (threadIdx.x == 0) {
-      // every CTA of the group is past its last barrier, so the generation can restart
+      // every CTA of the group is past its last barrier
+      ws->bar_count = 0u;
       ws->bar_gen = 0u;
       ws->cand_count = 0u;
       ws->done = 0u;
@@ -557,21 +589,18 @@ template <int SRC, int KS, int NTILE>
 __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t V, int64_t ebase, QueryWS* ws,
                                 float* sc, uint8_t* un, IdxShared& S) {
   const int64_t lo = (int64_t)j * V / G, hi = (int64_t)(j + 1) * V / G;
-  int64_t len = hi - lo;
+  int len = (int)min(hi - lo, (int64_t)p.seg_cap);
   const size_t tq = (size_t)t;
   int32_t* oi = p.out_idx + tq * p.k;
   float* os = p.out_score ? p.out_score + tq * p.k : nullptr;
   const int64_t keff = min((int64_t)p.k, V);
   if (j == 0)
-    for (int64_t i = keff + threadIdx.x; i < p.k; i += blockDim.x) {
+    for (int64_t i = keff + threadIdx.x; i < p.k; i += kIdxThreads) {
       oi[i] = -1;
       if (os) os[i] = 0.f;
     }
   if (keff == 0) return;
-  if (len > p.seg_cap) {
-    if (threadIdx.x == 0) flag(p.st, CSKV_DEV_CAPACITY);
-    len = p.seg_cap;
-  }
+  if (hi - lo > p.seg_cap && threadIdx.x == 0) flag(p.st, CSKV_DEV_CAPACITY);
   // ---- scores of this segment into shared memory
   if constexpr (SRC == kSrcFp8) {
     const uint8_t* kb = p.k_idx + (size_t)(ebase + lo) * (KS * 32);
@@ -583,7 +612,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     scan_f32(p, t, kb, ks, len, sc, S);
   } else {
     const float* src = p.scores + tq * p.ld_scores + lo;
-    copy_to_smem<false>(sc, src, len, threadIdx.x, blockDim.x);
+    copy_to_smem<false>(sc, src, len, threadIdx.x, kIdxThreads);
     __syncthreads();
   }
   // ---- everything kept: output position of entry e is e
@@ -593,7 +622,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   }
   unsigned* hist = reinterpret_cast<unsigned*>(un);
   unsigned long long* cands = reinterpret_cast<unsigned long long*>(un + kBins0 * 4);
-  auto own_key = [&](int64_t i) { return comp_key(sc[i], lo + i); };
+  auto own_key = [&](int i) { return comp_key(sc[i], lo + i); };
   uint64_t P = 0;
   int nb = 0;
   // ---- a single CTA owns the query: exact selection in shared memory
@@ -611,64 +640,34 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   //      (winners crowded into one segment, massive ties) the exact path below runs.
   // slot capacity per CTA: group-uniform (every CTA lays out and reads the slots alike)
   const int cap = (int)min((int64_t)(kCandMax / G), (V + G - 1) / G);
-  if (G <= (int)blockDim.x && cap >= 1 && (int64_t)cap * G >= keff) {
+  if (G <= kIdxThreads && cap >= 1 && (int64_t)cap * G >= keff) {
     // -- local range and histogram
     float mn = INFINITY, mx = -INFINITY;
-    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
+    for (int e = threadIdx.x; e < len; e += kIdxThreads) {
       mn = fminf(mn, sc[e]);
       mx = fmaxf(mx, sc[e]);
     }
-    for (int i = threadIdx.x; i < kLinBins; i += blockDim.x) hist[i] = 0u;
+    for (int i = threadIdx.x; i < kLinBins; i += kIdxThreads) hist[i] = 0u;
     float gmn, gmx;
     block_minmax(mn, mx, S, gmn, gmx);
     const float scl = gmx > gmn ? (float)kLinBins / (gmx - gmn) : 0.f;
-    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) atomicAdd(&hist[lin_bin(sc[e], gmn, scl)], 1u);
+    for (int e = threadIdx.x; e < len; e += kIdxThreads) atomicAdd(&hist[lin_bin(sc[e], gmn, scl)], 1u);
     __syncthreads();
-    // -- warp 0: lowest bin b whose suffix count stays within the per-CTA limit
+    // -- lowest bin whose suffix count stays within the per-CTA limit: one above the bin
+    //    where the count from the top first exceeds the limit
     const unsigned limit = (unsigned)min((int64_t)cap, (3 * keff * len + 2 * V - 1) / (2 * V) + 16);
-    if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;
-      constexpr int per = kLinBins / 32;
-      const int bhi = kLinBins - lane * per;  // lane 0 owns the highest bins
-      unsigned loc = 0;
-      for (int bb = bhi - 1; bb >= bhi - per; --bb) loc += hist[bb];
-      unsigned inc = loc;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
-      }
-      // suffix count before this lane's bins = inc - loc; walk down while within limit
-      unsigned cum = inc - loc;
-      int best = kLinBins;
-      unsigned bestc = 0;
-      if (cum <= limit) {
-        for (int bb = bhi - 1; bb >= bhi - per; --bb) {
-          if (cum + hist[bb] > limit) break;
-          cum += hist[bb];
-          best = bb;
-          bestc = cum;
-        }
-      }
-      // the lowest admissible bin over all lanes (suffix counts grow downwards)
-      int cand_b = best;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) cand_b = min(cand_b, __shfl_xor_sync(0xffffffffu, cand_b, o));
-      if (best == cand_b && best < kLinBins) {
-        S.ubuf[2] = (unsigned)best;
-        S.ubuf[3] = bestc;
-      }
-      if (lane == 0 && cand_b == kLinBins) {
-        S.ubuf[2] = kLinBins;
-        S.ubuf[3] = 0u;
-      }
+    if ((unsigned)len <= limit) {
+      if (threadIdx.x == 0) S.ubuf[2] = 0u;
+    } else {
+      const Crossing xl = find_crossing(hist, kLinBins, limit + 1u, S.red, &S.cross);
+      if (threadIdx.x == 0) S.ubuf[2] = xl.bin + 1u;
     }
     if (threadIdx.x == 0) S.ubuf[0] = 0u;  // proposal slot counter
     __syncthreads();
     const unsigned pb = S.ubuf[2];
     // -- proposals into this CTA's slots; best unproposed key
     uint64_t unp = 0;
-    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) {
+    for (int e = threadIdx.x; e < len; e += kIdxThreads) {
       const uint64_t ck = own_key(e);
       if (lin_bin(sc[e], gmn, scl) >= pb) {
         const unsigned slot = atomicAdd(&S.ubuf[0], 1u);
@@ -679,62 +678,62 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     }
     unp = block_max_u64(unp, S);
     if (threadIdx.x == 0) {
-      ws->prop[j] = min(S.ubuf[0], (unsigned)cap);
+      const unsigned n_prop = min(S.ubuf[0], (unsigned)cap);
+      ws->prop[j] = n_prop;
       ws->unp[j] = unp;
+      // a range that holds every proposal (bins of a range are monotone in the score, so a
+      // slightly loose lower edge only widens the first bin)
+      ws->plo[j] = n_prop ? (pb == 0 ? gmn : gmn + (float)pb / scl) : INFINITY;
+      ws->phi[j] = n_prop ? gmx : -INFINITY;
     }
     ok = group_barrier(ws, G, p.st, &S.flag);
     // -- gather every proposal (compact order = CTA order)
     unsigned np = 0;
     uint64_t u = 0;
+    float plo = INFINITY, phi = -INFINITY;
     if ((int)threadIdx.x < G) {
       np = __ldcg(&ws->prop[threadIdx.x]);
       u = __ldcg(&ws->unp[threadIdx.x]);
+      plo = __ldcg(&ws->plo[threadIdx.x]);
+      phi = __ldcg(&ws->phi[threadIdx.x]);
     }
+    for (int i = threadIdx.x; i < kBins0; i += kIdxThreads) hist[i] = 0u;
     unsigned total;
     const unsigned off = block_excl_scan(np, S.red, &total);
+    float qmn, qmx;
+    block_minmax(plo, phi, S, qmn, qmx);
     if ((int)threadIdx.x < G) {
       S.poff[threadIdx.x] = off;
       S.pcnt[threadIdx.x] = np;
+      if (total <= (unsigned)kCandMax)  // owner table: compact index -> proposing CTA
+        for (unsigned m = 0; m < np; ++m) S.owner[off + m] = (unsigned short)threadIdx.x;
     }
     __syncthreads();
     if (total >= (unsigned)keff && total <= (unsigned)kCandMax) {
-      // flat copy with 8 loads in flight per thread: compact index -> (owner CTA, slot)
-      for (unsigned b0 = threadIdx.x; b0 < total; b0 += blockDim.x * 8) {
+      // flat copy with 8 loads in flight per thread
+      for (unsigned b0 = threadIdx.x; b0 < total; b0 += kIdxThreads * 8) {
         unsigned long long v[8];
 #pragma unroll
         for (int uu = 0; uu < 8; ++uu) {
-          const unsigned c = b0 + uu * blockDim.x;
+          const unsigned c = b0 + uu * kIdxThreads;
           if (c < total) {
-            int lo_i = 0, hi_i = G - 1;  // last CTA whose block starts at or before c
-            while (lo_i < hi_i) {
-              const int mid = (lo_i + hi_i + 1) >> 1;
-              if (S.poff[mid] <= c) lo_i = mid; else hi_i = mid - 1;
-            }
-            v[uu] = __ldcg(ws->cand + (size_t)lo_i * cap + (c - S.poff[lo_i]));
+            const int o = S.owner[c];
+            v[uu] = __ldcg(ws->cand + (size_t)o * cap + (c - S.poff[o]));
           }
         }
 #pragma unroll
         for (int uu = 0; uu < 8; ++uu) {
-          const unsigned c = b0 + uu * blockDim.x;
+          const unsigned c = b0 + uu * kIdxThreads;
           if (c < total) cands[c] = v[uu];
         }
       }
       __syncthreads();
       // -- exact k-th best proposal: linear histogram, then rank inside the threshold bin
-      float cmn = INFINITY, cmx = -INFINITY;
-      for (unsigned i = threadIdx.x; i < total; i += blockDim.x) {
-        const float sv = key_score(cands[i]);
-        cmn = fminf(cmn, sv);
-        cmx = fmaxf(cmx, sv);
-      }
-      for (int i = threadIdx.x; i < kLinBins; i += blockDim.x) hist[i] = 0u;
-      float qmn, qmx;
-      block_minmax(cmn, cmx, S, qmn, qmx);
-      const float qscl = qmx > qmn ? (float)kLinBins / (qmx - qmn) : 0.f;
-      for (unsigned i = threadIdx.x; i < total; i += blockDim.x)
-        atomicAdd(&hist[lin_bin(key_score(cands[i]), qmn, qscl)], 1u);
+      const float qscl = qmx > qmn ? (float)kBins0 / (qmx - qmn) : 0.f;
+      for (unsigned i = threadIdx.x; i < total; i += kIdxThreads)
+        atomicAdd(&hist[lin_bin4k(key_score(cands[i]), qmn, qscl)], 1u);
       __syncthreads();
-      const Crossing x = find_crossing(hist, kLinBins, (unsigned)keff, S.red, &S.cross);
+      const Crossing x = find_crossing(hist, kBins0, (unsigned)keff, S.red, &S.cross);
       const unsigned rr = (unsigned)keff - x.above;  // rank wanted inside bin x.bin (1-based)
       const bool bin_fits = x.cnt <= (unsigned)kCandMax - total;
       // collect the threshold bin's keys
@@ -742,8 +741,8 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       __syncthreads();
       unsigned long long* bin_keys = cands + total;  // scratch after the proposals
       const unsigned bin_cap = (unsigned)kCandMax - total;
-      for (unsigned i = threadIdx.x; i < total; i += blockDim.x)
-        if (lin_bin(key_score(cands[i]), qmn, qscl) == x.bin) {
+      for (unsigned i = threadIdx.x; i < total; i += kIdxThreads)
+        if (lin_bin4k(key_score(cands[i]), qmn, qscl) == x.bin) {
           const unsigned sl = atomicAdd(&S.ubuf[1], 1u);
           if (sl < bin_cap) bin_keys[sl] = cands[i];
         }
@@ -752,43 +751,47 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       uint64_t Tstar = ~0ull;
       if (!bin_fits) {
         // the threshold bin does not fit the scratch: leave T* at "select nothing", which the
-        // check below rejects (every CTA has an unproposed or proposed key below it)
-      } else if (nbk <= 32) {
-        if (threadIdx.x < 32) {
-          const uint64_t mine = threadIdx.x < nbk ? (uint64_t)bin_keys[threadIdx.x] : 0ull;
-          unsigned rank = 0;  // keys strictly better than mine
+        // check below rejects
+      } else if (nbk <= (unsigned)kIdxThreads) {
+        // thread i ranks key i against the bin (keys are distinct: exactly one has rank rr-1)
+        if (threadIdx.x < nbk) {
+          const uint64_t mine = bin_keys[threadIdx.x];
+          unsigned rank = 0;
           for (unsigned m = 0; m < nbk; ++m) rank += (uint64_t)bin_keys[m] > mine;
-          if (threadIdx.x < nbk && rank + 1 == rr) S.tstar = mine;
+          if (rank + 1 == rr) S.tstar = mine;
         }
-        __syncthreads();  // (every key is distinct, so exactly one lane matches)
+        __syncthreads();
         Tstar = S.tstar;
       } else {
         // radix select inside the bin, then T* = the smallest selected key exactly (a bare
         // prefix threshold could also admit keys of lower linear bins)
         uint64_t P2;
         int nb2;
-        local_select([&](int64_t i) { return (uint64_t)bin_keys[i]; }, nbk, rr, P2, nb2, hist, S);
+        local_select([&](int i) { return (uint64_t)bin_keys[i]; }, nbk, rr, P2, nb2, hist, S);
         uint64_t mnk = ~0ull;
-        for (unsigned i = threadIdx.x; i < nbk; i += blockDim.x) {
+        for (unsigned i = threadIdx.x; i < nbk; i += kIdxThreads) {
           const uint64_t kk = bin_keys[i];
           if (key_selected(kk, P2, nb2) && kk < mnk) mnk = kk;
         }
         Tstar = ~block_max_u64(~mnk, S);
       }
       // -- accepted when no CTA kept back a key >= T*
-      unsigned bad = bin_fits ? 0u : 1u;
-      if ((int)threadIdx.x < G) bad += u >= Tstar;
-      unsigned nbad;
-      block_excl_scan(bad, S.red, &nbad);
-      if (nbad == 0 && ok) {
+      // one block scan carries both the validity count (high bits) and this CTA's output
+      // base = proposals of lower CTAs that are kept (low 16 bits; at most kCandMax)
+      unsigned packed = 0;
+      if ((int)threadIdx.x < G) packed += (unsigned)(u >= Tstar) << 16;
+      if (threadIdx.x == 0 && !bin_fits) packed += 1u << 16;
+      {
         const unsigned my_off = S.poff[j];
-        unsigned c = 0;
-        for (unsigned i = threadIdx.x; i < my_off; i += blockDim.x) c += cands[i] >= Tstar;
-        unsigned base;
-        block_excl_scan(c, S.red, &base);
+        for (unsigned i = threadIdx.x; i < my_off; i += kIdxThreads) packed += cands[i] >= Tstar;
+      }
+      unsigned tot;
+      block_excl_scan(packed, S.red, &tot);
+      if ((tot >> 16) == 0 && ok) {
+        const unsigned base = tot & 0xFFFFu;
         // emit keys >= T*: the rule "top 64 bits >= T*"
         emit(sc, len, lo, false, Tstar, 64, base, keff, oi, os, S);
-        group_cleanup(ws, G, 0, (unsigned)G * cap, S);
+        group_cleanup(ws, G, false, 0, S);
         return;
       }
     }
@@ -796,17 +799,17 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     // candidate slots are reused
   }
   // ---- exact path: 12-bit digit histogram of the whole group
-  for (int i = threadIdx.x; i < kBins0; i += blockDim.x) hist[i] = 0u;
+  for (int i = threadIdx.x; i < kBins0; i += kIdxThreads) hist[i] = 0u;
   __syncthreads();
-  for (int64_t b0 = threadIdx.x - (threadIdx.x & 31); b0 < len; b0 += blockDim.x) {
-    const int64_t e = b0 + (threadIdx.x & 31);
+  for (int b0 = threadIdx.x - (threadIdx.x & 31); b0 < len; b0 += kIdxThreads) {
+    const int e = b0 + (threadIdx.x & 31);
     hist_add(hist, e < len ? score_key(sc[e]) >> 20 : 0u, e < len);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kBins0; i += blockDim.x)
+  for (int i = threadIdx.x; i < kBins0; i += kIdxThreads)
     if (hist[i]) atomicAdd(&ws->hist0[i], hist[i]);
   ok = group_barrier(ws, G, p.st, &S.flag) && ok;
-  copy_to_smem<true>(hist, ws->hist0, kBins0, threadIdx.x, blockDim.x);
+  copy_to_smem<true>(hist, ws->hist0, kBins0, threadIdx.x, kIdxThreads);
   __syncthreads();
   unsigned r = (unsigned)keff;
   Crossing x = find_crossing(hist, kBins0, r, S.red, &S.cross);
@@ -822,10 +825,10 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     // compaction of the threshold bin's entries into the group's candidate list
     const unsigned b0 = x.bin;
     unsigned above = 0, mine = 0;
-    for (int64_t e = threadIdx.x; e < len; e += blockDim.x) above += (score_key(sc[e]) >> 20) > b0;
-    const int64_t per = (len + blockDim.x - 1) / blockDim.x;
-    const int64_t a = min(len, (int64_t)threadIdx.x * per), b = min(len, a + per);
-    for (int64_t e = a; e < b; ++e) mine += (score_key(sc[e]) >> 20) == b0;
+    for (int e = threadIdx.x; e < len; e += kIdxThreads) above += (score_key(sc[e]) >> 20) > b0;
+    const int per = (len + kIdxThreads - 1) / kIdxThreads;
+    const int a = min(len, (int)threadIdx.x * per), b = min(len, a + per);
+    for (int e = a; e < b; ++e) mine += (score_key(sc[e]) >> 20) == b0;
     unsigned tot_above, tot_mine;
     block_excl_scan(above, S.red, &tot_above);
     const unsigned off = block_excl_scan(mine, S.red, &tot_mine);
@@ -835,7 +838,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     }
     __syncthreads();
     unsigned slot = S.ubuf[0] + off;
-    for (int64_t e = a; e < b; ++e)
+    for (int e = a; e < b; ++e)
       if ((score_key(sc[e]) >> 20) == b0) {
         if (slot < (unsigned)kCandMax) ws->cand[slot] = own_key(e);
         ++slot;
@@ -843,17 +846,17 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     ok = group_barrier(ws, G, p.st, &S.flag) && ok;
     const unsigned n_c = min(__ldcg(&ws->cand_count), (unsigned)kCandMax);
     cands_used = n_c;
-    copy_to_smem<true>(cands, ws->cand, n_c, threadIdx.x, blockDim.x);
+    copy_to_smem<true>(cands, ws->cand, n_c, threadIdx.x, kIdxThreads);
     __syncthreads();
-    while (!done) done = local_pass([&](int64_t i) { return (uint64_t)cands[i]; }, n_c, P, nb, r, hist, S);
+    while (!done) done = local_pass([&](int i) { return (uint64_t)cands[i]; }, n_c, P, nb, r, hist, S);
     // output base = selected entries of lower segments
     unsigned c = 0;
-    for (unsigned i = threadIdx.x; i < n_c; i += blockDim.x) {
+    for (unsigned i = threadIdx.x; i < n_c; i += kIdxThreads) {
       const uint64_t ck = cands[i];
       const int64_t e = (int64_t)(0xFFFFFFFFu - (uint32_t)(ck & 0xFFFFFFFFull));
       c += (e < lo && key_selected(ck, P, nb)) ? 1u : 0u;
     }
-    for (int i = threadIdx.x; i < j; i += blockDim.x) c += __ldcg(&ws->above[i]);
+    for (int i = threadIdx.x; i < j; i += kIdxThreads) c += __ldcg(&ws->above[i]);
     unsigned tot;
     block_excl_scan(c, S.red, &tot);
     base = tot;
@@ -863,20 +866,20 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     while (!done && ok) {
       const int w = min(10, 64 - nb);
       const int nbins = 1 << w;
-      for (int i = threadIdx.x; i < nbins; i += blockDim.x) hist[i] = 0u;
+      for (int i = threadIdx.x; i < nbins; i += kIdxThreads) hist[i] = 0u;
       __syncthreads();
-      for (int64_t b0 = threadIdx.x - (threadIdx.x & 31); b0 < len; b0 += blockDim.x) {
-        const int64_t e = b0 + (threadIdx.x & 31);
+      for (int b0 = threadIdx.x - (threadIdx.x & 31); b0 < len; b0 += kIdxThreads) {
+        const int e = b0 + (threadIdx.x & 31);
         const uint64_t c = e < len ? own_key(e) : 0ull;
         hist_add(hist, (unsigned)((c >> (64 - nb - w)) & (uint64_t)(nbins - 1)), e < len && (c >> (64 - nb)) == P);
       }
       __syncthreads();
       unsigned* gh = ws->histp[used_passes];
-      for (int i = threadIdx.x; i < nbins; i += blockDim.x)
+      for (int i = threadIdx.x; i < nbins; i += kIdxThreads)
         if (hist[i]) atomicAdd(&gh[i], hist[i]);
       ++used_passes;
       ok = group_barrier(ws, G, p.st, &S.flag) && ok;
-      copy_to_smem<true>(hist, gh, nbins, threadIdx.x, blockDim.x);
+      copy_to_smem<true>(hist, gh, nbins, threadIdx.x, kIdxThreads);
       __syncthreads();
       const Crossing y = find_crossing(hist, nbins, r, S.red, &S.cross);
       P = (P << w) | y.bin;
@@ -891,13 +894,13 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     if (threadIdx.x == 0) ws->above[j] = mine;
     ok = group_barrier(ws, G, p.st, &S.flag) && ok;
     unsigned c = 0;
-    for (int i = threadIdx.x; i < j; i += blockDim.x) c += __ldcg(&ws->above[i]);
+    for (int i = threadIdx.x; i < j; i += kIdxThreads) c += __ldcg(&ws->above[i]);
     unsigned tot;
     block_excl_scan(c, S.red, &tot);
     base = tot;
   }
   emit(sc, len, lo, false, P, nb, base, keff, oi, os, S);
-  group_cleanup(ws, G, used_passes, max(cands_used, (unsigned)kCandMax), S);
+  group_cleanup(ws, G, true, used_passes, S);
 }
 
 __device__ __forceinline__ int64_t visible_of(const IdxParams& p, int t, int64_t* ebase) {

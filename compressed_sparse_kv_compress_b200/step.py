@@ -8,8 +8,9 @@ as cited in the C header):
              -> lindex_score_topk -> hybrid_decode_attn(CSA)
   HCA layer: hca_compress -> hybrid_decode_attn(HCA)
 
-The HCA layer does not depend on the indexer, so with ``two_streams`` it runs
-on a second stream that forks from and joins the caller's stream.  The whole
+The HCA layer and the CSA entry compression do not depend on the indexer, so
+with ``two_streams`` they run on side streams that fork from and join the
+caller's stream (CSA attention waits for the compressed entries).  The whole
 step can be captured into a CUDA graph and replayed.
 
 Tensor names (all device tensors, int64 offsets unless noted):
@@ -51,6 +52,7 @@ class DecodeStep:
         self.ws_h = api.attn_workspace(api.HCA, T, H, 0, self.W, self.max_hca_visible, dev)
         self.two_streams = two_streams
         self.side = torch.cuda.Stream(device=dev) if two_streams else None
+        self.side2 = torch.cuda.Stream(device=dev) if two_streams else None
         self.graph = None
 
     # ------------------------------------------------------------------
@@ -66,19 +68,30 @@ class DecodeStep:
                          max_blocks=max_hca_entries, bias=t.get("bias_h"), tok0=t["hca_t0"],
                          dev_status=self.status, stream=stream)
 
-    def csa_layer(self, stream=None):
+    def csa_compress(self, stream=None):
         t = self.t
         api.csa_compress(t["x_a"], t["z_a"], t["x_b"], t["z_b"], t["csa_x_off"], t["csa_off"], t["cmp_c"],
                          max_blocks=self.max_csa_blocks, bias_a=t.get("bias_a"), bias_b=t.get("bias_b"),
                          tok0=t["csa_t0"], first_block=t["csa_first"], num_blocks=t["csa_num"],
                          dev_status=self.status, stream=stream)
+
+    def csa_select(self, stream=None):
+        t = self.t
         api.lindex_score_topk(t["q_idx"], t["k_idx"], t["q_seq"], t["q_pos"], t["csa_off"], self.idx, self.ws_idx,
                               max_entries=self.max_csa_visible, q_scale=t.get("q_scale"), k_scale=t.get("k_scale"),
                               head_w=t.get("head_w"), out_score=self.score, dev_status=self.status, stream=stream)
+
+    def csa_attend(self, stream=None):
+        t = self.t
         api.hybrid_decode_attn(api.CSA, t["q_c"], t["cmp_c"], t["csa_off"], t["raw_c"], t["raw_off"], t["q_seq"],
                                t["q_pos"], self.o_c, self.ws_c, window=self.W, idx=self.idx, raw_tok0=t["raw_t0"],
                                sink=t.get("sink_c"), scale=self.scale, lse=self.lse_c, dev_status=self.status,
                                stream=stream)
+
+    def csa_layer(self, stream=None):
+        self.csa_compress(stream)
+        self.csa_select(stream)
+        self.csa_attend(stream)
 
     def hca_layer(self, stream=None):
         t = self.t
@@ -98,9 +111,15 @@ class DecodeStep:
             self.csa_layer(main)
             self.hca_layer(main)
             return
+        # HCA layer and the CSA entry compression run beside the indexer, which needs
+        # neither; CSA attention waits for the compressed entries.
         self.side.wait_stream(main)
+        self.side2.wait_stream(main)
         self.hca_layer(self.side)
-        self.csa_layer(main)
+        self.csa_compress(self.side2)
+        self.csa_select(main)
+        main.wait_stream(self.side2)
+        self.csa_attend(main)
         main.wait_stream(self.side)
 
     # ------------------------------------------------------------------

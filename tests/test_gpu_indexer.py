@@ -29,7 +29,13 @@ def _run_indexer(w, dev=None):
                           head_w=dev["head_w"], out_score=sc, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    assert int(ws.count_nonzero().item()) == 0
+    first = idx.clone()
+    # a second call on the same workspace gives the same selection
+    api.lindex_score_topk(dev["q_idx"], dev["k_idx"], dev["q_seq"], dev["q_pos"], dev["csa_off"], idx, ws,
+                          max_entries=b["max_csa_visible"], q_scale=dev["q_scale"], k_scale=dev["k_scale"],
+                          head_w=dev["head_w"], out_score=sc, dev_status=st)
+    torch.cuda.synchronize()
+    assert torch.equal(first, idx)
     return idx.cpu().numpy(), sc.cpu().numpy()
 
 
