@@ -158,49 +158,81 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) 
 // Merge the splits of each query ([TR] §3.1), the sink once ([SW] §十二):
 //   M = max(max_s m_s, sink), L = sum_s 2^{m_s - M} l_s + 2^{sink - M},
 //   o = sum_s 2^{m_s - M} acc_s / L,   lse = ln 2 * (M + log2 L).
-// CTA (dimension block, query), thread h = head: kCombineDims output dimensions per CTA,
-// so a query's partials are read by d / kCombineDims CTAs with coalesced loads.
+// CTA (block of kCombineDims output dimensions, query); thread (head h, split group g):
+// group g folds splits g, g + kCombineGroups, ... with a running (M, L, o) -- rescaling when a
+// split's max exceeds the running one, as the online softmax does -- so its loads stream
+// without a separate max pass; the groups are then merged through shared memory.
 constexpr int kCombineDims = 4;
+constexpr int kCombineGroups = 4;
 
-__global__ void __launch_bounds__(128) attn_combine_kernel(AttnParams p) {
-  const int t = blockIdx.y, j0 = blockIdx.x * kCombineDims, h = threadIdx.x;
+__global__ void __launch_bounds__(128 * kCombineGroups) attn_combine_kernel(AttnParams p) {
+  __shared__ float sM[kCombineGroups][128], sL[kCombineGroups][128], sO[kCombineGroups][kCombineDims][128];
+  const int t = blockIdx.y, j0 = blockIdx.x * kCombineDims;
+  const int h = threadIdx.x & 127, g = threadIdx.x >> 7;
   const int H = p.H;
-  if (h >= H) return;
   const QueryRows q = query_rows(p, t);
   int S = q.s < 0 ? 0 : (int)((q.n_rows + p.rows_per_split - 1) / p.rows_per_split);
   if (S > p.max_splits) {
-    if (h == 0 && j0 == 0) flag(p.st, CSKV_DEV_CAPACITY);
+    if (threadIdx.x == 0 && j0 == 0) flag(p.st, CSKV_DEV_CAPACITY);
     S = p.max_splits;
   }
-  const size_t sb0 = (size_t)t * p.max_splits;
-  const float* mrow = p.part_ml + sb0 * 2 * H + h;  // m of split s at mrow[s * 2H], l at mrow[s * 2H + H]
-  const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
-  float M = sk;
-#pragma unroll 8
-  for (int s = 0; s < S; ++s) M = fmaxf(M, __ldg(mrow + (size_t)s * 2 * H));
-  float L = 0.f, o[kCombineDims] = {};
-  if (M != -INFINITY) {
-    if (p.sink) L = exp2f(sk - M);
+  float M = -INFINITY, L = 0.f, o[kCombineDims] = {};
+  if (h < H) {
+    const size_t sb0 = (size_t)t * p.max_splits;
+    const float* mrow = p.part_ml + sb0 * 2 * H + h;  // m of split s at mrow[s * 2H], l at + H
     const float* acc = p.part_acc + sb0 * kHeadDim * H + (size_t)j0 * H + h;
 #pragma unroll 4
-    for (int s = 0; s < S; ++s) {
+    for (int s = g; s < S; s += kCombineGroups) {
       const float ms = __ldg(mrow + (size_t)s * 2 * H);
-      const float f = ms == -INFINITY ? 0.f : exp2f(ms - M);
-      L = fmaf(__ldg(mrow + (size_t)s * 2 * H + H), f, L);
+      const float ls = __ldg(mrow + (size_t)s * 2 * H + H);
+      float a[kCombineDims];
 #pragma unroll
-      for (int jj = 0; jj < kCombineDims; ++jj)
-        o[jj] = fmaf(__ldg(acc + (size_t)s * kHeadDim * H + (size_t)jj * H), f, o[jj]);
+      for (int jj = 0; jj < kCombineDims; ++jj) a[jj] = __ldg(acc + (size_t)s * kHeadDim * H + (size_t)jj * H);
+      if (ms == -INFINITY) continue;
+      if (ms > M) {
+        const float r = exp2f(M - ms);  // 0 on the first live split
+        L *= r;
+#pragma unroll
+        for (int jj = 0; jj < kCombineDims; ++jj) o[jj] *= r;
+        M = ms;
+      }
+      const float f = exp2f(ms - M);
+      L = fmaf(ls, f, L);
+#pragma unroll
+      for (int jj = 0; jj < kCombineDims; ++jj) o[jj] = fmaf(a[jj], f, o[jj]);
     }
   }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
+  sM[g][h] = M;
+  sL[g][h] = L;
+#pragma unroll
+  for (int jj = 0; jj < kCombineDims; ++jj) sO[g][jj][h] = o[jj];
+  __syncthreads();
+  if (g != 0 || h >= H) return;
+  const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+  float Mt = sk;
+#pragma unroll
+  for (int gg = 0; gg < kCombineGroups; ++gg) Mt = fmaxf(Mt, sM[gg][h]);
+  float Lt = 0.f, ot[kCombineDims] = {};
+  if (Mt != -INFINITY) {
+    if (p.sink) Lt = exp2f(sk - Mt);
+#pragma unroll
+    for (int gg = 0; gg < kCombineGroups; ++gg) {
+      if (sM[gg][h] == -INFINITY) continue;
+      const float f = exp2f(sM[gg][h] - Mt);
+      Lt = fmaf(sL[gg][h], f, Lt);
+#pragma unroll
+      for (int jj = 0; jj < kCombineDims; ++jj) ot[jj] = fmaf(sO[gg][jj][h], f, ot[jj]);
+    }
+  }
+  const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
   float* dst = p.out + ((size_t)t * H + h) * kHeadDim + j0;
 #pragma unroll
-  for (int jj = 0; jj < kCombineDims; ++jj) dst[jj] = o[jj] * inv;
-  if (j0 == 0 && p.lse) p.lse[(size_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  for (int jj = 0; jj < kCombineDims; ++jj) dst[jj] = ot[jj] * inv;
+  if (j0 == 0 && p.lse) p.lse[(size_t)t * H + h] = Lt > 0.f ? (Mt + log2f(Lt)) * 0.69314718055994531f : -INFINITY;
 }
 
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream) {
-  attn_combine_kernel<<<dim3(kHeadDim / kCombineDims, p.T), 128, 0, stream>>>(p);
+  attn_combine_kernel<<<dim3(kHeadDim / kCombineDims, p.T), 128 * kCombineGroups, 0, stream>>>(p);
   note_launch();
   return cudaGetLastError();
 }

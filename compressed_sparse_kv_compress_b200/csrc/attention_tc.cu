@@ -132,7 +132,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     tc_fence_after();
     // ---- online softmax of row tid over the nc columns (log2 units)
     const float sl2 = p.scale_log2;
-    float mx = -INFINITY;
+    // pass 1: masked row max over the chunk, four independent max chains per 32 columns
+    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     for (int cc = 0; cc < nc; cc += 32) {
       const uint32_t vm = row_mask[cc >> 5];
       uint32_t v[32];
@@ -140,12 +141,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i)
-        if ((vm >> i) & 1u) mx = fmaxf(mx, __uint_as_float(v[i]) * sl2);
+        if ((vm >> i) & 1u) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(v[i]) * sl2);
     }
+    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
     const float m_new = fmaxf(m_run, mx);
     const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
     const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-    float lsum = 0.f;
+    // pass 2: P = 2^(s - m) as bf16 into the P tile; four independent partial sums
+    float ls4[4] = {0.f, 0.f, 0.f, 0.f};
     for (int cc = 0; cc < nc; cc += 32) {
       const uint32_t vm = row_mask[cc >> 5];
       uint32_t v[32];
@@ -161,13 +164,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
           for (int e = 0; e < 2; ++e) {
             const int col = g * 8 + i * 2 + e;
             pr[e] = ((vm >> col) & 1u) ? fast_exp2(__uint_as_float(v[col]) * sl2 - m_use) : 0.f;
-            lsum += pr[e];
+            ls4[col & 3] += pr[e];
           }
           w4[i] = pack_bf16(pr[0], pr[1]);
         }
         *reinterpret_cast<uint4*>(Ps + core_off(tid, (cc >> 3) + g)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
     }
+    const float lsum = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
     // O of the previous chunks is complete (its MMA was waited on).  TMEM loads and stores are
     // warp-collective, so a warp rescales when any of its rows needs it (alpha = 1 elsewhere).
     if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {

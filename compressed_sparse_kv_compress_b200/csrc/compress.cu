@@ -77,10 +77,13 @@ __device__ __forceinline__ SeqRange seq_range(int b, int ratio, const int64_t* t
 }
 
 // ------------------------------------------------------------------ CSA
-// grid (ceil(max_blocks / 8), batch), 256 threads: warp w of CTA x computes entry
-// first + 8x + w of sequence blockIdx.y.
+// grid (ceil(max_blocks / kCsaWarps), batch), 32 * kCsaWarps threads: warp w of CTA x
+// computes entry first + kCsaWarps * x + w of sequence blockIdx.y.  Small CTAs keep the
+// register footprint low enough to run beside the indexer in a decode step.
+constexpr int kCsaWarps = 2;
+
 template <typename TI, typename TO, bool kTwo>
-__global__ void __launch_bounds__(256) csa_compress_kernel(
+__global__ void __launch_bounds__(32 * kCsaWarps) csa_compress_kernel(
     const TI* __restrict__ xa, const TI* __restrict__ za, const TI* __restrict__ xb,
     const TI* __restrict__ zb, const float* __restrict__ ba, const float* __restrict__ bb,
     const int64_t* __restrict__ tok_off, const int64_t* __restrict__ tok0,
@@ -91,7 +94,7 @@ __global__ void __launch_bounds__(256) csa_compress_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SeqRange s = seq_range(b, 4, tok_off, tok0, ent_off, first_block, num_blocks);
   if (blockIdx.x == 0 && threadIdx.x == 0 && s.num > max_blocks) flag(st, CSKV_DEV_CAPACITY);
-  const int64_t local = (int64_t)blockIdx.x * 8 + warp;
+  const int64_t local = (int64_t)blockIdx.x * kCsaWarps + warp;
   if (local >= s.num) return;
   const int64_t i = s.first + local;
   if (i < 0 || 4 * i >= s.n || i >= s.ent_cap) {
@@ -146,20 +149,57 @@ __global__ void __launch_bounds__(256) csa_compress_kernel(
 }
 
 // ------------------------------------------------------------------ HCA
-// grid (max_blocks, batch), 512 threads: CTA x computes entry first + x; warp w owns
-// tokens 8w .. 8w+7 of the block and lane l dims 8l .. 8l+7; the 16 warp partials
-// (max, sum, weighted sum) per dimension are merged through shared memory.
-constexpr int kHcaWarps = 16;
+// Raw 4-value slice of a row kept in registers until used (bf16: one uint2).
+template <typename T>
+struct Raw4;
+
+template <>
+struct Raw4<__nv_bfloat16> {
+  uint2 v;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { v = __ldg(reinterpret_cast<const uint2*>(p)); }
+  __device__ __forceinline__ float get(int i) const {
+    const uint32_t w = (i < 2) ? v.x : v.y;
+    return (i & 1) ? __uint_as_float(w & 0xffff0000u) : __uint_as_float(w << 16);
+  }
+};
+
+template <>
+struct Raw4<float> {
+  float4 a;
+  __device__ __forceinline__ void load(const float* p) { a = __ldg(reinterpret_cast<const float4*>(p)); }
+  __device__ __forceinline__ float get(int i) const {
+    switch (i) {
+      case 0: return a.x; case 1: return a.y; case 2: return a.z; default: return a.w;
+    }
+  }
+};
+
+__device__ __forceinline__ void load_bias4(const float* bias, int slot, int j0, float (&b)[4]) {
+  if (bias == nullptr) {
+    b[0] = b[1] = b[2] = b[3] = 0.f;
+    return;
+  }
+  const float4 u = __ldg(reinterpret_cast<const float4*>(bias + (size_t)slot * kRow + j0));
+  b[0] = u.x; b[1] = u.y; b[2] = u.z; b[3] = u.w;
+}
+
+// grid (max_blocks, batch), 256 threads: CTA x computes entry first + x.  Warp w covers
+// dimension half (w & 1) -- lane l owns its dims 4l .. 4l+3 -- and token quarter (w >> 1),
+// 32 tokens streamed eight at a time with a running max; the four quarter partials
+// (max, sum, weighted sum) per dimension are merged through shared memory.  The small
+// per-thread state keeps the CTA within 64 registers, so it fits beside the indexer.
+constexpr int kHcaWarps = 8;
+constexpr int kHcaQuarters = 4;
 
 template <typename TI, typename TO>
-__global__ void __launch_bounds__(512) hca_compress_kernel(
+__global__ void __launch_bounds__(32 * kHcaWarps, 4) hca_compress_kernel(
     const TI* __restrict__ x, const TI* __restrict__ z, const float* __restrict__ bias,
     const int64_t* __restrict__ tok_off, const int64_t* __restrict__ tok0,
     const int64_t* __restrict__ ent_off, const int64_t* __restrict__ first_block,
     const int64_t* __restrict__ num_blocks, int64_t max_blocks, TO* __restrict__ out, int* st) {
-  constexpr int kTokPerWarp = 128 / kHcaWarps;             // 8
-  constexpr int kGroup = sizeof(TI) == 2 ? kTokPerWarp : 4;  // tokens loaded per round
-  __shared__ float sm_m[kHcaWarps][kRow], sm_s[kHcaWarps][kRow], sm_a[kHcaWarps][kRow];
+  constexpr int kTokPerQuarter = 128 / kHcaQuarters;  // 32
+  constexpr int kGroup = sizeof(TI) == 2 ? 8 : 4;     // tokens loaded per round
+  __shared__ float sm_m[kHcaQuarters][kRow], sm_s[kHcaQuarters][kRow], sm_a[kHcaQuarters][kRow];
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SeqRange s = seq_range(b, 128, tok_off, tok0, ent_off, first_block, num_blocks);
@@ -175,17 +215,18 @@ __global__ void __launch_bounds__(512) hca_compress_kernel(
     if (threadIdx.x == 0) flag(st, CSKV_DEV_TAIL_MISSING);
     return;
   }
-  const int j0 = lane * 8;
-  float m[8], den[8], num[8];
+  const int quarter = warp >> 1;
+  const int j0 = (warp & 1) * 128 + lane * 4;
+  float m[4], den[4], num[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) { m[j] = -INFINITY; den[j] = 0.f; num[j] = 0.f; }
-#pragma unroll
-  for (int g0 = 0; g0 < kTokPerWarp; g0 += kGroup) {
-    Raw8<TI> xr[kGroup], zr[kGroup];
+  for (int j = 0; j < 4; ++j) { m[j] = -INFINITY; den[j] = 0.f; num[j] = 0.f; }
+#pragma unroll 1
+  for (int g0 = 0; g0 < kTokPerQuarter; g0 += kGroup) {
+    Raw4<TI> xr[kGroup], zr[kGroup];
     bool ok[kGroup];
 #pragma unroll
     for (int u = 0; u < kGroup; ++u) {
-      const int slot = warp * kTokPerWarp + g0 + u;
+      const int slot = quarter * kTokPerQuarter + g0 + u;
       const int64_t t = 128 * i + slot;
       ok[u] = t < s.n;
       if (ok[u]) {
@@ -194,19 +235,16 @@ __global__ void __launch_bounds__(512) hca_compress_kernel(
         zr[u].load(z + row);
       }
     }
-    float l2[kGroup][8];
 #pragma unroll
-    for (int u = 0; u < kGroup; ++u) {
-      float bb[8];
-      load_bias8(bias, warp * kTokPerWarp + g0 + u, j0, bb);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) l2[u][j] = ok[u] ? (zr[u].get(j) + bb[j]) * kLog2e : -INFINITY;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
+      float l2[kGroup];
       float mg = m[j];
 #pragma unroll
-      for (int u = 0; u < kGroup; ++u) mg = fmaxf(mg, l2[u][j]);
+      for (int u = 0; u < kGroup; ++u) {
+        const float bb = bias ? __ldg(bias + (size_t)(quarter * kTokPerQuarter + g0 + u) * kRow + j0 + j) : 0.f;
+        l2[u] = ok[u] ? (zr[u].get(j) + bb) * kLog2e : -INFINITY;
+        mg = fmaxf(mg, l2[u]);
+      }
       if (mg != -INFINITY) {
         const float r = exp2f(m[j] - mg);  // rescale of the running sums (0 on the first group)
         den[j] *= r;
@@ -215,7 +253,7 @@ __global__ void __launch_bounds__(512) hca_compress_kernel(
 #pragma unroll
         for (int u = 0; u < kGroup; ++u)
           if (ok[u]) {
-            const float w = exp2f(l2[u][j] - mg);
+            const float w = exp2f(l2[u] - mg);
             den[j] += w;
             num[j] = fmaf(w, xr[u].get(j), num[j]);
           }
@@ -223,20 +261,20 @@ __global__ void __launch_bounds__(512) hca_compress_kernel(
     }
   }
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    sm_m[warp][j0 + j] = m[j];
-    sm_s[warp][j0 + j] = den[j];
-    sm_a[warp][j0 + j] = num[j];
+  for (int j = 0; j < 4; ++j) {
+    sm_m[quarter][j0 + j] = m[j];
+    sm_s[quarter][j0 + j] = den[j];
+    sm_a[quarter][j0 + j] = num[j];
   }
   __syncthreads();
-  if (threadIdx.x < kRow) {
-    const int j = threadIdx.x;
+  {
+    const int j = threadIdx.x;  // 256 threads, one per dimension
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kHcaWarps; ++w) M = fmaxf(M, sm_m[w][j]);
+    for (int w = 0; w < kHcaQuarters; ++w) M = fmaxf(M, sm_m[w][j]);
     float S = 0.f, A = 0.f;
 #pragma unroll
-    for (int w = 0; w < kHcaWarps; ++w) {
+    for (int w = 0; w < kHcaQuarters; ++w) {
       const float mw = sm_m[w][j];
       if (mw != -INFINITY) {
         const float f = exp2f(mw - M);
@@ -259,13 +297,13 @@ static cudaError_t launch_csa_t(const void* xa, const void* za, const void* xb, 
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
                                 void* out, int* st, cudaStream_t stream) {
-  dim3 grid((unsigned)((max_blocks + 7) / 8), (unsigned)batch);
+  dim3 grid((unsigned)((max_blocks + kCsaWarps - 1) / kCsaWarps), (unsigned)batch);
   if (xb != nullptr)
-    csa_compress_kernel<TI, TO, true><<<grid, 256, 0, stream>>>(
+    csa_compress_kernel<TI, TO, true><<<grid, 32 * kCsaWarps, 0, stream>>>(
         (const TI*)xa, (const TI*)za, (const TI*)xb, (const TI*)zb, ba, bb, tok_off, tok0, ent_off,
         first, num, max_blocks, (TO*)out, st);
   else
-    csa_compress_kernel<TI, TO, false><<<grid, 256, 0, stream>>>(
+    csa_compress_kernel<TI, TO, false><<<grid, 32 * kCsaWarps, 0, stream>>>(
         (const TI*)xa, (const TI*)za, nullptr, nullptr, ba, bb, tok_off, tok0, ent_off, first, num,
         max_blocks, (TO*)out, st);
   note_launch();
@@ -296,7 +334,7 @@ static cudaError_t launch_hca_t(const void* x, const void* z, const float* bias,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
                                 void* out, int* st, cudaStream_t stream) {
   dim3 grid((unsigned)max_blocks, (unsigned)batch);
-  hca_compress_kernel<TI, TO><<<grid, 512, 0, stream>>>((const TI*)x, (const TI*)z, bias, tok_off, tok0,
+  hca_compress_kernel<TI, TO><<<grid, 32 * kHcaWarps, 0, stream>>>((const TI*)x, (const TI*)z, bias, tok_off, tok0,
                                                        ent_off, first, num, max_blocks, (TO*)out, st);
   note_launch();
   return cudaGetLastError();

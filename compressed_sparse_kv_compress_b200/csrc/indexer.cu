@@ -43,7 +43,7 @@ constexpr int kIdxTile = 16 * kIdxConsumerWarps;          // entries per ring st
 constexpr int kBins0 = 4096;                              // first digit: 12 bits
 constexpr int kBinsP = 1024;                              // later digits: 10 bits
 constexpr int kMaxPasses = 7;                             // 12 + 5 * 10 + 2 = 64 bits
-constexpr int kCandMax = 8192;  // candidates exchanged per query group (global and shared)
+constexpr int kCandMax = 4096;  // candidates exchanged per query group (global and shared)
 constexpr int kMaxGroup = 1024;
 constexpr int kMinSeg = 256;
 constexpr int kMaxSplitQueries = 128;
@@ -64,15 +64,23 @@ struct alignas(16) QueryWS {
 };
 
 
-// TMA ring depth: 96 KiB of k_idx tiles in flight per CTA whatever Di is.
-__host__ __device__ constexpr int idx_stages(int Di) { return (96 * 1024) / (kIdxTile * Di); }
+// TMA ring depth: 64 KiB of k_idx tiles in flight per CTA whatever Di is.
+__host__ __device__ constexpr int idx_stages(int Di) { return (64 * 1024) / (kIdxTile * Di); }
+
+// Layout of the shared region after the scan: histogram, candidate keys, then a scratch
+// area used first as the owner table of the gathered proposals, then for the keys of the
+// threshold bin.
+constexpr size_t kUnHist = 0;
+constexpr size_t kUnCand = (size_t)kBins0 * 4;
+constexpr size_t kUnAux = kUnCand + (size_t)kCandMax * 8;
+constexpr int kAuxKeys = 1024;  // 8 KiB: kCandMax owner entries (2 B) or kAuxKeys keys (8 B)
+constexpr size_t kUnSelBytes = kUnAux + (size_t)kAuxKeys * 8;
 
 // Bytes of the shared region used first as the TMA ring, then for the histogram and the
 // candidate keys.
 __host__ __device__ constexpr size_t idx_union_bytes(int Di) {
-  return (size_t)idx_stages(Di) * kIdxTile * Di > (size_t)kBins0 * 4 + (size_t)kCandMax * 8
-             ? (size_t)idx_stages(Di) * kIdxTile * Di
-             : (size_t)kBins0 * 4 + (size_t)kCandMax * 8;
+  return (size_t)idx_stages(Di) * kIdxTile * Di > kUnSelBytes ? (size_t)idx_stages(Di) * kIdxTile * Di
+                                                                : kUnSelBytes;
 }
 
 // ------------------------------------------------------------------ keys
@@ -151,7 +159,7 @@ struct Crossing {
 // highest bin downwards first reaches r (1 <= r <= sum of hist).  Two block barriers;
 // `red` (>= 9 words) must not be used by anything else until the next barrier after return.
 __device__ Crossing find_crossing(const unsigned* hist, int nbins, unsigned r, unsigned* red, Crossing* out) {
-  const int per = nbins >= 256 ? nbins / 256 : 1;
+  const int per = nbins >= 512 ? nbins / 512 : 1;
   const int nthr = nbins / per;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned local = 0;
@@ -228,7 +236,6 @@ struct IdxShared {
   float fred[64];
   unsigned long long ured[32];
   float pmin[kIdxThreads], pmax[kIdxThreads];
-  unsigned short owner[kCandMax];
   unsigned long long tstar;
   unsigned poff[kIdxThreads];
   unsigned pcnt[kIdxThreads];
@@ -237,7 +244,6 @@ struct IdxShared {
   unsigned ubuf[4];
   int plan_t, plan_j, plan_G;
   long long plan_V[kMaxSplitQueries];
-  float q_f32[kIdxMaxHeads * kIdxMaxDim];
 };
 
 // ------------------------------------------------------------------ scan: E4M3 via TMA + MMA
@@ -399,9 +405,9 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
 
 // ------------------------------------------------------------------ scan: fp32 (CUDA cores)
 __device__ void scan_f32(const IdxParams& p, int t, const float* kbase, const float* kscale, int len,
-                         float* sc, IdxShared& S) {
+                         float* sc, float* q_f32, IdxShared& S) {
   const int Hi = p.Hi, Di = p.Di;
-  copy_to_smem<false>(S.q_f32, reinterpret_cast<const float*>(p.q_idx) + (size_t)t * Hi * Di, Hi * Di, threadIdx.x,
+  copy_to_smem<false>(q_f32, reinterpret_cast<const float*>(p.q_idx) + (size_t)t * Hi * Di, Hi * Di, threadIdx.x,
                       kIdxThreads);
   __syncthreads();
   float sq[kIdxMaxHeads], wh[kIdxMaxHeads];
@@ -420,7 +426,7 @@ __device__ void scan_f32(const IdxParams& p, int t, const float* kbase, const fl
 #pragma unroll
       for (int h = 0; h < kIdxMaxHeads; ++h)
         if (h < Hi) {
-          const float* q = S.q_f32 + h * Di + 4 * d4;
+          const float* q = q_f32 + h * Di + 4 * d4;
           acc[h] = fmaf(q[0], kv.x, acc[h]);
           acc[h] = fmaf(q[1], kv.y, acc[h]);
           acc[h] = fmaf(q[2], kv.z, acc[h]);
@@ -609,7 +615,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   } else if constexpr (SRC == kSrcF32) {
     const float* kb = reinterpret_cast<const float*>(p.k_idx) + (size_t)(ebase + lo) * p.Di;
     const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
-    scan_f32(p, t, kb, ks, len, sc, S);
+    scan_f32(p, t, kb, ks, len, sc, reinterpret_cast<float*>(un), S);
   } else {
     const float* src = p.scores + tq * p.ld_scores + lo;
     copy_to_smem<false>(sc, src, len, threadIdx.x, kIdxThreads);
@@ -620,8 +626,9 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     emit(sc, len, lo, true, 0, 0, lo, keff, oi, os, S);
     return;
   }
-  unsigned* hist = reinterpret_cast<unsigned*>(un);
-  unsigned long long* cands = reinterpret_cast<unsigned long long*>(un + kBins0 * 4);
+  unsigned* hist = reinterpret_cast<unsigned*>(un + kUnHist);
+  unsigned long long* cands = reinterpret_cast<unsigned long long*>(un + kUnCand);
+  unsigned short* owner = reinterpret_cast<unsigned short*>(un + kUnAux);
   auto own_key = [&](int i) { return comp_key(sc[i], lo + i); };
   uint64_t P = 0;
   int nb = 0;
@@ -706,7 +713,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       S.poff[threadIdx.x] = off;
       S.pcnt[threadIdx.x] = np;
       if (total <= (unsigned)kCandMax)  // owner table: compact index -> proposing CTA
-        for (unsigned m = 0; m < np; ++m) S.owner[off + m] = (unsigned short)threadIdx.x;
+        for (unsigned m = 0; m < np; ++m) owner[off + m] = (unsigned short)threadIdx.x;
     }
     __syncthreads();
     if (total >= (unsigned)keff && total <= (unsigned)kCandMax) {
@@ -717,7 +724,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
         for (int uu = 0; uu < 8; ++uu) {
           const unsigned c = b0 + uu * kIdxThreads;
           if (c < total) {
-            const int o = S.owner[c];
+            const int o = owner[c];
             v[uu] = __ldcg(ws->cand + (size_t)o * cap + (c - S.poff[o]));
           }
         }
@@ -728,6 +735,10 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
         }
       }
       __syncthreads();
+      // Every read of the group's shared state by this CTA is complete: announce it now
+      // (the result is only needed at the very end, so the round trip overlaps the work below).
+      unsigned done_prev = 0;
+      if (threadIdx.x == 0) done_prev = atomicAdd(&ws->done, 1u);
       // -- exact k-th best proposal: linear histogram, then rank inside the threshold bin
       const float qscl = qmx > qmn ? (float)kBins0 / (qmx - qmn) : 0.f;
       for (unsigned i = threadIdx.x; i < total; i += kIdxThreads)
@@ -735,12 +746,13 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       __syncthreads();
       const Crossing x = find_crossing(hist, kBins0, (unsigned)keff, S.red, &S.cross);
       const unsigned rr = (unsigned)keff - x.above;  // rank wanted inside bin x.bin (1-based)
-      const bool bin_fits = x.cnt <= (unsigned)kCandMax - total;
+      const bool bin_fits = x.cnt <= (unsigned)kAuxKeys;
       // collect the threshold bin's keys
       if (threadIdx.x == 0) S.ubuf[1] = 0u;
       __syncthreads();
-      unsigned long long* bin_keys = cands + total;  // scratch after the proposals
-      const unsigned bin_cap = (unsigned)kCandMax - total;
+      // the owner table is no longer needed: its area holds the threshold bin's keys
+      unsigned long long* bin_keys = reinterpret_cast<unsigned long long*>(un + kUnAux);
+      const unsigned bin_cap = (unsigned)kAuxKeys;
       for (unsigned i = threadIdx.x; i < total; i += kIdxThreads)
         if (lin_bin4k(key_score(cands[i]), qmn, qscl) == x.bin) {
           const unsigned sl = atomicAdd(&S.ubuf[1], 1u);
@@ -791,9 +803,17 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
         const unsigned base = tot & 0xFFFFu;
         // emit keys >= T*: the rule "top 64 bits >= T*"
         emit(sc, len, lo, false, Tstar, 64, base, keff, oi, os, S);
-        group_cleanup(ws, G, false, 0, S);
+        if (threadIdx.x == 0 && done_prev == (unsigned)(G - 1)) {
+          // the last CTA to announce: every CTA of the group is past the barrier and done
+          // reading, so the synchronisation state can return to zero
+          ws->bar_count = 0u;
+          ws->done = 0u;
+        }
         return;
       }
+      // rejected (uniformly across the group): withdraw the announcement; the exact path
+      // below announces again at its own end
+      if (threadIdx.x == 0) atomicSub(&ws->done, 1u);
     }
     // fall through: the next group barrier orders every read of the proposals before the
     // candidate slots are reused
@@ -931,7 +951,9 @@ __device__ __forceinline__ int64_t visible_of(const IdxParams& p, int t, int64_t
 }
 
 template <int SRC, int KS, int NTILE>
-__global__ void __launch_bounds__(kIdxThreads, 1) lindex_topk_kernel(IdxParams p) {
+// At most 88 registers per thread: 544 x 88 leaves room on the SM's register file for a
+// 128-thread attention CTA to run beside the indexer in a decode step.
+__global__ void __maxnreg__(88) lindex_topk_kernel(IdxParams p) {
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ IdxShared S;
   uint8_t* un = dsm;                                              // ring / histogram / candidates
@@ -1067,7 +1089,9 @@ static cudaError_t launch_one(const IdxParams& p, int grid, bool coop, size_t sm
 template <int SRC, int KS, int NTILE>
 static cudaError_t run_topk(IdxParams p, int T, cudaStream_t stream) {
   const DevInfo d = dev_info();
-  const int P = d.sms;
+  // Two SMs stay out of the cooperative grid, so the small compression kernels that run
+  // beside the indexer in a decode step do not hold up its (all-CTAs-resident) launch.
+  const int P = d.sms > 8 ? d.sms - 2 : d.sms;
   const int Di = SRC == kSrcFp8 ? KS * 32 : 64;
   int64_t seg_cap = 0;
   const int Tb = split_queries_per_launch(T, p.max_entries, Di, P, &seg_cap);
