@@ -6,8 +6,14 @@ A step = every row of the hot path on one batch of synthetic input: CSA
 compression of the entries the new tokens complete, the Lightning Indexer
 scan + exact top-k, CSA attention (top-k + window + sink), HCA compression,
 HCA dense attention (+ window + sink), split merges.  Inputs are resident in
-HBM; the step is replayed from a CUDA graph; L2 is flushed (a 256 MiB write)
-before every timed step, outside its events.  Prints one JSON line on rank 0.
+HBM; the step is replayed from a CUDA graph.  Prints one JSON line on rank 0.
+
+L2 discipline (--l2): "rotate" (default) keeps R device replicas of the whole
+workload, each with its own captured graph, and replays them round-robin, R
+chosen so that the other replicas' step bytes exceed three L2 capacities: every
+step reads inputs that are not in L2, and L2 holds what a real model leaves
+there (mostly clean lines).  "flush" instead writes a 256 MiB buffer before
+every timed step, outside its events, which leaves L2 full of dirty lines.
 
 --impl reference times the CPU oracle (plain fp64 numpy) on the machine's host
 cores on a bounded sample of the same workload.
@@ -18,9 +24,11 @@ workload (weak scaling); the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -39,6 +47,8 @@ METRIC = "hybrid decode attention query-tokens/s at 1M ctx"
 UNIT = "query-tokens/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
+INDEXER_PROFILE = os.path.join(ROOT, "profiles", "lindex_topk_b1_ctx1m.md")
+INDEXER_SOURCES = ("indexer.cu", "sm100.cuh", "common.cuh", "launch.cuh")
 
 
 def peaks():
@@ -48,6 +58,32 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def indexer_digest() -> str:
+    """Digest of the sources the indexer kernel is compiled from."""
+    h = hashlib.sha256()
+    for f in INDEXER_SOURCES:
+        with open(os.path.join(ROOT, "compressed_sparse_kv_compress_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes (read + write) per indexer launch from the committed ncu summary, when it
+    was taken on this workload and the kernel's sources are unchanged since; else None."""
+    if workload != "b1_ctx1m":
+        return None
+    try:
+        with open(INDEXER_PROFILE) as f:
+            text = f.read()
+    except OSError:
+        return None
+    dg = re.search(r"source digest: (\w+)", text)
+    tb = re.search(r"dram bytes per launch \(read \+ write\): (\d+)", text)
+    if not dg or not tb or dg.group(1) != indexer_digest():
+        return None
+    return int(tb.group(1))
 
 
 # ---------------------------------------------------------------------- byte model
@@ -142,8 +178,8 @@ def oracle_sample(w: Workload, budget_s: float = 12.0, max_queries: int = 64):
     dt = {"kv": w.spec.dtype, "idx": w.spec.idx_dtype}
     t0 = time.perf_counter()
     done = 0
-    for t in range(min(w.meta["T"], max_queries)):
-        ostep.run_step(w.meta, a, dt, queries=[t])
+    for j in range(max_queries):  # cycles over the workload's queries until the budget is spent
+        ostep.run_step(w.meta, a, dt, queries=[j % w.meta["T"]])
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
@@ -180,6 +216,12 @@ def reduce_max(x: float, ws: int) -> float:
     return float(t.item())
 
 
+def whole_job_rate(units_per_rank: int, ws: int, ms_max: float) -> float:
+    """Units all ranks processed per second, over the slowest rank's time (weak scaling:
+    every rank runs its own replica of the workload)."""
+    return units_per_rank * ws / (ms_max / 1e3)
+
+
 def barrier(ws: int):
     if ws > 1:
         import torch.distributed as dist
@@ -213,6 +255,17 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def replica_count(args, dev: dict, step_total: int) -> int:
+    """Replicas for the rotate discipline: the other R-1 replicas move >= 3 L2 capacities."""
+    if args.l2 != "rotate":
+        return 1
+    l2 = getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "L2_cache_size", 0) or (126 << 20)
+    per = sum(v.numel() * v.element_size() for v in dev.values() if torch.is_tensor(v))
+    r = math.ceil(3 * l2 / max(step_total, 1)) + 1
+    r = min(r, max(2, (40 << 30) // max(per, 1)))  # at most ~40 GB of replicas
+    return max(2, r)
+
+
 def run_cskv(args, ws, rank, local):
     from compressed_sparse_kv_compress_b200 import _lib, api
     from compressed_sparse_kv_compress_b200.step import DecodeStep
@@ -222,137 +275,169 @@ def run_cskv(args, ws, rank, local):
     spec = spec.replace(seed=spec.seed + rank)
     w = Workload(spec)
     m = w.meta
-    dev = w.device("cuda")
+    by = step_bytes(w)
+    dev0 = w.device("cuda")
+    R = replica_count(args, dev0, by["total"])
+    devs = [dev0] + [{k: (v.clone() if torch.is_tensor(v) else v) for k, v in dev0.items()} for _ in range(R - 1)]
     bd = dict(max_csa_blocks=max(m["csa_num"]), max_hca_blocks=max(m["hca_num"]),
               max_csa_visible=max((p + 1) // 4 for p in m["q_pos"]),
               max_hca_visible=max((p + 1) // 128 for p in m["q_pos"]))
-    step = DecodeStep(dev, k=m["k"], window=m["W"], scale=m["scale"], two_streams=not args.one_stream, **bd)
-    if spec.cache == "compress":
-        step.bulk_compress(max(m["ncsa"]), max(m["nhca"]))
-    torch.cuda.synchronize()
-    n0 = lib.cskv_launch_count()
-    step.capture()
-    launches_per_step = (lib.cskv_launch_count() - n0) // 2  # capture() runs the step once eagerly, once captured
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    steps = []
+    for dev in devs:
+        st = DecodeStep(dev, k=m["k"], window=m["W"], scale=m["scale"], two_streams=not args.one_stream, **bd)
+        if spec.cache == "compress":
+            st.bulk_compress(max(m["ncsa"]), max(m["nhca"]))
+        torch.cuda.synchronize()
+        n1 = lib.cskv_launch_count()
+        st.capture()
+        launches_per_step = (lib.cskv_launch_count() - n1) // 2  # capture() runs the step eagerly, then captures
+        steps.append(st)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if args.l2 == "flush" else None
     stream = torch.cuda.current_stream()
 
-    for i in range(args.warmup):
-        flush.fill_(i & 0xFF)
-        step.replay()
-    torch.cuda.synchronize()
-    if int(step.status.item()) != 0:
-        raise RuntimeError(f"device status {int(step.status.item())} during warm-up")
+    def pre(i):  # what runs before step i, outside its timing
+        if flush is not None:
+            flush.fill_(i & 0xFF)
 
-    # ---- timed region: K graph replays, each after an L2 flush outside its events
+    def timed(body, K):
+        """Device ms per step of body(i), i < K: one event pair around all K (rotate), or
+        one pair per step after an L2 flush outside it (flush)."""
+        torch.cuda.synchronize()
+        if flush is None:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(K):
+                body(i)
+            b.record(stream)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / K
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(K):
+            pre(i)
+            evs[i][0].record(stream)
+            body(i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(x.elapsed_time(y) for x, y in evs)
+
+    for i in range(max(args.warmup, R)):  # every replica's graph runs at least once before timing
+        pre(i)
+        steps[i % R].replay()
+    torch.cuda.synchronize()
+    for st in steps:
+        if int(st.status.item()) != 0:
+            raise RuntimeError(f"device status {int(st.status.item())} during warm-up")
+
+    # ---- timed region: K graph replays (replica i mod R)
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     time.sleep(0.3)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier(ws)
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.fill_((i + 1) & 0xFF)
-        evs[i][0].record(stream)
-        step.replay()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
+    ms_local = timed(lambda i: steps[i % R].replay(), args.steps)
     barrier(ws)
-    ms_steps = [a.elapsed_time(b) for a, b in evs]
-    ms_local = statistics.mean(ms_steps)
 
-    # ---- dominant kernel alone (indexer scan + top-k), same stream, same flush discipline
-    t = step.t
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.fill_((i + 7) & 0xFF)
-        kev[i][0].record(stream)
-        api.lindex_score_topk(t["q_idx"], t["k_idx"], t["q_seq"], t["q_pos"], t["csa_off"], step.idx, step.ws_idx,
-                              max_entries=step.max_csa_visible, q_scale=t.get("q_scale"), k_scale=t.get("k_scale"),
-                              head_w=t.get("head_w"), out_score=step.score, dev_status=step.status)
-        kev[i][1].record(stream)
-    torch.cuda.synchronize()
+    # ---- dominant kernel alone (indexer scan + top-k), same stream, same L2 discipline
+    kev = []
+
+    def one_indexer(i):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        steps[i % R].csa_select(stream)
+        b.record(stream)
+        kev.append((a, b))
+
+    timed(one_indexer, args.steps)
     idx_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in kev)
 
-    # ---- end to end through the public API with host buffers
-    pairs = []  # (pinned host tensor, device destination view)
+    # ---- end to end through the public API with host buffers: per step, the step's new
+    #      inputs go host -> device from pinned memory and both outputs come back
+    def host_pairs(st):
+        t = st.t
+        pairs = []  # (pinned host tensor, device destination view)
 
-    def add(dst):
-        h = torch.empty(dst.shape, dtype=dst.dtype, pin_memory=True)
-        h.copy_(dst.cpu())
-        pairs.append((h, dst))
+        def add(dst):
+            h = torch.empty(dst.shape, dtype=dst.dtype, pin_memory=True)
+            h.copy_(dst.cpu())
+            pairs.append((h, dst))
 
-    for name in ("q_c", "q_h", "q_idx", "q_scale"):
-        if t.get(name) is not None:
-            add(t[name])
-    for b in range(m["B"]):  # the newest token's rows of every per-token array
-        for name, off in (("x_a", "csa_x_off"), ("z_a", "csa_x_off"), ("x_b", "csa_x_off"), ("z_b", "csa_x_off"),
-                          ("x_h", "hca_x_off"), ("z_h", "hca_x_off"), ("raw_c", "raw_off"), ("raw_h", "raw_off")):
-            r = m[off][b + 1] - 1
-            add(t[name][r:r + 1])
-        e = m["ncsa"][b] - 1 + m["csa_off"][b]  # the indexer key of the newest entry
-        add(t["k_idx"][e:e + 1])
-        if t.get("k_scale") is not None:
-            add(t["k_scale"][e:e + 1])
-    outs = [(step.o_c, torch.empty(step.o_c.shape, dtype=step.o_c.dtype, pin_memory=True)),
-            (step.o_h, torch.empty(step.o_h.shape, dtype=step.o_h.dtype, pin_memory=True))]
-    h2d = sum(h.numel() * h.element_size() for h, _ in pairs)
-    d2h = sum(h.numel() * h.element_size() for _, h in outs)
-    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.fill_((i + 3) & 0xFF)
-        eev[i][0].record(stream)
+        for name in ("q_c", "q_h", "q_idx", "q_scale"):
+            if t.get(name) is not None:
+                add(t[name])
+        for b in range(m["B"]):  # the newest token's rows of every per-token array
+            for name, off in (("x_a", "csa_x_off"), ("z_a", "csa_x_off"), ("x_b", "csa_x_off"),
+                              ("z_b", "csa_x_off"), ("x_h", "hca_x_off"), ("z_h", "hca_x_off"),
+                              ("raw_c", "raw_off"), ("raw_h", "raw_off")):
+                r = m[off][b + 1] - 1
+                add(t[name][r:r + 1])
+            e = m["ncsa"][b] - 1 + m["csa_off"][b]  # the indexer key of the newest entry
+            add(t["k_idx"][e:e + 1])
+            if t.get("k_scale") is not None:
+                add(t["k_scale"][e:e + 1])
+        outs = [(st.o_c, torch.empty(st.o_c.shape, dtype=st.o_c.dtype, pin_memory=True)),
+                (st.o_h, torch.empty(st.o_h.shape, dtype=st.o_h.dtype, pin_memory=True))]
+        return pairs, outs
+
+    io = [host_pairs(st) for st in steps]
+    h2d = sum(h.numel() * h.element_size() for h, _ in io[0][0])
+    d2h = sum(h.numel() * h.element_size() for _, h in io[0][1])
+
+    def e2e_step(i):
+        pairs, outs = io[i % R]
         for h, d in pairs:
             d.copy_(h, non_blocking=True)
-        step.replay()
+        steps[i % R].replay()
         for d, h in outs:
             h.copy_(d, non_blocking=True)
-        eev[i][1].record(stream)
-    torch.cuda.synchronize()
-    ms_e2e = statistics.mean(a.elapsed_time(b) for a, b in eev)
+
+    ms_e2e = timed(e2e_step, args.steps)
     clk = clocks.stop()
 
     ms = reduce_max(ms_local, ws)
     ms_e2e = reduce_max(ms_e2e, ws)
     T = m["T"]
-    value = T * ws / (ms / 1e3)
-    by = step_bytes(w)
+    value = whole_job_rate(T, ws, ms)
     hbm, hbm_src = peaks()
     achieved = by["indexer"] / (idx_us * 1e-6) / 1e9
+    if flush is not None:
+        l2 = "flushed (256 MiB write) before every timed step, outside its events"
+    else:
+        l2 = (f"inputs larger than L2: {R} device replicas replayed round-robin "
+              f"({R - 1} x {by['total'] / 1e6:.1f} MB of step reads between two reads of a replica)")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if
         spec.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": args.workload, "batch": m["B"], "context": max(m["n"]), "query_tokens_per_step": T,
                    "heads": m["H"], "topk": m["k"], "window": m["W"], "indexer": f"{m['Hi']}x{m['di']} "
-                   f"{spec.idx_dtype}", "l2": "flushed (256 MiB write) before every timed step",
-                   "replay": "cuda graph", "streams": 1 if args.one_stream else 2},
+                   f"{spec.idx_dtype}", "l2": l2, "replay": "cuda graph", "streams": 1 if args.one_stream else 3},
         "step_hbm_bytes": by["total"], "step_gbs": by["total"] / (ms * 1e-3) / 1e9,
         "step_frac_of_measured_hbm": by["total"] / (ms * 1e-3) / 1e9 / hbm,
         "roofline": {"kernel": "lindex_topk_kernel (indexer scan + top-k)", "bound": "hbm", "achieved": achieved,
                      "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "peak_source": hbm_src,
-                     "bytes_per_launch": by["indexer"], "us_per_launch": idx_us, "traffic": None},
-        "e2e": {"value": T * ws / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                     "bytes_per_launch": by["indexer"], "us_per_launch": idx_us,
+                     "traffic": profiled_traffic(args.workload)},
+        "e2e": {"value": whole_job_rate(T, ws, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches_per_step) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_sample(w, budget_s=args.ref_budget, max_queries=4)
+        line["cpu_baseline"] = oracle_sample(w, budget_s=args.ref_budget, max_queries=10000)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del step
+    del steps
     torch.cuda.synchronize()
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="b1_ctx1m")
     ap.add_argument("--impl", default="cskv", choices=["cskv", "reference"])
     ap.add_argument("--one-stream", action="store_true")
+    ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=12.0)
     args = ap.parse_args()
