@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) 
   float* l_run = m_run + HP;                     // [HP]
   float* alpha = l_run + HP;                     // [HP]
   __shared__ int valid[kAttnTile];
+  pdl_launch_dependents();
+  pdl_wait();
 
   const int t = blockIdx.y, split = blockIdx.x, tid = threadIdx.x;
   const QueryRows q = query_rows(p, t);
@@ -158,11 +160,11 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) 
 // Merge the splits of each query ([TR] §3.1), the sink once ([SW] §十二):
 //   M = max(max_s m_s, sink), L = sum_s 2^{m_s - M} l_s + 2^{sink - M},
 //   o = sum_s 2^{m_s - M} acc_s / L,   lse = ln 2 * (M + log2 L).
-// CTA (block of kCombineDims output dimensions, query); thread (head h, split group g):
-// group g folds splits g, g + kCombineGroups, ... with a running (M, L, o) -- rescaling when a
-// split's max exceeds the running one, as the online softmax does -- so its loads stream
-// without a separate max pass; the groups are then merged through shared memory.
-constexpr int kCombineDims = 4;
+// CTA (block of kCombineDims output dimensions, query); thread (head h, split group g), group g
+// taking splits g, g + kCombineGroups, ...  Two passes with independent loads (so many are in
+// flight at once): the max over the splits' m, merged across groups in shared memory, then the
+// weighted sums of l and acc under that common max, summed across groups.
+constexpr int kCombineDims = 2;
 constexpr int kCombineGroups = 4;
 
 __global__ void __launch_bounds__(128 * kCombineGroups) attn_combine_kernel(AttnParams p) {
@@ -170,71 +172,78 @@ __global__ void __launch_bounds__(128 * kCombineGroups) attn_combine_kernel(Attn
   const int t = blockIdx.y, j0 = blockIdx.x * kCombineDims;
   const int h = threadIdx.x & 127, g = threadIdx.x >> 7;
   const int H = p.H;
+  pdl_launch_dependents();
+  pdl_wait();
   const QueryRows q = query_rows(p, t);
   int S = q.s < 0 ? 0 : (int)((q.n_rows + p.rows_per_split - 1) / p.rows_per_split);
   if (S > p.max_splits) {
     if (threadIdx.x == 0 && j0 == 0) flag(p.st, CSKV_DEV_CAPACITY);
     S = p.max_splits;
   }
-  float M = -INFINITY, L = 0.f, o[kCombineDims] = {};
+  const size_t sb0 = (size_t)t * p.max_splits;
+  const float* mrow = p.part_ml + sb0 * 2 * H + h;  // m of split s at mrow[s * 2H], l at + H
+  const float* acc = p.part_acc + sb0 * kHeadDim * H + (size_t)j0 * H + h;
+  // ---- pass 1: M = max over all splits of m (log2 units)
+  float M = -INFINITY;
   if (h < H) {
-    const size_t sb0 = (size_t)t * p.max_splits;
-    const float* mrow = p.part_ml + sb0 * 2 * H + h;  // m of split s at mrow[s * 2H], l at + H
-    const float* acc = p.part_acc + sb0 * kHeadDim * H + (size_t)j0 * H + h;
-#pragma unroll 4
+#pragma unroll 8
+    for (int s = g; s < S; s += kCombineGroups) M = fmaxf(M, __ldg(mrow + (size_t)s * 2 * H));
+  }
+  sM[g][h] = M;
+  __syncthreads();
+  M = sM[0][h];
+#pragma unroll
+  for (int gg = 1; gg < kCombineGroups; ++gg) M = fmaxf(M, sM[gg][h]);
+  // ---- pass 2: L = sum_s 2^(m_s - M) l_s, o = sum_s 2^(m_s - M) acc_s
+  float L = 0.f, o[kCombineDims] = {};
+  if (h < H && M != -INFINITY) {
+#pragma unroll 8
     for (int s = g; s < S; s += kCombineGroups) {
       const float ms = __ldg(mrow + (size_t)s * 2 * H);
       const float ls = __ldg(mrow + (size_t)s * 2 * H + H);
       float a[kCombineDims];
 #pragma unroll
       for (int jj = 0; jj < kCombineDims; ++jj) a[jj] = __ldg(acc + (size_t)s * kHeadDim * H + (size_t)jj * H);
-      if (ms == -INFINITY) continue;
-      if (ms > M) {
-        const float r = exp2f(M - ms);  // 0 on the first live split
-        L *= r;
+      if (ms != -INFINITY) {  // a split whose rows were all skipped holds nothing
+        const float f = exp2f(ms - M);
+        L = fmaf(ls, f, L);
 #pragma unroll
-        for (int jj = 0; jj < kCombineDims; ++jj) o[jj] *= r;
-        M = ms;
+        for (int jj = 0; jj < kCombineDims; ++jj) o[jj] = fmaf(a[jj], f, o[jj]);
       }
-      const float f = exp2f(ms - M);
-      L = fmaf(ls, f, L);
-#pragma unroll
-      for (int jj = 0; jj < kCombineDims; ++jj) o[jj] = fmaf(a[jj], f, o[jj]);
     }
   }
-  sM[g][h] = M;
   sL[g][h] = L;
 #pragma unroll
   for (int jj = 0; jj < kCombineDims; ++jj) sO[g][jj][h] = o[jj];
   __syncthreads();
   if (g != 0 || h >= H) return;
-  const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
-  float Mt = sk;
+  float Ls = 0.f, os[kCombineDims] = {};
 #pragma unroll
-  for (int gg = 0; gg < kCombineGroups; ++gg) Mt = fmaxf(Mt, sM[gg][h]);
-  float Lt = 0.f, ot[kCombineDims] = {};
-  if (Mt != -INFINITY) {
-    if (p.sink) Lt = exp2f(sk - Mt);
+  for (int gg = 0; gg < kCombineGroups; ++gg) {
+    Ls += sL[gg][h];
 #pragma unroll
-    for (int gg = 0; gg < kCombineGroups; ++gg) {
-      if (sM[gg][h] == -INFINITY) continue;
-      const float f = exp2f(sM[gg][h] - Mt);
-      Lt = fmaf(sL[gg][h], f, Lt);
-#pragma unroll
-      for (int jj = 0; jj < kCombineDims; ++jj) ot[jj] = fmaf(sO[gg][jj][h], f, ot[jj]);
-    }
+    for (int jj = 0; jj < kCombineDims; ++jj) os[jj] += sO[gg][jj][h];
   }
-  const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+  // ---- the sink joins the denominator once
+  const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+  const float Mt = fmaxf(M, sk);
+  float Lt = 0.f, fp = 0.f;
+  if (Mt != -INFINITY) {
+    fp = M == -INFINITY ? 0.f : exp2f(M - Mt);
+    Lt = Ls * fp + (p.sink ? exp2f(sk - Mt) : 0.f);
+  }
+  const float inv = Lt > 0.f ? fp / Lt : 0.f;
   float* dst = p.out + ((size_t)t * H + h) * kHeadDim + j0;
 #pragma unroll
-  for (int jj = 0; jj < kCombineDims; ++jj) dst[jj] = ot[jj] * inv;
+  for (int jj = 0; jj < kCombineDims; ++jj) dst[jj] = os[jj] * inv;
   if (j0 == 0 && p.lse) p.lse[(size_t)t * H + h] = Lt > 0.f ? (Mt + log2f(Lt)) * 0.69314718055994531f : -INFINITY;
 }
 
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream) {
-  attn_combine_kernel<<<dim3(kHeadDim / kCombineDims, p.T), 128 * kCombineGroups, 0, stream>>>(p);
+  const cudaError_t e = launch_dependent(attn_combine_kernel, dim3(kHeadDim / kCombineDims, p.T),
+                                         dim3(128 * kCombineGroups), 0, stream, p);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 // ------------------------------------------------------------------ host side
@@ -278,9 +287,9 @@ static cudaError_t launch_split(const AttnParams& p, cudaStream_t stream) {
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.max_splits, p.T);
-  kern<<<grid, kAttnThreads, smem, stream>>>(p);
+  e = launch_dependent(kern, grid, dim3(kAttnThreads), smem, stream, p);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t stream) {

@@ -9,13 +9,16 @@
 // real dense contraction: S = Q K^T is [H x rows] x [rows x 128] and O = P V the same size.
 // One CTA (4 warps) takes a split of the query's virtual row list (attn_rows.cuh) in chunks
 // of up to 128 rows:
-//   1. cp.async gathers the chunk's K and V halves (16-byte pieces) into shared memory in
-//      the no-swizzle core-matrix layout (8 rows x 16 bytes per core matrix);
+//   1. cp.async gathers the chunk's K||V rows into shared memory, one whole 512-byte row per
+//      warp instruction, in the 128-byte-swizzle layout (four 16 KiB regions of 128-byte rows:
+//      K dims 0-63, K 64-127, V 0-63, V 64-127; chunk c of row r at chunk c ^ (r & 7), so a
+//      row's 32 pieces land on all 32 banks);
 //   2. one thread issues tcgen05.mma: S[128 x nc] (fp32, TMEM) = Q[128 x 128] K^T (bf16);
 //   3. thread h (TMEM lane h) owns head h's row: masks skipped rows, updates the running
 //      max / sum (log2 units), rescales its O row in TMEM when the max grew, and writes
 //      P = 2^(s - m) as bf16 into shared memory;
 //   4. one thread issues O[128 x 128] (+)= P[128 x nc] V[nc x 128] (V read MN-major).
+// Q, K and P are K-major operands, V is MN-major; all four use the same swizzled layout.
 // The split's (m, l, O) go to the workspace; attn_combine_kernel merges the splits and the
 // sink.  Heads beyond H are zero rows of Q (M is always 128).
 #include "attn_rows.cuh"
@@ -25,14 +28,14 @@ namespace cskv {
 
 constexpr int kTcThreads = 128;
 constexpr int kTcChunk = 128;                      // rows per chunk (MMA N of S, K of PV)
-constexpr uint32_t kTileBytes = 128 * 128 * 2;     // one 128 x 128 bf16 operand tile
-constexpr uint32_t kCoreStride = 128;              // bytes between neighbouring core matrices (rows)
-constexpr uint32_t kColStride = 16 * kCoreStride;  // bytes between neighbouring 16-byte column groups
+constexpr uint32_t kRegion = 128 * 128;             // 128 rows x 128 bytes: one swizzled region
+constexpr uint32_t kTileBytes = 2 * kRegion;        // one 128 x 128 bf16 operand tile
 constexpr size_t kTcSmem = 4 * (size_t)kTileBytes + 1024;
 
-// Byte offset of element group (row r, 16-byte column group c) in a 128-row core-matrix tile.
-__device__ __forceinline__ uint32_t core_off(int r, int c) {
-  return (uint32_t)c * kColStride + (uint32_t)(r >> 3) * kCoreStride + (uint32_t)(r & 7) * 16;
+// Byte offset of 16-byte chunk c of row r (c < 16 for a 256-byte row, < 32 for a 512-byte
+// K||V row) in the 128-byte-swizzle layout.
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+  return (uint32_t)(c >> 3) * kRegion + (uint32_t)r * 128 + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -44,8 +47,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smraw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~(uintptr_t)1023);
   uint8_t* Qs = sm;                   // A of S = Q K^T   [128 heads x 128 d], K-major
-  uint8_t* Ks = sm + kTileBytes;      // B of S           [128 rows x 128 d], K-major
-  uint8_t* Vs = sm + 2 * kTileBytes;  // B of O = P V     [128 rows (K) x 128 d (N)], MN-major
+  uint8_t* KVs = sm + kTileBytes;     // K: B of S [128 rows x 128 d], K-major (regions 0-1);
+                                      // V: B of O = P V [128 rows (K) x 128 d (N)], MN-major (2-3)
   uint8_t* Ps = sm + 3 * kTileBytes;  // A of O = P V     [128 heads x 128 rows], K-major
   __shared__ uint64_t bar_s, bar_o;
   __shared__ uint32_t tmem_base;
@@ -54,19 +57,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   __shared__ uint32_t row_mask[kTcChunk / 32];  // bit r: chunk row r is attended
 
   const int t = blockIdx.y, split = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const QueryRows q = query_rows(p, t);
-  if (q.s < 0) {
-    if (split == 0 && tid == 0) flag(p.st, CSKV_DEV_BAD_INDEX);
-    return;
-  }
-  const int64_t r0 = (int64_t)split * p.rows_per_split;
-  if (r0 >= q.n_rows) return;
-  const int64_t r1 = min(q.n_rows, r0 + p.rows_per_split);
-  const int H = p.H;
-  const __nv_bfloat16* cmp = reinterpret_cast<const __nv_bfloat16*>(p.kv_cmp);
-  const __nv_bfloat16* raw = reinterpret_cast<const __nv_bfloat16*>(p.kv_raw);
-  const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(p.q) + (size_t)t * H * kHeadDim;
-
+  pdl_launch_dependents();
+  // ---- set-up that reads no input overlaps the previous kernel (dependent launch)
   if (warp == 0) {
     tmem_alloc(&tmem_base, 256);  // S: columns 0..127, O: columns 128..255
     tmem_relinquish();
@@ -76,15 +68,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     mbar_init(&bar_o, 1);
     fence_mbar_init();
   }
-  // Q tile: thread h copies head h (zero rows beyond H); the copies complete together with the
-  // first chunk's gather, and the barriers of that chunk publish the TMEM address.
-  for (int c = 0; c < 16; ++c)
-    cp_async16(Qs + core_off(tid, c), tid < H ? (const void*)(qg + (size_t)tid * kHeadDim + 8 * c) : (const void*)qg,
-               tid < H ? 16u : 0u);
+  pdl_wait();
+  const QueryRows q = query_rows(p, t);
+  if (q.s < 0 && split == 0 && tid == 0) flag(p.st, CSKV_DEV_BAD_INDEX);
+  const int64_t r0 = (int64_t)split * p.rows_per_split;
+  // a CTA without rows (bad query, or a split past the query's rows) runs no chunk and
+  // only releases its TMEM at the end
+  const int64_t r1 = q.s < 0 ? r0 : max(r0, min(q.n_rows, r0 + p.rows_per_split));
+  const int H = p.H;
+  const __nv_bfloat16* cmp = reinterpret_cast<const __nv_bfloat16*>(p.kv_cmp);
+  const __nv_bfloat16* raw = reinterpret_cast<const __nv_bfloat16*>(p.kv_raw);
+  const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(p.q) + (size_t)t * H * kHeadDim;
+
+  // Q tile: a warp instruction copies two 256-byte head rows (zero rows beyond H); the copies
+  // complete together with the first chunk's gather, and the barriers of that chunk publish
+  // the TMEM address.
+  if (r0 < r1)
+    for (int it = 0; it < 16; ++it) {
+      const int h = warp * 32 + it * 2 + (lane >> 4), c = lane & 15;
+      cp_async16(Qs + sw_off(h, c), h < H ? (const void*)(qg + (size_t)h * kHeadDim + 8 * c) : (const void*)qg,
+                 h < H ? 16u : 0u);
+    }
   tc_fence_before();
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
-  const uint32_t qs_a = smem_u32(Qs), ks_a = smem_u32(Ks), vs_a = smem_u32(Vs), ps_a = smem_u32(Ps);
+  const uint32_t qs_a = smem_u32(Qs), ks_a = smem_u32(KVs), vs_a = ks_a + 2 * kRegion, ps_a = smem_u32(Ps);
   float m_run = -INFINITY, l_run = 0.f;
   bool alive = true;
   int c = 0;
@@ -102,16 +110,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
       if (lane == 0) row_mask[warp] = bal;
     }
     __syncthreads();
-    // ---- gather K and V halves: per warp instruction 8 rows x 4 column groups, so every
-    //      quarter-warp fills one 128-byte core matrix and reads 64 contiguous bytes per row
-    for (int u = warp; u < (nc / 8) * 8; u += 4) {
-      const int rg = u >> 3, cg = u & 7;
-      const int r = rg * 8 + (lane & 7);
-      const int col = cg * 4 + (lane >> 3);  // 16-byte column group of the 512-byte row, 0..31
+    // ---- gather: one whole 512-byte K||V row per warp instruction (lane j copies its
+    //      16-byte piece j); skipped rows up to nc are zero-filled
+    for (int r = warp; r < nc; r += 4) {
       const int64_t off = row_src[r];
-      const __nv_bfloat16* src = off >= 0 ? (row_raw[r] ? raw : cmp) + off + 8 * col : qg;
-      uint8_t* dst = col < 16 ? Ks + core_off(r, col) : Vs + core_off(r, col - 16);
-      cp_async16(dst, src, off >= 0 ? 16u : 0u);
+      const __nv_bfloat16* src = off >= 0 ? (row_raw[r] ? raw : cmp) + off + 8 * lane : qg;
+      cp_async16(KVs + sw_off(r, lane), src, off >= 0 ? 16u : 0u);
     }
     cp_async_wait_all();
     fence_proxy_async_smem();
@@ -122,54 +126,63 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     // ---- S = Q K^T
     if (tid == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, nc, false, false);
+      // K steps of 16 elements (32 bytes): region kk / 4, offset 32 * (kk % 4) inside the row
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc_mma_f16(tS, smem_desc_noswz(qs_a + 2 * kk * kColStride, kColStride, kCoreStride),
-                   smem_desc_noswz(ks_a + 2 * kk * kColStride, kColStride, kCoreStride), idesc, kk > 0);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t koff = (uint32_t)(kk >> 2) * kRegion + (uint32_t)(kk & 3) * 32;
+        tc_mma_f16(tS, smem_desc_sw128(qs_a + koff, 16, 1024), smem_desc_sw128(ks_a + koff, 16, 1024), idesc,
+                   kk > 0);
+      }
       tc_commit(&bar_s);
     }
     if (!mbar_wait_bounded(&bar_s, c & 1)) flag(p.st, CSKV_DEV_TIMEOUT);
     tc_fence_after();
     // ---- online softmax of row tid over the nc columns (log2 units)
     const float sl2 = p.scale_log2;
-    // pass 1: masked row max over the chunk, four independent max chains per 32 columns
+    // pass 1: row max of the raw logits over the attended columns (the scale is positive, so
+    // it is applied once, to the max); four independent max chains.  Blocks of 32 columns
+    // that are all attended (the common case) skip the mask.
     float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     for (int cc = 0; cc < nc; cc += 32) {
       const uint32_t vm = row_mask[cc >> 5];
       uint32_t v[32];
       tmem_ld32(tS + lane_base + cc, v);
       tmem_ld_wait();
+      if (vm == 0xFFFFFFFFu) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if ((vm >> i) & 1u) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(v[i]) * sl2);
+        for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(v[i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          mx4[i & 3] = fmaxf(mx4[i & 3], ((vm >> i) & 1u) ? __uint_as_float(v[i]) : -INFINITY);
+      }
     }
-    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
     const float m_new = fmaxf(m_run, mx);
     const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
-    const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-    // pass 2: P = 2^(s - m) as bf16 into the P tile; four independent partial sums
+    const float nm = (m_new == -INFINITY) ? 0.f : -m_new;
+    // pass 2: P = 2^(s * scale - m) as bf16 into the P tile; four independent partial sums
     float ls4[4] = {0.f, 0.f, 0.f, 0.f};
     for (int cc = 0; cc < nc; cc += 32) {
       const uint32_t vm = row_mask[cc >> 5];
       uint32_t v[32];
       tmem_ld32(tS + lane_base + cc, v);
       tmem_ld_wait();
+      float pr[32];
+      if (vm == 0xFFFFFFFFu) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t w4[4];
+        for (int i = 0; i < 32; ++i) pr[i] = fast_exp2(fmaf(__uint_as_float(v[i]), sl2, nm));
+      } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float pr[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = g * 8 + i * 2 + e;
-            pr[e] = ((vm >> col) & 1u) ? fast_exp2(__uint_as_float(v[col]) * sl2 - m_use) : 0.f;
-            ls4[col & 3] += pr[e];
-          }
-          w4[i] = pack_bf16(pr[0], pr[1]);
-        }
-        *reinterpret_cast<uint4*>(Ps + core_off(tid, (cc >> 3) + g)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        for (int i = 0; i < 32; ++i) pr[i] = ((vm >> i) & 1u) ? fast_exp2(fmaf(__uint_as_float(v[i]), sl2, nm)) : 0.f;
       }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ls4[i & 3] += pr[i];
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+        *reinterpret_cast<uint4*>(Ps + sw_off(tid, (cc >> 3) + g)) =
+            make_uint4(pack_bf16(pr[8 * g], pr[8 * g + 1]), pack_bf16(pr[8 * g + 2], pr[8 * g + 3]),
+                       pack_bf16(pr[8 * g + 4], pr[8 * g + 5]), pack_bf16(pr[8 * g + 6], pr[8 * g + 7]));
     }
     const float lsum = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
     // O of the previous chunks is complete (its MMA was waited on).  TMEM loads and stores are
@@ -194,13 +207,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
-      // V tile read MN-major: the leading byte offset steps along K (row groups, 128 B apart),
-      // the stride byte offset along N (16-byte d groups, kColStride apart)
-      const uint32_t v_lbo = kCoreStride;
-      const uint32_t v_sbo = kColStride;
-      for (int kk = 0; kk < nc / 16; ++kk)
-        tc_mma_f16(tO, smem_desc_noswz(ps_a + 2 * kk * kColStride, kColStride, kCoreStride),
-                   smem_desc_noswz(vs_a + 2 * kk * kCoreStride, v_lbo, v_sbo), idesc, (c > 0 || kk > 0));
+      // P: K-major like Q.  V read MN-major: 64-dimension blocks one region apart (leading
+      // byte offset), 8-row groups 1024 bytes apart (stride byte offset); a K step of 16 rows
+      // advances 2048 bytes.
+      for (int kk = 0; kk < nc / 16; ++kk) {
+        const uint32_t koff = (uint32_t)(kk >> 2) * kRegion + (uint32_t)(kk & 3) * 32;
+        tc_mma_f16(tO, smem_desc_sw128(ps_a + koff, 16, 1024),
+                   smem_desc_sw128(vs_a + (uint32_t)kk * 2048, kRegion, 1024), idesc, (c > 0 || kk > 0));
+      }
       tc_commit(&bar_o);
     }
     const bool timed_out = !mbar_wait_bounded(&bar_o, c & 1);

@@ -13,6 +13,17 @@ constexpr int kRow = 256;      // packed K||V row width
 constexpr int kHeadDim = 128;  // d
 constexpr float kLog2e = 1.4426950408889634f;
 
+// ---------------------------------------------------------------- dependent launches
+// A kernel launched as a programmatic dependent launch may start while the kernel before it
+// on the stream still runs.  It calls pdl_wait() before its first read of any input (the wait
+// returns once every grid it depends on has completed and its writes are visible; without a
+// programmatic dependency it returns at once) and pdl_launch_dependents() early, so that the
+// next kernel's launch overlaps this one.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- status
 __device__ __forceinline__ void flag(int* st, int bit) {
   if (st) atomicOr(st, bit);

@@ -79,17 +79,19 @@ __device__ __forceinline__ SeqRange seq_range(int b, int ratio, const int64_t* t
 // ------------------------------------------------------------------ CSA
 // grid (ceil(max_blocks / kCsaWarps), batch), 32 * kCsaWarps threads: warp w of CTA x
 // computes entry first + kCsaWarps * x + w of sequence blockIdx.y.  Small CTAs keep the
-// register footprint low enough to run beside the indexer in a decode step.
+// register footprint low enough to run beside the indexer in a decode step (<= 144 registers).
 constexpr int kCsaWarps = 2;
 
 template <typename TI, typename TO, bool kTwo>
-__global__ void __launch_bounds__(32 * kCsaWarps) csa_compress_kernel(
+__global__ void __maxnreg__(144) csa_compress_kernel(
     const TI* __restrict__ xa, const TI* __restrict__ za, const TI* __restrict__ xb,
     const TI* __restrict__ zb, const float* __restrict__ ba, const float* __restrict__ bb,
     const int64_t* __restrict__ tok_off, const int64_t* __restrict__ tok0,
     const int64_t* __restrict__ ent_off, const int64_t* __restrict__ first_block,
     const int64_t* __restrict__ num_blocks, int64_t max_blocks, TO* __restrict__ out, int* st) {
   constexpr int kC = kTwo ? 8 : 4;  // candidates: 4 path-A (+ 4 path-B)
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SeqRange s = seq_range(b, 4, tok_off, tok0, ent_off, first_block, num_blocks);
@@ -149,144 +151,120 @@ __global__ void __launch_bounds__(32 * kCsaWarps) csa_compress_kernel(
 }
 
 // ------------------------------------------------------------------ HCA
-// Raw 4-value slice of a row kept in registers until used (bf16: one uint2).
+// An entry is cut into kHcaSlices slices of 16 dimensions, one CTA (4 warps) per slice:
+// a lane pair covers one token's 16-dimension slice (8 dims per lane, one 16-byte load per
+// array for bf16), a warp 16 tokens, the CTA 64 tokens per round, two rounds -- every load
+// of the CTA is in flight before any arithmetic.  The per-dimension softmax over the 128
+// tokens then takes two reductions (max, then sum and weighted sum): shuffles across the
+// 16 lanes that share dimensions, then shared memory across the 4 warps.  Many small CTAs
+// keep the latency of one entry short and fit beside the indexer's CTAs.
+constexpr int kHcaSlices = 16;
+constexpr int kHcaThreads = 128;
+
 template <typename T>
-struct Raw4;
-
-template <>
-struct Raw4<__nv_bfloat16> {
-  uint2 v;
-  __device__ __forceinline__ void load(const __nv_bfloat16* p) { v = __ldg(reinterpret_cast<const uint2*>(p)); }
-  __device__ __forceinline__ float get(int i) const {
-    const uint32_t w = (i < 2) ? v.x : v.y;
-    return (i & 1) ? __uint_as_float(w & 0xffff0000u) : __uint_as_float(w << 16);
-  }
-};
-
-template <>
-struct Raw4<float> {
-  float4 a;
-  __device__ __forceinline__ void load(const float* p) { a = __ldg(reinterpret_cast<const float4*>(p)); }
-  __device__ __forceinline__ float get(int i) const {
-    switch (i) {
-      case 0: return a.x; case 1: return a.y; case 2: return a.z; default: return a.w;
-    }
-  }
-};
-
-__device__ __forceinline__ void load_bias4(const float* bias, int slot, int j0, float (&b)[4]) {
-  if (bias == nullptr) {
-    b[0] = b[1] = b[2] = b[3] = 0.f;
-    return;
-  }
-  const float4 u = __ldg(reinterpret_cast<const float4*>(bias + (size_t)slot * kRow + j0));
-  b[0] = u.x; b[1] = u.y; b[2] = u.z; b[3] = u.w;
+__device__ __forceinline__ void load8f(const T* p, float (&v)[8]) {
+  Raw8<T> r;
+  r.load(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = r.get(i);
 }
 
-// grid (max_blocks, batch), 256 threads: CTA x computes entry first + x.  Warp w covers
-// dimension half (w & 1) -- lane l owns its dims 4l .. 4l+3 -- and token quarter (w >> 1),
-// 32 tokens streamed eight at a time with a running max; the four quarter partials
-// (max, sum, weighted sum) per dimension are merged through shared memory.  The small
-// per-thread state keeps the CTA within 64 registers, so it fits beside the indexer.
-constexpr int kHcaWarps = 8;
-constexpr int kHcaQuarters = 4;
-
 template <typename TI, typename TO>
-__global__ void __launch_bounds__(32 * kHcaWarps, 4) hca_compress_kernel(
+__global__ void __launch_bounds__(kHcaThreads, 8) hca_compress_kernel(
     const TI* __restrict__ x, const TI* __restrict__ z, const float* __restrict__ bias,
     const int64_t* __restrict__ tok_off, const int64_t* __restrict__ tok0,
     const int64_t* __restrict__ ent_off, const int64_t* __restrict__ first_block,
     const int64_t* __restrict__ num_blocks, int64_t max_blocks, TO* __restrict__ out, int* st) {
-  constexpr int kTokPerQuarter = 128 / kHcaQuarters;  // 32
-  constexpr int kGroup = sizeof(TI) == 2 ? 8 : 4;     // tokens loaded per round
-  __shared__ float sm_m[kHcaQuarters][kRow], sm_s[kHcaQuarters][kRow], sm_a[kHcaQuarters][kRow];
+  __shared__ float sm_max[4][16], sm_sum[4][16], sm_acc[4][16];
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, half = lane & 1;
+  const int slice = (int)(blockIdx.x % kHcaSlices);
+  const int j0 = slice * 16 + half * 8;  // this lane's first dimension
   const SeqRange s = seq_range(b, 128, tok_off, tok0, ent_off, first_block, num_blocks);
   if (blockIdx.x == 0 && threadIdx.x == 0 && s.num > max_blocks) flag(st, CSKV_DEV_CAPACITY);
-  const int64_t local = blockIdx.x;
-  if (local >= s.num) return;
-  const int64_t i = s.first + local;
-  if (i < 0 || 128 * i >= s.n || i >= s.ent_cap) {
-    if (threadIdx.x == 0) flag(st, CSKV_DEV_BAD_INDEX);
-    return;
-  }
-  if (128 * i < s.t0) {
-    if (threadIdx.x == 0) flag(st, CSKV_DEV_TAIL_MISSING);
-    return;
-  }
-  const int quarter = warp >> 1;
-  const int j0 = (warp & 1) * 128 + lane * 4;
-  float m[4], den[4], num[4];
+  const int64_t stride = gridDim.x / kHcaSlices;
+  for (int64_t local = blockIdx.x / kHcaSlices; local < s.num && local < max_blocks; local += stride) {
+    const int64_t i = s.first + local;
+    if (i < 0 || 128 * i >= s.n || i >= s.ent_cap) {
+      if (threadIdx.x == 0) flag(st, CSKV_DEV_BAD_INDEX);
+      continue;  // block-uniform
+    }
+    if (128 * i < s.t0) {
+      if (threadIdx.x == 0) flag(st, CSKV_DEV_TAIL_MISSING);
+      continue;
+    }
+    float lg[2][8], xv[2][8];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) { m[j] = -INFINITY; den[j] = 0.f; num[j] = 0.f; }
-#pragma unroll 1
-  for (int g0 = 0; g0 < kTokPerQuarter; g0 += kGroup) {
-    Raw4<TI> xr[kGroup], zr[kGroup];
-    bool ok[kGroup];
-#pragma unroll
-    for (int u = 0; u < kGroup; ++u) {
-      const int slot = quarter * kTokPerQuarter + g0 + u;
+    for (int r = 0; r < 2; ++r) {
+      const int slot = r * 64 + warp * 16 + (lane >> 1);
       const int64_t t = 128 * i + slot;
-      ok[u] = t < s.n;
-      if (ok[u]) {
+      if (t < s.n) {
         const size_t row = (size_t)(s.row0 + (t - s.t0)) * kRow + j0;
-        xr[u].load(x + row);
-        zr[u].load(z + row);
+        load8f(x + row, xv[r]);
+        load8f(z + row, lg[r]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          xv[r][e] = 0.f;
+          lg[r][e] = -INFINITY;
+        }
       }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float l2[kGroup];
-      float mg = m[j];
+    for (int r = 0; r < 2; ++r) {
+      const int slot = r * 64 + warp * 16 + (lane >> 1);
+      float bb[8];
+      load_bias8(bias, slot, j0, bb);
 #pragma unroll
-      for (int u = 0; u < kGroup; ++u) {
-        const float bb = bias ? __ldg(bias + (size_t)(quarter * kTokPerQuarter + g0 + u) * kRow + j0 + j) : 0.f;
-        l2[u] = ok[u] ? (zr[u].get(j) + bb) * kLog2e : -INFINITY;
-        mg = fmaxf(mg, l2[u]);
+      for (int e = 0; e < 8; ++e) lg[r][e] = (lg[r][e] + bb[e]) * kLog2e;  // -inf stays -inf
+    }
+    // ---- per-dimension max over the 128 tokens
+    float m[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float v = fmaxf(lg[0][e], lg[1][e]);
+#pragma unroll
+      for (int o = 2; o < 32; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+      m[e] = v;
+    }
+    if (lane < 2)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sm_max[warp][half * 8 + e] = m[e];
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      m[e] = fmaxf(fmaxf(sm_max[0][half * 8 + e], sm_max[1][half * 8 + e]),
+                   fmaxf(sm_max[2][half * 8 + e], sm_max[3][half * 8 + e]));
+    // ---- weights, sums and weighted sums (token 128i is present, so every max is finite)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float w0 = exp2f(lg[0][e] - m[e]), w1 = exp2f(lg[1][e] - m[e]);
+      float sw = w0 + w1;
+      float sa = fmaf(w0, xv[0][e], w1 * xv[1][e]);
+#pragma unroll
+      for (int o = 2; o < 32; o <<= 1) {
+        sw += __shfl_xor_sync(0xffffffffu, sw, o);
+        sa += __shfl_xor_sync(0xffffffffu, sa, o);
       }
-      if (mg != -INFINITY) {
-        const float r = exp2f(m[j] - mg);  // rescale of the running sums (0 on the first group)
-        den[j] *= r;
-        num[j] *= r;
-        m[j] = mg;
-#pragma unroll
-        for (int u = 0; u < kGroup; ++u)
-          if (ok[u]) {
-            const float w = exp2f(l2[u] - mg);
-            den[j] += w;
-            num[j] = fmaf(w, xr[u].get(j), num[j]);
-          }
+      if (lane < 2) {
+        sm_sum[warp][half * 8 + e] = sw;
+        sm_acc[warp][half * 8 + e] = sa;
       }
     }
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    sm_m[quarter][j0 + j] = m[j];
-    sm_s[quarter][j0 + j] = den[j];
-    sm_a[quarter][j0 + j] = num[j];
-  }
-  __syncthreads();
-  {
-    const int j = threadIdx.x;  // 256 threads, one per dimension
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kHcaQuarters; ++w) M = fmaxf(M, sm_m[w][j]);
-    float S = 0.f, A = 0.f;
-#pragma unroll
-    for (int w = 0; w < kHcaQuarters; ++w) {
-      const float mw = sm_m[w][j];
-      if (mw != -INFINITY) {
-        const float f = exp2f(mw - M);
-        S = fmaf(sm_s[w][j], f, S);
-        A = fmaf(sm_a[w][j], f, A);
-      }
+    __syncthreads();
+    if (threadIdx.x < 16) {
+      const int j = threadIdx.x;
+      const float S = (sm_sum[0][j] + sm_sum[1][j]) + (sm_sum[2][j] + sm_sum[3][j]);
+      const float A = (sm_acc[0][j] + sm_acc[1][j]) + (sm_acc[2][j] + sm_acc[3][j]);
+      TO* dst = out + (size_t)(s.ent0 + i) * kRow + slice * 16 + j;
+      if constexpr (sizeof(TO) == 2)
+        *dst = __float2bfloat16_rn(A / S);
+      else
+        *dst = A / S;
     }
-    TO* dst = out + (size_t)(s.ent0 + i) * kRow + j;
-    if constexpr (sizeof(TO) == 2)
-      *dst = __float2bfloat16_rn(A / S);
-    else
-      *dst = A / S;
+    __syncthreads();  // the shared arrays are reused by the next entry
   }
 }
 
@@ -298,16 +276,17 @@ static cudaError_t launch_csa_t(const void* xa, const void* za, const void* xb, 
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
                                 void* out, int* st, cudaStream_t stream) {
   dim3 grid((unsigned)((max_blocks + kCsaWarps - 1) / kCsaWarps), (unsigned)batch);
+  cudaError_t e;
   if (xb != nullptr)
-    csa_compress_kernel<TI, TO, true><<<grid, 32 * kCsaWarps, 0, stream>>>(
-        (const TI*)xa, (const TI*)za, (const TI*)xb, (const TI*)zb, ba, bb, tok_off, tok0, ent_off,
-        first, num, max_blocks, (TO*)out, st);
+    e = launch_dependent(csa_compress_kernel<TI, TO, true>, grid, dim3(32 * kCsaWarps), 0, stream, (const TI*)xa,
+                         (const TI*)za, (const TI*)xb, (const TI*)zb, ba, bb, tok_off, tok0, ent_off, first, num,
+                         max_blocks, (TO*)out, st);
   else
-    csa_compress_kernel<TI, TO, false><<<grid, 32 * kCsaWarps, 0, stream>>>(
-        (const TI*)xa, (const TI*)za, nullptr, nullptr, ba, bb, tok_off, tok0, ent_off, first, num,
-        max_blocks, (TO*)out, st);
+    e = launch_dependent(csa_compress_kernel<TI, TO, false>, grid, dim3(32 * kCsaWarps), 0, stream, (const TI*)xa,
+                         (const TI*)za, (const TI*)nullptr, (const TI*)nullptr, ba, bb, tok_off, tok0, ent_off,
+                         first, num, max_blocks, (TO*)out, st);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_csa_compress(const void* xa, const void* za, const void* xb, const void* zb,
@@ -333,11 +312,14 @@ static cudaError_t launch_hca_t(const void* x, const void* z, const float* bias,
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
                                 void* out, int* st, cudaStream_t stream) {
-  dim3 grid((unsigned)max_blocks, (unsigned)batch);
-  hca_compress_kernel<TI, TO><<<grid, 32 * kHcaWarps, 0, stream>>>((const TI*)x, (const TI*)z, bias, tok_off, tok0,
-                                                       ent_off, first, num, max_blocks, (TO*)out, st);
+  // slices of one entry are consecutive CTAs; very large bulk calls loop over entries
+  const int64_t entries = max_blocks < (int64_t)(1 << 26) ? max_blocks : (int64_t)(1 << 26);
+  dim3 grid((unsigned)(entries * kHcaSlices), (unsigned)batch);
+  const cudaError_t e = launch_dependent(hca_compress_kernel<TI, TO>, grid, dim3(kHcaThreads), 0, stream,
+                                         (const TI*)x, (const TI*)z, bias, tok_off, tok0, ent_off, first, num,
+                                         max_blocks, (TO*)out, st);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_hca_compress(const void* x, const void* z, const float* bias, const int64_t* tok_off,

@@ -27,8 +27,8 @@
 //  shared memory; otherwise further 10-bit global passes run (rare: massive ties).
 //  Output positions come from per-CTA counts, so the result needs no sort.
 //
-// Scan of E4M3 keys: a producer warp streams 128-entry tiles (8 KiB) of k_idx into a
-// shared-memory ring with TMA bulk copies; eight consumer warps each take 16 entries of
+// Scan of E4M3 keys: a producer warp streams 240-entry tiles (15 KiB at Di = 64) of k_idx into a
+// shared-memory ring with TMA bulk copies; fifteen consumer warps each take 16 entries of
 // a tile and run m16n8k32 E4M3 MMAs (entries x dims) x (dims x 8 heads) with fp32
 // accumulation -- the head dimension fills N = 8 exactly -- then apply scales, ReLU and
 // the head sum in registers.
@@ -37,7 +37,10 @@
 
 namespace cskv {
 
-constexpr int kIdxConsumerWarps = 16;
+// 15 MMA warps + 1 TMA warp = 16 warps, 4 per SM sub-partition: with at most 88 registers a
+// thread the indexer leaves 5120 registers on every sub-partition, so a 4-warp attention
+// CTA (<= 160 registers) or compression CTAs fit beside it on the same SM.
+constexpr int kIdxConsumerWarps = 15;
 constexpr int kIdxThreads = 32 * (kIdxConsumerWarps + 1);  // + one producer warp
 constexpr int kIdxTile = 16 * kIdxConsumerWarps;          // entries per ring stage
 constexpr int kBins0 = 4096;                              // first digit: 12 bits
@@ -52,15 +55,17 @@ constexpr int kIdxMaxDim = 128;
 
 enum IdxSrc { kSrcFp8 = 0, kSrcF32 = 1, kSrcScores = 2 };
 
+constexpr int kWarpTop = 6;   // candidates per consumer warp in the warp form of the proposals
+constexpr int kWarpKeys = 8;  // entries per lane in the warp form: warp slices up to 256 entries
+constexpr int kLaneTop = 3;   // best keys each lane keeps for the warp form
+
 struct alignas(16) QueryWS {
-  unsigned bar_count, bar_gen, done, cand_count;
+  unsigned bar_count, spare, done, cand_count;  // bar_count: group barrier (phase bit + arrivals)
   unsigned hist0[kBins0];
   unsigned histp[kMaxPasses - 1][kBinsP];
   unsigned above[kMaxGroup];
-  unsigned prop[kMaxGroup];            // speculative path: proposals of each CTA
   unsigned long long unp[kMaxGroup];   // speculative path: best key each CTA did not propose
-  float plo[kMaxGroup], phi[kMaxGroup];  // speculative path: score range of each CTA's proposals
-  unsigned long long cand[kCandMax];
+  unsigned long long cand[kCandMax];   // speculative path: `cap` proposal slots per CTA
 };
 
 
@@ -99,6 +104,14 @@ __device__ __forceinline__ float key_score(uint64_t c) {
 }
 __device__ __forceinline__ bool key_selected(uint64_t c, uint64_t P, int nb) {
   return (c >> (64 - nb)) >= P;
+}
+// Largest 64-bit key of the warp: the largest high half, then the largest low half among the
+// lanes that hold it.
+__device__ __forceinline__ uint64_t warp_max_key(uint64_t k) {
+  const unsigned hi = (unsigned)(k >> 32), lo = (unsigned)k;
+  const unsigned mh = __reduce_max_sync(0xffffffffu, hi);
+  const unsigned ml = __reduce_max_sync(0xffffffffu, hi == mh ? lo : 0u);
+  return ((uint64_t)mh << 32) | ml;
 }
 
 // ------------------------------------------------------------------ block helpers
@@ -201,26 +214,29 @@ __device__ Crossing find_crossing(const unsigned* hist, int nbins, unsigned r, u
   return *out;
 }
 
-// Barrier over the G CTAs of one query group (all co-resident: cooperative launch).  The
-// arrival counter only grows during a call: arrival number a belongs to the barrier that
-// completes when the counter reaches the next multiple of G.  Thread 0 publishes the CTA's
-// prior writes with a release fence (cumulative over the block barrier before it) and
-// acquires the others' after the wait.  Bounded: gives up after ~1 s (CSKV_DEV_TIMEOUT).
-__device__ bool group_barrier(QueryWS* ws, unsigned G, int* st, int* sm_flag) {
+// Barrier over the G CTAs of one query group (all co-resident: cooperative launch), on one
+// counter whose top bit is the barrier's phase.  Thread 0 reads the counter (the phase cannot
+// change before this CTA arrives), publishes the CTA's writes with a fence (cumulative over
+// the block barrier before it) and arrives with a reduction that needs no reply: CTA 0 of the
+// group adds 2^31 - (G - 1), every other CTA adds 1, so the sum of the G arrivals is exactly
+// 2^31 -- the phase bit flips when the last one lands and the low bits are back where they
+// were (zero), for any G, with no reset.  Waiters poll until the phase differs.  Bounded:
+// gives up after a few million polls, about a second (CSKV_DEV_TIMEOUT).
+__device__ bool group_barrier(QueryWS* ws, unsigned G, int j, int* st, int* sm_flag) {
   __syncthreads();
   if (threadIdx.x == 0) {
     bool ok = true;
+    const unsigned before = ld_acquire_gpu(&ws->bar_count);
+    const unsigned add = j == 0 ? 0x80000000u - (G - 1u) : 1u;
     __threadfence();
-    const unsigned arrived = atomicAdd(&ws->bar_count, 1u) + 1u;
-    const unsigned target = (arrived + G - 1) / G * G;
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(&ws->bar_count), "r"(add) : "memory");
     long it = 0;
-    while (ld_acquire_gpu(&ws->bar_count) < target) {
-      if (++it > (1L << 24)) {
+    while (((ld_acquire_gpu(&ws->bar_count) ^ before) & 0x80000000u) == 0u) {  // an L2 round trip each
+      if (++it > (1L << 22)) {
         ok = false;
         flag(st, CSKV_DEV_TIMEOUT);
         break;
       }
-      __nanosleep(32);
     }
     *sm_flag = ok ? 1 : 0;
   }
@@ -235,10 +251,12 @@ struct IdxShared {
   unsigned red[32];
   float fred[64];
   unsigned long long ured[32];
-  float pmin[kIdxThreads], pmax[kIdxThreads];
   unsigned long long tstar;
-  unsigned poff[kIdxThreads];
-  unsigned pcnt[kIdxThreads];
+  unsigned long long wcand[kIdxConsumerWarps * kWarpTop];  // warp proposals: each warp's best
+  unsigned long long wunp[kIdxConsumerWarps];  // warp proposals: best key after each warp's top
+  unsigned long long cunp;                     // warp proposals: best candidate past `cap`
+  int wcnt[kIdxConsumerWarps];                 // warp proposals: keys found by each warp
+  int fcnt[32];
   Crossing cross;
   int flag;
   unsigned ubuf[4];
@@ -249,7 +267,7 @@ struct IdxShared {
 // ------------------------------------------------------------------ scan: E4M3 via TMA + MMA
 template <int KS, int NTILE>
 __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, int len,
-                         float* sc, float* ssk, uint8_t* ring, IdxShared& S) {
+                         float* sc, uint8_t* ring, IdxShared& S) {
   constexpr int Di = KS * 32;
   constexpr int stages = idx_stages(Di);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -347,14 +365,21 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
         ska[kScalePF - 1] = e < len ? (kscale ? __ldg(kscale + e) : 1.f) : 0.f;
         skb[kScalePF - 1] = e + 8 < len ? (kscale ? __ldg(kscale + e + 8) : 1.f) : 0.f;
       }
+      // A fragments of this warp's 16 rows into registers, then the stage goes back to the
+      // producer at once (the arrive orders the loads before the next copy into the stage),
+      // so the refill overlaps the MMAs and the epilogue
+      uint4 ra[KS / 2], rb[KS / 2];
       if (r0 < rows) {
         const uint8_t* tile = ring + (size_t)s * kIdxTile * Di;
-        uint4 ra[KS / 2], rb[KS / 2];
 #pragma unroll
         for (int c = 0; c < KS / 2; ++c) {
           ra[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g) * Di + (tq + 4 * c) * 16);
           rb[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g + 8) * Di + (tq + 4 * c) * 16);
         }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[s]);
+      if (r0 < rows) {
         float acc[NTILE][4];
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt) {
@@ -384,8 +409,6 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
         if (tq == 0 && e_g < len) sc[e_g] = vg;
         if (tq == 1 && e_g8 < len) sc[e_g8] = vg8;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.empty[s]);
       if (++s == stages) {
         s = 0;
         ph ^= 1u;
@@ -511,8 +534,9 @@ __device__ unsigned count_selected(const float* sc, int len, int64_t lo, uint64_
 // ---- speculative exchange helpers
 constexpr int kLinBins = 1024;  // linear score bins (<= kBins0, shares the histogram buffer)
 
-// Block-wide min and max of one float per thread.
-__device__ void block_minmax(float mn, float mx, IdxShared& S, float& gmn, float& gmx) {
+// Block-wide min and max of one float per thread, and the sum of one count per thread.
+__device__ void block_minmax(float mn, float mx, IdxShared& S, float& gmn, float& gmx, int cnt = 0,
+                             int* gcnt = nullptr) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int nw = kIdxThreads / 32;
 #pragma unroll
@@ -520,19 +544,25 @@ __device__ void block_minmax(float mn, float mx, IdxShared& S, float& gmn, float
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
   if (lane == 0) {
     S.fred[warp] = mn;
     S.fred[32 + warp] = mx;
+    S.fcnt[warp] = cnt;
   }
   __syncthreads();
   gmn = INFINITY;
   gmx = -INFINITY;
+  int c = 0;
   for (int w = 0; w < nw; ++w) {
     gmn = fminf(gmn, S.fred[w]);
     gmx = fmaxf(gmx, S.fred[32 + w]);
+    c += S.fcnt[w];
   }
+  if (gcnt) *gcnt = c;
   __syncthreads();
 }
+
 
 // Block-wide max of one 64-bit key per thread.
 __device__ uint64_t block_max_u64(uint64_t v, IdxShared& S) {
@@ -580,14 +610,144 @@ __device__ void group_cleanup(QueryWS* ws, int G, bool used_hist0, int used_pass
     for (int q = 0; q < used_passes; ++q)
       for (int i = threadIdx.x; i < kBinsP; i += kIdxThreads) ws->histp[q][i] = 0u;
     if (threadIdx.x == 0) {
-      // every CTA of the group is past its last barrier
-      ws->bar_count = 0u;
-      ws->bar_gen = 0u;
+      // every CTA of the group is past its last use of these
       ws->cand_count = 0u;
       ws->done = 0u;
     }
   }
   __syncthreads();
+}
+
+// ---- speculative proposals.  Both forms fill this CTA's `cap` slots (its best keys; 0 in
+//      unused slots) and return the best key of the segment they did not propose (0: none).
+
+// Warp form, for groups where a consumer warp's slice holds about one winner or fewer: every
+// consumer warp finds the kWarpTop best keys of its contiguous slice of the segment and the
+// best key after them (each lane keeps its best few, then repeated warp maxima of the lanes'
+// heads); the CTA ranks the candidates and proposes its best `cap` of them in rank order.
+__device__ uint64_t propose_warp(const float* sc, int len, int64_t lo, int cap, unsigned long long* slots,
+                                 IdxShared& S) {
+  constexpr int NW = kIdxConsumerWarps, NC = NW * kWarpTop;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned long long* cand_sm = S.wcand;
+  if (threadIdx.x == 0) S.cunp = 0ull;
+  if (warp < NW) {
+    const int wb = (int)((int64_t)warp * len / NW), we = (int)((int64_t)(warp + 1) * len / NW);
+    // The lane's kLaneTop best entries, sorted, and the best entry it lets go.  The lane reads
+    // its entries in increasing index order, so comparing score keys strictly (an equal score
+    // comes with a higher index and ranks lower) orders them as the full keys do.
+    uint32_t tsk[kLaneTop], tix[kLaneTop];  // score keys (0: empty) and segment entries
+#pragma unroll
+    for (int i = 0; i < kLaneTop; ++i) tsk[i] = tix[i] = 0u;
+    uint32_t gsk = 0u, gix = 0u;
+    for (int e = wb + lane; e < we; e += 32) {
+      uint32_t ks = score_key(sc[e]), ki = (uint32_t)e;
+#pragma unroll
+      for (int i = 0; i < kLaneTop; ++i)
+        if (ks > tsk[i]) {
+          const uint32_t a = tsk[i], b = tix[i];
+          tsk[i] = ks;
+          tix[i] = ki;
+          ks = a;
+          ki = b;
+        }
+      if (ks > gsk) {
+        gsk = ks;
+        gix = ki;
+      }
+    }
+    uint64_t top[kLaneTop];
+#pragma unroll
+    for (int i = 0; i < kLaneTop; ++i)
+      top[i] = tsk[i] ? ((uint64_t)tsk[i] << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)(lo + tix[i])) : 0ull;
+    const uint64_t gone = gsk ? ((uint64_t)gsk << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)(lo + gix)) : 0ull;
+    // the warp's kWarpTop best kept keys (repeated warp maxima of the lanes' heads), then the
+    // best key not among them: the next kept one or the best one let go
+    int found = 0;
+#pragma unroll 1
+    for (int r = 0; r < kWarpTop; ++r) {
+      const uint64_t m = warp_max_key(top[0]);
+      if (m != 0ull && top[0] == m) {
+#pragma unroll
+        for (int i = 0; i + 1 < kLaneTop; ++i) top[i] = top[i + 1];
+        top[kLaneTop - 1] = 0ull;
+      }
+      if (lane == 0) cand_sm[warp * kWarpTop + r] = m;
+      found += m != 0ull;
+    }
+    const uint64_t nxt = warp_max_key(top[0] > gone ? top[0] : gone);
+    if (lane == 0) {
+      S.wunp[warp] = nxt;
+      S.wcnt[warp] = found;
+    }
+  }
+  __syncthreads();
+  int nvalid = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) nvalid += S.wcnt[w];
+  if ((int)threadIdx.x < NC) {
+    const uint64_t key = cand_sm[threadIdx.x];
+    if (key != 0ull) {
+      int rank = 0;
+      for (int m = 0; m < NC; ++m) rank += cand_sm[m] > key;
+      if (rank < cap)
+        slots[rank] = key;
+      else if (rank == cap)
+        S.cunp = key;
+    }
+  }
+  for (int i = min(nvalid, cap) + (int)threadIdx.x; i < cap; i += kIdxThreads) slots[i] = 0ull;
+  __syncthreads();
+  uint64_t unp = S.cunp;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) unp = S.wunp[w] > unp ? S.wunp[w] : unp;
+  return unp;
+}
+
+// Histogram form: the entries in the top bins of a 1024-bin linear histogram over the CTA's own
+// score range, as many bins as keep the count within a limit (<= cap) sized from the CTA's
+// expected share of winners.
+__device__ uint64_t propose_hist(const float* sc, int len, int64_t lo, int cap, int64_t keff, int64_t V,
+                                 unsigned long long* slots, unsigned* hist, IdxShared& S) {
+  float mn = INFINITY, mx = -INFINITY;
+  for (int e = threadIdx.x; e < len; e += kIdxThreads) {
+    mn = fminf(mn, sc[e]);
+    mx = fmaxf(mx, sc[e]);
+  }
+  for (int i = threadIdx.x; i < kLinBins; i += kIdxThreads) hist[i] = 0u;
+  float gmn, gmx;
+  block_minmax(mn, mx, S, gmn, gmx);
+  const float scl = gmx > gmn ? (float)kLinBins / (gmx - gmn) : 0.f;
+  for (int e = threadIdx.x; e < len; e += kIdxThreads) atomicAdd(&hist[lin_bin(sc[e], gmn, scl)], 1u);
+  __syncthreads();
+  // lowest bin whose suffix count stays within the limit: one above the bin where the count
+  // from the top first exceeds it
+  const unsigned limit = (unsigned)min((int64_t)cap, (3 * keff * len + 2 * V - 1) / (2 * V) + 16);
+  if ((unsigned)len <= limit) {
+    if (threadIdx.x == 0) S.ubuf[2] = 0u;
+  } else {
+    const Crossing xl = find_crossing(hist, kLinBins, limit + 1u, S.red, &S.cross);
+    if (threadIdx.x == 0) S.ubuf[2] = xl.bin + 1u;
+  }
+  if (threadIdx.x == 0) S.ubuf[0] = 0u;  // proposal slot counter
+  __syncthreads();
+  const unsigned pb = S.ubuf[2];
+  uint64_t unp = 0;
+  for (int e = threadIdx.x; e < len; e += kIdxThreads) {
+    const uint64_t ck = comp_key(sc[e], lo + e);
+    bool put = false;
+    if (lin_bin(sc[e], gmn, scl) >= pb) {
+      const unsigned slot = atomicAdd(&S.ubuf[0], 1u);
+      if (slot < (unsigned)cap) {
+        slots[slot] = ck;
+        put = true;
+      }
+    }
+    if (!put) unp = ck > unp ? ck : unp;
+  }
+  unp = block_max_u64(unp, S);
+  for (int i = (int)min(S.ubuf[0], (unsigned)cap) + (int)threadIdx.x; i < cap; i += kIdxThreads) slots[i] = 0ull;
+  return unp;
 }
 
 // ------------------------------------------------------------------ one segment
@@ -607,11 +767,15 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     }
   if (keff == 0) return;
   if (hi - lo > p.seg_cap && threadIdx.x == 0) flag(p.st, CSKV_DEV_CAPACITY);
+  // speculative proposals in the warp form when a consumer warp's share of the segment holds
+  // about one winner or fewer (group-uniform)
+  const bool warp_form = (V + G - 1) / G <= (int64_t)kIdxConsumerWarps * 32 * kWarpKeys &&
+                         keff <= (int64_t)G * kIdxConsumerWarps;
   // ---- scores of this segment into shared memory
   if constexpr (SRC == kSrcFp8) {
     const uint8_t* kb = p.k_idx + (size_t)(ebase + lo) * (KS * 32);
     const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
-    scan_fp8<KS, NTILE>(p, t, kb, ks, len, sc, sc + p.seg_cap, un, S);
+    scan_fp8<KS, NTILE>(p, t, kb, ks, len, sc, un, S);
   } else if constexpr (SRC == kSrcF32) {
     const float* kb = reinterpret_cast<const float*>(p.k_idx) + (size_t)(ebase + lo) * p.Di;
     const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
@@ -628,7 +792,6 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   }
   unsigned* hist = reinterpret_cast<unsigned*>(un + kUnHist);
   unsigned long long* cands = reinterpret_cast<unsigned long long*>(un + kUnCand);
-  unsigned short* owner = reinterpret_cast<unsigned short*>(un + kUnAux);
   auto own_key = [&](int i) { return comp_key(sc[i], lo + i); };
   uint64_t P = 0;
   int nb = 0;
@@ -639,125 +802,71 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     return;
   }
   bool ok = true;
-  // ---- speculative exchange (one group barrier).  Every CTA proposes its best entries
-  //      (those in the top bins of a linear histogram over its own score range, at most
-  //      `cap`) and reports the best key it did NOT propose.  After the barrier every CTA
-  //      finds the exact k-th best proposal T*; when no CTA holds an unproposed key >= T*,
-  //      the selection is exactly {key >= T*} and no second exchange is needed.  Otherwise
-  //      (winners crowded into one segment, massive ties) the exact path below runs.
+  // ---- speculative exchange (one group barrier).  Every CTA proposes its best entries (at
+  //      most `cap`, into its own slots) and reports the best key it did NOT propose.  After
+  //      the barrier every CTA finds the exact k-th best proposal T*; when no CTA holds an
+  //      unproposed key >= T*, the selection is exactly {key >= T*} and no second exchange is
+  //      needed.  Otherwise (winners crowded into one segment, massive ties) the exact path
+  //      below runs.
   // slot capacity per CTA: group-uniform (every CTA lays out and reads the slots alike)
   const int cap = (int)min((int64_t)(kCandMax / G), (V + G - 1) / G);
   if (G <= kIdxThreads && cap >= 1 && (int64_t)cap * G >= keff) {
-    // -- local range and histogram
+    unsigned long long* slots = ws->cand + (size_t)j * cap;
+    const uint64_t unp = warp_form ? propose_warp(sc, len, lo, cap, slots, S)
+                                   : propose_hist(sc, len, lo, cap, keff, V, slots, hist, S);
+    if (threadIdx.x == 0) ws->unp[j] = unp;
+    for (int i = threadIdx.x; i < kBins0; i += kIdxThreads) hist[i] = 0u;  // for T*, set while waiting
+    ok = group_barrier(ws, G, j, p.st, &S.flag);
+    // -- gather every CTA's slots (CTA order; 0 marks an unused slot), count the proposals
+    //    and find their score range
+    const unsigned total = (unsigned)G * (unsigned)cap;
+    const uint64_t u = (int)threadIdx.x < G ? __ldcg(&ws->unp[threadIdx.x]) : 0ull;
     float mn = INFINITY, mx = -INFINITY;
-    for (int e = threadIdx.x; e < len; e += kIdxThreads) {
-      mn = fminf(mn, sc[e]);
-      mx = fmaxf(mx, sc[e]);
-    }
-    for (int i = threadIdx.x; i < kLinBins; i += kIdxThreads) hist[i] = 0u;
-    float gmn, gmx;
-    block_minmax(mn, mx, S, gmn, gmx);
-    const float scl = gmx > gmn ? (float)kLinBins / (gmx - gmn) : 0.f;
-    for (int e = threadIdx.x; e < len; e += kIdxThreads) atomicAdd(&hist[lin_bin(sc[e], gmn, scl)], 1u);
-    __syncthreads();
-    // -- lowest bin whose suffix count stays within the per-CTA limit: one above the bin
-    //    where the count from the top first exceeds the limit
-    const unsigned limit = (unsigned)min((int64_t)cap, (3 * keff * len + 2 * V - 1) / (2 * V) + 16);
-    if ((unsigned)len <= limit) {
-      if (threadIdx.x == 0) S.ubuf[2] = 0u;
-    } else {
-      const Crossing xl = find_crossing(hist, kLinBins, limit + 1u, S.red, &S.cross);
-      if (threadIdx.x == 0) S.ubuf[2] = xl.bin + 1u;
-    }
-    if (threadIdx.x == 0) S.ubuf[0] = 0u;  // proposal slot counter
-    __syncthreads();
-    const unsigned pb = S.ubuf[2];
-    // -- proposals into this CTA's slots; best unproposed key
-    uint64_t unp = 0;
-    for (int e = threadIdx.x; e < len; e += kIdxThreads) {
-      const uint64_t ck = own_key(e);
-      if (lin_bin(sc[e], gmn, scl) >= pb) {
-        const unsigned slot = atomicAdd(&S.ubuf[0], 1u);
-        if (slot < (unsigned)cap) ws->cand[(size_t)j * cap + slot] = ck;
-      } else {
-        unp = ck > unp ? ck : unp;
+    int cnt = 0;
+    for (unsigned b0 = threadIdx.x; b0 < total; b0 += kIdxThreads * 8) {
+      unsigned long long v[8];
+#pragma unroll
+      for (int uu = 0; uu < 8; ++uu) {
+        const unsigned c = b0 + uu * kIdxThreads;
+        v[uu] = c < total ? __ldcg(ws->cand + c) : 0ull;
+      }
+#pragma unroll
+      for (int uu = 0; uu < 8; ++uu) {
+        const unsigned c = b0 + uu * kIdxThreads;
+        if (c < total) cands[c] = v[uu];
+        if (v[uu] != 0ull) {
+          const float f = key_score(v[uu]);
+          mn = fminf(mn, f);
+          mx = fmaxf(mx, f);
+          ++cnt;
+        }
       }
     }
-    unp = block_max_u64(unp, S);
-    if (threadIdx.x == 0) {
-      const unsigned n_prop = min(S.ubuf[0], (unsigned)cap);
-      ws->prop[j] = n_prop;
-      ws->unp[j] = unp;
-      // a range that holds every proposal (bins of a range are monotone in the score, so a
-      // slightly loose lower edge only widens the first bin)
-      ws->plo[j] = n_prop ? (pb == 0 ? gmn : gmn + (float)pb / scl) : INFINITY;
-      ws->phi[j] = n_prop ? gmx : -INFINITY;
-    }
-    ok = group_barrier(ws, G, p.st, &S.flag);
-    // -- gather every proposal (compact order = CTA order)
-    unsigned np = 0;
-    uint64_t u = 0;
-    float plo = INFINITY, phi = -INFINITY;
-    if ((int)threadIdx.x < G) {
-      np = __ldcg(&ws->prop[threadIdx.x]);
-      u = __ldcg(&ws->unp[threadIdx.x]);
-      plo = __ldcg(&ws->plo[threadIdx.x]);
-      phi = __ldcg(&ws->phi[threadIdx.x]);
-    }
-    for (int i = threadIdx.x; i < kBins0; i += kIdxThreads) hist[i] = 0u;
-    unsigned total;
-    const unsigned off = block_excl_scan(np, S.red, &total);
     float qmn, qmx;
-    block_minmax(plo, phi, S, qmn, qmx);
-    if ((int)threadIdx.x < G) {
-      S.poff[threadIdx.x] = off;
-      S.pcnt[threadIdx.x] = np;
-      if (total <= (unsigned)kCandMax)  // owner table: compact index -> proposing CTA
-        for (unsigned m = 0; m < np; ++m) owner[off + m] = (unsigned short)threadIdx.x;
-    }
-    __syncthreads();
-    if (total >= (unsigned)keff && total <= (unsigned)kCandMax) {
-      // flat copy with 8 loads in flight per thread
-      for (unsigned b0 = threadIdx.x; b0 < total; b0 += kIdxThreads * 8) {
-        unsigned long long v[8];
-#pragma unroll
-        for (int uu = 0; uu < 8; ++uu) {
-          const unsigned c = b0 + uu * kIdxThreads;
-          if (c < total) {
-            const int o = owner[c];
-            v[uu] = __ldcg(ws->cand + (size_t)o * cap + (c - S.poff[o]));
-          }
-        }
-#pragma unroll
-        for (int uu = 0; uu < 8; ++uu) {
-          const unsigned c = b0 + uu * kIdxThreads;
-          if (c < total) cands[c] = v[uu];
-        }
-      }
-      __syncthreads();
-      // Every read of the group's shared state by this CTA is complete: announce it now
-      // (the result is only needed at the very end, so the round trip overlaps the work below).
-      unsigned done_prev = 0;
-      if (threadIdx.x == 0) done_prev = atomicAdd(&ws->done, 1u);
+    int nprop;
+    block_minmax(mn, mx, S, qmn, qmx, cnt, &nprop);  // its barriers also publish cands[]
+    if (nprop >= keff) {  // group-uniform: every CTA gathered the same slots
       // -- exact k-th best proposal: linear histogram, then rank inside the threshold bin
       const float qscl = qmx > qmn ? (float)kBins0 / (qmx - qmn) : 0.f;
-      for (unsigned i = threadIdx.x; i < total; i += kIdxThreads)
-        atomicAdd(&hist[lin_bin4k(key_score(cands[i]), qmn, qscl)], 1u);
+      for (unsigned i = threadIdx.x; i < total; i += kIdxThreads) {
+        const uint64_t c = cands[i];
+        if (c != 0ull) atomicAdd(&hist[lin_bin4k(key_score(c), qmn, qscl)], 1u);
+      }
+      if (threadIdx.x == 0) S.ubuf[1] = 0u;
       __syncthreads();
       const Crossing x = find_crossing(hist, kBins0, (unsigned)keff, S.red, &S.cross);
       const unsigned rr = (unsigned)keff - x.above;  // rank wanted inside bin x.bin (1-based)
       const bool bin_fits = x.cnt <= (unsigned)kAuxKeys;
       // collect the threshold bin's keys
-      if (threadIdx.x == 0) S.ubuf[1] = 0u;
-      __syncthreads();
-      // the owner table is no longer needed: its area holds the threshold bin's keys
       unsigned long long* bin_keys = reinterpret_cast<unsigned long long*>(un + kUnAux);
       const unsigned bin_cap = (unsigned)kAuxKeys;
-      for (unsigned i = threadIdx.x; i < total; i += kIdxThreads)
-        if (lin_bin4k(key_score(cands[i]), qmn, qscl) == x.bin) {
+      for (unsigned i = threadIdx.x; i < total; i += kIdxThreads) {
+        const uint64_t c = cands[i];
+        if (c != 0ull && lin_bin4k(key_score(c), qmn, qscl) == x.bin) {
           const unsigned sl = atomicAdd(&S.ubuf[1], 1u);
-          if (sl < bin_cap) bin_keys[sl] = cands[i];
+          if (sl < bin_cap) bin_keys[sl] = c;
         }
+      }
       __syncthreads();
       const unsigned nbk = min(S.ubuf[1], bin_cap);
       uint64_t Tstar = ~0ull;
@@ -793,30 +902,40 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       unsigned packed = 0;
       if ((int)threadIdx.x < G) packed += (unsigned)(u >= Tstar) << 16;
       if (threadIdx.x == 0 && !bin_fits) packed += 1u << 16;
-      {
-        const unsigned my_off = S.poff[j];
-        for (unsigned i = threadIdx.x; i < my_off; i += kIdxThreads) packed += cands[i] >= Tstar;
-      }
+      const unsigned my_off = (unsigned)j * (unsigned)cap;
+      for (unsigned i = threadIdx.x; i < my_off; i += kIdxThreads) packed += cands[i] >= Tstar;
       unsigned tot;
       block_excl_scan(packed, S.red, &tot);
       if ((tot >> 16) == 0 && ok) {
         const unsigned base = tot & 0xFFFFu;
-        // emit keys >= T*: the rule "top 64 bits >= T*"
-        emit(sc, len, lo, false, Tstar, 64, base, keff, oi, os, S);
-        if (threadIdx.x == 0 && done_prev == (unsigned)(G - 1)) {
-          // the last CTA to announce: every CTA of the group is past the barrier and done
-          // reading, so the synchronisation state can return to zero
-          ws->bar_count = 0u;
-          ws->done = 0u;
+        if (cap <= 64) {
+          // every kept entry of this segment is one of its proposals: its output position is
+          // the base plus the kept proposals of this CTA with a lower index
+          const unsigned long long* own = cands + my_off;
+          if ((int)threadIdx.x < cap) {
+            const uint64_t key = own[threadIdx.x];
+            if (key >= Tstar) {
+              const uint32_t kl = (uint32_t)key;  // inverted index: larger = lower index
+              unsigned pos = base;
+              for (int m = 0; m < cap; ++m) {
+                const uint64_t o = own[m];
+                pos += (o >= Tstar && (uint32_t)o > kl) ? 1u : 0u;
+              }
+              if (pos < (unsigned)keff) {
+                oi[pos] = (int32_t)(0xFFFFFFFFu - kl);
+                if (os) os[pos] = key_score(key);
+              }
+            }
+          }
+        } else {
+          // emit keys >= T*: the rule "top 64 bits >= T*"
+          emit(sc, len, lo, false, Tstar, 64, base, keff, oi, os, S);
         }
         return;
       }
-      // rejected (uniformly across the group): withdraw the announcement; the exact path
-      // below announces again at its own end
-      if (threadIdx.x == 0) atomicSub(&ws->done, 1u);
     }
-    // fall through: the next group barrier orders every read of the proposals before the
-    // candidate slots are reused
+    // rejected (uniformly across the group); the next group barrier orders every read of the
+    // proposals before the exact path reuses the candidate slots
   }
   // ---- exact path: 12-bit digit histogram of the whole group
   for (int i = threadIdx.x; i < kBins0; i += kIdxThreads) hist[i] = 0u;
@@ -828,7 +947,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   __syncthreads();
   for (int i = threadIdx.x; i < kBins0; i += kIdxThreads)
     if (hist[i]) atomicAdd(&ws->hist0[i], hist[i]);
-  ok = group_barrier(ws, G, p.st, &S.flag) && ok;
+  ok = group_barrier(ws, G, j, p.st, &S.flag) && ok;
   copy_to_smem<true>(hist, ws->hist0, kBins0, threadIdx.x, kIdxThreads);
   __syncthreads();
   unsigned r = (unsigned)keff;
@@ -863,7 +982,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
         if (slot < (unsigned)kCandMax) ws->cand[slot] = own_key(e);
         ++slot;
       }
-    ok = group_barrier(ws, G, p.st, &S.flag) && ok;
+    ok = group_barrier(ws, G, j, p.st, &S.flag) && ok;
     const unsigned n_c = min(__ldcg(&ws->cand_count), (unsigned)kCandMax);
     cands_used = n_c;
     copy_to_smem<true>(cands, ws->cand, n_c, threadIdx.x, kIdxThreads);
@@ -898,7 +1017,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       for (int i = threadIdx.x; i < nbins; i += kIdxThreads)
         if (hist[i]) atomicAdd(&gh[i], hist[i]);
       ++used_passes;
-      ok = group_barrier(ws, G, p.st, &S.flag) && ok;
+      ok = group_barrier(ws, G, j, p.st, &S.flag) && ok;
       copy_to_smem<true>(hist, gh, nbins, threadIdx.x, kIdxThreads);
       __syncthreads();
       const Crossing y = find_crossing(hist, nbins, r, S.red, &S.cross);
@@ -912,7 +1031,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     // per-segment selected counts -> output offsets
     const unsigned mine = count_selected(sc, len, lo, P, nb, S);
     if (threadIdx.x == 0) ws->above[j] = mine;
-    ok = group_barrier(ws, G, p.st, &S.flag) && ok;
+    ok = group_barrier(ws, G, j, p.st, &S.flag) && ok;
     unsigned c = 0;
     for (int i = threadIdx.x; i < j; i += kIdxThreads) c += __ldcg(&ws->above[i]);
     unsigned tot;
@@ -951,11 +1070,12 @@ __device__ __forceinline__ int64_t visible_of(const IdxParams& p, int t, int64_t
 }
 
 template <int SRC, int KS, int NTILE>
-// At most 88 registers per thread: 544 x 88 leaves room on the SM's register file for a
-// 128-thread attention CTA to run beside the indexer in a decode step.
+// At most 88 registers per thread (see kIdxConsumerWarps): other kernels of a decode step
+// run beside the indexer on the same SMs.
 __global__ void __maxnreg__(88) lindex_topk_kernel(IdxParams p) {
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ IdxShared S;
+  pdl_launch_dependents();  // the kernel after the indexer may start its set-up now
   uint8_t* un = dsm;                                              // ring / histogram / candidates
   float* sc = reinterpret_cast<float*>(dsm + idx_union_bytes(KS * 32));  // segment scores
   if (p.split) {

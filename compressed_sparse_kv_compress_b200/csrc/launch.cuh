@@ -18,6 +18,25 @@ cudaError_t ensure_smem(K kern, size_t bytes) {
   return ensure_smem_raw(reinterpret_cast<const void*>(kern), bytes);
 }
 
+// kern<<<grid, block, smem, stream>>>(args...) as a programmatic dependent launch: the grid
+// may be scheduled while the previous kernel on the stream runs; the kernel itself waits
+// (pdl_wait) before reading inputs, so stream order is unchanged.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // compress.cu
 cudaError_t launch_csa_compress(const void* xa, const void* za, const void* xb, const void* zb,
                                 const float* ba, const float* bb, const int64_t* tok_off,

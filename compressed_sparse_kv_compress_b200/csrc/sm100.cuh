@@ -123,6 +123,14 @@ __device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Shared-memory matrix descriptor for the 128-byte swizzle: rows of 128 bytes, 8-row atoms of
+// 1024 bytes (1024-byte aligned), 16-byte chunk c of row r stored at chunk c ^ (r & 7).
+// K-major: sbo = stride between 8-row groups, lbo unused (16); MN-major: lbo = stride between
+// 64-element column blocks, sbo = stride between 8-row groups along K.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc_noswz(saddr, lbo, sbo) | ((uint64_t)2 << 61);
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |

@@ -140,9 +140,10 @@ CSKV_API int hca_compress(const void* x, const void* z, const float* bias,
  *           ascending index order, then -1 padding.
  * out_score : [T, k] fp32 or NULL: the score of each kept entry (0 on padding).
  * workspace : lindex_workspace_size(T, k, max_entries) bytes, zero-filled before
- *           its first use; every call returns its synchronisation counters and
- *           histograms to zero (the rest is scratch), so it can be reused as is,
- *           unless the call flagged CSKV_DEV_TIMEOUT (zero-fill it again then).
+ *           its first use; every call leaves it ready for the next (arrival
+ *           counters and histograms back at zero, barrier generations advanced,
+ *           the rest scratch), so it can be reused as is, unless the call flagged
+ *           CSKV_DEV_TIMEOUT (zero-fill it again then).
  *           Calls sharing a workspace must be ordered on one stream.
  * ------------------------------------------------------------------------ */
 CSKV_API int lindex_score_topk(const void* q_idx, const float* q_scale, const void* k_idx, const float* k_scale,
