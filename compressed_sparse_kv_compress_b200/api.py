@@ -67,13 +67,17 @@ def lindex_workspace(T: int, k: int, max_entries: int, device="cuda") -> torch.T
 
 
 def lindex_score_topk(q_idx, k_idx, q_seq, q_pos, ent_off, out_idx, workspace, *, max_entries, q_scale=None,
-                      k_scale=None, head_w=None, out_score=None, dev_status=None, stream=None):
+                      k_scale=None, head_w=None, out_score=None, prefetch_rows=None, dev_status=None, stream=None):
+    """prefetch_rows: optional [entries, ...] tensor indexed like k_idx (e.g. the compressed
+    CSA cache); the rows of the kept entries are prefetched into L2 (a hint)."""
     T, Hi, Di = q_idx.shape
     lib = _lib.load()
+    pf_bytes = 0 if prefetch_rows is None else prefetch_rows[0].numel() * prefetch_rows.element_size()
     st = lib.lindex_score_topk(_ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(head_w), _ptr(q_seq),
                                _ptr(q_pos), _ptr(ent_off), ent_off.numel() - 1, T, Hi, Di, out_idx.shape[1],
-                               _dt(q_idx), int(max_entries), _ptr(out_idx), _ptr(out_score), _ptr(workspace),
-                               workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream))
+                               _dt(q_idx), int(max_entries), _ptr(out_idx), _ptr(out_score), _ptr(prefetch_rows),
+                               pf_bytes, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _ptr(dev_status), _stream(stream))
     _lib.check("lindex_score_topk", st)
     return out_idx
 

@@ -28,6 +28,11 @@ cudaError_t cskv::ensure_smem_raw(const void* kern, size_t bytes) {
   for (const Entry& x : done)
     if (x.kern == kern && x.dev == dev && x.bytes >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  // Every kernel asks for the largest shared-memory carve-out: an SM runs CTAs of different
+  // kernels side by side only under one carve-out, and the decode step relies on the indexer,
+  // the attention and the compression CTAs sharing SMs.
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) done.push_back(Entry{kern, dev, bytes});
   return e;
 }
@@ -126,12 +131,15 @@ static int check_topk_common(int T, int k, int64_t max_entries, const int32_t* o
 int lindex_score_topk(const void* q_idx, const float* q_scale, const void* k_idx, const float* k_scale,
                       const float* head_w, const int32_t* q_seq, const int64_t* q_pos, const int64_t* ent_off,
                       int batch, int T, int Hi, int Di, int k, int dtype, int64_t max_entries, int32_t* out_idx,
-                      float* out_score, void* workspace, size_t ws_bytes, int* dev_status,
-                      cskv_stream_t stream) {
+                      float* out_score, const void* prefetch_rows, int64_t prefetch_row_bytes, void* workspace,
+                      size_t ws_bytes, int* dev_status, cskv_stream_t stream) {
   if (dtype != CSKV_F32 && dtype != CSKV_FP8E4M3 && dtype != CSKV_BF16) return CSKV_ERR_INVALID_ARG;
   if (!lindex_shape_supported(dtype, Hi, Di)) return CSKV_ERR_UNSUPPORTED;
   if (T > 0 && (!q_idx || !k_idx || !q_seq || !q_pos || !ent_off || batch < 1)) return CSKV_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(k_idx)) return CSKV_ERR_INVALID_ARG;
+  if (prefetch_rows && (!aligned16(prefetch_rows) || prefetch_row_bytes <= 0 || prefetch_row_bytes % 16 != 0 ||
+                        prefetch_row_bytes > (1 << 20)))
+    return CSKV_ERR_INVALID_ARG;
   int rc = check_topk_common(T, k, max_entries, out_idx, workspace, ws_bytes);
   if (rc || T == 0) return rc;
   IdxParams p = {};
@@ -150,6 +158,8 @@ int lindex_score_topk(const void* q_idx, const float* q_scale, const void* k_idx
   p.max_entries = max_entries;
   p.out_idx = out_idx;
   p.out_score = out_score;
+  p.pf_rows = prefetch_rows ? (const uint8_t*)prefetch_rows : nullptr;
+  p.pf_row_bytes = prefetch_rows ? prefetch_row_bytes : 0;
   p.ws = (QueryWS*)workspace;
   p.st = dev_status;
   return launch_status(launch_lindex(p, dtype, T, (cudaStream_t)stream));

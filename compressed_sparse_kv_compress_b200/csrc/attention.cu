@@ -38,7 +38,6 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) 
   float* l_run = m_run + HP;                     // [HP]
   float* alpha = l_run + HP;                     // [HP]
   __shared__ int valid[kAttnTile];
-  pdl_launch_dependents();
   pdl_wait();
 
   const int t = blockIdx.y, split = blockIdx.x, tid = threadIdx.x;
@@ -155,6 +154,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) 
     p.part_ml[sb * 2 * H + h] = m_run[h];
     p.part_ml[(sb * 2 + 1) * H + h] = l_run[h];
   }
+  pdl_launch_dependents();  // the merge kernel waits for this grid before it reads
 }
 
 // Merge the splits of each query ([TR] §3.1), the sink once ([SW] §十二):
@@ -240,7 +240,9 @@ __global__ void __launch_bounds__(128 * kCombineGroups) attn_combine_kernel(Attn
 }
 
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream) {
-  const cudaError_t e = launch_dependent(attn_combine_kernel, dim3(kHeadDim / kCombineDims, p.T),
+  cudaError_t e = ensure_smem(attn_combine_kernel, 0);
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(attn_combine_kernel, dim3(kHeadDim / kCombineDims, p.T),
                                          dim3(128 * kCombineGroups), 0, stream, p);
   note_launch();
   return e;

@@ -52,12 +52,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   uint8_t* Ps = sm + 3 * kTileBytes;  // A of O = P V     [128 heads x 128 rows], K-major
   __shared__ uint64_t bar_s, bar_o;
   __shared__ uint32_t tmem_base;
-  __shared__ int64_t row_src[kTcChunk];  // element offset of each chunk row, -1 = skipped
-  __shared__ uint8_t row_raw[kTcChunk];
+  __shared__ const __nv_bfloat16* row_src[kTcChunk];  // address of each chunk row, null = skipped
   __shared__ uint32_t row_mask[kTcChunk / 32];  // bit r: chunk row r is attended
 
   const int t = blockIdx.y, split = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  pdl_launch_dependents();
   // ---- set-up that reads no input overlaps the previous kernel (dependent launch)
   if (warp == 0) {
     tmem_alloc(&tmem_base, 256);  // S: columns 0..127, O: columns 128..255
@@ -104,18 +102,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
       int64_t off = -1;
       bool is_raw = false;
       if (tid < rows) off = resolve_row(p, q, t, a + tid, &is_raw);
-      row_src[tid] = off;
-      row_raw[tid] = is_raw;
+      row_src[tid] = off >= 0 ? (is_raw ? raw : cmp) + off : nullptr;
       const uint32_t bal = __ballot_sync(0xffffffffu, off >= 0);
       if (lane == 0) row_mask[warp] = bal;
     }
     __syncthreads();
     // ---- gather: one whole 512-byte K||V row per warp instruction (lane j copies its
-    //      16-byte piece j); skipped rows up to nc are zero-filled
+    //      16-byte piece j), eight rows in flight per warp; skipped rows up to nc are
+    //      zero-filled
+#pragma unroll 8
     for (int r = warp; r < nc; r += 4) {
-      const int64_t off = row_src[r];
-      const __nv_bfloat16* src = off >= 0 ? (row_raw[r] ? raw : cmp) + off + 8 * lane : qg;
-      cp_async16(KVs + sw_off(r, lane), src, off >= 0 ? 16u : 0u);
+      const __nv_bfloat16* row = row_src[r];
+      cp_async16(KVs + sw_off(r, lane), row ? (const void*)(row + 8 * lane) : (const void*)qg, row ? 16u : 0u);
     }
     cp_async_wait_all();
     fence_proxy_async_smem();
@@ -243,6 +241,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
       p.part_ml[(sb * 2 + 1) * H + tid] = l_run;
     }
   }
+  // the merge kernel may launch now; it waits for this grid to finish before it reads
+  // (launching it earlier would park its CTAs on SMs that other kernels of the step need)
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

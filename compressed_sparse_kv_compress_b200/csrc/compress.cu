@@ -90,6 +90,8 @@ __global__ void __maxnreg__(144) csa_compress_kernel(
     const int64_t* __restrict__ ent_off, const int64_t* __restrict__ first_block,
     const int64_t* __restrict__ num_blocks, int64_t max_blocks, TO* __restrict__ out, int* st) {
   constexpr int kC = kTwo ? 8 : 4;  // candidates: 4 path-A (+ 4 path-B)
+  // A few small CTAs: the next kernel (the indexer in a decode step) may launch at once and
+  // sit beside them; it waits for this grid before reading anything.
   pdl_launch_dependents();
   pdl_wait();
   const int b = blockIdx.y;
@@ -176,7 +178,6 @@ __global__ void __launch_bounds__(kHcaThreads, 8) hca_compress_kernel(
     const int64_t* __restrict__ ent_off, const int64_t* __restrict__ first_block,
     const int64_t* __restrict__ num_blocks, int64_t max_blocks, TO* __restrict__ out, int* st) {
   __shared__ float sm_max[4][16], sm_sum[4][16], sm_acc[4][16];
-  pdl_launch_dependents();
   pdl_wait();
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, half = lane & 1;
@@ -276,7 +277,8 @@ static cudaError_t launch_csa_t(const void* xa, const void* za, const void* xb, 
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
                                 void* out, int* st, cudaStream_t stream) {
   dim3 grid((unsigned)((max_blocks + kCsaWarps - 1) / kCsaWarps), (unsigned)batch);
-  cudaError_t e;
+  cudaError_t e = ensure_smem(xb != nullptr ? csa_compress_kernel<TI, TO, true> : csa_compress_kernel<TI, TO, false>, 0);
+  if (e != cudaSuccess) return e;
   if (xb != nullptr)
     e = launch_dependent(csa_compress_kernel<TI, TO, true>, grid, dim3(32 * kCsaWarps), 0, stream, (const TI*)xa,
                          (const TI*)za, (const TI*)xb, (const TI*)zb, ba, bb, tok_off, tok0, ent_off, first, num,
@@ -315,7 +317,9 @@ static cudaError_t launch_hca_t(const void* x, const void* z, const float* bias,
   // slices of one entry are consecutive CTAs; very large bulk calls loop over entries
   const int64_t entries = max_blocks < (int64_t)(1 << 26) ? max_blocks : (int64_t)(1 << 26);
   dim3 grid((unsigned)(entries * kHcaSlices), (unsigned)batch);
-  const cudaError_t e = launch_dependent(hca_compress_kernel<TI, TO>, grid, dim3(kHcaThreads), 0, stream,
+  cudaError_t e = ensure_smem(hca_compress_kernel<TI, TO>, 0);
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(hca_compress_kernel<TI, TO>, grid, dim3(kHcaThreads), 0, stream,
                                          (const TI*)x, (const TI*)z, bias, tok_off, tok0, ent_off, first, num,
                                          max_blocks, (TO*)out, st);
   note_launch();

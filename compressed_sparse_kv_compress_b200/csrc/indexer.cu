@@ -55,9 +55,6 @@ constexpr int kIdxMaxDim = 128;
 
 enum IdxSrc { kSrcFp8 = 0, kSrcF32 = 1, kSrcScores = 2 };
 
-constexpr int kWarpTop = 6;   // candidates per consumer warp in the warp form of the proposals
-constexpr int kWarpKeys = 8;  // entries per lane in the warp form: warp slices up to 256 entries
-constexpr int kLaneTop = 3;   // best keys each lane keeps for the warp form
 
 struct alignas(16) QueryWS {
   unsigned bar_count, spare, done, cand_count;  // bar_count: group barrier (phase bit + arrivals)
@@ -104,14 +101,6 @@ __device__ __forceinline__ float key_score(uint64_t c) {
 }
 __device__ __forceinline__ bool key_selected(uint64_t c, uint64_t P, int nb) {
   return (c >> (64 - nb)) >= P;
-}
-// Largest 64-bit key of the warp: the largest high half, then the largest low half among the
-// lanes that hold it.
-__device__ __forceinline__ uint64_t warp_max_key(uint64_t k) {
-  const unsigned hi = (unsigned)(k >> 32), lo = (unsigned)k;
-  const unsigned mh = __reduce_max_sync(0xffffffffu, hi);
-  const unsigned ml = __reduce_max_sync(0xffffffffu, hi == mh ? lo : 0u);
-  return ((uint64_t)mh << 32) | ml;
 }
 
 // ------------------------------------------------------------------ block helpers
@@ -252,10 +241,6 @@ struct IdxShared {
   float fred[64];
   unsigned long long ured[32];
   unsigned long long tstar;
-  unsigned long long wcand[kIdxConsumerWarps * kWarpTop];  // warp proposals: each warp's best
-  unsigned long long wunp[kIdxConsumerWarps];  // warp proposals: best key after each warp's top
-  unsigned long long cunp;                     // warp proposals: best candidate past `cap`
-  int wcnt[kIdxConsumerWarps];                 // warp proposals: keys found by each warp
   int fcnt[32];
   Crossing cross;
   int flag;
@@ -507,7 +492,7 @@ __device__ void local_select(Get get, int n, unsigned r, uint64_t& P, int& nb, u
 // Positions are bounded by k, so even an inconsistent threshold (after a timed-out
 // group barrier) cannot write outside the output row.
 __device__ void emit(const float* sc, int len, int64_t lo, bool all, uint64_t P, int nb, int64_t base,
-                     int64_t k, int32_t* oi, float* os, IdxShared& S) {
+                     int64_t k, int32_t* oi, float* os, const IdxParams& p, int64_t ebase, IdxShared& S) {
   const int per = (len + kIdxThreads - 1) / kIdxThreads;
   const int a = min(len, (int)threadIdx.x * per), b = min(len, a + per);
   unsigned c = 0;
@@ -518,6 +503,7 @@ __device__ void emit(const float* sc, int len, int64_t lo, bool all, uint64_t P,
       if (pos >= 0 && pos < k) {
         oi[pos] = (int32_t)(lo + e);
         if (os) os[pos] = sc[e];
+        if (p.pf_rows) prefetch_l2_bulk(p.pf_rows + (size_t)(ebase + lo + e) * p.pf_row_bytes, (unsigned)p.pf_row_bytes);
       }
       ++pos;
     }
@@ -618,94 +604,11 @@ __device__ void group_cleanup(QueryWS* ws, int G, bool used_hist0, int used_pass
   __syncthreads();
 }
 
-// ---- speculative proposals.  Both forms fill this CTA's `cap` slots (its best keys; 0 in
-//      unused slots) and return the best key of the segment they did not propose (0: none).
+// ---- speculative proposals: fill this CTA's `cap` slots (its best keys; 0 in unused slots)
+//      and return the best key of the segment that was not proposed (0: none).
 
-// Warp form, for groups where a consumer warp's slice holds about one winner or fewer: every
-// consumer warp finds the kWarpTop best keys of its contiguous slice of the segment and the
-// best key after them (each lane keeps its best few, then repeated warp maxima of the lanes'
-// heads); the CTA ranks the candidates and proposes its best `cap` of them in rank order.
-__device__ uint64_t propose_warp(const float* sc, int len, int64_t lo, int cap, unsigned long long* slots,
-                                 IdxShared& S) {
-  constexpr int NW = kIdxConsumerWarps, NC = NW * kWarpTop;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned long long* cand_sm = S.wcand;
-  if (threadIdx.x == 0) S.cunp = 0ull;
-  if (warp < NW) {
-    const int wb = (int)((int64_t)warp * len / NW), we = (int)((int64_t)(warp + 1) * len / NW);
-    // The lane's kLaneTop best entries, sorted, and the best entry it lets go.  The lane reads
-    // its entries in increasing index order, so comparing score keys strictly (an equal score
-    // comes with a higher index and ranks lower) orders them as the full keys do.
-    uint32_t tsk[kLaneTop], tix[kLaneTop];  // score keys (0: empty) and segment entries
-#pragma unroll
-    for (int i = 0; i < kLaneTop; ++i) tsk[i] = tix[i] = 0u;
-    uint32_t gsk = 0u, gix = 0u;
-    for (int e = wb + lane; e < we; e += 32) {
-      uint32_t ks = score_key(sc[e]), ki = (uint32_t)e;
-#pragma unroll
-      for (int i = 0; i < kLaneTop; ++i)
-        if (ks > tsk[i]) {
-          const uint32_t a = tsk[i], b = tix[i];
-          tsk[i] = ks;
-          tix[i] = ki;
-          ks = a;
-          ki = b;
-        }
-      if (ks > gsk) {
-        gsk = ks;
-        gix = ki;
-      }
-    }
-    uint64_t top[kLaneTop];
-#pragma unroll
-    for (int i = 0; i < kLaneTop; ++i)
-      top[i] = tsk[i] ? ((uint64_t)tsk[i] << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)(lo + tix[i])) : 0ull;
-    const uint64_t gone = gsk ? ((uint64_t)gsk << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)(lo + gix)) : 0ull;
-    // the warp's kWarpTop best kept keys (repeated warp maxima of the lanes' heads), then the
-    // best key not among them: the next kept one or the best one let go
-    int found = 0;
-#pragma unroll 1
-    for (int r = 0; r < kWarpTop; ++r) {
-      const uint64_t m = warp_max_key(top[0]);
-      if (m != 0ull && top[0] == m) {
-#pragma unroll
-        for (int i = 0; i + 1 < kLaneTop; ++i) top[i] = top[i + 1];
-        top[kLaneTop - 1] = 0ull;
-      }
-      if (lane == 0) cand_sm[warp * kWarpTop + r] = m;
-      found += m != 0ull;
-    }
-    const uint64_t nxt = warp_max_key(top[0] > gone ? top[0] : gone);
-    if (lane == 0) {
-      S.wunp[warp] = nxt;
-      S.wcnt[warp] = found;
-    }
-  }
-  __syncthreads();
-  int nvalid = 0;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) nvalid += S.wcnt[w];
-  if ((int)threadIdx.x < NC) {
-    const uint64_t key = cand_sm[threadIdx.x];
-    if (key != 0ull) {
-      int rank = 0;
-      for (int m = 0; m < NC; ++m) rank += cand_sm[m] > key;
-      if (rank < cap)
-        slots[rank] = key;
-      else if (rank == cap)
-        S.cunp = key;
-    }
-  }
-  for (int i = min(nvalid, cap) + (int)threadIdx.x; i < cap; i += kIdxThreads) slots[i] = 0ull;
-  __syncthreads();
-  uint64_t unp = S.cunp;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) unp = S.wunp[w] > unp ? S.wunp[w] : unp;
-  return unp;
-}
-
-// Histogram form: the entries in the top bins of a 1024-bin linear histogram over the CTA's own
-// score range, as many bins as keep the count within a limit (<= cap) sized from the CTA's
+// The proposals are the entries in the top bins of a 1024-bin linear histogram over the CTA's
+// own score range, as many bins as keep the count within a limit (<= cap) sized from the CTA's
 // expected share of winners.
 __device__ uint64_t propose_hist(const float* sc, int len, int64_t lo, int cap, int64_t keff, int64_t V,
                                  unsigned long long* slots, unsigned* hist, IdxShared& S) {
@@ -767,10 +670,6 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     }
   if (keff == 0) return;
   if (hi - lo > p.seg_cap && threadIdx.x == 0) flag(p.st, CSKV_DEV_CAPACITY);
-  // speculative proposals in the warp form when a consumer warp's share of the segment holds
-  // about one winner or fewer (group-uniform)
-  const bool warp_form = (V + G - 1) / G <= (int64_t)kIdxConsumerWarps * 32 * kWarpKeys &&
-                         keff <= (int64_t)G * kIdxConsumerWarps;
   // ---- scores of this segment into shared memory
   if constexpr (SRC == kSrcFp8) {
     const uint8_t* kb = p.k_idx + (size_t)(ebase + lo) * (KS * 32);
@@ -787,7 +686,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   }
   // ---- everything kept: output position of entry e is e
   if (keff == V) {
-    emit(sc, len, lo, true, 0, 0, lo, keff, oi, os, S);
+    emit(sc, len, lo, true, 0, 0, lo, keff, oi, os, p, ebase, S);
     return;
   }
   unsigned* hist = reinterpret_cast<unsigned*>(un + kUnHist);
@@ -798,7 +697,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   // ---- a single CTA owns the query: exact selection in shared memory
   if (G == 1) {
     local_select(own_key, len, (unsigned)keff, P, nb, hist, S);
-    emit(sc, len, lo, false, P, nb, 0, keff, oi, os, S);
+    emit(sc, len, lo, false, P, nb, 0, keff, oi, os, p, ebase, S);
     return;
   }
   bool ok = true;
@@ -812,8 +711,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   const int cap = (int)min((int64_t)(kCandMax / G), (V + G - 1) / G);
   if (G <= kIdxThreads && cap >= 1 && (int64_t)cap * G >= keff) {
     unsigned long long* slots = ws->cand + (size_t)j * cap;
-    const uint64_t unp = warp_form ? propose_warp(sc, len, lo, cap, slots, S)
-                                   : propose_hist(sc, len, lo, cap, keff, V, slots, hist, S);
+    const uint64_t unp = propose_hist(sc, len, lo, cap, keff, V, slots, hist, S);
     if (threadIdx.x == 0) ws->unp[j] = unp;
     for (int i = threadIdx.x; i < kBins0; i += kIdxThreads) hist[i] = 0u;  // for T*, set while waiting
     ok = group_barrier(ws, G, j, p.st, &S.flag);
@@ -873,6 +771,8 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       if (!bin_fits) {
         // the threshold bin does not fit the scratch: leave T* at "select nothing", which the
         // check below rejects
+      } else if (nbk == 1 && rr == 1) {
+        Tstar = bin_keys[0];  // the usual case: the threshold bin holds T* alone
       } else if (nbk <= (unsigned)kIdxThreads) {
         // thread i ranks key i against the bin (keys are distinct: exactly one has rank rr-1)
         if (threadIdx.x < nbk) {
@@ -922,14 +822,17 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
                 pos += (o >= Tstar && (uint32_t)o > kl) ? 1u : 0u;
               }
               if (pos < (unsigned)keff) {
-                oi[pos] = (int32_t)(0xFFFFFFFFu - kl);
+                const uint32_t e = 0xFFFFFFFFu - kl;
+                oi[pos] = (int32_t)e;
                 if (os) os[pos] = key_score(key);
+                if (p.pf_rows)
+                  prefetch_l2_bulk(p.pf_rows + (size_t)(ebase + e) * p.pf_row_bytes, (unsigned)p.pf_row_bytes);
               }
             }
           }
         } else {
           // emit keys >= T*: the rule "top 64 bits >= T*"
-          emit(sc, len, lo, false, Tstar, 64, base, keff, oi, os, S);
+          emit(sc, len, lo, false, Tstar, 64, base, keff, oi, os, p, ebase, S);
         }
         return;
       }
@@ -1038,7 +941,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     block_excl_scan(c, S.red, &tot);
     base = tot;
   }
-  emit(sc, len, lo, false, P, nb, base, keff, oi, os, S);
+  emit(sc, len, lo, false, P, nb, base, keff, oi, os, p, ebase, S);
   group_cleanup(ws, G, true, used_passes, S);
 }
 
@@ -1076,9 +979,19 @@ __global__ void __maxnreg__(88) lindex_topk_kernel(IdxParams p) {
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ IdxShared S;
   pdl_launch_dependents();  // the kernel after the indexer may start its set-up now
+  pdl_wait();
   uint8_t* un = dsm;                                              // ring / histogram / candidates
   float* sc = reinterpret_cast<float*>(dsm + idx_union_bytes(KS * 32));  // segment scores
-  if (p.split) {
+  if (p.split && p.T == 1) {
+    // one query: the whole grid is its group (the plan below reduces to this)
+    const int t = p.t_begin;
+    int64_t eb;
+    const int64_t V = visible_of(p, t, &eb);
+    const int64_t smax = V > kMinSeg ? (V + kMinSeg - 1) / kMinSeg : 1;
+    const int G = V > 0 ? (int)min(min((int64_t)gridDim.x, smax), (int64_t)kMaxGroup) : 1;
+    if ((int)blockIdx.x >= G) return;
+    process_segment<SRC, KS, NTILE>(p, t, (int)blockIdx.x, G, V, eb, p.ws, sc, un, S);
+  } else if (p.split) {
     // plan, in parallel over queries: visible counts, group sizes (one round), CTA ranges
     if (threadIdx.x == 0) S.plan_t = -1;
     int64_t v = 0;
@@ -1196,11 +1109,15 @@ static cudaError_t launch_one(const IdxParams& p, int grid, bool coop, size_t sm
   cfg.blockDim = dim3(kIdxThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  // cooperative (the CTAs of a query group wait on one another) and a dependent launch of
+  // the previous kernel on the stream (the kernel waits for it before reading any input)
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = coop ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kern, p);
   if (e == cudaSuccess) note_launch();
   return e;

@@ -10,8 +10,9 @@ struct QueryWS;
 // Host-side count of kernels this library has launched (api.cu).
 void note_launch();
 
-// Raises a kernel's dynamic shared-memory limit once per (kernel, device):
-// cudaFuncSetAttribute is a host round trip that repeated launches skip (api.cu).
+// Raises a kernel's dynamic shared-memory limit and asks for the largest shared-memory
+// carve-out, once per (kernel, device): cudaFuncSetAttribute is a host round trip that
+// repeated launches skip (api.cu).  Every kernel calls it before its first launch.
 cudaError_t ensure_smem_raw(const void* kern, size_t bytes);
 template <typename K>
 cudaError_t ensure_smem(K kern, size_t bytes) {
@@ -70,6 +71,8 @@ struct IdxParams {
   int stages;
   int32_t* out_idx;
   float* out_score;
+  const uint8_t* pf_rows;  // optional: rows (indexed like k_idx) of kept entries go to L2
+  int64_t pf_row_bytes;
   QueryWS* ws;
   int* st;
 };

@@ -8,10 +8,9 @@ as cited in the C header):
              -> lindex_score_topk -> hybrid_decode_attn(CSA)
   HCA layer: hca_compress -> hybrid_decode_attn(HCA)
 
-The HCA layer and the CSA entry compression do not depend on the indexer, so
-with ``two_streams`` they run on side streams that fork from and join the
-caller's stream (CSA attention waits for the compressed entries).  The whole
-step can be captured into a CUDA graph and replayed.
+The HCA layer does not depend on the CSA layer, so with ``two_streams`` it
+runs on a side stream that forks from and joins the caller's stream.  The
+whole step can be captured into a CUDA graph and replayed.
 
 Tensor names (all device tensors, int64 offsets unless noted):
   CSA rows  x_a z_a x_b z_b [rows, 256], csa_x_off [B+1], csa_t0 [B],
@@ -52,7 +51,6 @@ class DecodeStep:
         self.ws_h = api.attn_workspace(api.HCA, T, H, 0, self.W, self.max_hca_visible, dev)
         self.two_streams = two_streams
         self.side = torch.cuda.Stream(device=dev) if two_streams else None
-        self.side2 = torch.cuda.Stream(device=dev) if two_streams else None
         self.graph = None
 
     # ------------------------------------------------------------------
@@ -79,7 +77,8 @@ class DecodeStep:
         t = self.t
         api.lindex_score_topk(t["q_idx"], t["k_idx"], t["q_seq"], t["q_pos"], t["csa_off"], self.idx, self.ws_idx,
                               max_entries=self.max_csa_visible, q_scale=t.get("q_scale"), k_scale=t.get("k_scale"),
-                              head_w=t.get("head_w"), out_score=self.score, dev_status=self.status, stream=stream)
+                              head_w=t.get("head_w"), out_score=self.score, prefetch_rows=t["cmp_c"],
+                              dev_status=self.status, stream=stream)
 
     def csa_attend(self, stream=None):
         t = self.t
@@ -111,15 +110,12 @@ class DecodeStep:
             self.csa_layer(main)
             self.hca_layer(main)
             return
-        # HCA layer and the CSA entry compression run beside the indexer, which needs
-        # neither; CSA attention waits for the compressed entries.
+        # The HCA layer runs beside the CSA layer, which it does not depend on.  The CSA
+        # layer stays on one stream, so each of its kernels follows the previous one as a
+        # dependent launch (its set-up overlaps the previous kernel's tail).
         self.side.wait_stream(main)
-        self.side2.wait_stream(main)
         self.hca_layer(self.side)
-        self.csa_compress(self.side2)
-        self.csa_select(main)
-        main.wait_stream(self.side2)
-        self.csa_attend(main)
+        self.csa_layer(main)
         main.wait_stream(self.side)
 
     # ------------------------------------------------------------------

@@ -139,6 +139,11 @@ CSKV_API int hca_compress(const void* x, const void* z, const float* bias,
  * out_idx : [T, k] int32: the kept entries (indices within the sequence) in
  *           ascending index order, then -1 padding.
  * out_score : [T, k] fp32 or NULL: the score of each kept entry (0 on padding).
+ * prefetch_rows, prefetch_row_bytes : optional (NULL / 0 for none): a row array
+ *           indexed like k_idx (rows ent_off[b] + i, prefetch_row_bytes each, a
+ *           multiple of 16, 16-byte aligned) -- e.g. the compressed CSA cache that
+ *           the attention call gathers next.  The rows of the kept entries are
+ *           prefetched into L2 as they are emitted; a hint with no effect on results.
  * workspace : lindex_workspace_size(T, k, max_entries) bytes, zero-filled before
  *           its first use; every call leaves it ready for the next (arrival
  *           counters and histograms back at zero, barrier generations advanced,
@@ -150,6 +155,7 @@ CSKV_API int lindex_score_topk(const void* q_idx, const float* q_scale, const vo
                       const float* head_w, const int32_t* q_seq, const int64_t* q_pos,
                       const int64_t* ent_off, int batch, int T, int Hi, int Di, int k, int dtype,
                       int64_t max_entries, int32_t* out_idx, float* out_score,
+                      const void* prefetch_rows, int64_t prefetch_row_bytes,
                       void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream);
 
 /* ------------------------------------------------------------------------

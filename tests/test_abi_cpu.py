@@ -84,7 +84,8 @@ def test_indexer_validation(lib):
     def call(**kw):
         a = {**args, **kw}
         return lib.lindex_score_topk(_p(), nul, _p(), nul, nul, _p(), _p(), _p(), 1, kw.get("T", 1), a["Hi"], a["Di"],
-                                     a["k"], a["dtype"], 100, _p(), nul, _p(), 1 << 20, nul, nul)
+                                     a["k"], a["dtype"], 100, _p(), nul, kw.get("pf", nul), kw.get("pf_bytes", 0),
+                                     _p(), 1 << 20, nul, nul)
 
     assert call(dtype=9) == _lib.ERR_INVALID_ARG
     assert call(dtype=_lib.BF16) == _lib.ERR_UNSUPPORTED
@@ -92,6 +93,8 @@ def test_indexer_validation(lib):
     assert call(Hi=17) == _lib.ERR_UNSUPPORTED
     assert call(k=0) == _lib.ERR_INVALID_ARG
     assert call(T=0) == _lib.OK
+    assert call(pf=_p(0x1008), pf_bytes=512) == _lib.ERR_INVALID_ARG  # misaligned prefetch rows
+    assert call(pf=_p(), pf_bytes=100) == _lib.ERR_INVALID_ARG  # row size not a multiple of 16
     assert lib.lindex_topk_from_scores(nul, 10, _p(), 1, 4, 10, _p(), nul, _p(), 1 << 20, nul,
                                        nul) == _lib.ERR_INVALID_ARG
     assert lib.lindex_topk_from_scores(_p(), 5, _p(), 1, 4, 10, _p(), nul, _p(), 1 << 20, nul,
