@@ -358,7 +358,8 @@ def run_cskv(args, ws, rank, local):
     idx_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in kev)
 
     # ---- end to end through the public API with host buffers: per step, the step's new
-    #      inputs go host -> device from pinned memory and both outputs come back
+    #      inputs go host -> device from pinned memory and both outputs come back, all in the
+    #      step's graph (DecodeStep.capture_io)
     def host_pairs(st):
         t = st.t
         pairs = []  # (pinned host tensor, device destination view)
@@ -389,13 +390,12 @@ def run_cskv(args, ws, rank, local):
     h2d = sum(h.numel() * h.element_size() for h, _ in io[0][0])
     d2h = sum(h.numel() * h.element_size() for _, h in io[0][1])
 
+    for st, (pairs, outs) in zip(steps, io):  # staged upload, step and read-back in one graph
+        st.capture_io(pairs, outs)
+    torch.cuda.synchronize()
+
     def e2e_step(i):
-        pairs, outs = io[i % R]
-        for h, d in pairs:
-            d.copy_(h, non_blocking=True)
-        steps[i % R].replay()
-        for d, h in outs:
-            h.copy_(d, non_blocking=True)
+        steps[i % R].replay_io()
 
     ms_e2e = timed(e2e_step, args.steps)
     clk = clocks.stop()

@@ -29,6 +29,7 @@ SIGNATURES = {
     "cskv_last_cuda_error": (ctypes.c_char_p, []),
     "cskv_version": (_i32, []),
     "cskv_launch_count": (ctypes.c_ulonglong, []),
+    "cskv_copy_segments": (_i32, [_p, _p, _p, _p, _i32, _p]),
     "csa_compress": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p, _p, _p]),
     "hca_compress": (_i32, [_p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p, _p, _p]),
     "lindex_score_topk": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _i32, _i32, _i32, _i32, _i32, _i64,

@@ -118,3 +118,13 @@ def hybrid_decode_attn(mode, q, kv_cmp, cmp_off, kv_raw, raw_off, q_seq, q_pos, 
                                 _ptr(dev_status), _stream(stream))
     _lib.check("hybrid_decode_attn", st)
     return out
+
+
+def copy_segments(src, src_off, dst_ptrs, lens, stream=None):
+    """Scatter segments of the device byte buffer `src` (int64 device arrays src_off, lens and
+    dst_ptrs = destination addresses) with one kernel: the unpacking half of a staged
+    host-to-device copy of a step's new inputs."""
+    lib = _lib.load()
+    st = lib.cskv_copy_segments(_ptr(src), _ptr(src_off), _ptr(dst_ptrs), _ptr(lens), int(src_off.numel()),
+                                _stream(stream))
+    _lib.check("cskv_copy_segments", st)

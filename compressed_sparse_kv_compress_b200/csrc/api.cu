@@ -71,6 +71,13 @@ const char* cskv_last_cuda_error(void) { return g_cuda_err; }
 
 int cskv_version(void) { return 100; }
 
+int cskv_copy_segments(const void* src, const int64_t* src_off, void* const* dst, const int64_t* len, int n,
+                       cskv_stream_t stream) {
+  if (n < 0 || n > (1 << 30) || (n > 0 && (!src || !src_off || !dst || !len))) return CSKV_ERR_INVALID_ARG;
+  if (n == 0) return CSKV_OK;
+  return launch_status(launch_copy_segments(src, src_off, dst, len, n, (cudaStream_t)stream));
+}
+
 unsigned long long cskv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 static int check_compress_common(const void* x, const void* z, const int64_t* tok_off, int batch,

@@ -112,4 +112,7 @@ int attn_tc_rows_per_split(int mode, int T, int k, int window, int64_t max_entri
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
 int attn_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms);
 int attn_max_splits(int mode, int k, int window, int64_t max_entries, int R);
+// staging.cu
+cudaError_t launch_copy_segments(const void* src, const int64_t* src_off, void* const* dst, const int64_t* len, int n,
+                                 cudaStream_t stream);
 }  // namespace cskv

@@ -132,5 +132,49 @@ class DecodeStep:
         self.graph = g
         return g
 
+    def capture_io(self, h2d=(), d2h=()):
+        """Capture, into one CUDA graph, the upload of this step's new inputs, the step, and the
+        read-back of its results; replay with replay_io().
+
+        h2d: (host, device) pairs.  The host sides are packed into one pinned staging buffer:
+        the returned host tensors (views into it, initialised from the given ones) are where
+        the caller writes each step's new inputs.  A replay makes one host-to-device copy of
+        the buffer and one cskv_copy_segments launch that spreads it to the device tensors
+        (which must be contiguous).  d2h: (device, host pinned) pairs copied back after the
+        step.  A replay costs one launch on the host, whatever the number of tensors."""
+        if self.graph is None:
+            self.capture()  # sets kernel attributes and warms up outside capture
+        dev = self.o_c.device
+        sizes = [d.numel() * d.element_size() for _, d in h2d]
+        offs, total = [], 0
+        for nb in sizes:
+            offs.append(total)
+            total += (nb + 15) // 16 * 16
+        stage_h = torch.empty(max(total, 16), dtype=torch.uint8, pin_memory=True)
+        stage_d = torch.empty(max(total, 16), dtype=torch.uint8, device=dev)
+        views = []
+        for (h, d), o, nb in zip(h2d, offs, sizes):
+            assert d.is_contiguous()
+            v = stage_h[o:o + nb].view(d.dtype).view(d.shape)
+            v.copy_(h)
+            views.append(v)
+        self._io = (stage_h, stage_d, torch.tensor(offs, dtype=torch.int64, device=dev),
+                    torch.tensor([d.data_ptr() for _, d in h2d], dtype=torch.int64, device=dev),
+                    torch.tensor(sizes, dtype=torch.int64, device=dev))
+        _, _, src_off, dst_ptrs, lens = self._io
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if h2d:
+                stage_d.copy_(stage_h, non_blocking=True)
+                api.copy_segments(stage_d, src_off, dst_ptrs, lens)
+            self.run()
+            for d, h in d2h:
+                h.copy_(d, non_blocking=True)
+        self.graph_io = g
+        return views
+
+    def replay_io(self):
+        self.graph_io.replay()
+
     def replay(self):
         self.graph.replay()

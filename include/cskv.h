@@ -233,6 +233,22 @@ CSKV_API int hybrid_decode_attn_noalloc(int mode, const void* q, const void* kv_
                        int dtype, int64_t max_entries, float* out, float* lse,
                        int* dev_status, cskv_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * cskv_copy_segments -- device-side scatter of byte segments (input staging).
+ *
+ * Not a step of the method: plumbing for callers that move a decode step's new
+ * inputs (queries, the newest token rows, the newest indexer keys) to the GPU in
+ * one host->device copy of a packed staging buffer and then spread them to their
+ * places.  Segment i copies len[i] bytes from src + src_off[i] to dst[i].
+ * src     : device buffer holding the packed segments.
+ * src_off, len : [n] int64 device arrays; dst : [n] device array of device
+ *           pointers.  Segments must not overlap their destinations.
+ * n       : number of segments (0 launches nothing).
+ * Errors: CSKV_ERR_INVALID_ARG for a null pointer with n > 0 or n < 0.
+ * ------------------------------------------------------------------------ */
+CSKV_API int cskv_copy_segments(const void* src, const int64_t* src_off, void* const* dst, const int64_t* len, int n,
+                                cskv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

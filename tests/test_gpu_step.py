@@ -76,6 +76,29 @@ def test_small_bf16_two_streams_graph_equal_eager():
     assert torch.equal(s1.o_c, s2.o_c) and torch.equal(s1.o_h, s2.o_h)
 
 
+def test_graph_with_host_copies_equals_eager():
+    # capture_io: new queries copied from pinned host memory and both outputs read back, all
+    # inside the step's graph; replayed twice with different queries
+    spec = spec_by_name("ragged_b64").replace(batch=3, len_range=(3000, 20000), heads=64)
+    w = Workload(spec)
+    step, dev = decode_step(w, two_streams=True)
+    qs = [dev["q_c"].clone(), dev["q_c"].flip(1).contiguous()]  # two query sets (heads reversed)
+    h_q = torch.empty(dev["q_c"].shape, dtype=dev["q_c"].dtype, pin_memory=True)
+    h_oc = torch.empty(step.o_c.shape, dtype=step.o_c.dtype, pin_memory=True)
+    h_oh = torch.empty(step.o_h.shape, dtype=step.o_h.dtype, pin_memory=True)
+    views = step.capture_io([(h_q, dev["q_c"])], [(step.o_c, h_oc), (step.o_h, h_oh)])
+    for q in qs:
+        views[0].copy_(q.cpu())
+        step.replay_io()
+        torch.cuda.synchronize()
+        assert int(step.status.item()) == 0
+        got_c, got_h = h_oc.clone(), h_oh.clone()
+        dev["q_c"].copy_(q)
+        step.run()
+        torch.cuda.synchronize()
+        assert torch.equal(got_c, step.o_c.cpu()) and torch.equal(got_h, step.o_h.cpu())
+
+
 def test_b8_ctx64k_full():
     w = Workload(spec_by_name("b8_ctx64k"))
     step, dev = _run_gpu(w, two_streams=True)
