@@ -161,11 +161,13 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) 
 //   M = max(max_s m_s, sink), L = sum_s 2^{m_s - M} l_s + 2^{sink - M},
 //   o = sum_s 2^{m_s - M} acc_s / L,   lse = ln 2 * (M + log2 L).
 // CTA (block of kCombineDims output dimensions, query); thread (head h, split group g), group g
-// taking splits g, g + kCombineGroups, ...  Two passes with independent loads (so many are in
-// flight at once): the max over the splits' m, merged across groups in shared memory, then the
-// weighted sums of l and acc under that common max, summed across groups.
+// taking splits g, g + kCombineGroups, ...  With few splits every load is issued at once and
+// each group folds its splits under its own max; otherwise two passes with independent loads
+// (so many are in flight at once): the max over the splits' m, merged across groups in shared
+// memory, then the weighted sums of l and acc under that common max, summed across groups.
 constexpr int kCombineDims = 2;
 constexpr int kCombineGroups = 4;
+constexpr int kFewSplits = 5;  // splits per group folded in one round of loads
 
 __global__ void __launch_bounds__(128 * kCombineGroups) attn_combine_kernel(AttnParams p) {
   __shared__ float sM[kCombineGroups][128], sL[kCombineGroups][128], sO[kCombineGroups][kCombineDims][128];
@@ -183,6 +185,63 @@ __global__ void __launch_bounds__(128 * kCombineGroups) attn_combine_kernel(Attn
   const size_t sb0 = (size_t)t * p.max_splits;
   const float* mrow = p.part_ml + sb0 * 2 * H + h;  // m of split s at mrow[s * 2H], l at + H
   const float* acc = p.part_acc + sb0 * kHeadDim * H + (size_t)j0 * H + h;
+  if (S <= kFewSplits * kCombineGroups) {
+    // ---- few splits (decode): one round of loads; group g folds its <= kFewSplits splits under its
+    //      own max, then thread g = 0 rescales the groups to the common max
+    float mv[kFewSplits], lv[kFewSplits], av[kFewSplits][kCombineDims];
+#pragma unroll
+    for (int i = 0; i < kFewSplits; ++i) {
+      const int s = g + kCombineGroups * i;
+      const bool ok = h < H && s < S;
+      mv[i] = ok ? __ldg(mrow + (size_t)s * 2 * H) : -INFINITY;
+      lv[i] = ok ? __ldg(mrow + (size_t)s * 2 * H + H) : 0.f;
+#pragma unroll
+      for (int jj = 0; jj < kCombineDims; ++jj)
+        av[i][jj] = ok ? __ldg(acc + (size_t)s * kHeadDim * H + (size_t)jj * H) : 0.f;
+    }
+    float Mg = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kFewSplits; ++i) Mg = fmaxf(Mg, mv[i]);
+    float Lg = 0.f, og[kCombineDims] = {};
+    if (Mg != -INFINITY) {
+#pragma unroll
+      for (int i = 0; i < kFewSplits; ++i)
+        if (mv[i] != -INFINITY) {
+          const float f = exp2f(mv[i] - Mg);
+          Lg = fmaf(lv[i], f, Lg);
+#pragma unroll
+          for (int jj = 0; jj < kCombineDims; ++jj) og[jj] = fmaf(av[i][jj], f, og[jj]);
+        }
+    }
+    sM[g][h] = Mg;
+    sL[g][h] = Lg;
+#pragma unroll
+    for (int jj = 0; jj < kCombineDims; ++jj) sO[g][jj][h] = og[jj];
+    __syncthreads();
+    if (g != 0 || h >= H) return;
+    const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+    float Mt = sk;
+#pragma unroll
+    for (int gg = 0; gg < kCombineGroups; ++gg) Mt = fmaxf(Mt, sM[gg][h]);
+    float Lt = 0.f, ot[kCombineDims] = {};
+    if (Mt != -INFINITY) {
+      Lt = p.sink ? exp2f(sk - Mt) : 0.f;
+#pragma unroll
+      for (int gg = 0; gg < kCombineGroups; ++gg) {
+        if (sM[gg][h] == -INFINITY) continue;
+        const float f = exp2f(sM[gg][h] - Mt);
+        Lt = fmaf(sL[gg][h], f, Lt);
+#pragma unroll
+        for (int jj = 0; jj < kCombineDims; ++jj) ot[jj] = fmaf(sO[gg][jj][h], f, ot[jj]);
+      }
+    }
+    const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+    float* dst = p.out + ((size_t)t * H + h) * kHeadDim + j0;
+#pragma unroll
+    for (int jj = 0; jj < kCombineDims; ++jj) dst[jj] = ot[jj] * inv;
+    if (j0 == 0 && p.lse) p.lse[(size_t)t * H + h] = Lt > 0.f ? (Mt + log2f(Lt)) * 0.69314718055994531f : -INFINITY;
+    return;
+  }
   // ---- pass 1: M = max over all splits of m (log2 units)
   float M = -INFINITY;
   if (h < H) {
@@ -270,8 +329,11 @@ int attn_rows_per_split(int mode, int T, int k, int window, int64_t max_entries,
 int attn_tc_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms) {
   const int64_t rows_max = (mode == CSKV_CSA ? (int64_t)k : max_entries) + window;
   int64_t R = (rows_max * (int64_t)T + sms - 1) / sms;
-  R = (R + 127) / 128 * 128;
-  if (R < 128) R = 128;
+  // CSA splits may be a half chunk (64 rows): the few CTAs of a decode query then finish
+  // sooner; HCA splits stay whole chunks (their count is already large)
+  const int64_t g = mode == CSKV_CSA ? 64 : 128;
+  R = (R + g - 1) / g * g;
+  if (R < g) R = g;
   if (R > 1024) R = 1024;
   return (int)R;
 }
