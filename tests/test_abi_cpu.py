@@ -115,3 +115,15 @@ def test_attention_validation(lib):
     assert call(H=129) == _lib.ERR_INVALID_ARG
     assert call(idx=nul) == _lib.ERR_INVALID_ARG
     assert call(T=0) == _lib.OK
+
+
+def test_copy_segments_validation(lib):
+    # nothing is launched for these (no GPU needed): bad counts and missing arrays are
+    # refused on the host, an empty list is a no-op
+    nul = None
+    assert lib.cskv_copy_segments(_p(), _p(), _p(), _p(), -1, nul) == _lib.ERR_INVALID_ARG
+    assert lib.cskv_copy_segments(nul, _p(), _p(), _p(), 3, nul) == _lib.ERR_INVALID_ARG
+    assert lib.cskv_copy_segments(_p(), nul, _p(), _p(), 3, nul) == _lib.ERR_INVALID_ARG
+    assert lib.cskv_copy_segments(_p(), _p(), nul, _p(), 3, nul) == _lib.ERR_INVALID_ARG
+    assert lib.cskv_copy_segments(_p(), _p(), _p(), nul, 3, nul) == _lib.ERR_INVALID_ARG
+    assert lib.cskv_copy_segments(nul, nul, nul, nul, 0, nul) == _lib.OK
