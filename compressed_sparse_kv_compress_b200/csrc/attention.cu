@@ -330,8 +330,9 @@ int attn_tc_rows_per_split(int mode, int T, int k, int window, int64_t max_entri
   const int64_t rows_max = (mode == CSKV_CSA ? (int64_t)k : max_entries) + window;
   int64_t R = (rows_max * (int64_t)T + sms - 1) / sms;
   // CSA splits may be a half chunk (64 rows): the few CTAs of a decode query then finish
-  // sooner; HCA splits stay whole chunks (their count is already large)
-  const int64_t g = mode == CSKV_CSA ? 64 : 128;
+  // sooner.  HCA splits are two chunks at least: fewer, longer CTAs beside the indexer (the
+  // HCA layer runs in its shadow) and half the partials to merge.
+  const int64_t g = mode == CSKV_CSA ? 64 : 256;
   R = (R + g - 1) / g * g;
   if (R < g) R = g;
   if (R > 1024) R = 1024;

@@ -979,6 +979,20 @@ __global__ void __maxnreg__(88) lindex_topk_kernel(IdxParams p) {
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ IdxShared S;
   pdl_launch_dependents();  // the kernel after the indexer may start its set-up now
+  // While the previous kernel finishes: warm L2 with the lines the plan and the first tile
+  // need (the query's position, sequence and offsets, its indexer vectors).  Prefetches only
+  // move lines into L2, which stays coherent with the writes of the kernel being waited for.
+  if (blockIdx.x == 0 && !p.scores) {
+    const int t0 = p.t_begin;
+    const int lane = threadIdx.x;
+    if (lane == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_seq + t0));
+    if (lane == 1) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_pos + t0));
+    if (lane == 2) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.ent_off));
+    if (lane == 3 && p.q_scale) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_scale + (size_t)t0 * p.Hi));
+    const size_t qbytes = (size_t)p.Hi * p.Di * (SRC == kSrcFp8 ? 1 : 4);
+    for (size_t off = (size_t)(lane >= 4 ? lane - 4 : 0) * 128; lane >= 4 && off < qbytes; off += 124 * 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_idx + (size_t)t0 * qbytes + off));
+  }
   pdl_wait();
   uint8_t* un = dsm;                                              // ring / histogram / candidates
   float* sc = reinterpret_cast<float*>(dsm + idx_union_bytes(KS * 32));  // segment scores
