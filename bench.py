@@ -189,6 +189,51 @@ def oracle_sample(w: Workload, budget_s: float = 12.0, max_queries: int = 64):
                       f"full indexer scan + top-k, CSA and HCA attention), {el:.1f} s"}
 
 
+# ---------------------------------------------------------------------- bulk compression
+def bulk_compress_rate(n: int = 1 << 20, seed: int = 1234, reps: int = 5) -> dict:
+    """Compression of a whole n-token cache in one call per layer (CSA 4:1 two streams, HCA
+    128:1) from seeded rows generated on the device (x ~ N(0,1)/sqrt(128), z ~ N(0,1), bf16):
+    algorithmic bytes over event time, against the measured copy bandwidth."""
+    from compressed_sparse_kv_compress_b200 import api
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+
+    def rows(scale):
+        return (torch.randn(n, 256, generator=g, device="cuda") * scale).to(torch.bfloat16)
+
+    xa, za, xb, zb, xh, zh = rows(128 ** -0.5), rows(1.0), rows(128 ** -0.5), rows(1.0), rows(128 ** -0.5), rows(1.0)
+    nc, nh = (n + 3) // 4, (n + 127) // 128
+    i64 = dict(dtype=torch.int64, device="cuda")
+    tok_off, csa_off, hca_off = torch.tensor([0, n], **i64), torch.tensor([0, nc], **i64), torch.tensor([0, nh], **i64)
+    out_c = torch.empty(nc, 256, dtype=torch.bfloat16, device="cuda")
+    out_h = torch.empty(nh, 256, dtype=torch.bfloat16, device="cuda")
+    calls = {
+        "csa": (lambda: api.csa_compress(xa, za, xb, zb, tok_off, csa_off, out_c, max_blocks=nc),
+                4 * n * 512 + nc * 512),
+        "hca": (lambda: api.hca_compress(xh, zh, tok_off, hca_off, out_h, max_blocks=nh), 2 * n * 512 + nh * 512),
+    }
+    hbm, _ = peaks()
+    res = {"n_tokens": n, "data": "seeded normal rows generated on the device"}
+    for name, (fn, nbytes) in calls.items():
+        for _ in range(2):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) * 1e3 / reps
+        res[f"{name}_us"] = us
+        res[f"{name}_gbs"] = nbytes / (us * 1e-6) / 1e9
+        res[f"{name}_frac_of_measured_hbm"] = res[f"{name}_gbs"] / hbm
+        res[f"{name}_bytes"] = nbytes
+    del xa, za, xb, zb, xh, zh, out_c, out_h
+    torch.cuda.empty_cache()
+    return res
+
+
 # ---------------------------------------------------------------------- distributed
 def dist_setup():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -429,6 +474,8 @@ def run_cskv(args, ws, rank, local):
         "gpu_launches": int(launches_per_step) * args.steps,
         "clocks": clk,
     }
+    if rank == 0 and ws == 1 and not args.no_bulk:
+        line["bulk_compress"] = bulk_compress_rate()
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(w, budget_s=args.ref_budget, max_queries=10000)
     if rank == 0:
@@ -447,6 +494,7 @@ def main():
     ap.add_argument("--one-stream", action="store_true")
     ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bulk", action="store_true", help="skip the whole-cache compression figures")
     ap.add_argument("--ref-budget", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -81,6 +81,7 @@ __device__ __forceinline__ SeqRange seq_range(int b, int ratio, const int64_t* t
 // computes entry first + kCsaWarps * x + w of sequence blockIdx.y.  Small CTAs keep the
 // register footprint low enough to run beside the indexer in a decode step (<= 144 registers).
 constexpr int kCsaWarps = 2;
+constexpr int64_t kCsaGridCtas = 16384;  // grid bound of whole-cache calls (entries loop)
 
 template <typename TI, typename TO, bool kTwo>
 __global__ void __maxnreg__(144) csa_compress_kernel(
@@ -98,58 +99,60 @@ __global__ void __maxnreg__(144) csa_compress_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SeqRange s = seq_range(b, 4, tok_off, tok0, ent_off, first_block, num_blocks);
   if (blockIdx.x == 0 && threadIdx.x == 0 && s.num > max_blocks) flag(st, CSKV_DEV_CAPACITY);
-  const int64_t local = (int64_t)blockIdx.x * kCsaWarps + warp;
-  if (local >= s.num) return;
-  const int64_t i = s.first + local;
-  if (i < 0 || 4 * i >= s.n || i >= s.ent_cap) {
-    if (lane == 0) flag(st, CSKV_DEV_BAD_INDEX);
-    return;
-  }
-  const int64_t tfirst = (kTwo && i >= 1) ? 4 * (i - 1) : 4 * i;
-  if (tfirst < s.t0) {
-    if (lane == 0) flag(st, CSKV_DEV_TAIL_MISSING);
-    return;
-  }
-  const int j0 = lane * 8;
-  Raw8<TI> xr[kC], zr[kC];
-  bool ok[kC];
-#pragma unroll
-  for (int c = 0; c < kC; ++c) {
-    const bool pathA = c < 4;
-    const int64_t t = pathA ? 4 * i + c : 4 * (i - 1) + (c - 4);
-    ok[c] = pathA ? (t < s.n) : (i >= 1);
-    if (ok[c]) {
-      const size_t row = (size_t)(s.row0 + (t - s.t0)) * kRow + j0;
-      xr[c].load((pathA ? xa : xb) + row);
-      zr[c].load((pathA ? za : zb) + row);
+  // warp-strided over the entries (a decode call has a few; a whole-cache call loops)
+  for (int64_t local = (int64_t)blockIdx.x * kCsaWarps + warp; local < s.num && local < max_blocks;
+       local += (int64_t)gridDim.x * kCsaWarps) {
+    const int64_t i = s.first + local;
+    if (i < 0 || 4 * i >= s.n || i >= s.ent_cap) {
+      if (lane == 0) flag(st, CSKV_DEV_BAD_INDEX);
+      continue;
     }
-  }
-  float m[8], den[8], num[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) { m[j] = -INFINITY; den[j] = 0.f; num[j] = 0.f; }
-  float bias[kC][8];
-#pragma unroll
-  for (int c = 0; c < kC; ++c) load_bias8(c < 4 ? ba : bb, c & 3, j0, bias[c]);
-#pragma unroll
-  for (int c = 0; c < kC; ++c)
-    if (ok[c]) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) m[j] = fmaxf(m[j], (zr[c].get(j) + bias[c][j]) * kLog2e);
+    const int64_t tfirst = (kTwo && i >= 1) ? 4 * (i - 1) : 4 * i;
+    if (tfirst < s.t0) {
+      if (lane == 0) flag(st, CSKV_DEV_TAIL_MISSING);
+      continue;
     }
+    const int j0 = lane * 8;
+    Raw8<TI> xr[kC], zr[kC];
+    bool ok[kC];
 #pragma unroll
-  for (int c = 0; c < kC; ++c)
-    if (ok[c]) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float w = exp2f((zr[c].get(j) + bias[c][j]) * kLog2e - m[j]);
-        den[j] += w;
-        num[j] = fmaf(w, xr[c].get(j), num[j]);
+    for (int c = 0; c < kC; ++c) {
+      const bool pathA = c < 4;
+      const int64_t t = pathA ? 4 * i + c : 4 * (i - 1) + (c - 4);
+      ok[c] = pathA ? (t < s.n) : (i >= 1);
+      if (ok[c]) {
+        const size_t row = (size_t)(s.row0 + (t - s.t0)) * kRow + j0;
+        xr[c].load((pathA ? xa : xb) + row);
+        zr[c].load((pathA ? za : zb) + row);
       }
     }
-  float o[8];
+    float m[8], den[8], num[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) o[j] = num[j] / den[j];
-  Vec8<TO>::store(out + (size_t)(s.ent0 + i) * kRow + j0, o);
+    for (int j = 0; j < 8; ++j) { m[j] = -INFINITY; den[j] = 0.f; num[j] = 0.f; }
+    float bias[kC][8];
+#pragma unroll
+    for (int c = 0; c < kC; ++c) load_bias8(c < 4 ? ba : bb, c & 3, j0, bias[c]);
+#pragma unroll
+    for (int c = 0; c < kC; ++c)
+      if (ok[c]) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m[j] = fmaxf(m[j], (zr[c].get(j) + bias[c][j]) * kLog2e);
+      }
+#pragma unroll
+    for (int c = 0; c < kC; ++c)
+      if (ok[c]) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float w = exp2f((zr[c].get(j) + bias[c][j]) * kLog2e - m[j]);
+          den[j] += w;
+          num[j] = fmaf(w, xr[c].get(j), num[j]);
+        }
+      }
+    float o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] = num[j] / den[j];
+    Vec8<TO>::store(out + (size_t)(s.ent0 + i) * kRow + j0, o);
+  }
 }
 
 // ------------------------------------------------------------------ HCA
@@ -161,6 +164,7 @@ __global__ void __maxnreg__(144) csa_compress_kernel(
 // 16 lanes that share dimensions, then shared memory across the 4 warps.  Many small CTAs
 // keep the latency of one entry short and fit beside the indexer's CTAs.
 constexpr int kHcaSlices = 16;
+constexpr int64_t kHcaGridEntries = 1024;  // grid bound of whole-cache calls (entries loop)
 constexpr int kHcaThreads = 128;
 
 template <typename T>
@@ -276,7 +280,9 @@ static cudaError_t launch_csa_t(const void* xa, const void* za, const void* xb, 
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
                                 void* out, int* st, cudaStream_t stream) {
-  dim3 grid((unsigned)((max_blocks + kCsaWarps - 1) / kCsaWarps), (unsigned)batch);
+  // a whole-cache call runs a bounded grid whose warps loop over the entries
+  const int64_t ctas = (max_blocks + kCsaWarps - 1) / kCsaWarps;
+  dim3 grid((unsigned)(ctas < kCsaGridCtas ? ctas : kCsaGridCtas), (unsigned)batch);
   cudaError_t e = ensure_smem(xb != nullptr ? csa_compress_kernel<TI, TO, true> : csa_compress_kernel<TI, TO, false>, 0);
   if (e != cudaSuccess) return e;
   if (xb != nullptr)
@@ -314,8 +320,9 @@ static cudaError_t launch_hca_t(const void* x, const void* z, const float* bias,
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
                                 void* out, int* st, cudaStream_t stream) {
-  // slices of one entry are consecutive CTAs; very large bulk calls loop over entries
-  const int64_t entries = max_blocks < (int64_t)(1 << 26) ? max_blocks : (int64_t)(1 << 26);
+  // slices of one entry are consecutive CTAs; whole-cache calls run a bounded grid whose
+  // CTAs loop over the entries (fewer, longer-lived CTAs keep the copy engines of the SMs busy)
+  const int64_t entries = max_blocks < kHcaGridEntries ? max_blocks : kHcaGridEntries;
   dim3 grid((unsigned)(entries * kHcaSlices), (unsigned)batch);
   cudaError_t e = ensure_smem(hca_compress_kernel<TI, TO>, 0);
   if (e != cudaSuccess) return e;

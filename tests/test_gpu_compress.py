@@ -4,6 +4,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import codecs, compress
 from oracle import step as ostep
 from synth import Workload, spec_by_name
 
@@ -45,6 +46,31 @@ def test_bulk_bf16_ragged_with_biases(seed):
             ents, ref = new[(layer, b)]
             got = storage_rows(dev[key])[m[off][b] + ents]
             compress_tol_check(got, ref, "bf16", f"seq{b}/{layer}")
+
+
+def test_bulk_bf16_more_entries_than_one_grid():
+    # 140001 tokens: 35001 CSA entries (more than the 32768 warps of a whole-cache grid) and
+    # 1094 HCA entries (more than its 1024), so warps and CTAs loop over entries; checked on
+    # entries around the loops' wrap points and at both ends
+    spec = spec_by_name("tiny").replace(batch=1, seq_len=(140001,), dtype="bf16", heads=8, biases=True, seed=5)
+    w = Workload(spec)
+    step, dev = decode_step(w)
+    step.bulk_compress(*bulk_bounds(w))
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    m, a = w.meta, np_arrays(w)
+    n = m["n"][0]
+    dec = {k: codecs.decode(a[k], "bf16") for k in ("x_a", "z_a", "x_b", "z_b", "x_h", "z_h")}
+    bias = {k: np.asarray(a[k], dtype=np.float64) for k in ("bias_a", "bias_b", "bias_h")}
+    csa_ents = np.r_[0:3, 32766:32771, 35000:35001]
+    ref = compress.csa_compress(csa_ents, n, dec["x_a"], dec["z_a"], dec["x_b"], dec["z_b"], bias["bias_a"],
+                                bias["bias_b"])
+    got = storage_rows(dev["cmp_c"])[m["csa_off"][0] + csa_ents]
+    compress_tol_check(got, ref, "bf16", "large/csa")
+    hca_ents = np.r_[0:2, 1022:1027, 1093:1094]
+    ref = compress.hca_compress(hca_ents, n, dec["x_h"], dec["z_h"], bias["bias_h"])
+    got = storage_rows(dev["cmp_h"])[m["hca_off"][0] + hca_ents]
+    compress_tol_check(got, ref, "bf16", "large/hca")
 
 
 def test_incremental_tail_compress_touches_only_its_entries():
