@@ -61,11 +61,15 @@ def peaks():
 
 
 def indexer_digest() -> str:
-    """Digest of the sources the indexer kernel is compiled from."""
+    """Digest of the sources the indexer kernel is compiled from, comments and blank lines
+    left out (a comment edit does not change the kernel the counters were taken on)."""
     h = hashlib.sha256()
     for f in INDEXER_SOURCES:
-        with open(os.path.join(ROOT, "compressed_sparse_kv_compress_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "compressed_sparse_kv_compress_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update("\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip()).encode())
     return h.hexdigest()[:16]
 
 

@@ -9,10 +9,12 @@
 //        through path B (x_b, z_b + B_b[slot]) -- one joint softmax over <= 8 candidates;
 //   HCA: the 128 tokens of block i (x, z + B_h[slot]).
 //
-// Both kernels are pure HBM streams (every input row is read once, 512 B bf16 per row):
-// lanes own 8 consecutive dimensions, so each warp-wide 16-byte vector load covers one
-// whole 512-byte row, and every candidate's loads are in flight before any arithmetic.
-// Softmax runs in the log2 domain: l2 = (z + b) * log2(e), w = exp2(l2 - max).
+// Both kernels are pure HBM streams (every input row is read once, 512 B bf16 per row) and
+// put every load of a unit of work in flight before any arithmetic.  CSA: a warp per entry,
+// lanes own 8 consecutive dimensions, so each warp-wide 16-byte vector load covers one whole
+// 512-byte row.  HCA: an entry is cut into 16 slices of 16 dimensions, one small CTA each
+// (see below), so one entry's 128 tokens are read by many SMs at once.  Softmax runs in the
+// log2 domain: l2 = (z + b) * log2(e), w = exp2(l2 - max).
 #include "launch.cuh"
 
 namespace cskv {

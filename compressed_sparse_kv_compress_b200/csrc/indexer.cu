@@ -17,15 +17,21 @@
 //    gets one segment, groups sized in proportion to V_t;
 //  * row mode (many queries, prefill): every CTA owns whole queries (group of one)
 //    and loops over them.
-// A segment's scores never leave shared memory.  Selection is a most-significant-digit
-// radix select on the 64-bit key (order-preserving score bits << 32 | ~index), so the
-// selected set is "key >= threshold" and ties resolve to the lower index exactly:
-//  pass 0: 12-bit digit histogram of the group (shared atomics, then global atomics
-//          and one group barrier when the group has several CTAs);
-//  then, if the threshold bin holds <= kCandMax entries, they are compacted to global
-//  memory (second barrier) and every CTA finishes the selection on that small set in
-//  shared memory; otherwise further 10-bit global passes run (rare: massive ties).
-//  Output positions come from per-CTA counts, so the result needs no sort.
+// A segment's scores never leave shared memory.  Keys are 64-bit (order-preserving score
+// bits << 32 | ~index), so a selection "key >= threshold" resolves ties to the lower index
+// exactly.
+//  * a group of one CTA: most-significant-digit radix select in shared memory;
+//  * a group of several CTAs, speculative exchange: every CTA proposes its best keys (the
+//    top bins of a linear histogram of its own scores) into fixed slots and publishes the
+//    best key it kept back; after one group barrier every CTA gathers all slots, finds the
+//    exact k-th proposal T* and, when no CTA kept back a key >= T*, emits its keys >= T* at
+//    positions counted from the lower CTAs' proposals;
+//  * otherwise (winners crowded into a few segments, massive ties) the exact path: a 12-bit
+//    digit histogram of the group (global atomics, group barrier), compaction of the
+//    threshold bin's entries when they fit (second barrier), else further 10-bit global
+//    passes.  Output positions come from per-CTA counts, so the result needs no sort.
+// As kept entries are emitted, their rows of an optional array (the compressed CSA cache that
+// the attention gathers next) are prefetched into L2.
 //
 // Scan of E4M3 keys: a producer warp streams 240-entry tiles (15 KiB at Di = 64) of k_idx into a
 // shared-memory ring with TMA bulk copies; fifteen consumer warps each take 16 entries of
