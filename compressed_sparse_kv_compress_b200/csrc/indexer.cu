@@ -573,11 +573,16 @@ __device__ uint64_t block_max_u64(uint64_t v, IdxShared& S) {
   return m;
 }
 
-// Linear bin (of kBins0) of a score inside [lo, lo + kBins0/scl]; monotone in s.
-__device__ __forceinline__ unsigned lin_bin4k(float s, float lo, float scl) {
-  const float f = (s - lo) * scl;
-  return f <= 0.f ? 0u : (f >= (float)(kBins0 - 1) ? (unsigned)(kBins0 - 1) : (unsigned)f);
+// Bin (of kBins0) of a key by its score bits above the smallest proposal's: the score key
+// minus the lowest one, shifted so that the range fits.  Monotone in the key; for scores of
+// one sign the bins are about uniform in log(score), so a few outlying large scores (planted
+// or real) do not crowd every other proposal into a handful of bins.
+__device__ __forceinline__ unsigned key_bin4k(uint64_t c, uint32_t kmin, int shift) {
+  const uint32_t d = (uint32_t)(c >> 32) - kmin;
+  const uint32_t b = d >> shift;
+  return b < (uint32_t)kBins0 ? b : (uint32_t)(kBins0 - 1);
 }
+
 
 // Linear bin of a score inside [lo, lo + 1024/scl]; monotone in s.
 __device__ __forceinline__ unsigned lin_bin(float s, float lo, float scl) {
@@ -750,11 +755,14 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
     int nprop;
     block_minmax(mn, mx, S, qmn, qmx, cnt, &nprop);  // its barriers also publish cands[]
     if (nprop >= keff) {  // group-uniform: every CTA gathered the same slots
-      // -- exact k-th best proposal: linear histogram, then rank inside the threshold bin
-      const float qscl = qmx > qmn ? (float)kBins0 / (qmx - qmn) : 0.f;
+      // -- exact k-th best proposal: histogram over the proposals' score keys, then rank
+      //    inside the threshold bin
+      const uint32_t kmin = score_key(qmn), krange = score_key(qmx) - kmin;
+      int shift = 0;
+      while (shift < 32 && (krange >> shift) >= (uint32_t)kBins0) ++shift;
       for (unsigned i = threadIdx.x; i < total; i += kIdxThreads) {
         const uint64_t c = cands[i];
-        if (c != 0ull) atomicAdd(&hist[lin_bin4k(key_score(c), qmn, qscl)], 1u);
+        if (c != 0ull) atomicAdd(&hist[key_bin4k(c, kmin, shift)], 1u);
       }
       if (threadIdx.x == 0) S.ubuf[1] = 0u;
       __syncthreads();
@@ -766,7 +774,7 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       const unsigned bin_cap = (unsigned)kAuxKeys;
       for (unsigned i = threadIdx.x; i < total; i += kIdxThreads) {
         const uint64_t c = cands[i];
-        if (c != 0ull && lin_bin4k(key_score(c), qmn, qscl) == x.bin) {
+        if (c != 0ull && key_bin4k(c, kmin, shift) == x.bin) {
           const unsigned sl = atomicAdd(&S.ubuf[1], 1u);
           if (sl < bin_cap) bin_keys[sl] = c;
         }
