@@ -431,8 +431,7 @@ def run_cskv(args, ws, rank, local):
             add(t["k_idx"][e:e + 1])
             if t.get("k_scale") is not None:
                 add(t["k_scale"][e:e + 1])
-        outs = [(st.o_c, torch.empty(st.o_c.shape, dtype=st.o_c.dtype, pin_memory=True)),
-                (st.o_h, torch.empty(st.o_h.shape, dtype=st.o_h.dtype, pin_memory=True))]
+        outs = [(st.o_all, torch.empty(st.o_all.shape, dtype=st.o_all.dtype, pin_memory=True))]  # o_c and o_h
         return pairs, outs
 
     io = [host_pairs(st) for st in steps]

@@ -34,7 +34,8 @@
 // the attention gathers next) are prefetched into L2.
 //
 // Scan of E4M3 keys: a producer warp streams 240-entry tiles (15 KiB at Di = 64) of k_idx into a
-// shared-memory ring with TMA bulk copies; fifteen consumer warps each take 16 entries of
+// shared-memory ring with TMA bulk copies (each fill completes on the stage's mbarrier; the
+// consumers hand a stage back through its release counter); fifteen consumer warps each take 16 entries of
 // a tile and run m16n8k32 E4M3 MMAs (entries x dims) x (dims x 8 heads) with fp32
 // accumulation -- the head dimension fills N = 8 exactly -- then apply scales, ReLU and
 // the head sum in registers.
@@ -242,7 +243,7 @@ __device__ bool group_barrier(QueryWS* ws, unsigned G, int j, int* st, int* sm_f
 // ------------------------------------------------------------------ shared state
 struct IdxShared {
   uint64_t full[12];
-  uint64_t empty[12];
+  unsigned released[12];  // per ring stage: consumer warps done with it, all fills so far
   unsigned red[32];
   float fred[64];
   unsigned long long ured[32];
@@ -255,6 +256,32 @@ struct IdxShared {
   long long plan_V[kMaxSplitQueries];
 };
 
+// ------------------------------------------------------------------ ring stage release
+// A consumer warp releases a ring stage by adding one to the stage's counter (release
+// semantics: its reads of the stage are ordered before the increment).  The producer refills
+// the stage when the counter shows every consumer warp's release of every earlier fill; a
+// plain counter in shared memory can only move when a consumer warp of this CTA moves it.
+__device__ __forceinline__ void release_stage(unsigned* ctr) {
+  asm volatile("red.release.cta.shared::cta.add.u32 [%0], 1;" ::"r"(smem_u32(ctr)) : "memory");
+}
+
+// Waits until *ctr >= target, polling with an acquire load (backing off after a few polls);
+// gives up after about a second of polling (false).  The proxy fence then orders the
+// consumers' reads of the stage before the TMA unit's writes into it.
+__device__ __forceinline__ bool wait_released(unsigned* ctr, unsigned target) {
+  const uint32_t a = smem_u32(ctr);
+  for (long n = 0; n < (1L << 24); ++n) {
+    unsigned v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    if (v >= target) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      return true;
+    }
+    if (n >= 32) __nanosleep(64);
+  }
+  return false;
+}
+
 // ------------------------------------------------------------------ scan: E4M3 via TMA + MMA
 template <int KS, int NTILE>
 __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, int len,
@@ -266,7 +293,7 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], kIdxConsumerWarps);
+      S.released[s] = 0u;
     }
     fence_mbar_init();
   }
@@ -278,9 +305,9 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
     asm volatile("bar.sync 2, %0;" ::"n"(kIdxThreads) : "memory");  // consumers' scale loads issued
     if (lane == 0) {
       int s = 0;
-      unsigned ph = 0;
       for (int it = 0; it < ntiles; ++it) {
-        if (it >= stages && !mbar_wait_bounded(&S.empty[s], ph ^ 1u)) {
+        // the stage is refilled once every consumer warp has released its previous fill
+        if (it >= stages && !wait_released(&S.released[s], (unsigned)(kIdxConsumerWarps * (it / stages)))) {
           flag(p.st, CSKV_DEV_TIMEOUT);
           break;
         }
@@ -288,10 +315,7 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
         const unsigned bytes = (unsigned)(rows * Di);
         mbar_arrive_expect_tx(&S.full[s], bytes);
         tma_bulk_g2s(ring + (size_t)s * kIdxTile * Di, kbase + (size_t)it * kIdxTile * Di, bytes, &S.full[s]);
-        if (++s == stages) {
-          s = 0;
-          ph ^= 1u;
-        }
+        if (++s == stages) s = 0;
       }
     }
   } else {
@@ -356,21 +380,22 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
         ska[kScalePF - 1] = e < len ? (kscale ? __ldg(kscale + e) : 1.f) : 0.f;
         skb[kScalePF - 1] = e + 8 < len ? (kscale ? __ldg(kscale + e + 8) : 1.f) : 0.f;
       }
-      // A fragments of this warp's 16 rows into registers, then the stage goes back to the
-      // producer at once (the arrive orders the loads before the next copy into the stage),
-      // so the refill overlaps the MMAs and the epilogue
-      uint4 ra[KS / 2], rb[KS / 2];
-      if (r0 < rows) {
+      // A fragments of this warp's 16 rows into registers and the MMAs on them; the stage
+      // goes back to the producer only after the MMAs have consumed every lane's fragments
+      // (a warp-synchronous mma.sync cannot issue before all of its source loads have
+      // returned), so the next copy into the stage cannot overwrite data still being read.
+      // The epilogue then overlaps the refill.
+      if (r0 >= rows) {
+        __syncwarp();
+        if (lane == 0) release_stage(&S.released[s]);
+      } else {
+        uint4 ra[KS / 2], rb[KS / 2];
         const uint8_t* tile = ring + (size_t)s * kIdxTile * Di;
 #pragma unroll
         for (int c = 0; c < KS / 2; ++c) {
           ra[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g) * Di + (tq + 4 * c) * 16);
           rb[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g + 8) * Di + (tq + 4 * c) * 16);
         }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.empty[s]);
-      if (r0 < rows) {
         float acc[NTILE][4];
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt) {
@@ -384,6 +409,8 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
                            bq[nt][ks][0], bq[nt][ks][1]);
           }
         }
+        __syncwarp();
+        if (lane == 0) release_stage(&S.released[s]);
         const int e_g = it * kIdxTile + r0 + g, e_g8 = e_g + 8;
         float vg = 0.f, vg8 = 0.f;
 #pragma unroll
@@ -410,10 +437,8 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
   // Every copy issued has completed (each full barrier was waited on), so the ring can be
   // reused and the barriers retired.
   if (threadIdx.x == 0)
-    for (int s = 0; s < stages; ++s) {
+    for (int s = 0; s < stages; ++s)
       asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(&S.full[s])) : "memory");
-      asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(&S.empty[s])) : "memory");
-    }
   __syncthreads();
 }
 

@@ -41,8 +41,9 @@ class DecodeStep:
         self.T, self.H = T, H
         self.idx = torch.empty(T, self.k, dtype=torch.int32, device=dev)
         self.score = torch.empty(T, self.k, dtype=torch.float32, device=dev)
-        self.o_c = torch.empty(T, H, 128, dtype=torch.float32, device=dev)
-        self.o_h = torch.empty_like(self.o_c)
+        # both layers' outputs in one buffer, so a read-back is a single copy
+        self.o_all = torch.empty(2, T, H, 128, dtype=torch.float32, device=dev)
+        self.o_c, self.o_h = self.o_all[0], self.o_all[1]
         self.lse_c = torch.empty(T, H, dtype=torch.float32, device=dev)
         self.lse_h = torch.empty_like(self.lse_c)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)

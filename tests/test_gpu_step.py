@@ -124,3 +124,39 @@ def test_prefill_chunk_full_sampled():
     w = Workload(spec_by_name("prefill_4k_at_128k"))
     step, dev = _run_gpu(w)
     _check(w, step, dev, [0, 1, 2, 3, 1001, 2048, 4094, 4095])
+
+
+def _issue_layers(step, order):
+    main = torch.cuda.current_stream()
+    step.side.wait_stream(main)
+    if order == "csa_first":
+        step.csa_layer(main)
+        step.hca_layer(step.side)
+    else:
+        step.hca_layer(step.side)
+        step.csa_layer(main)
+    main.wait_stream(step.side)
+
+
+def test_ragged_b64_selection_stable_beside_hca_layer():
+    # The HCA layer's kernels share the SMs with the indexer when it runs on a second stream,
+    # issued before or after the CSA layer.  Every repetition must select exactly what a
+    # one-stream run selects (the selection is deterministic), and that run must match the
+    # oracle on sampled queries.
+    w = Workload(spec_by_name("ragged_b64"))
+    m, a = w.meta, np_arrays(w)
+    step, dev = decode_step(w)
+    step.run()
+    torch.cuda.synchronize()
+    ref = step.idx.clone()
+    for t in (5, 36, 42, 54):
+        check_selection(ref[t].cpu().numpy(), ostep.query_scores(m, a, dtypes(w), t), m["k"], f"query {t}")
+    step2, _ = decode_step(w, two_streams=True)
+    for order in ("csa_first", "hca_first", "csa_first", "csa_first"):
+        for rep in range(3):
+            step2.idx.fill_(-2)
+            _issue_layers(step2, order)
+            torch.cuda.synchronize()
+            assert int(step2.status.item()) == 0
+            bad = (step2.idx != ref).any(dim=1).nonzero().flatten().tolist()
+            assert not bad, f"{order} repetition {rep}: queries {bad} select differently"
