@@ -238,6 +238,16 @@ def bulk_compress_rate(n: int = 1 << 20, seed: int = 1234, reps: int = 5) -> dic
     return res
 
 
+def combined_rate(bulk: dict, step_bytes: float, step_ms: float, hbm: float) -> dict:
+    """Bytes and time of building the whole cache (both compressions) plus one decode step,
+    summed: the figure across compress + index/top-k + attention together, beside the two
+    it combines."""
+    nbytes = bulk["csa_bytes"] + bulk["hca_bytes"] + step_bytes
+    us = bulk["csa_us"] + bulk["hca_us"] + step_ms * 1e3
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"bytes": nbytes, "us": us, "gbs": gbs, "frac_of_measured_hbm": gbs / hbm}
+
+
 # ---------------------------------------------------------------------- distributed
 def dist_setup():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -479,6 +489,7 @@ def run_cskv(args, ws, rank, local):
     }
     if rank == 0 and ws == 1 and not args.no_bulk:
         line["bulk_compress"] = bulk_compress_rate()
+        line["bulk_compress"]["combined_with_one_step"] = combined_rate(line["bulk_compress"], by["total"], ms, hbm)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(w, budget_s=args.ref_budget, max_queries=10000)
     if rank == 0:

@@ -85,3 +85,12 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_combined_rate_sums_bytes_and_times():
+    bulk = {"csa_bytes": 2.0e9, "csa_us": 400.0, "hca_bytes": 1.0e9, "hca_us": 200.0}
+    c = bench.combined_rate(bulk, 23.0e6, 0.05, 6538.3)
+    assert c["bytes"] == pytest.approx(3.023e9)
+    assert c["us"] == pytest.approx(650.0)
+    assert c["gbs"] == pytest.approx(3.023e9 / 650e-6 / 1e9)
+    assert c["frac_of_measured_hbm"] == pytest.approx(c["gbs"] / 6538.3)
