@@ -61,6 +61,25 @@ def e4m3_decode(codes: np.ndarray) -> np.ndarray:
     return sign * mag
 
 
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """float64 -> uint8 OCP E4M3 codes: the nearest finite E4M3 value, ties to the even
+    code (the one whose mantissa's last bit is 0), magnitudes above 448 saturating to 448;
+    the sign is kept, zero results included (-0 -> 0x80); NaN -> 0x7F.
+
+    The positive finite values are those of codes 0x00..0x7E, ascending with the code, so
+    the encoding is a nearest-neighbour search in that table."""
+    x = np.asarray(x, dtype=np.float64)
+    table = e4m3_decode(np.arange(0x7F))            # 0, 2^-9, ..., 448 (ascending)
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.clip(np.searchsorted(table, a, side="left"), 0, 0x7E)   # first value >= a
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - table[lo], table[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    code = np.where(np.signbit(x), code | np.uint8(0x80), code).astype(np.uint8)
+    return np.where(np.isnan(x), np.uint8(0x7F), code).astype(np.uint8)
+
+
 def decode(arr: np.ndarray | None, dtype: str) -> np.ndarray | None:
     """Storage array -> float64.  dtype in {'bf16', 'f32', 'fp8'}."""
     if arr is None:

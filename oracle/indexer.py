@@ -24,13 +24,27 @@ Readings taken where the pages leave the form open:
   lower entry index.  The selected set is returned in ascending index order
   and padded with -1 to length k.
 
+Entry keys from per-token keys ([TR] §4.2: the indexer's keys are projected per
+token, then pooled with a 1-D pool whose kernel and stride are the block size, before
+the scores): readings taken --
+* the pool is the mean over the block's tokens (a partial last block: over the tokens
+  it has), block size 4, the CSA ratio;
+* the entry key is then stored as E4M3 codes with one fp32 scale per entry,
+  scale = amax / 448 (1 when the key is all zeros), code = E4M3(key / scale).
+  The codes are integers decided by floating point, so this step is computed in the
+  precision of the kernel that also produces them: fp32, summing the tokens in order
+  and dividing by their count, then one fp32 division per element.
+
 Parity: pinned (worked (8, -7) example, block-24 causal example, brute-force
-enumeration of k-subsets on tiny inputs, ties).
+enumeration of k-subsets on tiny inputs, ties; pooling: identical tokens, partial
+blocks, mean linearity; the E4M3 codec against the OFP8 values and torch's cast).
 """
 
 from __future__ import annotations
 
 import numpy as np
+
+from oracle import codecs
 
 
 def visible_entries(p: int, ratio: int) -> int:
@@ -81,3 +95,33 @@ def kth_score(scores: np.ndarray, k: int) -> float:
     if kk == 0:
         return -np.inf
     return float(np.asarray(scores, dtype=np.float64)[topk_order(scores)[kk - 1]])
+
+
+E4M3_MAX = 448.0
+
+
+def pool_keys(k_tok: np.ndarray, ratio: int = 4) -> np.ndarray:
+    """Per-token keys [n, Di] (values exactly representable in fp32) -> entry keys
+    [ceil(n/ratio), Di] float32: the mean of each block's tokens, summed in token order
+    in fp32 and divided by the block's token count in fp32."""
+    k = np.asarray(k_tok, dtype=np.float32)
+    n = k.shape[0]
+    out = np.zeros(((n + ratio - 1) // ratio, k.shape[1]), dtype=np.float32)
+    for i in range(out.shape[0]):
+        rows = k[ratio * i: min(n, ratio * (i + 1))]
+        acc = rows[0].copy()
+        for r in rows[1:]:
+            acc = (acc + r).astype(np.float32)
+        out[i] = (acc / np.float32(len(rows))).astype(np.float32)
+    return out
+
+
+def quantize_keys(keys: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Entry keys [V, Di] float32 -> (E4M3 codes [V, Di] uint8, fp32 scales [V]):
+    scale = amax / 448 in fp32 (1 for an all-zero key), code = E4M3(key / scale) with the
+    division in fp32."""
+    k = np.asarray(keys, dtype=np.float32)
+    amax = np.max(np.abs(k), axis=1)
+    scale = np.where(amax > 0, (amax / np.float32(E4M3_MAX)).astype(np.float32), np.float32(1.0)).astype(np.float32)
+    v = (k / scale[:, None]).astype(np.float32)
+    return codecs.e4m3_encode(v.astype(np.float64)), scale

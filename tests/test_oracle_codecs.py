@@ -64,3 +64,47 @@ def test_bf16_encode_rounds_doubles_once():
     got = codecs.bf16_decode(codecs.bf16_encode(x))
     assert got[0] == 1.0 + 2.0 ** -7
     assert got[1] == 1.0
+
+
+def test_e4m3_encode_spec_values_and_nan():
+    g = json.load(open(os.path.join(GOLD, "e4m3_values.json")))
+    for code, val in g["codes"].items():
+        assert codecs.e4m3_encode(np.array([val]))[0] == int(code, 16), code
+    assert codecs.e4m3_encode(np.array([np.nan]))[0] == 0x7F
+
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = codecs.e4m3_decode(codes)
+    fin = ~np.isnan(vals)
+    assert np.array_equal(codecs.e4m3_encode(vals[fin]), codes[fin])
+
+
+def test_e4m3_encode_ties_go_to_the_even_code():
+    vals = codecs.e4m3_decode(np.arange(0x7F))
+    mids = (vals[:-1] + vals[1:]) / 2           # exactly halfway between neighbours
+    got = codecs.e4m3_encode(mids)
+    lo = np.arange(0x7E)
+    assert np.array_equal(got, np.where(lo % 2 == 0, lo, lo + 1))
+    # just off the midpoint the nearer neighbour wins
+    eps = (vals[1:] - vals[:-1]) / 64
+    assert np.array_equal(codecs.e4m3_encode(mids - eps), lo)
+    assert np.array_equal(codecs.e4m3_encode(mids + eps), lo + 1)
+
+
+def test_e4m3_encode_saturates_and_keeps_sign():
+    big = np.array([448.0, 449.0, 464.0, 480.0, 1e6, np.inf])
+    assert np.all(codecs.e4m3_encode(big) == 0x7E)
+    assert np.all(codecs.e4m3_encode(-big) == 0xFE)
+    assert codecs.e4m3_encode(np.array([-1e-9]))[0] == 0x80   # rounds to -0
+    assert codecs.e4m3_encode(np.array([2.0 ** -10]))[0] == 0x00  # half of the least subnormal: even (0)
+    assert codecs.e4m3_encode(np.array([1.5 * 2.0 ** -9]))[0] == 0x02  # between 1 and 2 subnormal steps: even
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_e4m3_encode_matches_torch_cast_in_range(seed):
+    rng = np.random.default_rng(seed)
+    x = np.concatenate([rng.normal(0, 50, 50000), rng.normal(0, 0.01, 50000)]).astype(np.float32)
+    x = np.clip(x, -448, 448)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codecs.e4m3_encode(x.astype(np.float64)), ref)

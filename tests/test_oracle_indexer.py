@@ -8,7 +8,7 @@ import os
 import numpy as np
 import pytest
 
-from oracle import attention, indexer
+from oracle import attention, codecs, indexer
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -102,3 +102,46 @@ def test_topk_padding_and_order():
     # ties at the threshold go to the lower index
     t = np.array([1.0, 0.0, 1.0, 1.0, 2.0])
     assert list(indexer.topk_select(t, 3)) == [0, 2, 4]
+
+
+def test_pool_keys_means_blocks_including_a_partial_one():
+    # integer-valued tokens: every mean below is exact in fp32
+    k = np.array([[1, -2], [2, 0], [3, 4], [6, 2],       # entry 0: mean (3, 1)
+                  [5, 5], [5, 5], [5, 5], [5, 5],         # entry 1: identical tokens
+                  [8, -8], [0, 2]], dtype=np.float32)     # entry 2: partial, two tokens
+    got = indexer.pool_keys(k, 4)
+    assert got.dtype == np.float32 and got.shape == (3, 2)
+    assert np.array_equal(got, np.array([[3, 1], [5, 5], [4, -3]], dtype=np.float32))
+
+
+def test_pool_keys_is_linear_and_sums_in_token_order():
+    rng = np.random.default_rng(5)
+    a = rng.standard_normal((12, 16)).astype(np.float32)
+    # scaling by 2 is exact in fp32, so pooling commutes with it bit for bit
+    assert np.array_equal(indexer.pool_keys(2 * a), 2 * indexer.pool_keys(a))
+    # fp32 sum in token order, then one division
+    blk = a[4:8]
+    want = ((((blk[0] + blk[1]).astype(np.float32) + blk[2]).astype(np.float32) + blk[3]).astype(np.float32)
+            / np.float32(4)).astype(np.float32)
+    assert np.array_equal(indexer.pool_keys(a)[1], want)
+    assert np.allclose(indexer.pool_keys(a), a.reshape(3, 4, 16).mean(axis=1), rtol=1e-6, atol=1e-6)
+
+
+def test_quantize_keys_scale_and_error_bound():
+    rng = np.random.default_rng(6)
+    keys = rng.standard_normal((200, 64)).astype(np.float32)
+    keys[7] = 0.0
+    codes, scale = indexer.quantize_keys(keys)
+    assert codes.dtype == np.uint8 and scale.dtype == np.float32
+    assert scale[7] == 1.0 and np.all(codes[7] == 0)
+    # the largest magnitude of every non-zero key lands on +-448 (code 0x7E / 0xFE)
+    for i in (0, 1, 100):
+        j = int(np.argmax(np.abs(keys[i])))
+        assert codes[i, j] & 0x7F == 0x7E
+        assert scale[i] == np.float32(np.abs(keys[i]).max() / np.float32(448))
+    # decoded * scale is within half an E4M3 step: relative 2^-4 for normals, and an
+    # absolute 2^-10 * scale below the smallest normal
+    deq = codecs.e4m3_decode(codes) * scale[:, None].astype(np.float64)
+    err = np.abs(deq - keys.astype(np.float64))
+    bound = np.maximum(np.abs(keys) * 2.0 ** -4, 2.0 ** -10 * scale[:, None])
+    assert np.all(err <= bound * (1 + 1e-6))
