@@ -32,6 +32,7 @@ SIGNATURES = {
     "cskv_copy_segments": (_i32, [_p, _p, _p, _p, _i32, _p]),
     "csa_compress": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p, _p, _p]),
     "hca_compress": (_i32, [_p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p, _p, _p]),
+    "lindex_pool_keys": (_i32, [_p, _i32, _i32, _p, _p, _i32, _p, _p, _p, _i64, _p, _p, _p, _p]),
     "lindex_score_topk": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _i32, _i32, _i32, _i32, _i32, _i64,
                                  _p, _p, _p, _i64, _p, _sz, _p, _p]),
     "lindex_topk_from_scores": (_i32, [_p, _i64, _p, _i32, _i32, _i64, _p, _p, _p, _sz, _p, _p]),

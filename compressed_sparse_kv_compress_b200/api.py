@@ -57,6 +57,19 @@ def hca_compress(x, z, tok_off, ent_off, out, *, max_blocks, bias=None, tok0=Non
     return out
 
 
+def lindex_pool_keys(k_tok, tok_off, ent_off, out_codes, out_scale, *, max_blocks, tok0=None, first_block=None,
+                     num_blocks=None, dev_status=None, stream=None):
+    """Entry keys of the indexer from per-token keys k_tok [rows, Di] (fp32 or bf16): the mean
+    of each 4-token block as E4M3 codes (out_codes [*, Di] uint8) with one fp32 scale per
+    entry (out_scale [*])."""
+    lib = _lib.load()
+    st = lib.lindex_pool_keys(_ptr(k_tok), _dt(k_tok), int(k_tok.shape[-1]), _ptr(tok_off), _ptr(tok0),
+                              tok_off.numel() - 1, _ptr(ent_off), _ptr(first_block), _ptr(num_blocks),
+                              int(max_blocks), _ptr(out_codes), _ptr(out_scale), _ptr(dev_status), _stream(stream))
+    _lib.check("lindex_pool_keys", st)
+    return out_codes, out_scale
+
+
 def lindex_workspace_size(T: int, k: int, max_entries: int) -> int:
     return int(_lib.load().lindex_workspace_size(int(T), int(k), int(max_entries)))
 

@@ -107,6 +107,23 @@ int csa_compress(const void* x_a, const void* z_a, const void* x_b, const void* 
                                            dev_status, (cudaStream_t)stream));
 }
 
+int lindex_pool_keys(const void* k_tok, int in_dtype, int Di, const int64_t* tok_off, const int64_t* tok0,
+                     int batch, const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
+                     int64_t max_blocks, uint8_t* out_codes, float* out_scale, int* dev_status,
+                     cskv_stream_t stream) {
+  if (!k_tok || !tok_off || !ent_off || !out_codes || !out_scale) return CSKV_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || max_blocks < 0 || max_blocks > (1LL << 31) - 1) return CSKV_ERR_INVALID_ARG;
+  if (in_dtype != CSKV_F32 && in_dtype != CSKV_BF16)
+    return in_dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+  if (Di != 64 && Di != 128) return Di > 0 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+  if (!aligned16(k_tok) || !aligned16(out_codes) || (reinterpret_cast<uintptr_t>(out_scale) & 3u))
+    return CSKV_ERR_INVALID_ARG;
+  if (max_blocks == 0) return CSKV_OK;
+  return launch_status(launch_pool_keys(k_tok, in_dtype, Di, tok_off, tok0, batch, ent_off, first_block,
+                                        num_blocks, max_blocks, out_codes, out_scale, dev_status,
+                                        (cudaStream_t)stream));
+}
+
 int hca_compress(const void* x, const void* z, const float* bias, const int64_t* tok_off, const int64_t* tok0,
                  int batch, const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
                  int64_t max_blocks, int in_dtype, int out_dtype, void* out, int* dev_status,

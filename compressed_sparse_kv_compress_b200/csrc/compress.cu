@@ -15,6 +15,10 @@
 // 512-byte row.  HCA: an entry is cut into 16 slices of 16 dimensions, one small CTA each
 // (see below), so one entry's 128 tokens are read by many SMs at once.  Softmax runs in the
 // log2 domain: l2 = (z + b) * log2(e), w = exp2(l2 - max).
+//
+// Also here: the indexer's entry keys pooled from per-token keys ([TR] §4.2), a warp per entry.
+#include <cuda_fp8.h>
+
 #include "launch.cuh"
 
 namespace cskv {
@@ -275,6 +279,99 @@ __global__ void __launch_bounds__(kHcaThreads, 8) hca_compress_kernel(
   }
 }
 
+
+// ------------------------------------------------------------------ indexer keys of the entries
+// The Lightning Indexer's keys are projected per token and pooled to one key per CSA block
+// ([TR] §4.2, a 1-D pool with kernel = stride = the block size): the mean over the block's
+// tokens (a partial last block: over the tokens it has), stored as E4M3 codes with one fp32
+// scale per entry, amax / 448 (1 for an all-zero key).  One warp per entry; lane l holds
+// dimensions [l * DPL, l * DPL + DPL).  The codes are integers decided in fp32: tokens summed
+// in order, one division by the count, one division by the scale, then the E4M3 conversion
+// (round to nearest even, saturating to +-448).
+constexpr int kPoolWarps = 4;
+constexpr int64_t kPoolGridCtas = 16384;  // grid bound of whole-cache calls (entries loop)
+
+template <int BYTES>
+struct RawBytes;
+template <>
+struct RawBytes<4> { uint32_t v; };
+template <>
+struct RawBytes<8> { uint2 v; };
+template <>
+struct RawBytes<16> { uint4 v; };
+
+template <typename TI, int DPL>
+__device__ __forceinline__ void load_dims(const TI* p, float (&out)[DPL]) {
+  union {
+    RawBytes<DPL * sizeof(TI)> r;
+    TI e[DPL];
+  } u;
+  u.r = *reinterpret_cast<const RawBytes<DPL * sizeof(TI)>*>(p);
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) {
+    if constexpr (sizeof(TI) == 2)
+      out[j] = __bfloat162float(u.e[j]);
+    else
+      out[j] = u.e[j];
+  }
+}
+
+template <typename TI, int DPL>
+__global__ void __launch_bounds__(32 * kPoolWarps) pool_keys_kernel(
+    const TI* __restrict__ k_tok, const int64_t* __restrict__ tok_off, const int64_t* __restrict__ tok0,
+    const int64_t* __restrict__ ent_off, const int64_t* __restrict__ first_block,
+    const int64_t* __restrict__ num_blocks, int64_t max_blocks, uint8_t* __restrict__ codes,
+    float* __restrict__ scales, int* st) {
+  constexpr int Di = 32 * DPL;
+  pdl_launch_dependents();  // the indexer after it waits for this grid before reading the keys
+  pdl_wait();
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SeqRange s = seq_range(b, 4, tok_off, tok0, ent_off, first_block, num_blocks);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && s.num > max_blocks) flag(st, CSKV_DEV_CAPACITY);
+  for (int64_t local = (int64_t)blockIdx.x * kPoolWarps + warp; local < s.num && local < max_blocks;
+       local += (int64_t)gridDim.x * kPoolWarps) {
+    const int64_t i = s.first + local;
+    if (i < 0 || 4 * i >= s.n || i >= s.ent_cap) {
+      if (lane == 0) flag(st, CSKV_DEV_BAD_INDEX);
+      continue;
+    }
+    if (4 * i < s.t0) {
+      if (lane == 0) flag(st, CSKV_DEV_TAIL_MISSING);
+      continue;
+    }
+    const int cnt = (int)min((int64_t)4, s.n - 4 * i);
+    float v[4][DPL];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      if (c < cnt) load_dims<TI, DPL>(k_tok + (size_t)(s.row0 + (4 * i + c - s.t0)) * Di + lane * DPL, v[c]);
+    float key[DPL];
+    float amax = 0.f;
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) {
+      float acc = v[0][j];
+#pragma unroll
+      for (int c = 1; c < 4; ++c)
+        if (c < cnt) acc = __fadd_rn(acc, v[c][j]);
+      key[j] = __fdiv_rn(acc, (float)cnt);
+      amax = fmaxf(amax, fabsf(key[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    uint32_t packed = 0;
+#pragma unroll
+    for (int j = 0; j < DPL; ++j)
+      packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(key[j], scale), __NV_SATFINITE, __NV_E4M3) << (8 * j);
+    uint8_t* dst = codes + (size_t)(s.ent0 + i) * Di + lane * DPL;
+    if constexpr (DPL == 2)
+      *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+    else
+      *reinterpret_cast<uint32_t*>(dst) = packed;
+    if (lane == 0) scales[s.ent0 + i] = scale;
+  }
+}
+
 // ------------------------------------------------------------------ launchers
 template <typename TI, typename TO>
 static cudaError_t launch_csa_t(const void* xa, const void* za, const void* xb, const void* zb,
@@ -350,6 +447,34 @@ cudaError_t launch_hca_compress(const void* x, const void* z, const float* bias,
                                               max_blocks, out, st, stream);
   return launch_hca_t<float, float>(x, z, bias, tok_off, tok0, batch, ent_off, first, num, max_blocks,
                                     out, st, stream);
+}
+
+template <typename TI, int DPL>
+static cudaError_t launch_pool_t(const void* k_tok, const int64_t* tok_off, const int64_t* tok0, int batch,
+                                 const int64_t* ent_off, const int64_t* first, const int64_t* num,
+                                 int64_t max_blocks, uint8_t* codes, float* scales, int* st, cudaStream_t stream) {
+  const int64_t ctas = (max_blocks + kPoolWarps - 1) / kPoolWarps;
+  dim3 grid((unsigned)(ctas < kPoolGridCtas ? ctas : kPoolGridCtas), (unsigned)batch);
+  cudaError_t e = ensure_smem(pool_keys_kernel<TI, DPL>, 0);
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(pool_keys_kernel<TI, DPL>, grid, dim3(32 * kPoolWarps), 0, stream, (const TI*)k_tok,
+                       tok_off, tok0, ent_off, first, num, max_blocks, codes, scales, st);
+  note_launch();
+  return e;
+}
+
+cudaError_t launch_pool_keys(const void* k_tok, int in_dt, int Di, const int64_t* tok_off, const int64_t* tok0,
+                             int batch, const int64_t* ent_off, const int64_t* first, const int64_t* num,
+                             int64_t max_blocks, uint8_t* codes, float* scales, int* st, cudaStream_t stream) {
+  if (in_dt == CSKV_BF16)
+    return Di == 64 ? launch_pool_t<__nv_bfloat16, 2>(k_tok, tok_off, tok0, batch, ent_off, first, num, max_blocks,
+                                                      codes, scales, st, stream)
+                    : launch_pool_t<__nv_bfloat16, 4>(k_tok, tok_off, tok0, batch, ent_off, first, num, max_blocks,
+                                                      codes, scales, st, stream);
+  return Di == 64 ? launch_pool_t<float, 2>(k_tok, tok_off, tok0, batch, ent_off, first, num, max_blocks, codes,
+                                            scales, st, stream)
+                  : launch_pool_t<float, 4>(k_tok, tok_off, tok0, batch, ent_off, first, num, max_blocks, codes,
+                                            scales, st, stream);
 }
 
 }  // namespace cskv

@@ -120,6 +120,37 @@ CSKV_API int hca_compress(const void* x, const void* z, const float* bias,
                  int* dev_status, cskv_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * lindex_pool_keys -- the indexer's entry keys from per-token keys.
+ *
+ * [TR] §4.2 (LightningIndexer: per-token keys, then a 1-D pool whose kernel and
+ * stride are the block size): entry i of a sequence gets the mean of the
+ * per-token keys of tokens 4i..4i+3 (a partial last block: of the tokens it
+ * has), stored as OCP E4M3 codes with one fp32 scale per entry:
+ *     scale = amax_j |key_j| / 448 (1 for an all-zero key),
+ *     code_j = E4M3(key_j / scale), round to nearest even, saturating to +-448.
+ * fp32 arithmetic: the tokens are summed in order, divided once by their
+ * count, each element divided once by the scale.  The outputs are the k_idx /
+ * k_scale arrays lindex_score_topk reads.
+ *
+ * k_tok              : [rows, Di] in_dtype (CSKV_F32 or CSKV_BF16; CSKV_FP8E4M3
+ *                      is CSKV_ERR_UNSUPPORTED), 16-byte aligned; finite values.
+ * Di                 : 64 or 128 (other positive values: CSKV_ERR_UNSUPPORTED).
+ * tok_off, tok0, batch, ent_off, first_block, num_blocks, max_blocks : as
+ *                      csa_compress (rows of sequence b are its token tail from
+ *                      tok0[b]; entry i goes to row ent_off[b] + i).
+ * out_codes          : [*, Di] uint8 E4M3 codes, 16-byte aligned.
+ * out_scale          : [*] fp32, 4-byte aligned.
+ * Device checks: an entry outside the sequence or its ent_off range sets
+ * CSKV_DEV_BAD_INDEX, one whose tokens start before the provided tail sets
+ * CSKV_DEV_TAIL_MISSING (the entry is skipped), num_blocks above max_blocks
+ * sets CSKV_DEV_CAPACITY.  max_blocks == 0 launches nothing.
+ * ------------------------------------------------------------------------ */
+CSKV_API int lindex_pool_keys(const void* k_tok, int in_dtype, int Di, const int64_t* tok_off,
+                 const int64_t* tok0, int batch, const int64_t* ent_off, const int64_t* first_block,
+                 const int64_t* num_blocks, int64_t max_blocks, uint8_t* out_codes, float* out_scale,
+                 int* dev_status, cskv_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * lindex_score_topk -- Lightning Indexer scan fused with exact top-k.
  *
  * [SW] §六/§七/§十, [TR] §4.2, [AM]: query t (sequence q_seq[t], position

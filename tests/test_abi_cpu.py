@@ -127,3 +127,29 @@ def test_copy_segments_validation(lib):
     assert lib.cskv_copy_segments(_p(), _p(), nul, _p(), 3, nul) == _lib.ERR_INVALID_ARG
     assert lib.cskv_copy_segments(_p(), _p(), _p(), nul, 3, nul) == _lib.ERR_INVALID_ARG
     assert lib.cskv_copy_segments(nul, nul, nul, nul, 0, nul) == _lib.OK
+
+
+def test_pool_keys_validation(lib):
+    nul = None
+    # (k_tok, in_dtype, Di, tok_off, tok0, batch, ent_off, first, num, max_blocks, codes, scale, st, stream)
+    ok_args = [_p(), 1, 64, _p(), nul, 1, _p(), nul, nul, 4, _p(), _p(), nul, nul]
+
+    def call(**kw):
+        a = list(ok_args)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.lindex_pool_keys(*a)
+
+    assert call(a0=nul) == _lib.ERR_INVALID_ARG              # no rows
+    assert call(a10=nul) == _lib.ERR_INVALID_ARG             # no output codes
+    assert call(a11=nul) == _lib.ERR_INVALID_ARG             # no output scales
+    assert call(a1=2) == _lib.ERR_UNSUPPORTED                # fp8 per-token keys
+    assert call(a1=9) == _lib.ERR_INVALID_ARG                # bad dtype enum
+    assert call(a2=96) == _lib.ERR_UNSUPPORTED               # key width not implemented
+    assert call(a2=0) == _lib.ERR_INVALID_ARG
+    assert call(a0=_p(0x1008)) == _lib.ERR_INVALID_ARG       # rows not 16-byte aligned
+    assert call(a10=_p(0x1004)) == _lib.ERR_INVALID_ARG      # codes not 16-byte aligned
+    assert call(a11=_p(0x1002)) == _lib.ERR_INVALID_ARG      # scales not 4-byte aligned
+    assert call(a5=0) == _lib.ERR_INVALID_ARG                # empty batch
+    assert call(a9=-1) == _lib.ERR_INVALID_ARG
+    assert call(a9=0) == _lib.OK                             # nothing to do, nothing launched
