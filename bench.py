@@ -196,7 +196,8 @@ def oracle_sample(w: Workload, budget_s: float = 12.0, max_queries: int = 64):
 # ---------------------------------------------------------------------- bulk compression
 def bulk_compress_rate(n: int = 1 << 20, seed: int = 1234, reps: int = 5) -> dict:
     """Compression of a whole n-token cache in one call per layer (CSA 4:1 two streams, HCA
-    128:1) from seeded rows generated on the device (x ~ N(0,1)/sqrt(128), z ~ N(0,1), bf16):
+    128:1) from seeded rows generated on the device (x ~ N(0,1)/sqrt(128), z ~ N(0,1), bf16),
+    and the pooling of n per-token indexer keys (64 dims, bf16) into E4M3 entry keys:
     algorithmic bytes over event time, against the measured copy bandwidth."""
     from compressed_sparse_kv_compress_b200 import api
     g = torch.Generator(device="cuda")
@@ -207,6 +208,10 @@ def bulk_compress_rate(n: int = 1 << 20, seed: int = 1234, reps: int = 5) -> dic
 
     xa, za, xb, zb, xh, zh = rows(128 ** -0.5), rows(1.0), rows(128 ** -0.5), rows(1.0), rows(128 ** -0.5), rows(1.0)
     nc, nh = (n + 3) // 4, (n + 127) // 128
+    di = 64  # per-token indexer keys -> E4M3 entry keys + scales
+    kt = (torch.randn(n, di, generator=g, device="cuda") * di ** -0.5).to(torch.bfloat16)
+    k_codes = torch.empty(nc, di, dtype=torch.uint8, device="cuda")
+    k_scales = torch.empty(nc, dtype=torch.float32, device="cuda")
     i64 = dict(dtype=torch.int64, device="cuda")
     tok_off, csa_off, hca_off = torch.tensor([0, n], **i64), torch.tensor([0, nc], **i64), torch.tensor([0, nh], **i64)
     out_c = torch.empty(nc, 256, dtype=torch.bfloat16, device="cuda")
@@ -215,6 +220,8 @@ def bulk_compress_rate(n: int = 1 << 20, seed: int = 1234, reps: int = 5) -> dic
         "csa": (lambda: api.csa_compress(xa, za, xb, zb, tok_off, csa_off, out_c, max_blocks=nc),
                 4 * n * 512 + nc * 512),
         "hca": (lambda: api.hca_compress(xh, zh, tok_off, hca_off, out_h, max_blocks=nh), 2 * n * 512 + nh * 512),
+        "key_pool": (lambda: api.lindex_pool_keys(kt, tok_off, csa_off, k_codes, k_scales, max_blocks=nc),
+                     n * di * 2 + nc * (di + 4)),
     }
     hbm, _ = peaks()
     res = {"n_tokens": n, "data": "seeded normal rows generated on the device"}
@@ -233,7 +240,7 @@ def bulk_compress_rate(n: int = 1 << 20, seed: int = 1234, reps: int = 5) -> dic
         res[f"{name}_gbs"] = nbytes / (us * 1e-6) / 1e9
         res[f"{name}_frac_of_measured_hbm"] = res[f"{name}_gbs"] / hbm
         res[f"{name}_bytes"] = nbytes
-    del xa, za, xb, zb, xh, zh, out_c, out_h
+    del xa, za, xb, zb, xh, zh, out_c, out_h, kt, k_codes, k_scales
     torch.cuda.empty_cache()
     return res
 
