@@ -17,11 +17,14 @@ it (cited by page and section in each function):
        计算量降至原来的27%？" (ratios 4:1 / 128:1, top-1024, 128-token window).
 
 All arithmetic is float64 on values decoded exactly from their storage form
-(bf16, fp32, OCP E4M3).  Loops are vectorised with numpy but follow each
-definition term by term; nothing is blocked, fused or reordered beyond it.
+(bf16, fp32, OCP E4M3), with one exception: where floating point decides an
+integer -- the E4M3 codes of pooled indexer keys (indexer.quantize_keys) -- the
+steps are taken in fp32, the precision of the kernel that decides the same codes.
+Loops are vectorised with numpy but follow each definition term by term; nothing
+is blocked, fused or reordered beyond it.
 
 Parity status of each function is stated in its docstring; every function
 here is pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_*.py``.
 """
 
-from . import codecs, compress, indexer, attention, step  # noqa: F401
+from . import codecs, compress, indexer, attention, norm, step  # noqa: F401
