@@ -108,3 +108,74 @@ def test_e4m3_encode_matches_torch_cast_in_range(seed):
     x = np.clip(x, -448, 448)
     ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.array_equal(codecs.e4m3_encode(x.astype(np.float64)), ref)
+
+
+def _mx_gold():
+    return json.load(open(os.path.join(GOLD, "mx_fp4_values.json")))
+
+
+def test_e2m1_and_e8m0_values_from_spec():
+    g = _mx_gold()
+    for code, val in g["e2m1"].items():
+        c = np.array([int(code, 16)], np.uint8)
+        got = codecs.e2m1_decode(c)[0]
+        assert got == val and np.signbit(got) == np.signbit(val), code
+        assert codecs.e2m1_encode(np.array([val]))[0] == int(code, 16), code
+    for code, val in g["e8m0"].items():
+        assert codecs.e8m0_decode(np.array([int(code, 16)]))[0] == val, code
+    assert np.isnan(codecs.e8m0_decode(np.array([int(g["e8m0_nan"], 16)]))[0])
+    assert g["block_size"] == codecs.MX_BLOCK and g["e2m1_emax"] == codecs.E2M1_EMAX
+
+
+def test_e2m1_encode_ties_even_and_saturation():
+    # midpoints between neighbours go to the even code (the value with mantissa bit 0)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    assert list(codecs.e2m1_decode(codecs.e2m1_encode(mids))) == [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0]
+    assert list(codecs.e2m1_decode(codecs.e2m1_encode(-mids))) == [-0.0, -1.0, -1.0, -2.0, -2.0, -4.0, -4.0]
+    assert np.all(codecs.e2m1_encode(np.array([6.0, 6.5, 7.0, 100.0])) == 0x7)
+    assert codecs.e2m1_encode(np.array([-1e-9]))[0] == 0x8
+    # off the midpoints the nearer neighbour wins
+    assert list(codecs.e2m1_decode(codecs.e2m1_encode(np.array([0.26, 2.49, 4.99, 5.01])))) == [0.5, 2.0, 4.0, 6.0]
+
+
+def test_mx_fp4_shared_exponent_and_exact_powers_of_two():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((20, 64)) * np.ldexp(1.0, rng.integers(-20, 20, (20, 1)))
+    codes, scales = codecs.mx_fp4_quantize(x)
+    assert codes.shape == (20, 64) and scales.shape == (20, 2)
+    amax = np.abs(x).reshape(20, 2, 32).max(axis=2)
+    assert np.array_equal(scales.astype(np.int64) - 127, np.floor(np.log2(amax)).astype(np.int64) - 2)
+    # the block maximum lands in [4, 6] times the scale (6 when it saturates)
+    deq = codecs.mx_fp4_decode(codes, scales)
+    top = np.abs(deq).reshape(20, 2, 32).max(axis=2) / codecs.e8m0_decode(scales)
+    assert np.all((top >= 4.0) & (top <= 6.0))
+    # blocks of representable magnitudes times one power of two come back exactly
+    vals = codecs.e2m1_decode(rng.integers(0, 16, (5, 64)))
+    vals[:, 0] = 6.0
+    vals[:, 32] = -4.0
+    y = vals * np.ldexp(1.0, 9)
+    c2, s2 = codecs.mx_fp4_quantize(y)
+    assert np.array_equal(codecs.mx_fp4_decode(c2, s2), y)
+
+
+def test_mx_fp4_error_bound_and_zero_block():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((50, 64))
+    x[3, :32] = 0.0
+    codes, scales = codecs.mx_fp4_quantize(x)
+    assert scales[3, 0] == 0 and np.all(codes[3, :32] == 0)
+    X = np.repeat(codecs.e8m0_decode(scales), 32, axis=1)
+    r = np.abs(x) / X
+    deq = codecs.mx_fp4_decode(codes, scales)
+    # half the E2M1 spacing at the element's magnitude; above 6 the element saturates to 6
+    half = np.where(r < 2, 0.25, np.where(r < 4, 0.5, 1.0)) * X
+    inside = r <= 6
+    assert np.all(np.abs(deq - x)[inside] <= half[inside] * (1 + 1e-12))
+    assert np.all(np.abs(deq[~inside]) == 6 * X[~inside])
+
+
+def test_nibble_packing_order_and_round_trip():
+    c = np.arange(16, dtype=np.uint8)
+    p = codecs.pack_nibbles(c)
+    assert list(p) == [0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE]
+    assert np.array_equal(codecs.unpack_nibbles(p), c)
