@@ -125,10 +125,24 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu: str):
+        self.gpu = gpu  # nvidia-smi's -i selector: the GPU's UUID (or PCI bus id)
         self.proc = None
         self.path = None
+
+    @staticmethod
+    def selector(dev: int) -> str:
+        """The CUDA device's identity in a form nvidia-smi -i accepts whatever the two tools'
+        numbering: its UUID, else its PCI bus id.  (A CUDA index is relative to
+        CUDA_VISIBLE_DEVICES and CUDA's enumeration order, which nvidia-smi does not use.)"""
+        props = torch.cuda.get_device_properties(dev)
+        try:
+            u = str(props.uuid)
+            if u:
+                return u if u.startswith("GPU-") else f"GPU-{u}"
+        except Exception:
+            pass
+        return f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
 
     def start(self):
         try:
@@ -143,7 +157,7 @@ class ClockSampler:
 
     def stop(self) -> dict:
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "gpu": self.gpu}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -166,7 +180,7 @@ class ClockSampler:
                     reasons.add(nm)
         os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "gpu": self.gpu}
 
 
 # ---------------------------------------------------------------------- oracle timing
@@ -395,7 +409,7 @@ def run_cskv(args, ws, rank, local):
             raise RuntimeError(f"device status {int(st.status.item())} during warm-up")
 
     # ---- timed region: K graph replays (replica i mod R)
-    clocks = ClockSampler(torch.cuda.current_device())
+    clocks = ClockSampler(ClockSampler.selector(torch.cuda.current_device()))
     clocks.start()
     time.sleep(0.3)
     barrier(ws)
@@ -463,6 +477,14 @@ def run_cskv(args, ws, rank, local):
         steps[i % R].replay_io()
 
     ms_e2e = timed(e2e_step, args.steps)
+    # the same end-to-end steps by the host's wall clock: synchronised on both sides, so the
+    # figure includes every host-side cost of a replay and of waiting for the read-back
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    for i in range(args.steps):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    wall_us = (time.perf_counter() - w0) * 1e6 / args.steps
     clk = clocks.stop()
 
     ms = reduce_max(ms_local, ws)
@@ -490,7 +512,8 @@ def run_cskv(args, ws, rank, local):
                      "bytes_per_launch": by["indexer"], "us_per_launch": idx_us,
                      "traffic": profiled_traffic(args.workload)},
         "e2e": {"value": whole_job_rate(T, ws, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h, "device_us_per_step": ms_e2e * 1e3,
+                "host_wall_us_per_step": wall_us},
         "gpu_launches": int(launches_per_step) * args.steps,
         "clocks": clk,
     }

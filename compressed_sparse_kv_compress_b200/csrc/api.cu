@@ -235,21 +235,39 @@ size_t hybrid_attn_workspace_size(int mode, int T, int H, int d, int k, int wind
   return best;
 }
 
-int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off, const int32_t* idx,
-                       int k, const void* kv_raw, const int64_t* raw_off, const int64_t* raw_tok0, int window,
-                       const float* sink, float scale, const int32_t* q_seq, const int64_t* q_pos, int batch,
-                       int T, int H, int d, int dtype, int64_t max_entries, float* out, float* lse,
-                       void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream) {
+}  // extern "C"
+
+// Host-side checks of hybrid_decode_attn's arguments (everything but the workspace), shared
+// with the allocation-free variant so that both report the same error for the same mistake.
+int cskv::check_attn_args(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off, const int32_t* idx,
+                          int k, const void* kv_raw, const int64_t* raw_off, int window, float scale,
+                          const int32_t* q_seq, const int64_t* q_pos, int batch, int T, int H, int d, int dtype,
+                          int64_t max_entries, const float* out) {
   if (mode != CSKV_CSA && mode != CSKV_HCA) return CSKV_ERR_INVALID_ARG;
   if (dtype != CSKV_F32 && dtype != CSKV_BF16) return dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
   if (d != kHeadDim) return CSKV_ERR_UNSUPPORTED;
   if (H < 1 || H > 128 || T < 0 || window < 0 || window > (1 << 20) || batch < 1) return CSKV_ERR_INVALID_ARG;
   if (mode == CSKV_CSA && (k < 1 || k > (1 << 20) || !idx)) return CSKV_ERR_INVALID_ARG;
   if (mode == CSKV_HCA && (max_entries < 0 || max_entries > (1LL << 30))) return CSKV_ERR_INVALID_ARG;
+  // the softmax scale must be positive and finite: the kernels take the row maximum of the
+  // unscaled logits and scale it once, which is the maximum of the scaled logits only then
+  if (!(scale > 0.f) || !(scale < INFINITY)) return CSKV_ERR_INVALID_ARG;
   if (T == 0) return CSKV_OK;
   if (!q || !kv_cmp || !cmp_off || !kv_raw || !raw_off || !q_seq || !q_pos || !out) return CSKV_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(kv_cmp) || !aligned16(kv_raw)) return CSKV_ERR_INVALID_ARG;
-  if (!(scale == scale)) return CSKV_ERR_INVALID_ARG;
+  return CSKV_OK;
+}
+
+extern "C" {
+
+int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off, const int32_t* idx,
+                       int k, const void* kv_raw, const int64_t* raw_off, const int64_t* raw_tok0, int window,
+                       const float* sink, float scale, const int32_t* q_seq, const int64_t* q_pos, int batch,
+                       int T, int H, int d, int dtype, int64_t max_entries, float* out, float* lse,
+                       void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream) {
+  int arc = check_attn_args(mode, q, kv_cmp, cmp_off, idx, k, kv_raw, raw_off, window, scale, q_seq, q_pos, batch,
+                            T, H, d, dtype, max_entries, out);
+  if (arc != CSKV_OK || T == 0) return arc;
   const bool tc = dtype == CSKV_BF16;
   int R = 0, S = 0;
   int rc = attn_plan(mode, T, mode == CSKV_CSA ? k : 0, window, max_entries, tc, &R, &S);

@@ -14,7 +14,11 @@
 //    always written before they are read, so nothing needs clearing, but two calls that
 //    overlap on the GPU (different streams, no ordering between them) race on it;
 //  * the first call on each device looks up the array's device address with that device
-//    current (cudaGetSymbolAddress); make that first call before any stream capture.
+//    current (cudaGetSymbolAddress).  With lazy module loading (the CUDA 12 default) that
+//    lookup may be what loads this library's device code on the device and reserves the
+//    array, which allocates and can synchronise; so make one warm-up call per device at
+//    start-up, before any stream capture and before the point where allocation is
+//    forbidden.  Later calls allocate nothing.
 #include <mutex>
 
 #include "launch.cuh"
@@ -57,10 +61,11 @@ extern "C" int hybrid_decode_attn_noalloc(int mode, const void* q, const void* k
                                           const int32_t* q_seq, const int64_t* q_pos, int batch, int T, int H,
                                           int d, int dtype, int64_t max_entries, float* out, float* lse,
                                           int* dev_status, cskv_stream_t stream) {
-  if (T <= 0)  // nothing to launch: let the regular entry point validate and return
-    return hybrid_decode_attn(mode, q, kv_cmp, cmp_off, idx, k, kv_raw, raw_off, raw_tok0, window, sink, scale,
-                              q_seq, q_pos, batch, T, H, d, dtype, max_entries, out, lse, nullptr, 0, dev_status,
-                              stream);
+  // the same argument checks as the regular entry point, before the size check, so a bad
+  // argument is reported as such and not as a lack of scratch
+  const int arc = cskv::check_attn_args(mode, q, kv_cmp, cmp_off, idx, k, kv_raw, raw_off, window, scale, q_seq,
+                                        q_pos, batch, T, H, d, dtype, max_entries, out);
+  if (arc != CSKV_OK || T == 0) return arc;
   const size_t need = hybrid_attn_workspace_size(mode, T, H, d, mode == CSKV_CSA ? k : 0, window, max_entries);
   if (need > CSKV_NOALLOC_SCRATCH_BYTES) return CSKV_ERR_WORKSPACE;
   float* scratch = nullptr;

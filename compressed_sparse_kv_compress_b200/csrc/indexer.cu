@@ -244,6 +244,8 @@ __device__ bool group_barrier(QueryWS* ws, unsigned G, int j, int* st, int* sm_f
 struct IdxShared {
   uint64_t full[12];
   unsigned released[12];  // per ring stage: consumer warps done with it, all fills so far
+  int fills;              // fills the producer issued (read by the drain after a timeout)
+  int scan_err;           // a bounded wait of the scan gave up
   unsigned red[32];
   float fred[64];
   unsigned long long ured[32];
@@ -268,7 +270,8 @@ __device__ __forceinline__ void release_stage(unsigned* ctr) {
 // Waits until *ctr >= target, polling with an acquire load (backing off after a few polls);
 // gives up after about a second of polling (false).  The proxy fence then orders the
 // consumers' reads of the stage before the TMA unit's writes into it.
-__device__ __forceinline__ bool wait_released(unsigned* ctr, unsigned target) {
+// Also gives up (false) as soon as *err is set: a consumer warp that gave up never releases.
+__device__ __forceinline__ bool wait_released(unsigned* ctr, unsigned target, const int* err) {
   const uint32_t a = smem_u32(ctr);
   for (long n = 0; n < (1L << 24); ++n) {
     unsigned v;
@@ -277,14 +280,19 @@ __device__ __forceinline__ bool wait_released(unsigned* ctr, unsigned target) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       return true;
     }
+    if (*(const volatile int*)err) return false;
     if (n >= 32) __nanosleep(64);
   }
   return false;
 }
 
 // ------------------------------------------------------------------ scan: E4M3 via TMA + MMA
+// Returns false when a bounded wait gave up (CSKV_DEV_TIMEOUT is flagged).  The ring region is
+// then left untouched by the caller: every fill the producer issued has been waited for (the
+// drain below), or, when even that wait gave up, the barriers are not retired and the caller
+// must not touch the ring memory again.
 template <int KS, int NTILE>
-__device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, int len,
+__device__ bool scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, int len,
                          float* sc, uint8_t* ring, IdxShared& S) {
   constexpr int Di = KS * 32;
   constexpr int stages = idx_stages(Di);
@@ -295,6 +303,8 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
       mbar_init(&S.full[s], 1);
       S.released[s] = 0u;
     }
+    S.fills = 0;
+    S.scan_err = 0;
     fence_mbar_init();
   }
   // generic-proxy writes to the ring region (histograms of a previous segment) must be
@@ -304,11 +314,14 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
   if (warp == kIdxConsumerWarps) {
     asm volatile("bar.sync 2, %0;" ::"n"(kIdxThreads) : "memory");  // consumers' scale loads issued
     if (lane == 0) {
-      int s = 0;
-      for (int it = 0; it < ntiles; ++it) {
-        // the stage is refilled once every consumer warp has released its previous fill
-        if (it >= stages && !wait_released(&S.released[s], (unsigned)(kIdxConsumerWarps * (it / stages)))) {
+      int s = 0, it = 0;
+      for (; it < ntiles; ++it) {
+        // the stage is refilled once every consumer warp has released its previous fill; a
+        // consumer that gave up stops the producer too (no further fills are issued)
+        if (it >= stages && !wait_released(&S.released[s], (unsigned)(kIdxConsumerWarps * (it / stages)),
+                                           &S.scan_err)) {
           flag(p.st, CSKV_DEV_TIMEOUT);
+          S.scan_err = 1;
           break;
         }
         const int rows = min(kIdxTile, len - it * kIdxTile);
@@ -317,6 +330,7 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
         tma_bulk_g2s(ring + (size_t)s * kIdxTile * Di, kbase + (size_t)it * kIdxTile * Di, bytes, &S.full[s]);
         if (++s == stages) s = 0;
       }
+      S.fills = it;  // fills issued (the drain below needs the count)
     }
   } else {
     const int g = lane >> 2, tq = lane & 3;
@@ -365,6 +379,7 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
     for (int it = 0; it < ntiles && alive; ++it) {
       if (!mbar_wait_bounded(&S.full[s], ph)) {
         flag(p.st, CSKV_DEV_TIMEOUT);
+        *(volatile int*)&S.scan_err = 1;  // the producer stops issuing fills
         alive = false;
         break;
       }
@@ -434,12 +449,25 @@ __device__ void scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
     }
   }
   __syncthreads();
-  // Every copy issued has completed (each full barrier was waited on), so the ring can be
-  // reused and the barriers retired.
-  if (threadIdx.x == 0)
-    for (int s = 0; s < stages; ++s)
-      asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(&S.full[s])) : "memory");
+  // Without a timeout every fill was waited for by the consumers, so the ring can be reused
+  // and the barriers retired.  After a timeout some fills may still be in flight: thread 0
+  // waits (bounded) for the last fill issued to every stage before the barriers are retired;
+  // if that wait gives up too, the barriers stay live and the ring is never touched again.
+  if (threadIdx.x == 0) {
+    bool drained = true;
+    if (S.scan_err) {
+      const int fills = S.fills;
+      for (int s = 0; s < stages && drained; ++s) {
+        const int n = fills > s ? (fills - s + stages - 1) / stages : 0;  // fills of stage s
+        if (n > 0) drained = mbar_wait_bounded(&S.full[s], (unsigned)((n - 1) & 1));
+      }
+    }
+    if (drained)
+      for (int s = 0; s < stages; ++s)
+        asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(&S.full[s])) : "memory");
+  }
   __syncthreads();
+  return S.scan_err == 0;
 }
 
 // ------------------------------------------------------------------ scan: fp32 (CUDA cores)
@@ -710,7 +738,9 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   if constexpr (SRC == kSrcFp8) {
     const uint8_t* kb = p.k_idx + (size_t)(ebase + lo) * (KS * 32);
     const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
-    scan_fp8<KS, NTILE>(p, t, kb, ks, len, sc, un, S);
+    // after a timeout the ring (and the histograms that share its memory) is not touched
+    // again; the other CTAs of the group time out at their next group barrier
+    if (!scan_fp8<KS, NTILE>(p, t, kb, ks, len, sc, un, S)) return;
   } else if constexpr (SRC == kSrcF32) {
     const float* kb = reinterpret_cast<const float*>(p.k_idx) + (size_t)(ebase + lo) * p.Di;
     const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
@@ -1032,6 +1062,7 @@ __global__ void __maxnreg__(88) lindex_topk_kernel(IdxParams p) {
     for (size_t off = (size_t)(lane >= 4 ? lane - 4 : 0) * 128; lane >= 4 && off < qbytes; off += 124 * 128)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_idx + (size_t)t0 * qbytes + off));
   }
+  if (threadIdx.x == 0) S.scan_err = 0;  // read only after later block barriers
   pdl_wait();
   uint8_t* un = dsm;                                              // ring / histogram / candidates
   float* sc = reinterpret_cast<float*>(dsm + idx_union_bytes(KS * 32));  // segment scores
@@ -1084,6 +1115,7 @@ __global__ void __maxnreg__(88) lindex_topk_kernel(IdxParams p) {
       const int64_t V = visible_of(p, t, &eb);
       process_segment<SRC, KS, NTILE>(p, t, 0, 1, V, eb, nullptr, sc, un, S);
       __syncthreads();
+      if (S.scan_err) break;  // a scan gave up: its ring may not be reused (block-uniform)
     }
   }
 }

@@ -115,6 +115,11 @@ int attn_tc_rows_per_split(int mode, int T, int k, int window, int64_t max_entri
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
 int attn_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms);
 int attn_max_splits(int mode, int k, int window, int64_t max_entries, int R);
+// api.cu: host-side argument checks of hybrid_decode_attn (all but the workspace)
+int check_attn_args(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off, const int32_t* idx, int k,
+                    const void* kv_raw, const int64_t* raw_off, int window, float scale, const int32_t* q_seq,
+                    const int64_t* q_pos, int batch, int T, int H, int d, int dtype, int64_t max_entries,
+                    const float* out);
 // staging.cu
 cudaError_t launch_copy_segments(const void* src, const int64_t* src_off, void* const* dst, const int64_t* len, int n,
                                  cudaStream_t stream);

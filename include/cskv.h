@@ -222,7 +222,8 @@ CSKV_API size_t lindex_workspace_size(int T, int k, int64_t max_entries);
  * idx     : [T, k] int32 (mode CSA), NULL for HCA.
  * kv_raw  : [rows, 2d] dtype raw window rows; raw_off: [batch+1] int64;
  *           raw_tok0: [batch] int64 or NULL (0): token of sequence b's first row.
- * sink    : [H] fp32 or NULL (no sink).  scale: host float (1/sqrt(d) typical).
+ * sink    : [H] fp32 or NULL (no sink).  scale: host float, positive and finite
+ *           (1/sqrt(d) typical); anything else is CSKV_ERR_INVALID_ARG.
  * q_seq   : [T] int32; q_pos: [T] int64.
  * max_entries : host; mode HCA: >= every visible HCA entry count; mode CSA: unused.
  * out     : [T, H, d] fp32;  lse: [T, H] fp32 or NULL.
@@ -246,15 +247,20 @@ CSKV_API size_t hybrid_attn_workspace_size(int mode, int T, int H, int d, int k,
  * must never synchronise, as cudaMalloc/cudaFree can).  This variant takes the same
  * arguments as hybrid_decode_attn minus the workspace, and keeps its split-KV partials
  * in one array of CSKV_NOALLOC_SCRATCH_BYTES that the library declares in device memory.
- * It allocates nothing.
+ * After its first call on a device (below) it allocates nothing.
  * - A call whose hybrid_attn_workspace_size() exceeds CSKV_NOALLOC_SCRATCH_BYTES returns
  *   CSKV_ERR_WORKSPACE and launches nothing.
  * - Every GPU that loads the library holds the array until the process exits.
  * - All calls share the array, which keeps the last call's contents.  Nothing in it needs
  *   clearing (every partial is written before it is read), but calls that overlap on the
  *   GPU (unordered streams) race on it.
- * - The first call on a device looks up the array's address with that device current;
- *   make that first call before any stream capture.
+ * - The first call on a device looks up the array's address with that device current.
+ *   Under lazy module loading (the CUDA 12 default) that first lookup may load the
+ *   library's device code and reserve the array, which allocates and may synchronise: make
+ *   one warm-up call per device at start-up, before any stream capture and before
+ *   allocation becomes forbidden.  Every later call allocates nothing.
+ * - Arguments are checked exactly as hybrid_decode_attn checks them (CSKV_ERR_INVALID_ARG /
+ *   CSKV_ERR_UNSUPPORTED) before the scratch size is.
  * ------------------------------------------------------------------------ */
 #define CSKV_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 CSKV_API int hybrid_decode_attn_noalloc(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off,

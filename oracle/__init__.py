@@ -17,9 +17,11 @@ it (cited by page and section in each function):
        计算量降至原来的27%？" (ratios 4:1 / 128:1, top-1024, 128-token window).
 
 All arithmetic is float64 on values decoded exactly from their storage form
-(bf16, fp32, OCP E4M3), with one exception: where floating point decides an
-integer -- the E4M3 codes of pooled indexer keys (indexer.quantize_keys) -- the
-steps are taken in fp32, the precision of the kernel that decides the same codes.
+(bf16, fp32, OCP E4M3).  Where floating point decides an integer -- the E4M3 codes
+of pooled indexer keys -- the definition is exact (indexer.pool_keys_f64,
+quantize_keys_f64) and indexer.quotient_error_bound says where an fp32 evaluation
+may round to the neighbouring code; indexer.pool_keys / quantize_keys restate the
+same steps in fp32 (the kernel's precision) as a second, labelled check.
 Loops are vectorised with numpy but follow each definition term by term; nothing
 is blocked, fused or reordered beyond it.
 

@@ -31,13 +31,23 @@ the scores): readings taken --
   it has), block size 4, the CSA ratio;
 * the entry key is then stored as E4M3 codes with one fp32 scale per entry,
   scale = amax / 448 (1 when the key is all zeros), code = E4M3(key / scale).
-  The codes are integers decided by floating point, so this step is computed in the
-  precision of the kernel that also produces them: fp32, summing the tokens in order
-  and dividing by their count, then one fp32 division per element.
+
+Two forms of the pooling are given.  The definition (``pool_keys_f64`` and
+``quantize_keys_f64``) computes the mean, the scale and the quotient exactly in float64
+and encodes with the nearest-even E4M3 rule.  The codes are integers decided by floating
+point, so an fp32 evaluation (the kernel's precision) may land on the neighbouring code
+where the exact quotient lies within the fp32 rounding error of an E4M3 rounding
+boundary; ``quotient_error_bound`` bounds that error for any evaluation that sums the
+tokens in fp32 and divides in fp32, so a comparison can tell where either code is
+correct.  ``pool_keys`` / ``quantize_keys`` take the same steps in fp32 (tokens summed in
+order, one division by the count, one division by the scale): a second, labelled
+restatement in the kernel's precision, not the definition.
 
 Parity: pinned (worked (8, -7) example, block-24 causal example, brute-force
-enumeration of k-subsets on tiny inputs, ties; pooling: identical tokens, partial
-blocks, mean linearity; the E4M3 codec against the OFP8 values and torch's cast).
+enumeration of k-subsets on tiny inputs, ties; pooling: integer means, identical tokens,
+partial blocks, codes that land on printed E4M3 values, the nearest E4M3 value found by
+brute force over every finite code, the fp32 restatement agreeing outside the error band;
+the E4M3 codec against the OFP8 values and torch's cast).
 """
 
 from __future__ import annotations
@@ -125,3 +135,57 @@ def quantize_keys(keys: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     scale = np.where(amax > 0, (amax / np.float32(E4M3_MAX)).astype(np.float32), np.float32(1.0)).astype(np.float32)
     v = (k / scale[:, None]).astype(np.float32)
     return codecs.e4m3_encode(v.astype(np.float64)), scale
+
+
+def pool_keys_f64(k_tok: np.ndarray, ratio: int = 4) -> np.ndarray:
+    """Per-token keys [n, Di] -> entry keys [ceil(n/ratio), Di] float64: the exact mean of
+    each block's tokens (a partial last block: of the tokens it has)."""
+    k = np.asarray(k_tok, dtype=np.float64)
+    n = k.shape[0]
+    out = np.zeros(((n + ratio - 1) // ratio, k.shape[1]), dtype=np.float64)
+    for i in range(out.shape[0]):
+        out[i] = np.mean(k[ratio * i: min(n, ratio * (i + 1))], axis=0)
+    return out
+
+
+def quantize_keys_f64(keys: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Entry keys [V, Di] float64 -> (E4M3 codes [V, Di] uint8, scales [V] float64):
+    scale = amax / 448 (1 for an all-zero key), code = E4M3(key / scale), every step exact
+    in float64 before the one rounding of the encoder."""
+    k = np.asarray(keys, dtype=np.float64)
+    amax = np.max(np.abs(k), axis=1)
+    scale = np.where(amax > 0, amax / E4M3_MAX, 1.0)
+    return codecs.e4m3_encode(k / scale[:, None]), scale
+
+
+def quotient_error_bound(k_tok: np.ndarray, ratio: int = 4) -> tuple[np.ndarray, np.ndarray]:
+    """Bounds on how far an fp32 evaluation of the pooling can land from the exact values:
+    (tol_v [V, Di], tol_scale [V]) with |v32 - key/scale| <= tol_v for the quotient the
+    encoder rounds and |scale32 - scale| <= tol_scale.
+
+    Error analysis (u = 2^-24, the fp32 unit roundoff): summing c tokens in fp32 in any
+    order makes at most c - 1 roundings, each at most u times a partial sum, and every
+    partial sum is at most S = sum_c |token_c| in magnitude; the division by c adds u |key|.
+    So |key32 - key| <= e = u ((c - 1) S / c + |key|).  The largest magnitude moves by at
+    most max_j e_j, so the scale (amax / 448, one more rounding) moves by at most
+    d_s = max_j e_j / 448 + u scale, and the quotient key32 / scale32 (one more rounding)
+    by at most e / scale + |v| d_s / scale + u |v|, to first order; the bound returned is
+    twice that, which covers the second-order terms."""
+    k = np.asarray(k_tok, dtype=np.float64)
+    n = k.shape[0]
+    u = 2.0 ** -24
+    V = (n + ratio - 1) // ratio
+    key = pool_keys_f64(k, ratio)
+    _, scale = quantize_keys_f64(key)
+    tol_v = np.zeros_like(key)
+    tol_s = np.zeros(V)
+    for i in range(V):
+        rows = k[ratio * i: min(n, ratio * (i + 1))]
+        c = rows.shape[0]
+        S = np.sum(np.abs(rows), axis=0)
+        e = u * ((c - 1) * S / c + np.abs(key[i]))
+        ds = np.max(e) / E4M3_MAX + u * scale[i]
+        v = np.abs(key[i]) / scale[i]
+        tol_v[i] = 2.0 * (e / scale[i] + v * ds / scale[i] + u * v)
+        tol_s[i] = 2.0 * ds
+    return tol_v, tol_s

@@ -9,10 +9,10 @@ import torch
 from oracle import codecs, indexer
 from synth import Workload
 
-# SPEC §4 tolerances
-ATTN_MAX_REL = 1e-2      # max|d| <= 1e-2 * max|ref|
-ATTN_MEAN_ABS = 1e-3     # mean|d| <= 1e-3
-SEL_BAND = 1e-4          # selection may differ only within 1e-4 of the k-th score
+# Parity tolerances of the hot path (bf16 in, fp32 accumulate, against the fp64 oracle):
+ATTN_MAX_REL = 1e-2      # attention outputs: max|d| <= 1e-2 * max|ref|
+ATTN_MEAN_ABS = 1e-3     # attention outputs: mean|d| <= 1e-3
+SEL_BAND = 1e-4          # end-to-end top-k may differ only for entries within 1e-4 of the k-th score
 
 
 def np_arrays(w: Workload) -> dict:
@@ -97,3 +97,27 @@ def storage_rows(t: torch.Tensor) -> np.ndarray:
     if c.dtype == torch.bfloat16:
         return codecs.bf16_decode(c.view(torch.int16).numpy().view(np.uint16))
     return c.numpy().astype(np.float64)
+
+
+def check_pooled_keys(gpu_codes, gpu_scale, tok_f64, ratio=4, what=""):
+    """Pooled indexer keys from the GPU against the exact (fp64) definition.
+
+    Outside the fp32 error band (oracle.indexer.quotient_error_bound) every code must equal
+    the exact code; inside it, the decoded value must lie between the codes of the band's
+    two ends (the neighbouring code is as correct as the exact one there).  Scales must lie
+    within their bound.  Returns the number of elements inside the band."""
+    key = indexer.pool_keys_f64(tok_f64, ratio)
+    c64, s64 = indexer.quantize_keys_f64(key)
+    tol_v, tol_s = indexer.quotient_error_bound(tok_f64, ratio)
+    v64 = key / s64[:, None]
+    lo = codecs.e4m3_decode(codecs.e4m3_encode(v64 - tol_v))
+    hi = codecs.e4m3_decode(codecs.e4m3_encode(v64 + tol_v))
+    got = codecs.e4m3_decode(np.asarray(gpu_codes, dtype=np.uint8))
+    sure = lo == hi
+    off = sure & (got != codecs.e4m3_decode(c64))
+    assert not off.any(), f"{what}: {int(off.sum())} codes differ from the exact ones outside the band"
+    out = ~((got >= lo) & (got <= hi))
+    assert not out.any(), f"{what}: {int(out.sum())} codes outside the band"
+    ds = np.abs(np.asarray(gpu_scale, dtype=np.float64) - s64)
+    assert np.all(ds <= tol_s), f"{what}: scale off by {ds.max():.3e}"
+    return int((~sure).sum())

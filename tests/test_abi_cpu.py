@@ -104,17 +104,25 @@ def test_indexer_validation(lib):
 def test_attention_validation(lib):
     nul = None
 
-    def call(mode=0, d=128, H=16, dtype=1, idx=_p(), k=8, T=1):
-        return lib.hybrid_decode_attn(mode, _p(), _p(), _p(), idx, k, _p(), _p(), nul, 128, nul, 0.1, _p(), _p(), 1,
+    def call(mode=0, d=128, H=16, dtype=1, idx=_p(), k=8, T=1, scale=0.1, noalloc=False):
+        if noalloc:  # the allocation-free variant: same arguments minus the workspace
+            return lib.hybrid_decode_attn_noalloc(mode, _p(), _p(), _p(), idx, k, _p(), _p(), nul, 128, nul, scale,
+                                                  _p(), _p(), 1, T, H, d, dtype, 0, _p(), nul, nul, nul)
+        return lib.hybrid_decode_attn(mode, _p(), _p(), _p(), idx, k, _p(), _p(), nul, 128, nul, scale, _p(), _p(), 1,
                                       T, H, d, dtype, 0, _p(), nul, _p(), 1 << 20, nul, nul)
 
-    assert call(mode=5) == _lib.ERR_INVALID_ARG
-    assert call(d=64) == _lib.ERR_UNSUPPORTED
-    assert call(dtype=_lib.FP8E4M3) == _lib.ERR_UNSUPPORTED
-    assert call(H=0) == _lib.ERR_INVALID_ARG
-    assert call(H=129) == _lib.ERR_INVALID_ARG
-    assert call(idx=nul) == _lib.ERR_INVALID_ARG
-    assert call(T=0) == _lib.OK
+    for na in (False, True):  # both entry points report the same error for the same mistake
+        assert call(mode=5, noalloc=na) == _lib.ERR_INVALID_ARG
+        assert call(d=64, noalloc=na) == _lib.ERR_UNSUPPORTED
+        assert call(dtype=_lib.FP8E4M3, noalloc=na) == _lib.ERR_UNSUPPORTED
+        assert call(H=0, noalloc=na) == _lib.ERR_INVALID_ARG
+        assert call(H=129, noalloc=na) == _lib.ERR_INVALID_ARG
+        assert call(idx=nul, noalloc=na) == _lib.ERR_INVALID_ARG
+        assert call(k=0, noalloc=na) == _lib.ERR_INVALID_ARG
+        # the softmax scale must be positive and finite
+        for bad in (0.0, -0.1, float("inf"), float("nan")):
+            assert call(scale=bad, noalloc=na) == _lib.ERR_INVALID_ARG
+        assert call(T=0, noalloc=na) == _lib.OK
 
 
 def test_copy_segments_validation(lib):

@@ -138,25 +138,34 @@ def _issue_layers(step, order):
     main.wait_stream(step.side)
 
 
-def test_ragged_b64_selection_stable_beside_hca_layer():
+@pytest.mark.parametrize("name,reps", [("ragged_b64", 20), ("b8_ctx64k", 12), ("b1_ctx1m", 12)])
+def test_selection_stable_beside_hca_layer(name, reps):
     # The HCA layer's kernels share the SMs with the indexer when it runs on a second stream,
-    # issued before or after the CSA layer.  Every repetition must select exactly what a
-    # one-stream run selects (the selection is deterministic), and that run must match the
-    # oracle on sampled queries.
-    w = Workload(spec_by_name("ragged_b64"))
+    # issued before or after the CSA layer.  Every repetition, in both issue orders and as a
+    # replayed two-stream graph, must select exactly what a one-stream run selects (the
+    # selection is deterministic), and that run must match the oracle on sampled queries.
+    w = Workload(spec_by_name(name))
     m, a = w.meta, np_arrays(w)
     step, dev = decode_step(w)
     step.run()
     torch.cuda.synchronize()
     ref = step.idx.clone()
-    for t in (5, 36, 42, 54):
+    T = m["T"]
+    for t in sorted({0, T // 2, T - 1}):
         check_selection(ref[t].cpu().numpy(), ostep.query_scores(m, a, dtypes(w), t), m["k"], f"query {t}")
-    step2, _ = decode_step(w, two_streams=True)
-    for order in ("csa_first", "hca_first", "csa_first", "csa_first"):
-        for rep in range(3):
+    step2, _ = decode_step(w, dev=dev, two_streams=True)
+    for order in ("csa_first", "hca_first"):
+        for rep in range(reps):
             step2.idx.fill_(-2)
             _issue_layers(step2, order)
             torch.cuda.synchronize()
             assert int(step2.status.item()) == 0
             bad = (step2.idx != ref).any(dim=1).nonzero().flatten().tolist()
             assert not bad, f"{order} repetition {rep}: queries {bad} select differently"
+    step2.capture()
+    for rep in range(reps):
+        step2.idx.fill_(-2)
+        step2.replay()
+        torch.cuda.synchronize()
+        assert int(step2.status.item()) == 0
+        assert torch.equal(step2.idx, ref), f"graph replay {rep} selects differently"

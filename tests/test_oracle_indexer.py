@@ -145,3 +145,93 @@ def test_quantize_keys_scale_and_error_bound():
     err = np.abs(deq - keys.astype(np.float64))
     bound = np.maximum(np.abs(keys) * 2.0 ** -4, 2.0 ** -10 * scale[:, None])
     assert np.all(err <= bound * (1 + 1e-6))
+
+
+# ---- the exact (fp64) pooling definition and its fp32 error band
+
+
+def _e4m3_table():
+    """Every finite E4M3 code with its value (NaN codes left out)."""
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)
+    return codes, codecs.e4m3_decode(codes)
+
+
+def test_pool_f64_lands_on_printed_e4m3_values():
+    g = json.load(open(os.path.join(GOLD, "e4m3_values.json")))
+    vals = {int(c, 16): v for c, v in g["codes"].items() if c != "0x80"}
+    key = np.array(list(vals.values()), dtype=np.float64)          # amax 448 -> scale 1
+    offs = np.array([3.0, -1.0, -4.0, 2.0])                         # sum 0: the mean is the key
+    for mult in (1.0, 2.0, 0.25):                                   # scales 1, 2, 1/4 (exact)
+        tok = np.stack([mult * key + o * (1 if mult >= 1 else 0) for o in offs])
+        mean = indexer.pool_keys_f64(tok, 4)
+        assert np.array_equal(mean[0], mult * key)
+        codes, scale = indexer.quantize_keys_f64(mean)
+        assert scale[0] == mult * 448.0 / 448.0
+        assert [int(c) for c in codes[0]] == list(vals.keys())
+
+
+def test_pool_f64_integer_means_and_partial_block():
+    k = np.array([[1, -2], [2, 0], [3, 4], [6, 2], [8, -8], [0, 2]], dtype=np.float64)
+    assert np.array_equal(indexer.pool_keys_f64(k, 4), np.array([[3, 1], [4, -3]], dtype=np.float64))
+    codes, scale = indexer.quantize_keys_f64(np.zeros((1, 4)))
+    assert scale[0] == 1.0 and np.all(codes == 0)
+
+
+def test_pool_f64_codes_are_the_nearest_e4m3_values_by_brute_force():
+    table_c, table_v = _e4m3_table()
+    rng = np.random.default_rng(11)
+    tok = rng.standard_normal((4 * 40, 16)) / 8.0
+    codes, scale = indexer.quantize_keys_f64(indexer.pool_keys_f64(tok, 4))
+    key = indexer.pool_keys_f64(tok, 4)
+    for i in range(key.shape[0]):
+        for j in range(key.shape[1]):
+            dist = np.abs(table_v * scale[i] - key[i, j])
+            best = np.flatnonzero(dist == dist.min())
+            # ties between two neighbours go to the even mantissa; +-0 are one value
+            pick = [c for c in table_c[best] if c & 1 == 0] or list(table_c[best])
+            want = codecs.e4m3_decode(np.array(pick[:1], dtype=np.uint8))[0]
+            assert codecs.e4m3_decode(codes[i:i + 1, j])[0] == want, (i, j)
+
+
+def test_fp32_restatement_stays_inside_the_error_band():
+    rng = np.random.default_rng(12)
+    tok = (rng.standard_normal((4 * 3000, 64)) / 8.0).astype(np.float32)
+    # a few adversarial blocks: large tokens that cancel beside small ones
+    tok[0:4, :8] = np.array([[1e4], [1.0], [-1e4], [0.5]], dtype=np.float32)
+    tok[4:8, :8] = np.array([[3.0], [-3.0], [1e-3], [2e-3]], dtype=np.float32)
+    t64 = tok.astype(np.float64)
+    key64 = indexer.pool_keys_f64(t64, 4)
+    c64, s64 = indexer.quantize_keys_f64(key64)
+    tol_v, tol_s = indexer.quotient_error_bound(t64, 4)
+    c32, s32 = indexer.quantize_keys(indexer.pool_keys(tok, 4))
+    # the scale and the quotient of the fp32 steps lie inside the bounds
+    assert np.all(np.abs(s32.astype(np.float64) - s64) <= tol_s)
+    key32 = indexer.pool_keys(tok, 4)
+    v32 = (key32 / s32[:, None]).astype(np.float32).astype(np.float64)
+    v64 = key64 / s64[:, None]
+    assert np.all(np.abs(v32 - v64) <= tol_v)
+    # codes: equal to the exact ones outside the band, inside it between the codes of its ends
+    lo = codecs.e4m3_decode(codecs.e4m3_encode(v64 - tol_v))
+    hi = codecs.e4m3_decode(codecs.e4m3_encode(v64 + tol_v))
+    d32 = codecs.e4m3_decode(c32)
+    assert np.all((d32 >= lo) & (d32 <= hi))
+    sure = lo == hi
+    assert np.all(d32[sure] == codecs.e4m3_decode(c64)[sure])
+    assert (~sure).mean() < 1e-3  # the band is narrow: a handful of elements
+
+
+def test_error_band_catches_a_planted_off_by_one_code():
+    # a code one step off where the band is a single code must fail the band check
+    rng = np.random.default_rng(13)
+    tok = rng.standard_normal((16, 64)) / 8.0
+    key = indexer.pool_keys_f64(tok, 4)
+    c64, s64 = indexer.quantize_keys_f64(key)
+    tol_v, _ = indexer.quotient_error_bound(tok, 4)
+    v64 = key / s64[:, None]
+    lo = codecs.e4m3_decode(codecs.e4m3_encode(v64 - tol_v))
+    hi = codecs.e4m3_decode(codecs.e4m3_encode(v64 + tol_v))
+    bad = c64.copy()
+    j = int(np.argmax((lo == hi)[0] & (np.abs(v64[0]) > 1.0)))
+    bad[0, j] = bad[0, j] + 1 if bad[0, j] & 0x7F < 0x7E else bad[0, j] - 1
+    d = codecs.e4m3_decode(bad)
+    assert not np.all((d >= lo) & (d <= hi))

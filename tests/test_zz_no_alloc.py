@@ -36,7 +36,8 @@ def _noalloc(lib, mode, w, dev, idx, out, lse, status):
     return lib.hybrid_decode_attn_noalloc(
         mode, _p(dev["q_" + layer]), _p(dev["cmp_" + layer]), _p(off), _p(idx), 0 if idx is None else idx.shape[1],
         _p(dev["raw_" + layer]), _p(dev["raw_off"]), _p(dev["raw_t0"]), m["W"], _p(dev["sink_" + layer]),
-        m["scale"], _p(dev["q_seq"]), _p(dev["q_pos"]), m["B"], T, H, d, _lib.BF16,
+        m["scale"], _p(dev["q_seq"]), _p(dev["q_pos"]), m["B"], T, H, d,
+        _lib.BF16 if dev["q_" + layer].dtype == torch.bfloat16 else _lib.F32,
         bounds(w)["max_hca_visible"], _p(out), _p(lse), _p(status), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
@@ -52,9 +53,15 @@ def _regular(mode, w, dev, idx, out, lse):
                            max_entries=bounds(w)["max_hca_visible"])
 
 
-def test_noalloc_matches_regular_entry_point_twice():
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+def test_noalloc_matches_regular_entry_point_twice(kind):
+    """bf16 runs the tensor-core kernel, fp32 the CUDA-core one; both keep their partials in
+    the library's array."""
     lib = _lib.load()
-    w = Workload(spec_by_name("b8_ctx64k").replace(batch=4, seq_len=(65536, 40001, 9000, 300), heads=64))
+    if kind == "bf16":
+        w = Workload(spec_by_name("b8_ctx64k").replace(batch=4, seq_len=(65536, 40001, 9000, 300), heads=64))
+    else:
+        w = Workload(spec_by_name("tiny").replace(batch=3, seq_len=(4096, 2000, 700), heads=16, cache="random"))
     m, a = w.meta, np_arrays(w)
     dev = w.device("cuda")
     rows = np.stack([indexer.topk_select(ostep.query_scores(m, a, dtypes(w), t), m["k"]) for t in range(m["T"])])
@@ -90,3 +97,30 @@ def test_noalloc_refuses_more_scratch_than_it_holds():
     assert rc == _lib.ERR_WORKSPACE
     torch.cuda.synchronize()
     assert int(out.count_nonzero().item()) == 0  # nothing launched
+
+
+def test_noalloc_reports_bad_arguments_as_such():
+    # a bad argument is CSKV_ERR_INVALID_ARG, as from the regular entry point, even when the
+    # call would also need more scratch than the array holds; nothing is launched
+    lib = _lib.load()
+    w = Workload(spec_by_name("b8_ctx64k").replace(batch=2, seq_len=(8192, 5000), heads=64))
+    dev = w.device("cuda")
+    m = w.meta
+    T, H = m["T"], m["H"]
+    out = torch.zeros(T, H, 128, dtype=torch.float32, device="cuda")
+    idx = torch.zeros(T, m["k"], dtype=torch.int32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def call(mode=api.CSA, k=m["k"], H_=H, scale=m["scale"], window=m["W"]):
+        return lib.hybrid_decode_attn_noalloc(
+            mode, _p(dev["q_c"]), _p(dev["cmp_c"]), _p(dev["csa_off"]), _p(idx), k, _p(dev["raw_c"]),
+            _p(dev["raw_off"]), _p(dev["raw_t0"]), window, None, scale, _p(dev["q_seq"]), _p(dev["q_pos"]), m["B"],
+            T, H_, 128, _lib.BF16, 0, _p(out), None, None, stream)
+
+    assert call(mode=7) == _lib.ERR_INVALID_ARG
+    assert call(H_=129) == _lib.ERR_INVALID_ARG
+    assert call(k=0) == _lib.ERR_INVALID_ARG
+    assert call(scale=-1.0) == _lib.ERR_INVALID_ARG
+    assert call(k=(1 << 20) + 1) == _lib.ERR_INVALID_ARG  # also far beyond the array
+    torch.cuda.synchronize()
+    assert int(out.count_nonzero().item()) == 0
