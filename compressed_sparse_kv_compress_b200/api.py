@@ -38,21 +38,30 @@ def _stream(stream) -> int:
 
 
 def csa_compress(x_a, z_a, x_b, z_b, tok_off, ent_off, out, *, max_blocks, bias_a=None, bias_b=None, tok0=None,
-                 first_block=None, num_blocks=None, dev_status=None, stream=None):
+                 first_block=None, num_blocks=None, rmsnorm=False, norm_gamma=None, norm_eps=1e-6, k_tok=None,
+                 k_codes=None, k_scale=None, dev_status=None, stream=None):
+    """rmsnorm: normalise each entry's K and V halves (norm_gamma [256] fp32, K then V; None =
+    ones).  k_tok [rows, Di] (rows indexed like x_a): also pool the per-token indexer keys of
+    the same entries into k_codes [*, Di] uint8 (E4M3) and k_scale [*] fp32."""
     lib = _lib.load()
+    k_dt = _dt(k_tok) if k_tok is not None else F32
+    Di = int(k_tok.shape[-1]) if k_tok is not None else 0
     st = lib.csa_compress(_ptr(x_a), _ptr(z_a), _ptr(x_b), _ptr(z_b), _ptr(bias_a), _ptr(bias_b), _ptr(tok_off),
                           _ptr(tok0), tok_off.numel() - 1, _ptr(ent_off), _ptr(first_block), _ptr(num_blocks),
-                          int(max_blocks), _dt(x_a), _dt(out), _ptr(out), _ptr(dev_status), _stream(stream))
+                          int(max_blocks), _dt(x_a), _dt(out), _ptr(out), int(bool(rmsnorm)), _ptr(norm_gamma),
+                          float(norm_eps), _ptr(k_tok), k_dt, Di, _ptr(k_codes), _ptr(k_scale), _ptr(dev_status),
+                          _stream(stream))
     _lib.check("csa_compress", st)
     return out
 
 
 def hca_compress(x, z, tok_off, ent_off, out, *, max_blocks, bias=None, tok0=None, first_block=None,
-                 num_blocks=None, dev_status=None, stream=None):
+                 num_blocks=None, rmsnorm=False, norm_gamma=None, norm_eps=1e-6, dev_status=None, stream=None):
     lib = _lib.load()
     st = lib.hca_compress(_ptr(x), _ptr(z), _ptr(bias), _ptr(tok_off), _ptr(tok0), tok_off.numel() - 1,
                           _ptr(ent_off), _ptr(first_block), _ptr(num_blocks), int(max_blocks), _dt(x), _dt(out),
-                          _ptr(out), _ptr(dev_status), _stream(stream))
+                          _ptr(out), int(bool(rmsnorm)), _ptr(norm_gamma), float(norm_eps), _ptr(dev_status),
+                          _stream(stream))
     _lib.check("hca_compress", st)
     return out
 

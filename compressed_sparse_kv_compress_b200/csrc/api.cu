@@ -91,19 +91,39 @@ static int check_compress_common(const void* x, const void* z, const int64_t* to
   return CSKV_OK;
 }
 
+// RMSNorm arguments shared by both compressions.
+static int check_norm(int rmsnorm, const float* gamma, float eps) {
+  if (rmsnorm != 0 && rmsnorm != 1) return CSKV_ERR_INVALID_ARG;
+  if (rmsnorm && (!(eps >= 0.f) || !(eps < INFINITY))) return CSKV_ERR_INVALID_ARG;
+  if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)) return CSKV_ERR_INVALID_ARG;
+  return CSKV_OK;
+}
+
 int csa_compress(const void* x_a, const void* z_a, const void* x_b, const void* z_b, const float* bias_a,
                  const float* bias_b, const int64_t* tok_off, const int64_t* tok0, int batch,
                  const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
-                 int64_t max_blocks, int in_dtype, int out_dtype, void* out, int* dev_status,
-                 cskv_stream_t stream) {
+                 int64_t max_blocks, int in_dtype, int out_dtype, void* out, int rmsnorm, const float* norm_gamma,
+                 float norm_eps, const void* k_tok, int k_dtype, int Di, uint8_t* k_codes, float* k_scale,
+                 int* dev_status, cskv_stream_t stream) {
   int rc = check_compress_common(x_a, z_a, tok_off, batch, ent_off, max_blocks, in_dtype, out_dtype, out);
   if (rc) return rc;
   if ((x_b == nullptr) != (z_b == nullptr)) return CSKV_ERR_INVALID_ARG;
   if (x_b && (!aligned16(x_b) || !aligned16(z_b))) return CSKV_ERR_INVALID_ARG;
   if ((bias_a && !aligned16(bias_a)) || (bias_b && !aligned16(bias_b))) return CSKV_ERR_INVALID_ARG;
+  rc = check_norm(rmsnorm, norm_gamma, norm_eps);
+  if (rc) return rc;
+  if (k_tok) {
+    if (!k_codes || !k_scale) return CSKV_ERR_INVALID_ARG;
+    if (k_dtype != CSKV_F32 && k_dtype != CSKV_BF16)
+      return k_dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+    if (Di != 64 && Di != 128) return Di > 0 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+    if (!aligned16(k_tok) || !aligned16(k_codes) || (reinterpret_cast<uintptr_t>(k_scale) & 3u))
+      return CSKV_ERR_INVALID_ARG;
+  }
   if (max_blocks == 0) return CSKV_OK;
   return launch_status(launch_csa_compress(x_a, z_a, x_b, z_b, bias_a, bias_b, tok_off, tok0, batch, ent_off,
-                                           first_block, num_blocks, max_blocks, in_dtype, out_dtype, out,
+                                           first_block, num_blocks, max_blocks, in_dtype, out_dtype, out, rmsnorm,
+                                           norm_gamma, norm_eps, k_tok, k_dtype, k_tok ? Di : 0, k_codes, k_scale,
                                            dev_status, (cudaStream_t)stream));
 }
 
@@ -126,15 +146,17 @@ int lindex_pool_keys(const void* k_tok, int in_dtype, int Di, const int64_t* tok
 
 int hca_compress(const void* x, const void* z, const float* bias, const int64_t* tok_off, const int64_t* tok0,
                  int batch, const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
-                 int64_t max_blocks, int in_dtype, int out_dtype, void* out, int* dev_status,
-                 cskv_stream_t stream) {
+                 int64_t max_blocks, int in_dtype, int out_dtype, void* out, int rmsnorm, const float* norm_gamma,
+                 float norm_eps, int* dev_status, cskv_stream_t stream) {
   int rc = check_compress_common(x, z, tok_off, batch, ent_off, max_blocks, in_dtype, out_dtype, out);
   if (rc) return rc;
   if (bias && !aligned16(bias)) return CSKV_ERR_INVALID_ARG;
+  rc = check_norm(rmsnorm, norm_gamma, norm_eps);
+  if (rc) return rc;
   if (max_blocks == 0) return CSKV_OK;
   return launch_status(launch_hca_compress(x, z, bias, tok_off, tok0, batch, ent_off, first_block, num_blocks,
-                                           max_blocks, in_dtype, out_dtype, out, dev_status,
-                                           (cudaStream_t)stream));
+                                           max_blocks, in_dtype, out_dtype, out, rmsnorm, norm_gamma, norm_eps,
+                                           dev_status, (cudaStream_t)stream));
 }
 
 size_t lindex_workspace_size(int T, int k, int64_t max_entries) {

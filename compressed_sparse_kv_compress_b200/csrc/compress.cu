@@ -89,13 +89,26 @@ __device__ __forceinline__ SeqRange seq_range(int b, int ratio, const int64_t* t
 constexpr int kCsaWarps = 2;
 constexpr int64_t kCsaGridCtas = 16384;  // grid bound of whole-cache calls (entries loop)
 
+// Optional epilogues of the CSA kernels: RMSNorm of the entry's K and V halves, and the pooling
+// of the per-token indexer keys (rows indexed like x_a) into E4M3 entry keys.
+struct CsaExtras {
+  int norm;
+  const float* gamma;  // [256] (K then V) or NULL = ones
+  float eps;
+  const void* k_tok;  // [rows, Di] fp32 or bf16, or NULL
+  int k_f32;
+  int Di;
+  uint8_t* k_codes;
+  float* k_scale;
+};
+
 template <typename TI, typename TO, bool kTwo>
 __global__ void __maxnreg__(144) csa_compress_kernel(
     const TI* __restrict__ xa, const TI* __restrict__ za, const TI* __restrict__ xb,
     const TI* __restrict__ zb, const float* __restrict__ ba, const float* __restrict__ bb,
     const int64_t* __restrict__ tok_off, const int64_t* __restrict__ tok0,
     const int64_t* __restrict__ ent_off, const int64_t* __restrict__ first_block,
-    const int64_t* __restrict__ num_blocks, int64_t max_blocks, TO* __restrict__ out, int* st) {
+    const int64_t* __restrict__ num_blocks, int64_t max_blocks, TO* __restrict__ out, CsaExtras ex, int* st) {
   constexpr int kC = kTwo ? 8 : 4;  // candidates: 4 path-A (+ 4 path-B)
   // A few small CTAs: the next kernel (the indexer in a decode step) may launch at once and
   // sit beside them; it waits for this grid before reading anything.
@@ -157,7 +170,56 @@ __global__ void __maxnreg__(144) csa_compress_kernel(
     float o[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j] = num[j] / den[j];
+    if (ex.norm) {
+      // RMSNorm over each 128-dim half: lanes 0-15 hold K, lanes 16-31 hold V
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ss = fmaf(o[j], o[j], ss);
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const float r = rsqrtf(ss * (1.f / 128.f) + ex.eps);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = o[j] * r * (ex.gamma ? __ldg(ex.gamma + j0 + j) : 1.f);
+    }
     Vec8<TO>::store(out + (size_t)(s.ent0 + i) * kRow + j0, o);
+    if (ex.k_tok) {
+      // the entry's indexer key: mean of its tokens' keys (fp32, token order), E4M3 + scale
+      const int cnt = (int)min((int64_t)4, s.n - 4 * i);
+      const int dpl = ex.Di / 32;
+      const size_t kb = (size_t)ex.Di * (ex.k_f32 ? 4 : 2);
+      const uint8_t* krow = reinterpret_cast<const uint8_t*>(ex.k_tok) + (size_t)(s.row0 + 4 * i - s.t0) * kb;
+      float key[4] = {0.f, 0.f, 0.f, 0.f};
+      float amax = 0.f;
+#pragma unroll
+      for (int d = 0; d < 4; ++d) {
+        if (d < dpl) {
+          const int col = lane * dpl + d;
+          float acc = 0.f;
+          for (int q = 0; q < cnt; ++q) {
+            const uint8_t* r = krow + (size_t)q * kb;
+            const float v = ex.k_f32 ? __ldg(reinterpret_cast<const float*>(r) + col)
+                                     : __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16*>(r) + col));
+            acc = q == 0 ? v : __fadd_rn(acc, v);
+          }
+          key[d] = __fdiv_rn(acc, (float)cnt);
+          amax = fmaxf(amax, fabsf(key[d]));
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+      uint32_t packed = 0;
+#pragma unroll
+      for (int d = 0; d < 4; ++d)
+        if (d < dpl)
+          packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(key[d], scale), __NV_SATFINITE, __NV_E4M3) << (8 * d);
+      uint8_t* dst = ex.k_codes + (size_t)(s.ent0 + i) * ex.Di + lane * dpl;
+      if (dpl == 2)
+        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+      else
+        *reinterpret_cast<uint32_t*>(dst) = packed;
+      if (lane == 0) ex.k_scale[s.ent0 + i] = scale;
+    }
   }
 }
 
@@ -378,7 +440,7 @@ static cudaError_t launch_csa_t(const void* xa, const void* za, const void* xb, 
                                 const float* ba, const float* bb, const int64_t* tok_off,
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
-                                void* out, int* st, cudaStream_t stream) {
+                                void* out, const CsaExtras& ex, int* st, cudaStream_t stream) {
   // a whole-cache call runs a bounded grid whose warps loop over the entries
   const int64_t ctas = (max_blocks + kCsaWarps - 1) / kCsaWarps;
   dim3 grid((unsigned)(ctas < kCsaGridCtas ? ctas : kCsaGridCtas), (unsigned)batch);
@@ -387,11 +449,11 @@ static cudaError_t launch_csa_t(const void* xa, const void* za, const void* xb, 
   if (xb != nullptr)
     e = launch_dependent(csa_compress_kernel<TI, TO, true>, grid, dim3(32 * kCsaWarps), 0, stream, (const TI*)xa,
                          (const TI*)za, (const TI*)xb, (const TI*)zb, ba, bb, tok_off, tok0, ent_off, first, num,
-                         max_blocks, (TO*)out, st);
+                         max_blocks, (TO*)out, ex, st);
   else
     e = launch_dependent(csa_compress_kernel<TI, TO, false>, grid, dim3(32 * kCsaWarps), 0, stream, (const TI*)xa,
                          (const TI*)za, (const TI*)nullptr, (const TI*)nullptr, ba, bb, tok_off, tok0, ent_off,
-                         first, num, max_blocks, (TO*)out, st);
+                         first, num, max_blocks, (TO*)out, ex, st);
   note_launch();
   return e;
 }
@@ -400,18 +462,25 @@ cudaError_t launch_csa_compress(const void* xa, const void* za, const void* xb, 
                                 const float* ba, const float* bb, const int64_t* tok_off,
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
-                                int in_dt, int out_dt, void* out, int* st, cudaStream_t stream) {
+                                int in_dt, int out_dt, void* out, int norm, const float* gamma, float eps,
+                                const void* k_tok, int k_dt, int Di, uint8_t* k_codes, float* k_scale, int* st,
+                                cudaStream_t stream) {
+  // many entries: the TMA-ring kernel (one CTA per SM); a few (a decode step): warp per entry
+  if (max_blocks >= kCsaBulkMinEntries)
+    return launch_csa_bulk(xa, za, xb, zb, ba, bb, tok_off, tok0, batch, ent_off, first, num, max_blocks, in_dt,
+                           out_dt, out, gamma, eps, norm, k_tok, k_dt, Di, k_codes, k_scale, st, stream);
+  CsaExtras ex{norm, gamma, eps, k_tok, k_dt == CSKV_F32, Di, k_codes, k_scale};
   if (in_dt == CSKV_BF16 && out_dt == CSKV_BF16)
     return launch_csa_t<__nv_bfloat16, __nv_bfloat16>(xa, za, xb, zb, ba, bb, tok_off, tok0, batch,
-                                                      ent_off, first, num, max_blocks, out, st, stream);
+                                                      ent_off, first, num, max_blocks, out, ex, st, stream);
   if (in_dt == CSKV_BF16 && out_dt == CSKV_F32)
     return launch_csa_t<__nv_bfloat16, float>(xa, za, xb, zb, ba, bb, tok_off, tok0, batch, ent_off,
-                                              first, num, max_blocks, out, st, stream);
+                                              first, num, max_blocks, out, ex, st, stream);
   if (in_dt == CSKV_F32 && out_dt == CSKV_BF16)
     return launch_csa_t<float, __nv_bfloat16>(xa, za, xb, zb, ba, bb, tok_off, tok0, batch, ent_off,
-                                              first, num, max_blocks, out, st, stream);
+                                              first, num, max_blocks, out, ex, st, stream);
   return launch_csa_t<float, float>(xa, za, xb, zb, ba, bb, tok_off, tok0, batch, ent_off, first, num,
-                                    max_blocks, out, st, stream);
+                                    max_blocks, out, ex, st, stream);
 }
 
 template <typename TI, typename TO>
@@ -435,7 +504,13 @@ static cudaError_t launch_hca_t(const void* x, const void* z, const float* bias,
 cudaError_t launch_hca_compress(const void* x, const void* z, const float* bias, const int64_t* tok_off,
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
-                                int in_dt, int out_dt, void* out, int* st, cudaStream_t stream) {
+                                int in_dt, int out_dt, void* out, int norm, const float* gamma, float eps, int* st,
+                                cudaStream_t stream) {
+  // many entries, or RMSNorm (which needs a whole entry in one CTA): the TMA-ring kernel;
+  // a few entries (a decode step): sixteen small CTAs per entry
+  if (norm || max_blocks >= kHcaBulkMinEntries)
+    return launch_hca_bulk(x, z, bias, tok_off, tok0, batch, ent_off, first, num, max_blocks, in_dt, out_dt, out,
+                           gamma, eps, norm, st, stream);
   if (in_dt == CSKV_BF16 && out_dt == CSKV_BF16)
     return launch_hca_t<__nv_bfloat16, __nv_bfloat16>(x, z, bias, tok_off, tok0, batch, ent_off, first,
                                                       num, max_blocks, out, st, stream);

@@ -258,34 +258,6 @@ struct IdxShared {
   long long plan_V[kMaxSplitQueries];
 };
 
-// ------------------------------------------------------------------ ring stage release
-// A consumer warp releases a ring stage by adding one to the stage's counter (release
-// semantics: its reads of the stage are ordered before the increment).  The producer refills
-// the stage when the counter shows every consumer warp's release of every earlier fill; a
-// plain counter in shared memory can only move when a consumer warp of this CTA moves it.
-__device__ __forceinline__ void release_stage(unsigned* ctr) {
-  asm volatile("red.release.cta.shared::cta.add.u32 [%0], 1;" ::"r"(smem_u32(ctr)) : "memory");
-}
-
-// Waits until *ctr >= target, polling with an acquire load (backing off after a few polls);
-// gives up after about a second of polling (false).  The proxy fence then orders the
-// consumers' reads of the stage before the TMA unit's writes into it.
-// Also gives up (false) as soon as *err is set: a consumer warp that gave up never releases.
-__device__ __forceinline__ bool wait_released(unsigned* ctr, unsigned target, const int* err) {
-  const uint32_t a = smem_u32(ctr);
-  for (long n = 0; n < (1L << 24); ++n) {
-    unsigned v;
-    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-    if (v >= target) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      return true;
-    }
-    if (*(const volatile int*)err) return false;
-    if (n >= 32) __nanosleep(64);
-  }
-  return false;
-}
-
 // ------------------------------------------------------------------ scan: E4M3 via TMA + MMA
 // Returns false when a bounded wait gave up (CSKV_DEV_TIMEOUT is flagged).  The ring region is
 // then left untouched by the caller: every fill the producer issued has been waited for (the

@@ -38,16 +38,31 @@ cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-// compress.cu
+// compress.cu (a few entries: decode shapes) and compress_bulk.cu (many: TMA rings)
+constexpr int64_t kCsaBulkMinEntries = 512;  // at or above: the TMA-ring CSA kernel
+constexpr int64_t kHcaBulkMinEntries = 128;  // at or above: the TMA-ring HCA kernel
 cudaError_t launch_csa_compress(const void* xa, const void* za, const void* xb, const void* zb,
                                 const float* ba, const float* bb, const int64_t* tok_off,
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
-                                int in_dt, int out_dt, void* out, int* st, cudaStream_t stream);
+                                int in_dt, int out_dt, void* out, int norm, const float* gamma, float eps,
+                                const void* k_tok, int k_dt, int Di, uint8_t* k_codes, float* k_scale, int* st,
+                                cudaStream_t stream);
 cudaError_t launch_hca_compress(const void* x, const void* z, const float* bias, const int64_t* tok_off,
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
-                                int in_dt, int out_dt, void* out, int* st, cudaStream_t stream);
+                                int in_dt, int out_dt, void* out, int norm, const float* gamma, float eps, int* st,
+                                cudaStream_t stream);
+cudaError_t launch_csa_bulk(const void* xa, const void* za, const void* xb, const void* zb, const float* ba,
+                            const float* bb, const int64_t* tok_off, const int64_t* tok0, int batch,
+                            const int64_t* ent_off, const int64_t* first, const int64_t* num, int64_t max_blocks,
+                            int in_dt, int out_dt, void* out, const float* gamma, float eps, int norm,
+                            const void* k_tok, int k_dt, int Di, uint8_t* k_codes, float* k_scale, int* st,
+                            cudaStream_t stream);
+cudaError_t launch_hca_bulk(const void* x, const void* z, const float* bias, const int64_t* tok_off,
+                            const int64_t* tok0, int batch, const int64_t* ent_off, const int64_t* first,
+                            const int64_t* num, int64_t max_blocks, int in_dt, int out_dt, void* out,
+                            const float* gamma, float eps, int norm, int* st, cudaStream_t stream);
 cudaError_t launch_pool_keys(const void* k_tok, int in_dt, int Di, const int64_t* tok_off, const int64_t* tok0,
                              int batch, const int64_t* ent_off, const int64_t* first, const int64_t* num,
                              int64_t max_blocks, uint8_t* codes, float* scales, int* st, cudaStream_t stream);

@@ -98,12 +98,32 @@ CSKV_API unsigned long long cskv_launch_count(void);
  *                      skipped and flagged CSKV_DEV_CAPACITY.
  * out                : [*, 256] out_dtype (CSKV_F32 or CSKV_BF16; bf16 rounds to
  *                      nearest even).  fp32 arithmetic inside.
+ * rmsnorm, norm_gamma, norm_eps : [SW] §十四.3 (queries and KV are RMS-normalised
+ *                      so that attention logits cannot blow up).  rmsnorm = 1
+ *                      normalises every entry written, on its fp32 value before
+ *                      the output rounding, over its K half and over its V half
+ *                      separately: y = x / sqrt(mean(x^2) + norm_eps) * gamma, with
+ *                      norm_gamma [256] fp32 (K gains then V gains; NULL = ones,
+ *                      4-byte aligned) and norm_eps >= 0 finite.  rmsnorm = 0: no
+ *                      normalisation (norm_gamma / norm_eps unused).
+ * k_tok, k_dtype, Di, k_codes, k_scale : optional (k_tok NULL = off): also pool the
+ *                      indexer's per-token keys of the same entries, exactly as
+ *                      lindex_pool_keys does ([TR] §4.2): k_tok [rows, Di] k_dtype
+ *                      (CSKV_F32 / CSKV_BF16; rows indexed like x_a, 16-byte
+ *                      aligned), Di 64 or 128; entry i of sequence b writes
+ *                      k_codes[ent_off[b] + i, :] (E4M3, 16-byte aligned) and
+ *                      k_scale[ent_off[b] + i] (fp32).
+ * Many entries (max_blocks >= 512) run a TMA-ring kernel, one CTA per SM; a few
+ * (a decode step) run a warp per entry.  Both give the same results up to fp32
+ * rounding order.
  * ------------------------------------------------------------------------ */
 CSKV_API int csa_compress(const void* x_a, const void* z_a, const void* x_b, const void* z_b,
                  const float* bias_a, const float* bias_b,
                  const int64_t* tok_off, const int64_t* tok0, int batch,
                  const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
                  int64_t max_blocks, int in_dtype, int out_dtype, void* out,
+                 int rmsnorm, const float* norm_gamma, float norm_eps,
+                 const void* k_tok, int k_dtype, int Di, uint8_t* k_codes, float* k_scale,
                  int* dev_status, cskv_stream_t stream);
 
 /* ------------------------------------------------------------------------
@@ -111,12 +131,15 @@ CSKV_API int csa_compress(const void* x_a, const void* z_a, const void* x_b, con
  *
  * [SW] §三.3, [TR] §4.3 (HCA, no dual stream): entry i mixes the tokens of
  * block i (value x[t,j], logit z[t,j] + bias[t-128i, j]) with one softmax per
- * dimension.  Arguments as csa_compress; bias is [128, 256] fp32 or NULL.
+ * dimension.  Arguments as csa_compress (no key pooling); bias is [128, 256]
+ * fp32 or NULL.  Many entries (max_blocks >= 128) or rmsnorm = 1 run a TMA-ring
+ * kernel with one CTA per entry at a time; a few run sixteen small CTAs per entry.
  * ------------------------------------------------------------------------ */
 CSKV_API int hca_compress(const void* x, const void* z, const float* bias,
                  const int64_t* tok_off, const int64_t* tok0, int batch,
                  const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
                  int64_t max_blocks, int in_dtype, int out_dtype, void* out,
+                 int rmsnorm, const float* norm_gamma, float norm_eps,
                  int* dev_status, cskv_stream_t stream);
 
 /* ------------------------------------------------------------------------

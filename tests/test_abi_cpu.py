@@ -56,25 +56,35 @@ def _p(v=0x1000):
 
 def test_compress_validation(lib):
     nul = None
-    # null rows
-    assert lib.csa_compress(nul, _p(), nul, nul, nul, nul, _p(), nul, 1, _p(), nul, nul, 4, 1, 1, _p(), nul,
-                            nul) == _lib.ERR_INVALID_ARG
-    # x_b without z_b
-    assert lib.csa_compress(_p(), _p(), _p(), nul, nul, nul, _p(), nul, 1, _p(), nul, nul, 4, 1, 1, _p(), nul,
-                            nul) == _lib.ERR_INVALID_ARG
-    # misaligned output
-    assert lib.csa_compress(_p(), _p(), nul, nul, nul, nul, _p(), nul, 1, _p(), nul, nul, 4, 1, 1, _p(0x1004), nul,
-                            nul) == _lib.ERR_INVALID_ARG
-    # fp8 rows are not a compression input
-    assert lib.hca_compress(_p(), _p(), nul, _p(), nul, 1, _p(), nul, nul, 4, 2, 1, _p(), nul,
-                            nul) == _lib.ERR_UNSUPPORTED
-    # bad batch / bad enum
-    assert lib.hca_compress(_p(), _p(), nul, _p(), nul, 0, _p(), nul, nul, 4, 1, 1, _p(), nul,
-                            nul) == _lib.ERR_INVALID_ARG
-    assert lib.hca_compress(_p(), _p(), nul, _p(), nul, 1, _p(), nul, nul, 4, 7, 1, _p(), nul,
-                            nul) == _lib.ERR_INVALID_ARG
+
+    def csa(x=_p(), z=_p(), xb=nul, zb=nul, out=_p(), in_dt=1, out_dt=1, max_blocks=4, norm=0, gamma=nul, eps=1e-6,
+            k_tok=nul, k_dt=1, Di=64, codes=_p(), scale=_p()):
+        return lib.csa_compress(x, z, xb, zb, nul, nul, _p(), nul, 1, _p(), nul, nul, max_blocks, in_dt, out_dt, out,
+                                norm, gamma, eps, k_tok, k_dt, Di, codes, scale, nul, nul)
+
+    def hca(batch=1, in_dt=1, max_blocks=4, norm=0, gamma=nul, eps=1e-6):
+        return lib.hca_compress(_p(), _p(), nul, _p(), nul, batch, _p(), nul, nul, max_blocks, in_dt, 1, _p(), norm,
+                                gamma, eps, nul, nul)
+
+    assert csa(x=nul) == _lib.ERR_INVALID_ARG               # null rows
+    assert csa(xb=_p()) == _lib.ERR_INVALID_ARG             # x_b without z_b
+    assert csa(out=_p(0x1004)) == _lib.ERR_INVALID_ARG      # misaligned output
+    assert hca(in_dt=2) == _lib.ERR_UNSUPPORTED             # fp8 rows are not a compression input
+    assert hca(batch=0) == _lib.ERR_INVALID_ARG             # bad batch / bad enum
+    assert hca(in_dt=7) == _lib.ERR_INVALID_ARG
+    # RMSNorm arguments
+    assert csa(norm=2) == _lib.ERR_INVALID_ARG
+    assert hca(norm=1, eps=-1.0) == _lib.ERR_INVALID_ARG
+    assert hca(norm=1, eps=float("nan")) == _lib.ERR_INVALID_ARG
+    assert hca(norm=1, gamma=_p(0x1002)) == _lib.ERR_INVALID_ARG
+    # fused key pooling arguments
+    assert csa(k_tok=_p(), codes=nul) == _lib.ERR_INVALID_ARG
+    assert csa(k_tok=_p(), Di=96) == _lib.ERR_UNSUPPORTED
+    assert csa(k_tok=_p(), k_dt=2) == _lib.ERR_UNSUPPORTED
+    assert csa(k_tok=_p(0x1008)) == _lib.ERR_INVALID_ARG
     # nothing to do
-    assert lib.hca_compress(_p(), _p(), nul, _p(), nul, 1, _p(), nul, nul, 0, 1, 1, _p(), nul, nul) == _lib.OK
+    assert hca(max_blocks=0) == _lib.OK
+    assert csa(max_blocks=0, norm=1, k_tok=_p()) == _lib.OK
 
 
 def test_indexer_validation(lib):
