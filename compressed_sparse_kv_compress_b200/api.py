@@ -104,6 +104,24 @@ def lindex_score_topk(q_idx, k_idx, q_seq, q_pos, ent_off, out_idx, workspace, *
     return out_idx
 
 
+def lindex_score_topk_mxfp4(q_codes, q_bscale, k_codes, k_bscale, q_seq, q_pos, ent_off, out_idx, workspace, *,
+                            max_entries, q_scale=None, head_w=None, out_score=None, prefetch_rows=None,
+                            dev_status=None, stream=None):
+    """MXFP4 indexer vectors: q_codes [T, Hi, Di/2] / k_codes [Nc, Di/2] uint8 (two E2M1 codes a
+    byte) with E8M0 block scales q_bscale [T, Hi, Di/32] / k_bscale [Nc, Di/32] uint8."""
+    T, Hi, half = q_codes.shape
+    lib = _lib.load()
+    pf_bytes = 0 if prefetch_rows is None else prefetch_rows[0].numel() * prefetch_rows.element_size()
+    st = lib.lindex_score_topk_mxfp4(_ptr(q_codes), _ptr(q_bscale), _ptr(q_scale), _ptr(k_codes), _ptr(k_bscale),
+                                     _ptr(head_w), _ptr(q_seq), _ptr(q_pos), _ptr(ent_off), ent_off.numel() - 1, T,
+                                     Hi, 2 * half, out_idx.shape[1], int(max_entries), _ptr(out_idx),
+                                     _ptr(out_score), _ptr(prefetch_rows), pf_bytes, _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                     _stream(stream))
+    _lib.check("lindex_score_topk_mxfp4", st)
+    return out_idx
+
+
 def lindex_topk_from_scores(scores, n_valid, out_idx, workspace, *, max_entries, out_score=None, dev_status=None,
                             stream=None):
     T, ld = scores.shape

@@ -211,6 +211,48 @@ int lindex_score_topk(const void* q_idx, const float* q_scale, const void* k_idx
   return launch_status(launch_lindex(p, dtype, T, (cudaStream_t)stream));
 }
 
+int lindex_score_topk_mxfp4(const uint8_t* q_codes, const uint8_t* q_bscale, const float* q_scale,
+                            const uint8_t* k_codes, const uint8_t* k_bscale, const float* head_w,
+                            const int32_t* q_seq, const int64_t* q_pos, const int64_t* ent_off, int batch, int T,
+                            int Hi, int Di, int k, int64_t max_entries, int32_t* out_idx, float* out_score,
+                            const void* prefetch_rows, int64_t prefetch_row_bytes, void* workspace, size_t ws_bytes,
+                            int* dev_status, cskv_stream_t stream) {
+  if (Hi < 1 || Hi > 16 || (Di != 64 && Di != 128)) return Hi >= 1 && Di > 0 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+  if (T > 0 && (!q_codes || !q_bscale || !k_codes || !k_bscale || !q_seq || !q_pos || !ent_off || batch < 1))
+    return CSKV_ERR_INVALID_ARG;
+  // codes are read in 16-byte tiles and 4-byte words; a key's Di/32 scale bytes as one 2- or
+  // 4-byte word
+  if (!aligned16(q_codes) || !aligned16(k_codes) || (reinterpret_cast<uintptr_t>(k_bscale) % (Di / 32)))
+    return CSKV_ERR_INVALID_ARG;
+  if (prefetch_rows && (!aligned16(prefetch_rows) || prefetch_row_bytes <= 0 || prefetch_row_bytes % 16 != 0 ||
+                        prefetch_row_bytes > (1 << 20)))
+    return CSKV_ERR_INVALID_ARG;
+  int rc = check_topk_common(T, k, max_entries, out_idx, workspace, ws_bytes);
+  if (rc || T == 0) return rc;
+  IdxParams p = {};
+  p.q_idx = q_codes;
+  p.q_scale = q_scale;
+  p.k_idx = k_codes;
+  p.q_bs = q_bscale;
+  p.k_bs = k_bscale;
+  p.head_w = head_w;
+  p.q_seq = q_seq;
+  p.q_pos = q_pos;
+  p.ent_off = ent_off;
+  p.batch = batch;
+  p.Hi = Hi;
+  p.Di = Di;
+  p.k = k;
+  p.max_entries = max_entries;
+  p.out_idx = out_idx;
+  p.out_score = out_score;
+  p.pf_rows = prefetch_rows ? (const uint8_t*)prefetch_rows : nullptr;
+  p.pf_row_bytes = prefetch_rows ? prefetch_row_bytes : 0;
+  p.ws = (QueryWS*)workspace;
+  p.st = dev_status;
+  return launch_status(launch_lindex(p, CSKV_FP8E4M3, T, (cudaStream_t)stream));
+}
+
 int lindex_topk_from_scores(const float* scores, int64_t ld_scores, const int64_t* n_valid, int T, int k,
                             int64_t max_entries, int32_t* out_idx, float* out_score, void* workspace,
                             size_t ws_bytes, int* dev_status, cskv_stream_t stream) {

@@ -30,7 +30,9 @@ constexpr int kTcThreads = 128;
 constexpr int kTcChunk = 128;                      // rows per chunk (MMA N of S, K of PV)
 constexpr uint32_t kRegion = 128 * 128;             // 128 rows x 128 bytes: one swizzled region
 constexpr uint32_t kTileBytes = 2 * kRegion;        // one 128 x 128 bf16 operand tile
-constexpr size_t kTcSmem = 4 * (size_t)kTileBytes + 1024;
+// Q, K||V and P tiles; P takes K's place (K is dead once S = Q K^T has completed), so a CTA
+// needs ~97 KB and fits on an SM beside the indexer's CTA.
+constexpr size_t kTcSmem = 3 * (size_t)kTileBytes + 1024;
 
 // Byte offset of 16-byte chunk c of row r (c < 16 for a 256-byte row, < 32 for a 512-byte
 // K||V row) in the 128-byte-swizzle layout.
@@ -49,7 +51,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   uint8_t* Qs = sm;                   // A of S = Q K^T   [128 heads x 128 d], K-major
   uint8_t* KVs = sm + kTileBytes;     // K: B of S [128 rows x 128 d], K-major (regions 0-1);
                                       // V: B of O = P V [128 rows (K) x 128 d (N)], MN-major (2-3)
-  uint8_t* Ps = sm + 3 * kTileBytes;  // A of O = P V     [128 heads x 128 rows], K-major
+  uint8_t* Ps = KVs;                  // A of O = P V     [128 heads x 128 rows], K-major: K's regions,
+                                      // written only after the S MMA has read K (bar_s)
   __shared__ uint64_t bar_s, bar_o;
   __shared__ uint32_t tmem_base;
   __shared__ const __nv_bfloat16* row_src[kTcChunk];  // address of each chunk row, null = skipped

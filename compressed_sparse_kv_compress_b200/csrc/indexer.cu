@@ -39,6 +39,8 @@
 // a tile and run m16n8k32 E4M3 MMAs (entries x dims) x (dims x 8 heads) with fp32
 // accumulation -- the head dimension fills N = 8 exactly -- then apply scales, ReLU and
 // the head sum in registers.
+#include <type_traits>
+
 #include "launch.cuh"
 #include "sm100.cuh"
 
@@ -60,7 +62,7 @@ constexpr int kMaxSplitQueries = 128;
 constexpr int kIdxMaxHeads = 16;
 constexpr int kIdxMaxDim = 128;
 
-enum IdxSrc { kSrcFp8 = 0, kSrcF32 = 1, kSrcScores = 2 };
+enum IdxSrc { kSrcFp8 = 0, kSrcF32 = 1, kSrcScores = 2, kSrcFp4 = 3 };
 
 
 struct alignas(16) QueryWS {
@@ -73,8 +75,10 @@ struct alignas(16) QueryWS {
 };
 
 
-// TMA ring depth: 64 KiB of k_idx tiles in flight per CTA whatever Di is.
+// TMA ring depth: at least 64 KiB of k_idx tiles in flight per CTA whatever Di is; deeper (up
+// to kIdxMaxStages, the whole segment when it fits) where shared memory allows (run_topk).
 __host__ __device__ constexpr int idx_stages(int Di) { return (64 * 1024) / (kIdxTile * Di); }
+constexpr int kIdxMaxStages = 16;
 
 // Layout of the shared region after the scan: histogram, candidate keys, then a scratch
 // area used first as the owner table of the gathered proposals, then for the keys of the
@@ -85,11 +89,25 @@ constexpr size_t kUnAux = kUnCand + (size_t)kCandMax * 8;
 constexpr int kAuxKeys = 1024;  // 8 KiB: kCandMax owner entries (2 B) or kAuxKeys keys (8 B)
 constexpr size_t kUnSelBytes = kUnAux + (size_t)kAuxKeys * 8;
 
-// Bytes of the shared region used first as the TMA ring, then for the histogram and the
-// candidate keys.
-__host__ __device__ constexpr size_t idx_union_bytes(int Di) {
-  return (size_t)idx_stages(Di) * kIdxTile * Di > kUnSelBytes ? (size_t)idx_stages(Di) * kIdxTile * Di
-                                                                : kUnSelBytes;
+// Bytes of the shared region used first as the TMA ring (`stages` tiles), then for the
+// histogram and the candidate keys.
+__host__ __device__ constexpr size_t idx_union_bytes(int Di, int stages) {
+  return (size_t)stages * kIdxTile * Di > kUnSelBytes ? (size_t)stages * kIdxTile * Di : kUnSelBytes;
+}
+
+// ------------------------------------------------------------------ MXFP4 helpers
+// Four E2M1 codes (code i in bits 4i..4i+3: sign bit 3, exponent bits 2..1 with bias 1,
+// mantissa bit 0; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) -> the four E4M3 bytes of the same
+// values (every E2M1 value is exact in E4M3): a byte permute over the table of the eight
+// magnitudes' E4M3 codes, then the sign bits moved to bit 7 of each byte.
+__device__ __forceinline__ uint32_t e2m1x4_to_e4m3x4(uint32_t c) {
+  const uint32_t mag = __byte_perm(0x3C383000u, 0x4C484440u, c & 0x7777u);
+  const uint32_t spread = (c & 0x000Fu) | ((c & 0x00F0u) << 4) | ((c & 0x0F00u) << 8) | ((c & 0xF000u) << 12);
+  return mag | ((spread << 4) & 0x80808080u);
+}
+// E8M0 scale code -> 2^(code - 127) (code 0 is the subnormal 2^-127, 0xFF is NaN).
+__device__ __forceinline__ float e8m0_to_float(uint32_t c) {
+  return c == 0u ? __uint_as_float(0x00400000u) : (c == 255u ? __uint_as_float(0x7fc00000u) : __uint_as_float(c << 23));
 }
 
 // ------------------------------------------------------------------ keys
@@ -211,21 +229,23 @@ __device__ Crossing find_crossing(const unsigned* hist, int nbins, unsigned r, u
 }
 
 // Barrier over the G CTAs of one query group (all co-resident: cooperative launch), on one
-// counter whose top bit is the barrier's phase.  Thread 0 reads the counter (the phase cannot
-// change before this CTA arrives), publishes the CTA's writes with a fence (cumulative over
-// the block barrier before it) and arrives with a reduction that needs no reply: CTA 0 of the
-// group adds 2^31 - (G - 1), every other CTA adds 1, so the sum of the G arrivals is exactly
-// 2^31 -- the phase bit flips when the last one lands and the low bits are back where they
-// were (zero), for any G, with no reset.  Waiters poll until the phase differs.  Bounded:
+// counter whose top bit is the barrier's phase.  Thread 0 arrives with one atomic add that is a
+// release (it publishes the CTA's writes) and returns the counter before it, whose phase bit is
+// the phase being completed (it cannot change before this CTA arrives): CTA 0 of the group adds
+// 2^31 - (G - 1), every other CTA adds 1, so the sum of the G arrivals is exactly 2^31 -- the
+// phase bit flips when the last one lands and the low bits are back where they were (zero), for
+// any G, with no reset.  Waiters poll (acquire) until the phase differs.  Bounded:
 // gives up after a few million polls, about a second (CSKV_DEV_TIMEOUT).
 __device__ bool group_barrier(QueryWS* ws, unsigned G, int j, int* st, int* sm_flag) {
   __syncthreads();
   if (threadIdx.x == 0) {
     bool ok = true;
-    const unsigned before = ld_acquire_gpu(&ws->bar_count);
     const unsigned add = j == 0 ? 0x80000000u - (G - 1u) : 1u;
-    __threadfence();
-    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(&ws->bar_count), "r"(add) : "memory");
+    // the arrival is a release (cumulative over the block barrier before it: every write of the
+    // CTA is visible before it) and returns the counter, whose top bit is the phase this CTA
+    // arrives in
+    unsigned before;
+    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(before) : "l"(&ws->bar_count), "r"(add) : "memory");
     long it = 0;
     while (((ld_acquire_gpu(&ws->bar_count) ^ before) & 0x80000000u) == 0u) {  // an L2 round trip each
       if (++it > (1L << 22)) {
@@ -242,8 +262,8 @@ __device__ bool group_barrier(QueryWS* ws, unsigned G, int j, int* st, int* sm_f
 
 // ------------------------------------------------------------------ shared state
 struct IdxShared {
-  uint64_t full[12];
-  unsigned released[12];  // per ring stage: consumer warps done with it, all fills so far
+  uint64_t full[kIdxMaxStages];
+  unsigned released[kIdxMaxStages];  // per ring stage: consumer warps done with it, all fills so far
   int fills;              // fills the producer issued (read by the drain after a timeout)
   int scan_err;           // a bounded wait of the scan gave up
   unsigned red[32];
@@ -263,11 +283,22 @@ struct IdxShared {
 // then left untouched by the caller: every fill the producer issued has been waited for (the
 // drain below), or, when even that wait gave up, the barriers are not retired and the caller
 // must not touch the ring memory again.
-template <int KS, int NTILE>
-__device__ bool scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, int len,
-                         float* sc, uint8_t* ring, IdxShared& S) {
+//
+// FP4 = false: E4M3 keys and queries ([SW] §六.1 FP8), fp32 scales per entry (kscale) and per
+// (query, head).  FP4 = true: OCP MXFP4 keys and queries ([SW] §六.1 / §十三.4 and [TR] §4.2: the
+// indexer's QK path may run in FP4): E2M1 codes two per byte (element 2j in the low nibble) with
+// one E8M0 scale per 32 elements (kbs: the entry's Di/32 scale bytes; p.q_bs for the queries).
+// E2M1 values are exact in E4M3, so the codes are widened in registers and the same E4M3 MMA
+// runs once per 32-element block: thread (g, tq) takes elements 32b + 8tq .. 32b + 8tq + 7 of
+// block b for its rows and heads (one 32-bit load of codes), which keeps every MMA inside one
+// block; the block's dot product is then multiplied by the two power-of-two scales.
+template <int KS, int NTILE, bool FP4>
+__device__ bool scan_mma(const IdxParams& p, int t, const uint8_t* kbase, const float* kscale, const uint8_t* kbs,
+                         int len, float* sc, uint8_t* ring, IdxShared& S) {
   constexpr int Di = KS * 32;
-  constexpr int stages = idx_stages(Di);
+  constexpr int RB = FP4 ? Di / 2 : Di;  // key bytes per entry in the tile
+  constexpr int NB = Di / 32;            // MX blocks per key (FP4)
+  const int stages = p.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = (len + kIdxTile - 1) / kIdxTile;
   if (threadIdx.x == 0) {
@@ -297,9 +328,9 @@ __device__ bool scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
           break;
         }
         const int rows = min(kIdxTile, len - it * kIdxTile);
-        const unsigned bytes = (unsigned)(rows * Di);
+        const unsigned bytes = (unsigned)(rows * RB);
         mbar_arrive_expect_tx(&S.full[s], bytes);
-        tma_bulk_g2s(ring + (size_t)s * kIdxTile * Di, kbase + (size_t)it * kIdxTile * Di, bytes, &S.full[s]);
+        tma_bulk_g2s(ring + (size_t)s * kIdxTile * RB, kbase + (size_t)it * kIdxTile * RB, bytes, &S.full[s]);
         if (++s == stages) s = 0;
       }
       S.fills = it;  // fills issued (the drain below needs the count)
@@ -309,20 +340,33 @@ __device__ bool scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
     // B fragments (the query's heads) and per-head scale / weight, loaded once.
     uint32_t bq[NTILE][KS][2];
     float sq[NTILE][2], wh[NTILE][2];
-    const uint8_t* qrow = p.q_idx + (size_t)t * p.Hi * Di;
+    float fq[NTILE][2][FP4 ? NB : 1];  // FP4: the query heads' block scales
+    const uint8_t* qrow = p.q_idx + (size_t)t * p.Hi * RB;
 #pragma unroll
     for (int nt = 0; nt < NTILE; ++nt) {
       const int h = nt * 8 + g;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        const int chunk = tq + 4 * (ks >> 1), wp = (ks & 1) * 2;
-        if (h < p.Hi) {
+        if (h >= p.Hi) {
+          bq[nt][ks][0] = bq[nt][ks][1] = 0u;
+        } else if constexpr (FP4) {
+          // block ks, elements 32 ks + 8 tq .. + 7: widened to E4M3 (k 4tq.. then 16 + 4tq..)
+          const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(qrow + (size_t)h * RB + 16 * ks + 4 * tq));
+          bq[nt][ks][0] = e2m1x4_to_e4m3x4(w & 0xFFFFu);
+          bq[nt][ks][1] = e2m1x4_to_e4m3x4(w >> 16);
+        } else {
+          const int chunk = tq + 4 * (ks >> 1), wp = (ks & 1) * 2;
           const uint32_t* src = reinterpret_cast<const uint32_t*>(qrow + (size_t)h * Di + chunk * 16);
           bq[nt][ks][0] = __ldg(src + wp);
           bq[nt][ks][1] = __ldg(src + wp + 1);
-        } else {
-          bq[nt][ks][0] = bq[nt][ks][1] = 0u;
         }
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int hh = nt * 8 + 2 * tq + c;
+#pragma unroll
+        for (int bb = 0; bb < (FP4 ? NB : 1); ++bb)
+          fq[nt][c][bb] = (FP4 && hh < p.Hi) ? e8m0_to_float(__ldg(p.q_bs + ((size_t)t * p.Hi + hh) * NB + bb)) : 1.f;
       }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -335,14 +379,25 @@ __device__ bool scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
     // Entry scales of this warp's rows for the next kScalePF tiles, held in registers and
     // shifted along; the first batch is requested before the producer starts streaming, so
     // these small loads are not queued behind the tile traffic.
+    // (FP4: the rows' block-scale bytes, NB per entry, instead of an fp32 scale.)
     constexpr int kScalePF = 8;
     const int r0 = warp * 16;
-    float ska[kScalePF], skb[kScalePF];
+    using SK = typename std::conditional<FP4, uint32_t, float>::type;
+    auto ld_sk = [&](int e) -> SK {
+      if constexpr (FP4) {
+        if (e >= len) return 0u;
+        return NB == 2 ? (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(kbs) + e)
+                       : __ldg(reinterpret_cast<const uint32_t*>(kbs) + e);
+      } else {
+        return e < len ? (kscale ? __ldg(kscale + e) : 1.f) : 0.f;
+      }
+    };
+    SK ska[kScalePF], skb[kScalePF];
 #pragma unroll
     for (int i = 0; i < kScalePF; ++i) {
       const int e = i * kIdxTile + r0 + g;
-      ska[i] = e < len ? (kscale ? __ldg(kscale + e) : 1.f) : 0.f;
-      skb[i] = e + 8 < len ? (kscale ? __ldg(kscale + e + 8) : 1.f) : 0.f;
+      ska[i] = ld_sk(e);
+      skb[i] = ld_sk(e + 8);
     }
     asm volatile("bar.arrive 2, %0;" ::"n"(kIdxThreads) : "memory");
     bool alive = true;
@@ -356,7 +411,7 @@ __device__ bool scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
         break;
       }
       const int rows = min(kIdxTile, len - it * kIdxTile);
-      const float skg = ska[0], skg8 = skb[0];
+      const SK skg = ska[0], skg8 = skb[0];
 #pragma unroll
       for (int i = 0; i + 1 < kScalePF; ++i) {
         ska[i] = ska[i + 1];
@@ -364,8 +419,8 @@ __device__ bool scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
       }
       {
         const int e = (it + kScalePF) * kIdxTile + r0 + g;
-        ska[kScalePF - 1] = e < len ? (kscale ? __ldg(kscale + e) : 1.f) : 0.f;
-        skb[kScalePF - 1] = e + 8 < len ? (kscale ? __ldg(kscale + e + 8) : 1.f) : 0.f;
+        ska[kScalePF - 1] = ld_sk(e);
+        skb[kScalePF - 1] = ld_sk(e + 8);
       }
       // A fragments of this warp's 16 rows into registers and the MMAs on them; the stage
       // goes back to the producer only after the MMAs have consumed every lane's fragments
@@ -376,36 +431,73 @@ __device__ bool scan_fp8(const IdxParams& p, int t, const uint8_t* kbase, const 
         __syncwarp();
         if (lane == 0) release_stage(&S.released[s]);
       } else {
-        uint4 ra[KS / 2], rb[KS / 2];
-        const uint8_t* tile = ring + (size_t)s * kIdxTile * Di;
-#pragma unroll
-        for (int c = 0; c < KS / 2; ++c) {
-          ra[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g) * Di + (tq + 4 * c) * 16);
-          rb[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g + 8) * Di + (tq + 4 * c) * 16);
-        }
+        const uint8_t* tile = ring + (size_t)s * kIdxTile * RB;
         float acc[NTILE][4];
+        float accb[FP4 ? NB : 1][NTILE][4];  // FP4: one accumulator per block
+        if constexpr (FP4) {
+          uint32_t wa[NB], wb[NB];
 #pragma unroll
-        for (int nt = 0; nt < NTILE; ++nt) {
-          acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+          for (int bb = 0; bb < NB; ++bb) {
+            wa[bb] = *reinterpret_cast<const uint32_t*>(tile + (size_t)(r0 + g) * RB + 16 * bb + 4 * tq);
+            wb[bb] = *reinterpret_cast<const uint32_t*>(tile + (size_t)(r0 + g + 8) * RB + 16 * bb + 4 * tq);
+          }
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            const uint4& A = ra[ks >> 1];
-            const uint4& B = rb[ks >> 1];
-            const bool hiw = ks & 1;
-            mma_e4m3_16832(acc[nt], hiw ? A.z : A.x, hiw ? B.z : B.x, hiw ? A.w : A.y, hiw ? B.w : B.y,
-                           bq[nt][ks][0], bq[nt][ks][1]);
+          for (int bb = 0; bb < NB; ++bb) {
+            const uint32_t a0 = e2m1x4_to_e4m3x4(wa[bb] & 0xFFFFu), a2 = e2m1x4_to_e4m3x4(wa[bb] >> 16);
+            const uint32_t a1 = e2m1x4_to_e4m3x4(wb[bb] & 0xFFFFu), a3 = e2m1x4_to_e4m3x4(wb[bb] >> 16);
+#pragma unroll
+            for (int nt = 0; nt < NTILE; ++nt) {
+              accb[bb][nt][0] = accb[bb][nt][1] = accb[bb][nt][2] = accb[bb][nt][3] = 0.f;
+              mma_e4m3_16832(accb[bb][nt], a0, a1, a2, a3, bq[nt][bb][0], bq[nt][bb][1]);
+            }
+          }
+        } else {
+          uint4 ra[KS / 2], rb[KS / 2];
+#pragma unroll
+          for (int c = 0; c < KS / 2; ++c) {
+            ra[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g) * Di + (tq + 4 * c) * 16);
+            rb[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g + 8) * Di + (tq + 4 * c) * 16);
+          }
+#pragma unroll
+          for (int nt = 0; nt < NTILE; ++nt) {
+            acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+              const uint4& A = ra[ks >> 1];
+              const uint4& B = rb[ks >> 1];
+              const bool hiw = ks & 1;
+              mma_e4m3_16832(acc[nt], hiw ? A.z : A.x, hiw ? B.z : B.x, hiw ? A.w : A.y, hiw ? B.w : B.y,
+                             bq[nt][ks][0], bq[nt][ks][1]);
+            }
           }
         }
         __syncwarp();
         if (lane == 0) release_stage(&S.released[s]);
+        if constexpr (FP4) {
+          // each block's exact dot product times 2^(query exponent) * 2^(key exponent)
+#pragma unroll
+          for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              float dg = 0.f, dg8 = 0.f;
+#pragma unroll
+              for (int bb = 0; bb < NB; ++bb) {
+                dg = fmaf(accb[bb][nt][c] * e8m0_to_float((skg >> (8 * bb)) & 0xFFu), fq[nt][c][bb], dg);
+                dg8 = fmaf(accb[bb][nt][2 + c] * e8m0_to_float((skg8 >> (8 * bb)) & 0xFFu), fq[nt][c][bb], dg8);
+              }
+              acc[nt][c] = dg;
+              acc[nt][2 + c] = dg8;
+            }
+        }
         const int e_g = it * kIdxTile + r0 + g, e_g8 = e_g + 8;
+        const float kg = FP4 ? 1.f : (float)skg, kg8 = FP4 ? 1.f : (float)skg8;
         float vg = 0.f, vg8 = 0.f;
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt)
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            vg = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * skg) * acc[nt][c]), vg);
-            vg8 = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * skg8) * acc[nt][2 + c]), vg8);
+            vg = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * kg) * acc[nt][c]), vg);
+            vg8 = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * kg8) * acc[nt][2 + c]), vg8);
           }
         vg += __shfl_xor_sync(0xffffffffu, vg, 1);
         vg += __shfl_xor_sync(0xffffffffu, vg, 2);
@@ -549,38 +641,6 @@ __device__ unsigned count_selected(const float* sc, int len, int64_t lo, uint64_
 }
 
 // ---- speculative exchange helpers
-constexpr int kLinBins = 1024;  // linear score bins (<= kBins0, shares the histogram buffer)
-
-// Block-wide min and max of one float per thread, and the sum of one count per thread.
-__device__ void block_minmax(float mn, float mx, IdxShared& S, float& gmn, float& gmx, int cnt = 0,
-                             int* gcnt = nullptr) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int nw = kIdxThreads / 32;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  }
-  cnt = __reduce_add_sync(0xffffffffu, cnt);
-  if (lane == 0) {
-    S.fred[warp] = mn;
-    S.fred[32 + warp] = mx;
-    S.fcnt[warp] = cnt;
-  }
-  __syncthreads();
-  gmn = INFINITY;
-  gmx = -INFINITY;
-  int c = 0;
-  for (int w = 0; w < nw; ++w) {
-    gmn = fminf(gmn, S.fred[w]);
-    gmx = fmaxf(gmx, S.fred[32 + w]);
-    c += S.fcnt[w];
-  }
-  if (gcnt) *gcnt = c;
-  __syncthreads();
-}
-
-
 // Block-wide max of one 64-bit key per thread.
 __device__ uint64_t block_max_u64(uint64_t v, IdxShared& S) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -598,21 +658,74 @@ __device__ uint64_t block_max_u64(uint64_t v, IdxShared& S) {
   return m;
 }
 
-// Bin (of kBins0) of a key by its score bits above the smallest proposal's: the score key
-// minus the lowest one, shifted so that the range fits.  Monotone in the key; for scores of
-// one sign the bins are about uniform in log(score), so a few outlying large scores (planted
-// or real) do not crowd every other proposal into a handful of bins.
-__device__ __forceinline__ unsigned key_bin4k(uint64_t c, uint32_t kmin, int shift) {
-  const uint32_t d = (uint32_t)(c >> 32) - kmin;
-  const uint32_t b = d >> shift;
-  return b < (uint32_t)kBins0 ? b : (uint32_t)(kBins0 - 1);
+// Log-scale bins below a maximum score key: for scores of one sign the score key grows by 2^23
+// per octave, so (key_max - key) >> shift puts 2^(23 - shift) bins in every octave.  Monotone
+// (decreasing) in the key; keys more than the range below the maximum share the last bin.
+__device__ __forceinline__ unsigned log_bin(uint32_t kmax, uint32_t key, int shift, unsigned nbins) {
+  const uint32_t b = (kmax - key) >> shift;
+  return b < nbins ? b : nbins - 1u;
 }
+constexpr int kPropBins = 1024;  // proposal bins below the CTA's best score: 128 per octave
+constexpr int kPropShift = 16;
+constexpr int kTBins = kBins0;   // T* bins below the group's best proposal, sized to the proposals' range
 
-
-// Linear bin of a score inside [lo, lo + 1024/scl]; monotone in s.
-__device__ __forceinline__ unsigned lin_bin(float s, float lo, float scl) {
-  const float f = (s - lo) * scl;
-  return f <= 0.f ? 0u : (f >= (float)(kLinBins - 1) ? (unsigned)(kLinBins - 1) : (unsigned)f);
+// Over NB bins ordered from the best scores down, the first bin at which the running count
+// exceeds `limit`: *out = {that bin, the count of the bins before it, its count}, or {NB, the
+// total, 0} when the count never exceeds the limit.  All threads take part: thread t holds bins
+// [t * NB / kIdxThreads, ...) in registers (one or two vector loads: no bank conflicts), one
+// block scan, then the thread whose bins hold the cut writes it.  Two block barriers.
+template <int NB>
+__device__ void block_cut(const unsigned* hist, unsigned limit, Crossing* out, IdxShared& S) {
+  constexpr int per = NB / kIdxThreads;
+  static_assert(per == 2 || per == 8, "bins per thread");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned v[per];
+  if constexpr (per == 2) {
+    const uint2 w = reinterpret_cast<const uint2*>(hist)[tid];
+    v[0] = w.x;
+    v[1] = w.y;
+  } else {
+    const uint4 w0 = reinterpret_cast<const uint4*>(hist)[2 * tid], w1 = reinterpret_cast<const uint4*>(hist)[2 * tid + 1];
+    v[0] = w0.x; v[1] = w0.y; v[2] = w0.z; v[3] = w0.w;
+    v[4] = w1.x; v[5] = w1.y; v[6] = w1.z; v[7] = w1.w;
+  }
+  unsigned loc = 0;
+#pragma unroll
+  for (int i = 0; i < per; ++i) loc += v[i];
+  unsigned inc = loc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) S.red[warp] = inc;
+  __syncthreads();
+  unsigned excl = inc - loc, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kIdxThreads / 32; ++w) {
+    const unsigned r = S.red[w];
+    excl += w < warp ? r : 0u;
+    tot += r;
+  }
+  if (excl <= limit && excl + loc > limit) {
+    unsigned c = excl;
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+      if (c + v[i] > limit) {
+        out->bin = (unsigned)(tid * per + i);
+        out->above = c;
+        out->cnt = v[i];
+        break;
+      }
+      c += v[i];
+    }
+  }
+  if (tid == 0 && tot <= limit) {
+    out->bin = (unsigned)NB;
+    out->above = tot;
+    out->cnt = 0u;
+  }
+  __syncthreads();
 }
 
 // Returns the group's synchronisation state (and any global histogram it used) to zero;
@@ -640,248 +753,101 @@ __device__ void group_cleanup(QueryWS* ws, int G, bool used_hist0, int used_pass
   __syncthreads();
 }
 
-// ---- speculative proposals: fill this CTA's `cap` slots (its best keys; 0 in unused slots)
-//      and return the best key of the segment that was not proposed (0: none).
-
-// The proposals are the entries in the top bins of a 1024-bin linear histogram over the CTA's
-// own score range, as many bins as keep the count within a limit (<= cap) sized from the CTA's
-// expected share of winners.
-__device__ uint64_t propose_hist(const float* sc, int len, int64_t lo, int cap, int64_t keff, int64_t V,
-                                 unsigned long long* slots, unsigned* hist, IdxShared& S) {
-  float mn = INFINITY, mx = -INFINITY;
-  for (int e = threadIdx.x; e < len; e += kIdxThreads) {
-    mn = fminf(mn, sc[e]);
-    mx = fmaxf(mx, sc[e]);
-  }
-  for (int i = threadIdx.x; i < kLinBins; i += kIdxThreads) hist[i] = 0u;
-  float gmn, gmx;
-  block_minmax(mn, mx, S, gmn, gmx);
-  const float scl = gmx > gmn ? (float)kLinBins / (gmx - gmn) : 0.f;
-  for (int e = threadIdx.x; e < len; e += kIdxThreads) atomicAdd(&hist[lin_bin(sc[e], gmn, scl)], 1u);
-  __syncthreads();
-  // lowest bin whose suffix count stays within the limit: one above the bin where the count
-  // from the top first exceeds it
-  const unsigned limit = (unsigned)min((int64_t)cap, (3 * keff * len + 2 * V - 1) / (2 * V) + 16);
-  if ((unsigned)len <= limit) {
-    if (threadIdx.x == 0) S.ubuf[2] = 0u;
-  } else {
-    const Crossing xl = find_crossing(hist, kLinBins, limit + 1u, S.red, &S.cross);
-    if (threadIdx.x == 0) S.ubuf[2] = xl.bin + 1u;
-  }
+// ---- speculative proposals: fill this CTA's first slots (its best keys) in global memory and in
+//      `own` (shared), leave their number in S.ubuf[0] (final after the next block barrier), and
+//      return an upper bound of every key of the segment that was not proposed (0: none).
+// The proposals are the entries in the top bins of a histogram of log-scale bins below the CTA's
+// best score (32 per octave), as many bins from the top as keep the count within `limit` (<= cap;
+// sized from the CTA's expected share of winners).  Log-scale bins keep a few outlying large
+// scores from crowding every other score into one bin.
+__device__ uint64_t propose_log(const float* sc, int len, int64_t lo, int cap, unsigned limit,
+                                unsigned long long* slots, unsigned long long* own, unsigned* hist, IdxShared& S) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int nw = kIdxThreads / 32;
+  float mx = -INFINITY;
+  for (int e = threadIdx.x; e < len; e += kIdxThreads) mx = fmaxf(mx, sc[e]);
+  for (int i = threadIdx.x; i < kPropBins; i += kIdxThreads) hist[i] = 0u;
+  mx = warp_max(mx);
+  if (lane == 0) S.fred[warp] = mx;
   if (threadIdx.x == 0) S.ubuf[0] = 0u;  // proposal slot counter
   __syncthreads();
-  const unsigned pb = S.ubuf[2];
-  uint64_t unp = 0;
-  for (int e = threadIdx.x; e < len; e += kIdxThreads) {
-    const uint64_t ck = comp_key(sc[e], lo + e);
-    bool put = false;
-    if (lin_bin(sc[e], gmn, scl) >= pb) {
-      const unsigned slot = atomicAdd(&S.ubuf[0], 1u);
-      if (slot < (unsigned)cap) {
-        slots[slot] = ck;
-        put = true;
-      }
+  float gmx = S.fred[0];
+#pragma unroll
+  for (int w = 1; w < nw; ++w) gmx = fmaxf(gmx, S.fred[w]);
+  const uint32_t kmx = score_key(gmx);
+  for (int e = threadIdx.x; e < len; e += kIdxThreads)
+    atomicAdd(&hist[log_bin(kmx, score_key(sc[e]), kPropShift, kPropBins)], 1u);
+  __syncthreads();
+  // pb = the number of bins from the top whose entries together stay within the limit
+  block_cut<kPropBins>(hist, limit, &S.cross, S);
+  const unsigned pb = S.cross.bin;
+  for (int b0 = threadIdx.x - lane; b0 < len; b0 += kIdxThreads) {  // warp-uniform trip count
+    const int e = b0 + lane;
+    const bool valid = e < len;
+    const uint32_t k32 = valid ? score_key(sc[e]) : 0u;
+    const uint64_t ck = ((uint64_t)k32 << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)(lo + e));
+    const bool prop = valid && log_bin(kmx, k32, kPropShift, kPropBins) < pb;
+    // one slot reservation per warp
+    const unsigned mask = __ballot_sync(0xffffffffu, prop);
+    unsigned slot = 0;
+    if (mask) {
+      unsigned base = 0;
+      if (lane == __ffs(mask) - 1) base = atomicAdd(&S.ubuf[0], (unsigned)__popc(mask));
+      base = __shfl_sync(0xffffffffu, base, __ffs(mask) - 1);
+      slot = base + (unsigned)__popc(mask & ((1u << lane) - 1u));
     }
-    if (!put) unp = ck > unp ? ck : unp;
+    if (prop && slot < (unsigned)cap) {
+      slots[slot] = ck;
+      own[slot] = ck;
+    }
   }
-  unp = block_max_u64(unp, S);
-  for (int i = (int)min(S.ubuf[0], (unsigned)cap) + (int)threadIdx.x; i < cap; i += kIdxThreads) slots[i] = 0ull;
-  return unp;
+  // An upper bound of every key not proposed (no reduction needed): the top of the first bin
+  // not proposed; 0 when every entry was proposed.  (A bound a little above the best key kept
+  // back can only turn an exact acceptance into the exact path, never the reverse.)
+  if (pb >= (unsigned)kPropBins) return 0ull;
+  const uint32_t drop = pb << kPropShift;
+  const uint32_t top = kmx >= drop ? kmx - drop : kmx;
+  return ((uint64_t)top << 32) | 0xFFFFFFFFull;
 }
 
-// ------------------------------------------------------------------ one segment
-template <int SRC, int KS, int NTILE>
-__device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t V, int64_t ebase, QueryWS* ws,
-                                float* sc, uint8_t* un, IdxShared& S) {
-  const int64_t lo = (int64_t)j * V / G, hi = (int64_t)(j + 1) * V / G;
-  int len = (int)min(hi - lo, (int64_t)p.seg_cap);
-  const size_t tq = (size_t)t;
-  int32_t* oi = p.out_idx + tq * p.k;
-  float* os = p.out_score ? p.out_score + tq * p.k : nullptr;
-  const int64_t keff = min((int64_t)p.k, V);
-  if (j == 0)
-    for (int64_t i = keff + threadIdx.x; i < p.k; i += kIdxThreads) {
-      oi[i] = -1;
-      if (os) os[i] = 0.f;
-    }
-  if (keff == 0) return;
-  if (hi - lo > p.seg_cap && threadIdx.x == 0) flag(p.st, CSKV_DEV_CAPACITY);
-  // ---- scores of this segment into shared memory
-  if constexpr (SRC == kSrcFp8) {
-    const uint8_t* kb = p.k_idx + (size_t)(ebase + lo) * (KS * 32);
-    const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
-    // after a timeout the ring (and the histograms that share its memory) is not touched
-    // again; the other CTAs of the group time out at their next group barrier
-    if (!scan_fp8<KS, NTILE>(p, t, kb, ks, len, sc, un, S)) return;
-  } else if constexpr (SRC == kSrcF32) {
-    const float* kb = reinterpret_cast<const float*>(p.k_idx) + (size_t)(ebase + lo) * p.Di;
-    const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
-    scan_f32(p, t, kb, ks, len, sc, reinterpret_cast<float*>(un), S);
-  } else {
-    const float* src = p.scores + tq * p.ld_scores + lo;
-    copy_to_smem<false>(sc, src, len, threadIdx.x, kIdxThreads);
-    __syncthreads();
+// ---- cold paths, kept out of line: the speculative exchange's code stays compact (a launch
+//      runs the selection once, so its instructions come from the instruction caches cold)
+
+// A single CTA owns the query: radix select over the segment's keys, then emission.
+__device__ __noinline__ void select_single(const IdxParams& p, const float* sc, int len, int64_t lo, int64_t keff,
+                                           int32_t* oi, float* os, int64_t ebase, unsigned* hist, IdxShared& S) {
+  uint64_t P = 0;
+  int nb = 0;
+  local_select([&](int i) { return comp_key(sc[i], lo + i); }, len, (unsigned)keff, P, nb, hist, S);
+  emit(sc, len, lo, false, P, nb, 0, keff, oi, os, p, ebase, S);
+}
+
+// The rr-th best of the nbk keys of a crowded threshold bin: radix select inside the bin, then
+// the smallest selected key exactly (a bare prefix threshold could also admit keys of lower bins).
+__device__ __noinline__ uint64_t rank_in_big_bin(const unsigned long long* bin_keys, unsigned nbk, unsigned rr,
+                                                 unsigned* hist, IdxShared& S) {
+  uint64_t P2;
+  int nb2;
+  local_select([&](int i) { return (uint64_t)bin_keys[i]; }, nbk, rr, P2, nb2, hist, S);
+  uint64_t mnk = ~0ull;
+  for (unsigned i = threadIdx.x; i < nbk; i += kIdxThreads) {
+    const uint64_t kk = bin_keys[i];
+    if (key_selected(kk, P2, nb2) && kk < mnk) mnk = kk;
   }
-  // ---- everything kept: output position of entry e is e
-  if (keff == V) {
-    emit(sc, len, lo, true, 0, 0, lo, keff, oi, os, p, ebase, S);
-    return;
-  }
+  return ~block_max_u64(~mnk, S);
+}
+
+// The exact path over a group of CTAs (the speculative exchange was rejected: winners crowded
+// into a few segments, massive ties).
+__device__ __noinline__ void exact_group_select(const IdxParams& p, const float* sc, int len, int64_t lo, int j, int G,
+                                                int64_t keff, int32_t* oi, float* os, int64_t ebase, QueryWS* ws,
+                                                uint8_t* un, bool ok, IdxShared& S) {
   unsigned* hist = reinterpret_cast<unsigned*>(un + kUnHist);
   unsigned long long* cands = reinterpret_cast<unsigned long long*>(un + kUnCand);
   auto own_key = [&](int i) { return comp_key(sc[i], lo + i); };
   uint64_t P = 0;
   int nb = 0;
-  // ---- a single CTA owns the query: exact selection in shared memory
-  if (G == 1) {
-    local_select(own_key, len, (unsigned)keff, P, nb, hist, S);
-    emit(sc, len, lo, false, P, nb, 0, keff, oi, os, p, ebase, S);
-    return;
-  }
-  bool ok = true;
-  // ---- speculative exchange (one group barrier).  Every CTA proposes its best entries (at
-  //      most `cap`, into its own slots) and reports the best key it did NOT propose.  After
-  //      the barrier every CTA finds the exact k-th best proposal T*; when no CTA holds an
-  //      unproposed key >= T*, the selection is exactly {key >= T*} and no second exchange is
-  //      needed.  Otherwise (winners crowded into one segment, massive ties) the exact path
-  //      below runs.
-  // slot capacity per CTA: group-uniform (every CTA lays out and reads the slots alike)
-  const int cap = (int)min((int64_t)(kCandMax / G), (V + G - 1) / G);
-  if (G <= kIdxThreads && cap >= 1 && (int64_t)cap * G >= keff) {
-    unsigned long long* slots = ws->cand + (size_t)j * cap;
-    const uint64_t unp = propose_hist(sc, len, lo, cap, keff, V, slots, hist, S);
-    if (threadIdx.x == 0) ws->unp[j] = unp;
-    for (int i = threadIdx.x; i < kBins0; i += kIdxThreads) hist[i] = 0u;  // for T*, set while waiting
-    ok = group_barrier(ws, G, j, p.st, &S.flag);
-    // -- gather every CTA's slots (CTA order; 0 marks an unused slot), count the proposals
-    //    and find their score range
-    const unsigned total = (unsigned)G * (unsigned)cap;
-    const uint64_t u = (int)threadIdx.x < G ? __ldcg(&ws->unp[threadIdx.x]) : 0ull;
-    float mn = INFINITY, mx = -INFINITY;
-    int cnt = 0;
-    for (unsigned b0 = threadIdx.x; b0 < total; b0 += kIdxThreads * 8) {
-      unsigned long long v[8];
-#pragma unroll
-      for (int uu = 0; uu < 8; ++uu) {
-        const unsigned c = b0 + uu * kIdxThreads;
-        v[uu] = c < total ? __ldcg(ws->cand + c) : 0ull;
-      }
-#pragma unroll
-      for (int uu = 0; uu < 8; ++uu) {
-        const unsigned c = b0 + uu * kIdxThreads;
-        if (c < total) cands[c] = v[uu];
-        if (v[uu] != 0ull) {
-          const float f = key_score(v[uu]);
-          mn = fminf(mn, f);
-          mx = fmaxf(mx, f);
-          ++cnt;
-        }
-      }
-    }
-    float qmn, qmx;
-    int nprop;
-    block_minmax(mn, mx, S, qmn, qmx, cnt, &nprop);  // its barriers also publish cands[]
-    if (nprop >= keff) {  // group-uniform: every CTA gathered the same slots
-      // -- exact k-th best proposal: histogram over the proposals' score keys, then rank
-      //    inside the threshold bin
-      const uint32_t kmin = score_key(qmn), krange = score_key(qmx) - kmin;
-      int shift = 0;
-      while (shift < 32 && (krange >> shift) >= (uint32_t)kBins0) ++shift;
-      for (unsigned i = threadIdx.x; i < total; i += kIdxThreads) {
-        const uint64_t c = cands[i];
-        if (c != 0ull) atomicAdd(&hist[key_bin4k(c, kmin, shift)], 1u);
-      }
-      if (threadIdx.x == 0) S.ubuf[1] = 0u;
-      __syncthreads();
-      const Crossing x = find_crossing(hist, kBins0, (unsigned)keff, S.red, &S.cross);
-      const unsigned rr = (unsigned)keff - x.above;  // rank wanted inside bin x.bin (1-based)
-      const bool bin_fits = x.cnt <= (unsigned)kAuxKeys;
-      // collect the threshold bin's keys
-      unsigned long long* bin_keys = reinterpret_cast<unsigned long long*>(un + kUnAux);
-      const unsigned bin_cap = (unsigned)kAuxKeys;
-      for (unsigned i = threadIdx.x; i < total; i += kIdxThreads) {
-        const uint64_t c = cands[i];
-        if (c != 0ull && key_bin4k(c, kmin, shift) == x.bin) {
-          const unsigned sl = atomicAdd(&S.ubuf[1], 1u);
-          if (sl < bin_cap) bin_keys[sl] = c;
-        }
-      }
-      __syncthreads();
-      const unsigned nbk = min(S.ubuf[1], bin_cap);
-      uint64_t Tstar = ~0ull;
-      if (!bin_fits) {
-        // the threshold bin does not fit the scratch: leave T* at "select nothing", which the
-        // check below rejects
-      } else if (nbk == 1 && rr == 1) {
-        Tstar = bin_keys[0];  // the usual case: the threshold bin holds T* alone
-      } else if (nbk <= (unsigned)kIdxThreads) {
-        // thread i ranks key i against the bin (keys are distinct: exactly one has rank rr-1)
-        if (threadIdx.x < nbk) {
-          const uint64_t mine = bin_keys[threadIdx.x];
-          unsigned rank = 0;
-          for (unsigned m = 0; m < nbk; ++m) rank += (uint64_t)bin_keys[m] > mine;
-          if (rank + 1 == rr) S.tstar = mine;
-        }
-        __syncthreads();
-        Tstar = S.tstar;
-      } else {
-        // radix select inside the bin, then T* = the smallest selected key exactly (a bare
-        // prefix threshold could also admit keys of lower linear bins)
-        uint64_t P2;
-        int nb2;
-        local_select([&](int i) { return (uint64_t)bin_keys[i]; }, nbk, rr, P2, nb2, hist, S);
-        uint64_t mnk = ~0ull;
-        for (unsigned i = threadIdx.x; i < nbk; i += kIdxThreads) {
-          const uint64_t kk = bin_keys[i];
-          if (key_selected(kk, P2, nb2) && kk < mnk) mnk = kk;
-        }
-        Tstar = ~block_max_u64(~mnk, S);
-      }
-      // -- accepted when no CTA kept back a key >= T*
-      // one block scan carries both the validity count (high bits) and this CTA's output
-      // base = proposals of lower CTAs that are kept (low 16 bits; at most kCandMax)
-      unsigned packed = 0;
-      if ((int)threadIdx.x < G) packed += (unsigned)(u >= Tstar) << 16;
-      if (threadIdx.x == 0 && !bin_fits) packed += 1u << 16;
-      const unsigned my_off = (unsigned)j * (unsigned)cap;
-      for (unsigned i = threadIdx.x; i < my_off; i += kIdxThreads) packed += cands[i] >= Tstar;
-      unsigned tot;
-      block_excl_scan(packed, S.red, &tot);
-      if ((tot >> 16) == 0 && ok) {
-        const unsigned base = tot & 0xFFFFu;
-        if (cap <= 64) {
-          // every kept entry of this segment is one of its proposals: its output position is
-          // the base plus the kept proposals of this CTA with a lower index
-          const unsigned long long* own = cands + my_off;
-          if ((int)threadIdx.x < cap) {
-            const uint64_t key = own[threadIdx.x];
-            if (key >= Tstar) {
-              const uint32_t kl = (uint32_t)key;  // inverted index: larger = lower index
-              unsigned pos = base;
-              for (int m = 0; m < cap; ++m) {
-                const uint64_t o = own[m];
-                pos += (o >= Tstar && (uint32_t)o > kl) ? 1u : 0u;
-              }
-              if (pos < (unsigned)keff) {
-                const uint32_t e = 0xFFFFFFFFu - kl;
-                oi[pos] = (int32_t)e;
-                if (os) os[pos] = key_score(key);
-                if (p.pf_rows)
-                  prefetch_l2_bulk(p.pf_rows + (size_t)(ebase + e) * p.pf_row_bytes, (unsigned)p.pf_row_bytes);
-              }
-            }
-          }
-        } else {
-          // emit keys >= T*: the rule "top 64 bits >= T*"
-          emit(sc, len, lo, false, Tstar, 64, base, keff, oi, os, p, ebase, S);
-        }
-        return;
-      }
-    }
-    // rejected (uniformly across the group); the next group barrier orders every read of the
-    // proposals before the exact path reuses the candidate slots
-  }
-  // ---- exact path: 12-bit digit histogram of the whole group
+  // ---- 12-bit digit histogram of the whole group
   for (int i = threadIdx.x; i < kBins0; i += kIdxThreads) hist[i] = 0u;
   __syncthreads();
   for (int b0 = threadIdx.x - (threadIdx.x & 31); b0 < len; b0 += kIdxThreads) {
@@ -901,7 +867,6 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   r -= x.above;
   bool done = (x.cnt == r);
   int used_passes = 0;
-  unsigned cands_used = 0;
   int64_t base = 0;
   bool have_base = false;
   if (!done && x.cnt <= kCandMax) {
@@ -928,7 +893,6 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
       }
     ok = group_barrier(ws, G, j, p.st, &S.flag) && ok;
     const unsigned n_c = min(__ldcg(&ws->cand_count), (unsigned)kCandMax);
-    cands_used = n_c;
     copy_to_smem<true>(cands, ws->cand, n_c, threadIdx.x, kIdxThreads);
     __syncthreads();
     while (!done) done = local_pass([&](int i) { return (uint64_t)cands[i]; }, n_c, P, nb, r, hist, S);
@@ -986,6 +950,236 @@ __device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t
   group_cleanup(ws, G, true, used_passes, S);
 }
 
+// ------------------------------------------------------------------ one segment
+template <int SRC, int KS, int NTILE>
+__device__ void process_segment(const IdxParams& p, int t, int j, int G, int64_t V, int64_t ebase, QueryWS* ws,
+                                float* sc, uint8_t* un, IdxShared& S) {
+  const int64_t lo = (int64_t)j * V / G, hi = (int64_t)(j + 1) * V / G;
+  int len = (int)min(hi - lo, (int64_t)p.seg_cap);
+  const size_t tq = (size_t)t;
+  int32_t* oi = p.out_idx + tq * p.k;
+  float* os = p.out_score ? p.out_score + tq * p.k : nullptr;
+  const int64_t keff = min((int64_t)p.k, V);
+  if (j == 0)
+    for (int64_t i = keff + threadIdx.x; i < p.k; i += kIdxThreads) {
+      oi[i] = -1;
+      if (os) os[i] = 0.f;
+    }
+  if (keff == 0) return;
+  if (hi - lo > p.seg_cap && threadIdx.x == 0) flag(p.st, CSKV_DEV_CAPACITY);
+  // speculative exchange sizes, computed before the scan (its copies are in flight meanwhile):
+  // slots per CTA (group-uniform: every CTA lays out and reads the slots alike), and this CTA's
+  // proposal limit -- its expected share of winners, half as many again and 16 more
+  const unsigned V32 = (unsigned)min(V, (int64_t)0x7FFFFFFF);
+  const int cap = (int)min((unsigned)(kCandMax / G), (V32 + (unsigned)G - 1u) / (unsigned)G);
+  const unsigned limit = (unsigned)min((float)cap, 1.5f * (float)keff * (float)len / (float)V32 + 17.f);
+  // ---- scores of this segment into shared memory
+  if constexpr (SRC == kSrcFp8 || SRC == kSrcFp4) {
+    constexpr bool fp4 = SRC == kSrcFp4;
+    const uint8_t* kb = p.k_idx + (size_t)(ebase + lo) * (fp4 ? KS * 16 : KS * 32);
+    const float* ks = (!fp4 && p.k_scale) ? p.k_scale + ebase + lo : nullptr;
+    const uint8_t* kbs = fp4 ? p.k_bs + (size_t)(ebase + lo) * KS : nullptr;
+    // after a timeout the ring (and the histograms that share its memory) is not touched
+    // again; the other CTAs of the group time out at their next group barrier
+    if (!scan_mma<KS, NTILE, fp4>(p, t, kb, ks, kbs, len, sc, un, S)) return;
+  } else if constexpr (SRC == kSrcF32) {
+    const float* kb = reinterpret_cast<const float*>(p.k_idx) + (size_t)(ebase + lo) * p.Di;
+    const float* ks = p.k_scale ? p.k_scale + ebase + lo : nullptr;
+    scan_f32(p, t, kb, ks, len, sc, reinterpret_cast<float*>(un), S);
+  } else {
+    const float* src = p.scores + tq * p.ld_scores + lo;
+    copy_to_smem<false>(sc, src, len, threadIdx.x, kIdxThreads);
+    __syncthreads();
+  }
+  // ---- everything kept: output position of entry e is e
+  if (keff == V) {
+    emit(sc, len, lo, true, 0, 0, lo, keff, oi, os, p, ebase, S);
+    return;
+  }
+  unsigned* hist = reinterpret_cast<unsigned*>(un + kUnHist);
+  // ---- a single CTA owns the query: exact selection in shared memory
+  if (G == 1) {
+    select_single(p, sc, len, lo, keff, oi, os, ebase, hist, S);
+    return;
+  }
+  bool ok = true;
+  // ---- speculative exchange (one group barrier).  Every CTA proposes its best entries (at
+  //      most `cap`, into its own slots) and reports the best key it did NOT propose.  After
+  //      the barrier every CTA finds the exact k-th best proposal T*; when no CTA holds an
+  //      unproposed key >= T*, the selection is exactly {key >= T*} and no second exchange is
+  //      needed.  Otherwise (winners crowded into one segment, massive ties) the exact path
+  //      below runs.
+  // slot capacity per CTA: group-uniform (every CTA lays out and reads the slots alike)
+  if (G <= kIdxThreads && cap >= 1 && (int64_t)cap * G >= keff) {
+    unsigned long long* slots = ws->cand + (size_t)j * cap;
+    unsigned long long* own = reinterpret_cast<unsigned long long*>(un + kUnCand);  // this CTA's proposals
+    const uint64_t unp = propose_log(sc, len, lo, cap, limit, slots, own, hist, S);
+    for (int i = threadIdx.x; i < kTBins; i += kIdxThreads) hist[i] = 0u;  // for T*, set while waiting
+    __syncthreads();  // the slot count is final
+    const int nprop_own = (int)min(S.ubuf[0], (unsigned)cap);
+    for (int i = nprop_own + (int)threadIdx.x; i < cap; i += kIdxThreads) {
+      slots[i] = 0ull;  // 0 marks an unused slot
+      own[i] = 0ull;
+    }
+    if (threadIdx.x == 0) ws->unp[j] = unp;
+    ok = group_barrier(ws, G, j, p.st, &S.flag);  // its first block barrier orders the writes above
+    // -- gather every CTA's slots into registers (thread t: slots t + kIdxThreads * uu, in CTA
+    //    order; 0 marks an unused slot), with the best key and the number of proposals
+    const unsigned total = (unsigned)G * (unsigned)cap;  // <= kCandMax = 8 * kIdxThreads
+    const uint64_t u = (int)threadIdx.x < G ? __ldcg(&ws->unp[threadIdx.x]) : 0ull;
+    unsigned long long v[8];
+#pragma unroll
+    for (int uu = 0; uu < 8; ++uu) {
+      const unsigned c = threadIdx.x + uu * kIdxThreads;
+      v[uu] = c < total ? __ldcg(ws->cand + c) : 0ull;
+    }
+    unsigned kmx = 0u, kmn = 0xFFFFFFFFu, cnt = 0u;
+#pragma unroll
+    for (int uu = 0; uu < 8; ++uu)
+      if (v[uu] != 0ull) {
+        kmx = max(kmx, (unsigned)(v[uu] >> 32));
+        kmn = min(kmn, (unsigned)(v[uu] >> 32));
+        ++cnt;
+      }
+    {
+      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+      kmx = __reduce_max_sync(0xffffffffu, kmx);
+      kmn = __reduce_min_sync(0xffffffffu, kmn);
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (lane == 0) {
+        S.red[warp] = kmx;
+        S.ured[warp] = kmn;
+        S.fcnt[warp] = (int)cnt;
+      }
+    }
+    if (threadIdx.x == 0) S.ubuf[1] = 0u;
+    __syncthreads();
+    unsigned gkmx = 0u, gkmn = 0xFFFFFFFFu;
+    int nprop = 0;
+#pragma unroll
+    for (int w = 0; w < kIdxThreads / 32; ++w) {
+      gkmx = max(gkmx, S.red[w]);
+      gkmn = min(gkmn, (unsigned)S.ured[w]);
+      nprop += S.fcnt[w];
+    }
+    if (nprop >= keff) {  // group-uniform: every CTA gathered the same slots
+      // -- exact k-th best proposal: histogram of log-scale bins below the best proposal
+      //    (256 per octave), then the rank inside the threshold bin
+      // bins from the best proposal down to the worst, as fine as kTBins bins over that range
+      // allow (uniform in the score key: about uniform in log(score) for scores of one
+      // sign); warp 0 finds the bin holding the k-th best proposal and the count above it
+      int tshift = 0;
+      while (tshift < 32 && ((gkmx - gkmn) >> tshift) >= (uint32_t)kTBins) ++tshift;
+      auto tbin = [&](uint64_t c) { return log_bin(gkmx, (uint32_t)(c >> 32), tshift, kTBins); };
+#pragma unroll
+      for (int uu = 0; uu < 8; ++uu)
+        if (v[uu] != 0ull) atomicAdd(&hist[tbin(v[uu])], 1u);
+      __syncthreads();
+      block_cut<kTBins>(hist, (unsigned)keff - 1u, &S.cross, S);  // the first bin passing k - 1
+      const Crossing x = S.cross;
+      const unsigned rr = (unsigned)keff - x.above;  // rank wanted inside bin x.bin (1-based)
+      const bool bin_fits = x.bin < (unsigned)kTBins && x.cnt <= (unsigned)kAuxKeys;
+      // collect the threshold bin's keys
+      unsigned long long* bin_keys = reinterpret_cast<unsigned long long*>(un + kUnAux);
+      const unsigned bin_cap = (unsigned)kAuxKeys;
+#pragma unroll
+      for (int uu = 0; uu < 8; ++uu) {
+        const uint64_t c = v[uu];
+        if (c != 0ull && tbin(c) == x.bin) {
+          const unsigned sl = atomicAdd(&S.ubuf[1], 1u);
+          if (sl < bin_cap) bin_keys[sl] = c;
+        }
+      }
+      __syncthreads();
+      const unsigned nbk = min(S.ubuf[1], bin_cap);
+      uint64_t Tstar = ~0ull;
+      if (!bin_fits) {
+        // the threshold bin does not fit the scratch: leave T* at "select nothing", which the
+        // check below rejects
+      } else if (nbk == 1 && rr == 1) {
+        Tstar = bin_keys[0];  // the usual case: the threshold bin holds T* alone
+      } else if (nbk <= (unsigned)kIdxThreads) {
+        // thread i ranks key i against the bin (keys are distinct: exactly one has rank rr-1)
+        if (threadIdx.x < nbk) {
+          const uint64_t mine = bin_keys[threadIdx.x];
+          unsigned rank = 0;
+          for (unsigned m = 0; m < nbk; ++m) rank += (uint64_t)bin_keys[m] > mine;
+          if (rank + 1 == rr) S.tstar = mine;
+        }
+        __syncthreads();
+        Tstar = S.tstar;
+      } else {
+        Tstar = rank_in_big_bin(bin_keys, nbk, rr, hist, S);
+      }
+      // -- accepted when no CTA kept back a key >= T*
+      // one block scan carries both the validity count (high bits) and this CTA's output
+      // base = proposals of lower CTAs that are kept (low 16 bits; at most kCandMax)
+      unsigned packed = 0;
+      if ((int)threadIdx.x < G) packed += (unsigned)(u >= Tstar) << 16;
+      if (threadIdx.x == 0 && !bin_fits) packed += 1u << 16;
+      const unsigned my_off = (unsigned)j * (unsigned)cap;
+#pragma unroll
+      for (int uu = 0; uu < 8; ++uu)
+        packed += (threadIdx.x + uu * kIdxThreads < my_off && v[uu] >= Tstar) ? 1u : 0u;
+      unsigned tot;
+      block_excl_scan(packed, S.red, &tot);
+      if ((tot >> 16) == 0 && ok) {
+        const unsigned base = tot & 0xFFFFu;
+        if (cap <= 32) {
+          // every kept entry of this segment is one of its proposals: its output position is
+          // the base plus the kept proposals of this CTA with a lower index; warp 0 holds one
+          // proposal a lane and ranks them with shuffles
+          if (threadIdx.x < 32) {
+            const uint64_t key = (int)threadIdx.x < cap ? own[threadIdx.x] : 0ull;
+            const bool kept = key != 0ull && key >= Tstar;
+            const uint32_t kl = (uint32_t)key;  // inverted index: larger = lower index
+            unsigned pos = base;
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+              const uint64_t o = __shfl_sync(0xffffffffu, key, m);
+              pos += (o != 0ull && o >= Tstar && (uint32_t)o > kl) ? 1u : 0u;
+            }
+            if (kept && pos < (unsigned)keff) {
+              const uint32_t e = 0xFFFFFFFFu - kl;
+              oi[pos] = (int32_t)e;
+              if (os) os[pos] = key_score(key);
+              if (p.pf_rows)
+                prefetch_l2_bulk(p.pf_rows + (size_t)(ebase + e) * p.pf_row_bytes, (unsigned)p.pf_row_bytes);
+            }
+          }
+        } else if (cap <= 64) {
+          // as above, a thread a proposal
+          if ((int)threadIdx.x < cap) {
+            const uint64_t key = own[threadIdx.x];
+            if (key >= Tstar) {
+              const uint32_t kl = (uint32_t)key;  // inverted index: larger = lower index
+              unsigned pos = base;
+              for (int m = 0; m < cap; ++m) {
+                const uint64_t o = own[m];
+                pos += (o >= Tstar && (uint32_t)o > kl) ? 1u : 0u;
+              }
+              if (pos < (unsigned)keff) {
+                const uint32_t e = 0xFFFFFFFFu - kl;
+                oi[pos] = (int32_t)e;
+                if (os) os[pos] = key_score(key);
+                if (p.pf_rows)
+                  prefetch_l2_bulk(p.pf_rows + (size_t)(ebase + e) * p.pf_row_bytes, (unsigned)p.pf_row_bytes);
+              }
+            }
+          }
+        } else {
+          // emit keys >= T*: the rule "top 64 bits >= T*"
+          emit(sc, len, lo, false, Tstar, 64, base, keff, oi, os, p, ebase, S);
+        }
+        return;
+      }
+    }
+    // rejected (uniformly across the group); the next group barrier orders every read of the
+    // proposals before the exact path reuses the candidate slots
+  }
+  exact_group_select(p, sc, len, lo, j, G, keff, oi, os, ebase, ws, un, ok, S);
+}
+
 __device__ __forceinline__ int64_t visible_of(const IdxParams& p, int t, int64_t* ebase) {
   if (p.scores) {
     *ebase = 0;
@@ -996,15 +1190,18 @@ __device__ __forceinline__ int64_t visible_of(const IdxParams& p, int t, int64_t
     }
     return v;
   }
+  // the query's sequence, position and (speculatively, for sequence 0) entry range are loaded
+  // together: one round trip instead of two dependent ones in the common one-sequence case
   const int s = __ldg(p.q_seq + t);
+  const int64_t pos = __ldg(p.q_pos + t);
+  const int64_t z0 = __ldg(p.ent_off), z1 = __ldg(p.ent_off + 1);
   if (s < 0 || s >= p.batch) {
     flag(p.st, CSKV_DEV_BAD_INDEX);
     *ebase = 0;
     return 0;
   }
-  const int64_t e0 = __ldg(p.ent_off + s), e1 = __ldg(p.ent_off + s + 1);
+  const int64_t e0 = s == 0 ? z0 : __ldg(p.ent_off + s), e1 = s == 0 ? z1 : __ldg(p.ent_off + s + 1);
   *ebase = e0;
-  const int64_t pos = __ldg(p.q_pos + t);
   int64_t v = pos >= 0 ? (pos + 1) / 4 : 0;
   if (v > e1 - e0) {
     flag(p.st, CSKV_DEV_BAD_INDEX);
@@ -1030,14 +1227,14 @@ __global__ void __maxnreg__(88) lindex_topk_kernel(IdxParams p) {
     if (lane == 1) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_pos + t0));
     if (lane == 2) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.ent_off));
     if (lane == 3 && p.q_scale) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_scale + (size_t)t0 * p.Hi));
-    const size_t qbytes = (size_t)p.Hi * p.Di * (SRC == kSrcFp8 ? 1 : 4);
+    const size_t qbytes = SRC == kSrcFp4 ? (size_t)p.Hi * p.Di / 2 : (size_t)p.Hi * p.Di * (SRC == kSrcFp8 ? 1 : 4);
     for (size_t off = (size_t)(lane >= 4 ? lane - 4 : 0) * 128; lane >= 4 && off < qbytes; off += 124 * 128)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_idx + (size_t)t0 * qbytes + off));
   }
   if (threadIdx.x == 0) S.scan_err = 0;  // read only after later block barriers
   pdl_wait();
   uint8_t* un = dsm;                                              // ring / histogram / candidates
-  float* sc = reinterpret_cast<float*>(dsm + idx_union_bytes(KS * 32));  // segment scores
+  float* sc = reinterpret_cast<float*>(dsm + p.un_bytes);  // segment scores
   if (p.split && p.T == 1) {
     // one query: the whole grid is its group (the plan below reduces to this)
     const int t = p.t_begin;
@@ -1120,8 +1317,25 @@ static DevInfo dev_info() {
   return info;
 }
 
-// ring/histogram region + the segment's scores + its entry scales
-static size_t idx_dyn_smem(int Di, int64_t seg_cap) { return idx_union_bytes(Di) + (size_t)seg_cap * 8; }
+// ring/histogram region + the segment's scores
+static size_t idx_dyn_smem(int Di, int64_t seg_cap, int stages) {
+  return idx_union_bytes(Di, stages) + (size_t)seg_cap * 4;
+}
+
+// Shared memory an indexer CTA of a split-mode launch may take when choosing a deeper ring: a
+// tensor-core attention CTA (~97 KB) of a decode step must still fit on the same SM (228 KB,
+// 1 KB of it reserved per CTA).
+constexpr size_t kIdxDeepRingSmem = 127 * 1024;
+
+// Ring stages of a launch: the minimum (64 KiB), deepened towards the whole segment (every
+// fill issued at once) while the CTA stays within kIdxDeepRingSmem.
+static int idx_ring_stages(int Di, int64_t seg_cap) {
+  const int base = idx_stages(Di);
+  const int need = (int)min((seg_cap + kIdxTile - 1) / kIdxTile, (int64_t)kIdxMaxStages);
+  int st = base;
+  while (st < need && idx_dyn_smem(Di, seg_cap, st + 1) <= kIdxDeepRingSmem) ++st;
+  return st;
+}
 
 static size_t idx_smem_budget() {
   const DevInfo d = dev_info();
@@ -1138,7 +1352,7 @@ static int split_queries_per_launch(int T, int64_t max_entries, int Di, int P, i
     int64_t cap = (int64_t)Tb * max_entries / (P - Tb) + 1;
     cap = max(cap, (int64_t)2 * kMinSeg);
     cap = min(cap, max_entries);
-    if (idx_dyn_smem(Di, cap) <= budget) {
+    if (idx_dyn_smem(Di, cap, idx_stages(Di)) <= budget) {
       *seg_cap = cap;
       return Tb;
     }
@@ -1186,18 +1400,20 @@ static cudaError_t run_topk(IdxParams p, int T, cudaStream_t stream) {
   // Two SMs stay out of the cooperative grid, so the small compression kernels that run
   // beside the indexer in a decode step do not hold up its (all-CTAs-resident) launch.
   const int P = d.sms > 8 ? d.sms - 2 : d.sms;
-  const int Di = SRC == kSrcFp8 ? KS * 32 : 64;
+  // bytes of one key in the scan's tiles ("Di" of the ring and shared-memory plan)
+  const int Di = SRC == kSrcFp8 ? KS * 32 : SRC == kSrcFp4 ? KS * 16 : 64;
   int64_t seg_cap = 0;
   const int Tb = split_queries_per_launch(T, p.max_entries, Di, P, &seg_cap);
-  const bool row_fits = idx_dyn_smem(Di, p.max_entries) <= idx_smem_budget();
-  p.stages = idx_stages(Di);
+  const bool row_fits = idx_dyn_smem(Di, p.max_entries, idx_stages(Di)) <= idx_smem_budget();
   if (Tb >= 1 && (Tb == T || !row_fits)) {
     p.split = 1;
     p.seg_cap = seg_cap;
+    p.stages = (SRC == kSrcFp8 || SRC == kSrcFp4) ? idx_ring_stages(Di, seg_cap) : idx_stages(Di);
+    p.un_bytes = (int64_t)idx_union_bytes(Di, p.stages);
     for (int t0 = 0; t0 < T; t0 += Tb) {
       p.t_begin = t0;
       p.T = min(Tb, T - t0);
-      cudaError_t e = launch_one<SRC, KS, NTILE>(p, P, true, idx_dyn_smem(Di, seg_cap), stream);
+      cudaError_t e = launch_one<SRC, KS, NTILE>(p, P, true, idx_dyn_smem(Di, seg_cap, p.stages), stream);
       if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -1205,9 +1421,11 @@ static cudaError_t run_topk(IdxParams p, int T, cudaStream_t stream) {
   if (!row_fits) return cudaErrorInvalidValue;
   p.split = 0;
   p.seg_cap = max(p.max_entries, (int64_t)1);
+  p.stages = idx_stages(Di);
+  p.un_bytes = (int64_t)idx_union_bytes(Di, p.stages);
   p.t_begin = 0;
   p.T = T;
-  return launch_one<SRC, KS, NTILE>(p, min(T, P), false, idx_dyn_smem(Di, p.seg_cap), stream);
+  return launch_one<SRC, KS, NTILE>(p, min(T, P), false, idx_dyn_smem(Di, p.seg_cap, p.stages), stream);
 }
 
 bool lindex_shape_supported(int dtype, int Hi, int Di) {
@@ -1222,7 +1440,7 @@ bool lindex_capacity_ok(int64_t max_entries, int T) {
   if (d.sms < 2) return false;
   int64_t cap;
   const bool split = split_queries_per_launch(T, max_entries, 128, d.sms, &cap) >= 1;
-  const bool row = idx_dyn_smem(128, max_entries) <= idx_smem_budget();
+  const bool row = idx_dyn_smem(128, max_entries, idx_stages(128)) <= idx_smem_budget();
   return split || row;
 }
 
@@ -1232,6 +1450,12 @@ cudaError_t launch_lindex(const IdxParams& p0, int dtype, int T, cudaStream_t st
   if (dtype == CSKV_F32) return run_topk<kSrcF32, 2, 1>(p, T, stream);
   const int ks = p.Di / 32;
   const int nt = p.Hi > 8 ? 2 : 1;
+  if (p.k_bs) {  // MXFP4
+    if (ks == 2 && nt == 1) return run_topk<kSrcFp4, 2, 1>(p, T, stream);
+    if (ks == 2 && nt == 2) return run_topk<kSrcFp4, 2, 2>(p, T, stream);
+    if (ks == 4 && nt == 1) return run_topk<kSrcFp4, 4, 1>(p, T, stream);
+    return run_topk<kSrcFp4, 4, 2>(p, T, stream);
+  }
   if (ks == 2 && nt == 1) return run_topk<kSrcFp8, 2, 1>(p, T, stream);
   if (ks == 2 && nt == 2) return run_topk<kSrcFp8, 2, 2>(p, T, stream);
   if (ks == 4 && nt == 1) return run_topk<kSrcFp8, 4, 1>(p, T, stream);

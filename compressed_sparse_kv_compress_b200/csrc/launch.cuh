@@ -73,6 +73,8 @@ struct IdxParams {
   const float* q_scale;
   const uint8_t* k_idx;
   const float* k_scale;
+  const uint8_t* q_bs;  // MXFP4: E8M0 block scales of the queries [T, Hi, Di/32] and keys [Nc, Di/32]
+  const uint8_t* k_bs;
   const float* head_w;
   const float* scores;
   int64_t ld_scores;
@@ -86,7 +88,8 @@ struct IdxParams {
   int64_t max_entries;
   int64_t seg_cap;
   int split;
-  int stages;
+  int stages;        // TMA ring stages of the fp8 scan
+  int64_t un_bytes;  // shared bytes of the ring / selection region (the scores follow it)
   int32_t* out_idx;
   float* out_score;
   const uint8_t* pf_rows;  // optional: rows (indexed like k_idx) of kept entries go to L2

@@ -9,8 +9,10 @@ as cited in the C header):
   HCA layer: hca_compress -> hybrid_decode_attn(HCA)
 
 The HCA layer does not depend on the CSA layer, so with ``two_streams`` it
-runs on a side stream that forks from and joins the caller's stream.  The
-whole step can be captured into a CUDA graph and replayed.
+runs on a side stream that forks from and joins the caller's stream; the
+CSA compression runs on a second side stream beside the indexer (which reads
+the entry keys, not the compressed cache), and the CSA attention waits for
+both.  The whole step can be captured into a CUDA graph and replayed.
 
 Tensor names (all device tensors, int64 offsets unless noted):
   CSA rows  x_a z_a x_b z_b [rows, 256], csa_x_off [B+1], csa_t0 [B],
@@ -52,6 +54,8 @@ class DecodeStep:
         self.ws_h = api.attn_workspace(api.HCA, T, H, 0, self.W, self.max_hca_visible, dev)
         self.two_streams = two_streams
         self.side = torch.cuda.Stream(device=dev) if two_streams else None
+        self.side_c = torch.cuda.Stream(device=dev) if two_streams else None
+        self.ev_c = torch.cuda.Event() if two_streams else None
         self.graph = None
 
     # ------------------------------------------------------------------
@@ -111,13 +115,21 @@ class DecodeStep:
             self.csa_layer(main)
             self.hca_layer(main)
             return
-        # The HCA layer runs beside the CSA layer, which it does not depend on.  The CSA
-        # layer stays on one stream, so each of its kernels follows the previous one as a
-        # dependent launch (its set-up overlaps the previous kernel's tail).
+        # The HCA layer runs beside the CSA layer, which it does not depend on.  Inside the CSA
+        # layer the indexer reads the entry keys, not the compressed cache, so it starts at
+        # once on the main stream while the compression of the newest entries runs on a
+        # second side stream; the CSA attention (a dependent launch of the indexer) also waits
+        # for that compression.
         self.side.wait_stream(main)
+        self.side_c.wait_stream(main)
         self.hca_layer(self.side)
-        self.csa_layer(main)
+        self.csa_compress(self.side_c)
+        self.ev_c.record(self.side_c)
+        self.csa_select(main)
+        main.wait_event(self.ev_c)
+        self.csa_attend(main)
         main.wait_stream(self.side)
+        main.wait_stream(self.side_c)
 
     # ------------------------------------------------------------------
     def capture(self):

@@ -213,6 +213,31 @@ CSKV_API int lindex_score_topk(const void* q_idx, const float* q_scale, const vo
                       void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * lindex_score_topk_mxfp4 -- the same scan and selection on FP4 indexer vectors.
+ *
+ * [SW] §六.1 / §十三.4, [TR] §4.2: the indexer only ranks entries, so its QK path may run
+ * in FP4.  Keys and queries are OCP MXFP4: E2M1 elements (sign, 2 exponent bits with bias
+ * 1, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), two per byte (element 2j in
+ * the low nibble of byte j), and one E8M0 scale 2^(e - 127) per 32 elements (e = 0xFF is
+ * NaN).  With decoded values q[t,h,:] and k[i,:]:
+ *     s_i = sum_h head_w[h] * ReLU(q_scale[t,h] * <q[t,h,:], k[i,:]>)
+ * (per-block dot products exact, then fp32), and the selection, outputs and workspace are
+ * exactly those of lindex_score_topk.
+ * q_codes  : [T, Hi, Di/2] uint8, 16-byte aligned;  q_bscale: [T, Hi, Di/32] uint8.
+ * q_scale  : [T, Hi] fp32 or NULL (1).
+ * k_codes  : [sum entries, Di/2] uint8, 16-byte aligned;  k_bscale: [sum entries, Di/32]
+ *            uint8, aligned to Di/32 bytes (a key's scales are read as one word).
+ * Hi in 1..16, Di 64 or 128 (else CSKV_ERR_UNSUPPORTED).  Other arguments: as
+ * lindex_score_topk.
+ * ------------------------------------------------------------------------ */
+CSKV_API int lindex_score_topk_mxfp4(const uint8_t* q_codes, const uint8_t* q_bscale, const float* q_scale,
+                      const uint8_t* k_codes, const uint8_t* k_bscale, const float* head_w,
+                      const int32_t* q_seq, const int64_t* q_pos, const int64_t* ent_off, int batch, int T,
+                      int Hi, int Di, int k, int64_t max_entries, int32_t* out_idx, float* out_score,
+                      const void* prefetch_rows, int64_t prefetch_row_bytes,
+                      void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * lindex_topk_from_scores -- the selection half of lindex_score_topk alone.
  *
  * Keeps, for every row t, the min(k, n_valid[t]) largest of scores[t, 0..n_valid[t]-1]

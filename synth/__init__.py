@@ -7,4 +7,4 @@ both the CUDA library's tests and the CPU oracle can be fed from it without
 sharing any computation.
 """
 
-from .workloads import SPECS, Spec, Workload, spec_by_name  # noqa: F401
+from .workloads import SPECS, Spec, Workload, mxfp4_random, spec_by_name  # noqa: F401

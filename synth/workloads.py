@@ -137,6 +137,18 @@ def _quant_e4m3(x: np.ndarray) -> tuple[torch.Tensor, torch.Tensor]:
     return codes.contiguous(), scale.squeeze(-1).contiguous()
 
 
+def mxfp4_random(seed: int, tag: str, rows: int, di: int, exp_lo: int = 121, exp_hi: int = 126):
+    """Random MXFP4 vectors: E2M1 codes drawn uniformly over all 16 codes, packed two per byte
+    (element 2j in the low nibble), and E8M0 block exponents drawn uniformly in
+    [exp_lo, exp_hi] (scales 2^-6 .. 2^-1), one per 32 elements.  Returns
+    (codes uint8 [rows, di/2], scales uint8 [rows, di/32]) as torch tensors."""
+    g = _stream(seed, tag, 0)
+    nib = g.integers(0, 16, size=(rows, di), dtype=np.uint8)
+    codes = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    scales = g.integers(exp_lo, exp_hi + 1, size=(rows, di // 32), dtype=np.uint8)
+    return torch.from_numpy(codes), torch.from_numpy(scales)
+
+
 class Workload:
     """Host-side tensors and sizes of one named workload.
 

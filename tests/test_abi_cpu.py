@@ -105,6 +105,19 @@ def test_indexer_validation(lib):
     assert call(T=0) == _lib.OK
     assert call(pf=_p(0x1008), pf_bytes=512) == _lib.ERR_INVALID_ARG  # misaligned prefetch rows
     assert call(pf=_p(), pf_bytes=100) == _lib.ERR_INVALID_ARG  # row size not a multiple of 16
+    # the MXFP4 variant
+    def fp4(Hi=8, Di=64, k=16, T=1, kbs=_p(), qc=_p()):
+        return lib.lindex_score_topk_mxfp4(qc, _p(), nul, _p(), kbs, nul, _p(), _p(), _p(), 1, T, Hi, Di, k, 100,
+                                           _p(), nul, nul, 0, _p(), 1 << 20, nul, nul)
+
+    assert fp4(Di=96) == _lib.ERR_UNSUPPORTED
+    assert fp4(Hi=17) == _lib.ERR_UNSUPPORTED
+    assert fp4(Hi=0) == _lib.ERR_INVALID_ARG
+    assert fp4(k=0) == _lib.ERR_INVALID_ARG
+    assert fp4(qc=nul) == _lib.ERR_INVALID_ARG
+    assert fp4(qc=_p(0x1008)) == _lib.ERR_INVALID_ARG     # codes not 16-byte aligned
+    assert fp4(Di=128, kbs=_p(0x1002)) == _lib.ERR_INVALID_ARG  # 4 scale bytes per key: 4-aligned
+    assert fp4(T=0) == _lib.OK
     assert lib.lindex_topk_from_scores(nul, 10, _p(), 1, 4, 10, _p(), nul, _p(), 1 << 20, nul,
                                        nul) == _lib.ERR_INVALID_ARG
     assert lib.lindex_topk_from_scores(_p(), 5, _p(), 1, 4, 10, _p(), nul, _p(), 1 << 20, nul,
