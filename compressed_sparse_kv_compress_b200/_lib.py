@@ -33,6 +33,7 @@ SIGNATURES = {
     "csa_compress": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p,
                             _i32, _p, _f, _p, _i32, _i32, _p, _p, _p, _p]),
     "hca_compress": (_i32, [_p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p, _i32, _p, _f, _p, _p]),
+    "rmsnorm_heads": (_i32, [_p, _i32, _i64, _i32, _p, _f, _p, _p]),
     "lindex_pool_keys": (_i32, [_p, _i32, _i32, _p, _p, _i32, _p, _p, _p, _i64, _p, _p, _p, _p]),
     "lindex_score_topk": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _i32, _i32, _i32, _i32, _i32, _i64,
                                  _p, _p, _p, _i64, _p, _sz, _p, _p]),

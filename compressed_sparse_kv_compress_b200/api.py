@@ -66,6 +66,17 @@ def hca_compress(x, z, tok_off, ent_off, out, *, max_blocks, bias=None, tok0=Non
     return out
 
 
+def rmsnorm_heads(x, out=None, *, gamma=None, eps=1e-6, stream=None):
+    """RMSNorm of every 128-dimension row of x ([..., 128], fp32 or bf16) into out (default:
+    in place): x / sqrt(mean(x^2) + eps) * gamma."""
+    out = x if out is None else out
+    lib = _lib.load()
+    st = lib.rmsnorm_heads(_ptr(x), _dt(x), x.numel() // x.shape[-1], int(x.shape[-1]), _ptr(gamma), float(eps),
+                           _ptr(out), _stream(stream))
+    _lib.check("rmsnorm_heads", st)
+    return out
+
+
 def lindex_pool_keys(k_tok, tok_off, ent_off, out_codes, out_scale, *, max_blocks, tok0=None, first_block=None,
                      num_blocks=None, dev_status=None, stream=None):
     """Entry keys of the indexer from per-token keys k_tok [rows, Di] (fp32 or bf16): the mean

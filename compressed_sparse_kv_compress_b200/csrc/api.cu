@@ -159,6 +159,17 @@ int hca_compress(const void* x, const void* z, const float* bias, const int64_t*
                                            dev_status, (cudaStream_t)stream));
 }
 
+int rmsnorm_heads(const void* x, int dtype, int64_t rows, int d, const float* gamma, float eps, void* out,
+                  cskv_stream_t stream) {
+  if (dtype != CSKV_F32 && dtype != CSKV_BF16) return dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+  if (d != kHeadDim) return d > 0 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+  if (rows < 0 || !(eps >= 0.f) || !(eps < INFINITY)) return CSKV_ERR_INVALID_ARG;
+  if (rows == 0) return CSKV_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out) || (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)))
+    return CSKV_ERR_INVALID_ARG;
+  return launch_status(launch_rmsnorm_rows(x, dtype, rows, gamma, eps, out, (cudaStream_t)stream));
+}
+
 size_t lindex_workspace_size(int T, int k, int64_t max_entries) {
   (void)k;
   if (T < 1) return 0;

@@ -553,3 +553,61 @@ cudaError_t launch_pool_keys(const void* k_tok, int in_dt, int Di, const int64_t
 }
 
 }  // namespace cskv
+
+namespace cskv {
+
+// ------------------------------------------------------------------ RMSNorm of head vectors
+// [SW] §十四.3: the queries (and the KV, see the compression epilogues) are RMS-normalised so
+// that attention logits cannot blow up: y = x / sqrt(mean(x^2) + eps) * gamma over each
+// 128-dimension row (a query head).  A warp per row, a lane per 4 dimensions; fp32 inside.
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const T* __restrict__ x, int64_t rows,
+                                                           const float* __restrict__ gamma, float eps,
+                                                           T* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    float v[4];
+    const T* src = x + (size_t)r * kHeadDim + 4 * lane;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = to_f(src[i]);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ss = fmaf(v[i], v[i], ss);
+    ss = warp_sum(ss);
+    const float rr = rsqrtf(ss * (1.f / kHeadDim) + eps);
+    T* dst = out + (size_t)r * kHeadDim + 4 * lane;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float y = v[i] * rr * (gamma ? __ldg(gamma + 4 * lane + i) : 1.f);
+      if constexpr (sizeof(T) == 2)
+        dst[i] = __float2bfloat16_rn(y);
+      else
+        dst[i] = y;
+    }
+  }
+}
+
+cudaError_t launch_rmsnorm_rows(const void* x, int dtype, int64_t rows, const float* gamma, float eps, void* out,
+                                cudaStream_t stream) {
+  const int64_t blocks = (rows + 7) / 8;
+  const dim3 grid((unsigned)(blocks < 16384 ? blocks : 16384));
+  cudaError_t e;
+  if (dtype == CSKV_BF16) {
+    e = ensure_smem(rmsnorm_rows_kernel<__nv_bfloat16>, 0);
+    if (e == cudaSuccess)
+      e = launch_dependent(rmsnorm_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, stream,
+                           (const __nv_bfloat16*)x, rows, gamma, eps, (__nv_bfloat16*)out);
+  } else {
+    e = ensure_smem(rmsnorm_rows_kernel<float>, 0);
+    if (e == cudaSuccess)
+      e = launch_dependent(rmsnorm_rows_kernel<float>, grid, dim3(256), 0, stream, (const float*)x, rows, gamma, eps,
+                           (float*)out);
+  }
+  note_launch();
+  return e;
+}
+
+}  // namespace cskv

@@ -400,113 +400,121 @@ __device__ bool scan_mma(const IdxParams& p, int t, const uint8_t* kbase, const 
       skb[i] = ld_sk(e + 8);
     }
     asm volatile("bar.arrive 2, %0;" ::"n"(kIdxThreads) : "memory");
+    // A fragments of this warp's 16 rows of a tile into registers and the MMAs on them (FP4: the
+    // block scales applied to each block's dot product).
+    auto mma_tile = [&](const uint8_t* tile, SK skg, SK skg8, float (&acc)[NTILE][4]) {
+      if constexpr (FP4) {
+        uint32_t wa[NB], wb[NB];
+#pragma unroll
+        for (int bb = 0; bb < NB; ++bb) {
+          wa[bb] = *reinterpret_cast<const uint32_t*>(tile + (size_t)(r0 + g) * RB + 16 * bb + 4 * tq);
+          wb[bb] = *reinterpret_cast<const uint32_t*>(tile + (size_t)(r0 + g + 8) * RB + 16 * bb + 4 * tq);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+        for (int bb = 0; bb < NB; ++bb) {
+          const uint32_t a0 = e2m1x4_to_e4m3x4(wa[bb] & 0xFFFFu), a2 = e2m1x4_to_e4m3x4(wa[bb] >> 16);
+          const uint32_t a1 = e2m1x4_to_e4m3x4(wb[bb] & 0xFFFFu), a3 = e2m1x4_to_e4m3x4(wb[bb] >> 16);
+          const float kb0 = e8m0_to_float((skg >> (8 * bb)) & 0xFFu), kb8 = e8m0_to_float((skg8 >> (8 * bb)) & 0xFFu);
+#pragma unroll
+          for (int nt = 0; nt < NTILE; ++nt) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_e4m3_16832(d, a0, a1, a2, a3, bq[nt][bb][0], bq[nt][bb][1]);
+            // each block's exact dot product times 2^(key exponent) * 2^(query exponent)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              acc[nt][c] = fmaf(d[c] * kb0, fq[nt][c][bb], acc[nt][c]);
+              acc[nt][2 + c] = fmaf(d[2 + c] * kb8, fq[nt][c][bb], acc[nt][2 + c]);
+            }
+          }
+        }
+      } else {
+        uint4 ra[KS / 2], rb[KS / 2];
+#pragma unroll
+        for (int c = 0; c < KS / 2; ++c) {
+          ra[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g) * Di + (tq + 4 * c) * 16);
+          rb[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g + 8) * Di + (tq + 4 * c) * 16);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt) {
+          acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const uint4& A = ra[ks >> 1];
+            const uint4& B = rb[ks >> 1];
+            const bool hiw = ks & 1;
+            mma_e4m3_16832(acc[nt], hiw ? A.z : A.x, hiw ? B.z : B.x, hiw ? A.w : A.y, hiw ? B.w : B.y,
+                           bq[nt][ks][0], bq[nt][ks][1]);
+          }
+        }
+      }
+    };
+    // Scales, ReLU and the weighted head sum of rows g and g + 8; lanes tq 0 / 1 store them.
+    auto epilogue = [&](int it, SK skg, SK skg8, const float (&acc)[NTILE][4]) {
+      const int e_g = it * kIdxTile + r0 + g, e_g8 = e_g + 8;
+      const float kg = FP4 ? 1.f : (float)skg, kg8 = FP4 ? 1.f : (float)skg8;
+      float vg = 0.f, vg8 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          vg = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * kg) * acc[nt][c]), vg);
+          vg8 = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * kg8) * acc[nt][2 + c]), vg8);
+        }
+      vg += __shfl_xor_sync(0xffffffffu, vg, 1);
+      vg += __shfl_xor_sync(0xffffffffu, vg, 2);
+      vg8 += __shfl_xor_sync(0xffffffffu, vg8, 1);
+      vg8 += __shfl_xor_sync(0xffffffffu, vg8, 2);
+      if (tq == 0 && e_g < len) sc[e_g] = vg;
+      if (tq == 1 && e_g8 < len) sc[e_g8] = vg8;
+    };
+    // Two ring stages a pass (one when one is left): the two tiles' load -> MMA -> epilogue
+    // chains are independent, so the warp overlaps them.  A stage goes back to the producer
+    // only after the MMAs have consumed every lane's fragments (a warp-synchronous mma.sync
+    // cannot issue before all of its source loads have returned), so the next copy into it
+    // cannot overwrite data still being read; the epilogues then overlap the refills.
     bool alive = true;
     int s = 0;
     unsigned ph = 0;
-    for (int it = 0; it < ntiles && alive; ++it) {
-      if (!mbar_wait_bounded(&S.full[s], ph)) {
+    for (int it = 0; it < ntiles && alive; it += 2) {
+      const int n2 = min(2, ntiles - it);
+      const int s1 = s + 1 == stages ? 0 : s + 1;
+      const unsigned ph1 = s + 1 == stages ? ph ^ 1u : ph;
+      if (!mbar_wait_bounded(&S.full[s], ph) || (n2 == 2 && !mbar_wait_bounded(&S.full[s1], ph1))) {
         flag(p.st, CSKV_DEV_TIMEOUT);
         *(volatile int*)&S.scan_err = 1;  // the producer stops issuing fills
         alive = false;
         break;
       }
-      const int rows = min(kIdxTile, len - it * kIdxTile);
-      const SK skg = ska[0], skg8 = skb[0];
+      const SK ska0 = ska[0], skb0 = skb[0], ska1 = ska[1], skb1 = skb[1];
 #pragma unroll
-      for (int i = 0; i + 1 < kScalePF; ++i) {
-        ska[i] = ska[i + 1];
-        skb[i] = skb[i + 1];
+      for (int i = 0; i + 2 < kScalePF; ++i) {
+        ska[i] = ska[i + 2];
+        skb[i] = skb[i + 2];
       }
       {
         const int e = (it + kScalePF) * kIdxTile + r0 + g;
-        ska[kScalePF - 1] = ld_sk(e);
-        skb[kScalePF - 1] = ld_sk(e + 8);
+        ska[kScalePF - 2] = ld_sk(e);
+        skb[kScalePF - 2] = ld_sk(e + 8);
+        ska[kScalePF - 1] = ld_sk(e + kIdxTile);
+        skb[kScalePF - 1] = ld_sk(e + kIdxTile + 8);
       }
-      // A fragments of this warp's 16 rows into registers and the MMAs on them; the stage
-      // goes back to the producer only after the MMAs have consumed every lane's fragments
-      // (a warp-synchronous mma.sync cannot issue before all of its source loads have
-      // returned), so the next copy into the stage cannot overwrite data still being read.
-      // The epilogue then overlaps the refill.
-      if (r0 >= rows) {
-        __syncwarp();
-        if (lane == 0) release_stage(&S.released[s]);
-      } else {
-        const uint8_t* tile = ring + (size_t)s * kIdxTile * RB;
-        float acc[NTILE][4];
-        float accb[FP4 ? NB : 1][NTILE][4];  // FP4: one accumulator per block
-        if constexpr (FP4) {
-          uint32_t wa[NB], wb[NB];
-#pragma unroll
-          for (int bb = 0; bb < NB; ++bb) {
-            wa[bb] = *reinterpret_cast<const uint32_t*>(tile + (size_t)(r0 + g) * RB + 16 * bb + 4 * tq);
-            wb[bb] = *reinterpret_cast<const uint32_t*>(tile + (size_t)(r0 + g + 8) * RB + 16 * bb + 4 * tq);
-          }
-#pragma unroll
-          for (int bb = 0; bb < NB; ++bb) {
-            const uint32_t a0 = e2m1x4_to_e4m3x4(wa[bb] & 0xFFFFu), a2 = e2m1x4_to_e4m3x4(wa[bb] >> 16);
-            const uint32_t a1 = e2m1x4_to_e4m3x4(wb[bb] & 0xFFFFu), a3 = e2m1x4_to_e4m3x4(wb[bb] >> 16);
-#pragma unroll
-            for (int nt = 0; nt < NTILE; ++nt) {
-              accb[bb][nt][0] = accb[bb][nt][1] = accb[bb][nt][2] = accb[bb][nt][3] = 0.f;
-              mma_e4m3_16832(accb[bb][nt], a0, a1, a2, a3, bq[nt][bb][0], bq[nt][bb][1]);
-            }
-          }
-        } else {
-          uint4 ra[KS / 2], rb[KS / 2];
-#pragma unroll
-          for (int c = 0; c < KS / 2; ++c) {
-            ra[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g) * Di + (tq + 4 * c) * 16);
-            rb[c] = *reinterpret_cast<const uint4*>(tile + (size_t)(r0 + g + 8) * Di + (tq + 4 * c) * 16);
-          }
-#pragma unroll
-          for (int nt = 0; nt < NTILE; ++nt) {
-            acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-              const uint4& A = ra[ks >> 1];
-              const uint4& B = rb[ks >> 1];
-              const bool hiw = ks & 1;
-              mma_e4m3_16832(acc[nt], hiw ? A.z : A.x, hiw ? B.z : B.x, hiw ? A.w : A.y, hiw ? B.w : B.y,
-                             bq[nt][ks][0], bq[nt][ks][1]);
-            }
-          }
-        }
-        __syncwarp();
-        if (lane == 0) release_stage(&S.released[s]);
-        if constexpr (FP4) {
-          // each block's exact dot product times 2^(query exponent) * 2^(key exponent)
-#pragma unroll
-          for (int nt = 0; nt < NTILE; ++nt)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              float dg = 0.f, dg8 = 0.f;
-#pragma unroll
-              for (int bb = 0; bb < NB; ++bb) {
-                dg = fmaf(accb[bb][nt][c] * e8m0_to_float((skg >> (8 * bb)) & 0xFFu), fq[nt][c][bb], dg);
-                dg8 = fmaf(accb[bb][nt][2 + c] * e8m0_to_float((skg8 >> (8 * bb)) & 0xFFu), fq[nt][c][bb], dg8);
-              }
-              acc[nt][c] = dg;
-              acc[nt][2 + c] = dg8;
-            }
-        }
-        const int e_g = it * kIdxTile + r0 + g, e_g8 = e_g + 8;
-        const float kg = FP4 ? 1.f : (float)skg, kg8 = FP4 ? 1.f : (float)skg8;
-        float vg = 0.f, vg8 = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < NTILE; ++nt)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            vg = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * kg) * acc[nt][c]), vg);
-            vg8 = fmaf(wh[nt][c], fmaxf(0.f, (sq[nt][c] * kg8) * acc[nt][2 + c]), vg8);
-          }
-        vg += __shfl_xor_sync(0xffffffffu, vg, 1);
-        vg += __shfl_xor_sync(0xffffffffu, vg, 2);
-        vg8 += __shfl_xor_sync(0xffffffffu, vg8, 1);
-        vg8 += __shfl_xor_sync(0xffffffffu, vg8, 2);
-        if (tq == 0 && e_g < len) sc[e_g] = vg;
-        if (tq == 1 && e_g8 < len) sc[e_g8] = vg8;
+      const bool act0 = r0 < min(kIdxTile, len - it * kIdxTile);
+      const bool act1 = n2 == 2 && r0 < min(kIdxTile, len - (it + 1) * kIdxTile);
+      float acc0[NTILE][4], acc1[NTILE][4];
+      if (act0) mma_tile(ring + (size_t)s * kIdxTile * RB, ska0, skb0, acc0);
+      if (act1) mma_tile(ring + (size_t)s1 * kIdxTile * RB, ska1, skb1, acc1);
+      __syncwarp();
+      if (lane == 0) {
+        release_stage(&S.released[s]);
+        if (n2 == 2) release_stage(&S.released[s1]);
       }
-      if (++s == stages) {
+      if (act0) epilogue(it, ska0, skb0, acc0);
+      if (act1) epilogue(it + 1, ska1, skb1, acc1);
+      s = s1;
+      ph = ph1;
+      if (n2 == 2 && ++s == stages) {
         s = 0;
         ph ^= 1u;
       }

@@ -63,6 +63,8 @@ cudaError_t launch_hca_bulk(const void* x, const void* z, const float* bias, con
                             const int64_t* tok0, int batch, const int64_t* ent_off, const int64_t* first,
                             const int64_t* num, int64_t max_blocks, int in_dt, int out_dt, void* out,
                             const float* gamma, float eps, int norm, int* st, cudaStream_t stream);
+cudaError_t launch_rmsnorm_rows(const void* x, int dtype, int64_t rows, const float* gamma, float eps, void* out,
+                                cudaStream_t stream);
 cudaError_t launch_pool_keys(const void* k_tok, int in_dt, int Di, const int64_t* tok_off, const int64_t* tok0,
                              int batch, const int64_t* ent_off, const int64_t* first, const int64_t* num,
                              int64_t max_blocks, uint8_t* codes, float* scales, int* st, cudaStream_t stream);

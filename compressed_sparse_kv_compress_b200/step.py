@@ -19,7 +19,9 @@ Tensor names (all device tensors, int64 offsets unless noted):
             bias_a bias_b [4, 256] fp32 or None, csa_first csa_num [B]
   HCA rows  x_h z_h, hca_x_off, hca_t0, bias_h [128, 256] or None, hca_first hca_num
   caches    cmp_c [sum ceil(n/4), 256] + csa_off [B+1]; cmp_h + hca_off
-  indexer   k_idx [entries, Di] (+ k_scale), q_idx [T, Hi, Di] (+ q_scale), head_w
+  indexer   k_idx [entries, Di] (+ k_scale), q_idx [T, Hi, Di] (+ q_scale), head_w;
+            optional k_tok [rows, Di] bf16 per-token keys (rows like x_a): the step pools
+            its entries' keys from them inside the CSA compression
   window    raw_c raw_h [rows, 256], raw_off [B+1], raw_t0 [B]
   queries   q_c q_h [T, H, 128], sink_c sink_h [H] or None, q_seq [T] int32, q_pos [T]
 """
@@ -72,11 +74,15 @@ class DecodeStep:
                          dev_status=self.status, stream=stream)
 
     def csa_compress(self, stream=None):
+        """The CSA entries the new tokens complete; with per-token indexer keys (k_tok) the
+        same kernel also pools those entries' indexer keys into k_idx / k_scale."""
         t = self.t
+        pool = t.get("k_tok") is not None
         api.csa_compress(t["x_a"], t["z_a"], t["x_b"], t["z_b"], t["csa_x_off"], t["csa_off"], t["cmp_c"],
                          max_blocks=self.max_csa_blocks, bias_a=t.get("bias_a"), bias_b=t.get("bias_b"),
                          tok0=t["csa_t0"], first_block=t["csa_first"], num_blocks=t["csa_num"],
-                         dev_status=self.status, stream=stream)
+                         k_tok=t["k_tok"] if pool else None, k_codes=t["k_idx"] if pool else None,
+                         k_scale=t["k_scale"] if pool else None, dev_status=self.status, stream=stream)
 
     def csa_select(self, stream=None):
         t = self.t
@@ -125,6 +131,8 @@ class DecodeStep:
         self.hca_layer(self.side)
         self.csa_compress(self.side_c)
         self.ev_c.record(self.side_c)
+        if self.t.get("k_tok") is not None:
+            main.wait_event(self.ev_c)  # the indexer reads the keys the compression pools
         self.csa_select(main)
         main.wait_event(self.ev_c)
         self.csa_attend(main)

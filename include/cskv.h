@@ -143,6 +143,21 @@ CSKV_API int hca_compress(const void* x, const void* z, const float* bias,
                  int* dev_status, cskv_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * rmsnorm_heads -- RMSNorm of head vectors (the query-side pass).
+ *
+ * [SW] §十四.3: queries and KV are RMS-normalised so that attention logits cannot
+ * blow up.  Every row of x (one query head: d = 128 values) becomes
+ *     out = x / sqrt(mean(x^2) + eps) * gamma
+ * in fp32, rounded to the storage type.  (The KV side is the compression
+ * epilogue: csa_compress / hca_compress with rmsnorm = 1.)
+ * x, out : [rows, 128] dtype (CSKV_F32 or CSKV_BF16), 16-byte aligned; out may be x.
+ * gamma  : [128] fp32 or NULL (ones), 4-byte aligned.  eps >= 0, finite.
+ * rows == 0 launches nothing; d other than 128 is CSKV_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------ */
+CSKV_API int rmsnorm_heads(const void* x, int dtype, int64_t rows, int d, const float* gamma, float eps, void* out,
+                           cskv_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * lindex_pool_keys -- the indexer's entry keys from per-token keys.
  *
  * [TR] §4.2 (LightningIndexer: per-token keys, then a 1-D pool whose kernel and

@@ -69,13 +69,32 @@ def compress_step(meta, arrays, dtypes, bulk=False, seqs=None):
     return cmp_c, cmp_h, new
 
 
+def pooled_step_keys(meta, arrays, b):
+    """With per-token indexer keys (``k_tok``, rows indexed like x_a): the step's CSA entries of
+    sequence b get keys pooled from their tokens ([TR] §4.2; the exact definition,
+    indexer.pool_keys_f64 / quantize_keys_f64).  Returns (entries, E4M3 codes, scales)."""
+    first, num = meta["csa_first"][b], meta["csa_num"][b]
+    ents = np.arange(first, first + num)
+    t0, n = meta["csa_t0"][b], meta["n"][b]
+    o = meta["csa_x_off"][b]
+    tok = codecs.decode(arrays["k_tok"][o + 4 * first - t0: o + n - t0], "bf16")
+    codes, scales = indexer.quantize_keys_f64(indexer.pool_keys_f64(tok, compress.CSA_RATIO))
+    return ents, codes, scales
+
+
 def query_scores(meta, arrays, dtypes, t):
-    """Indexer scores [V] of query t over its visible CSA entries."""
+    """Indexer scores [V] of query t over its visible CSA entries (with ``k_tok``: the step's
+    entries scored with their pooled keys)."""
     b, p = meta["q_seq"][t], meta["q_pos"][t]
     V = min(indexer.visible_entries(p, compress.CSA_RATIO), meta["ncsa"][b])
     off = meta["csa_off"][b]
     k_idx = codecs.decode(arrays["k_idx"][off: off + V], dtypes["idx"])
-    k_scale = None if arrays.get("k_scale") is None else arrays["k_scale"][off: off + V]
+    k_scale = None if arrays.get("k_scale") is None else np.array(arrays["k_scale"][off: off + V], dtype=np.float64)
+    if arrays.get("k_tok") is not None:
+        ents, codes, scales = pooled_step_keys(meta, arrays, b)
+        keep = ents < V
+        k_idx[ents[keep]] = codecs.e4m3_decode(codes[keep])
+        k_scale[ents[keep]] = scales[keep]
     q_idx = codecs.decode(arrays["q_idx"][t], dtypes["idx"])
     q_scale = None if arrays.get("q_scale") is None else arrays["q_scale"][t]
     return indexer.index_scores(q_idx, k_idx, q_scale, k_scale, arrays.get("head_w"))

@@ -21,7 +21,9 @@ Layout (all row-major, sequences concatenated in order):
   * raw window rows ``raw_c`` / ``raw_h`` hold the tail from ``raw_t0[b]``;
   * indexer keys ``k_idx`` [sum ceil(n/4), 64] with ``k_scale``;
   * queries ``q_c`` / ``q_h`` [T, H, 128], indexer queries ``q_idx``
-    [T, Hi, 64] with ``q_scale`` [T, Hi].
+    [T, Hi, 64] with ``q_scale`` [T, Hi];
+  * with ``pool_keys``: per-token indexer keys ``k_tok`` [rows, 64] bf16 of the CSA
+    tail rows (indexed like ``x_a``), from which the step pools its entries' keys.
 """
 
 from __future__ import annotations
@@ -58,6 +60,7 @@ class Spec:
     biases: bool = False           # position biases ~N(0,1) instead of 0
     cache: str = "random"          # random: cache state drawn directly; compress: built from full rows
     needles: int = 0
+    pool_keys: bool = False        # the step pools its entries' indexer keys from per-token keys (k_tok)
     seed: int = 0
 
     def replace(self, **kw) -> "Spec":
@@ -260,6 +263,10 @@ class Workload:
             a["k_idx"], a["k_scale"] = torch.from_numpy(ki).clone(), None
             a["q_idx"], a["q_scale"] = torch.from_numpy(qi).clone(), None
 
+        if s.pool_keys:
+            # per-token indexer keys of the CSA tail rows (rows indexed like x_a), bf16
+            a["k_tok"] = _normal(seed, "k_tok", rows_c, di, 1.0 / math.sqrt(di))
+            a["k_tok"] = _to_storage(a["k_tok"], "bf16")
         a["head_w"] = torch.ones(Hi, dtype=torch.float32)
         if s.sink == "one":
             v = _normal(seed, "sink", 1, 1, 1.0)[0, 0]

@@ -82,6 +82,12 @@ def test_compress_validation(lib):
     assert csa(k_tok=_p(), Di=96) == _lib.ERR_UNSUPPORTED
     assert csa(k_tok=_p(), k_dt=2) == _lib.ERR_UNSUPPORTED
     assert csa(k_tok=_p(0x1008)) == _lib.ERR_INVALID_ARG
+    # the query-side RMSNorm
+    assert lib.rmsnorm_heads(_p(), 2, 10, 128, nul, 1e-6, _p(), nul) == _lib.ERR_UNSUPPORTED  # fp8
+    assert lib.rmsnorm_heads(_p(), 1, 10, 64, nul, 1e-6, _p(), nul) == _lib.ERR_UNSUPPORTED
+    assert lib.rmsnorm_heads(_p(), 1, 10, 128, nul, -1.0, _p(), nul) == _lib.ERR_INVALID_ARG
+    assert lib.rmsnorm_heads(_p(0x1008), 1, 10, 128, nul, 1e-6, _p(), nul) == _lib.ERR_INVALID_ARG
+    assert lib.rmsnorm_heads(nul, 1, 0, 128, nul, 1e-6, nul, nul) == _lib.OK
     # nothing to do
     assert hca(max_blocks=0) == _lib.OK
     assert csa(max_blocks=0, norm=1, k_tok=_p()) == _lib.OK

@@ -220,3 +220,23 @@ def test_bulk_capacity_flag():
     ents, ref = _csa_ref(c, 0, [0], [CSA_BULK_MIN], False)
     compress_tol_check(got[ents], ref, "bf16", "entries within the bound")
     assert np.all(got[CSA_BULK_MIN:] == 0)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_rmsnorm_heads_query_side(dtype):
+    # the query-side pass: every 128-dimension head vector, gains and eps, in place and not
+    rng = np.random.default_rng(31)
+    q = torch.from_numpy((rng.standard_normal((37, 16, 128)) / np.sqrt(128)).astype(np.float32))
+    q[3, 5] = 0.0  # a zero head: stays zero
+    q = q.to(torch.bfloat16) if dtype == "bf16" else q
+    gamma = torch.from_numpy(rng.uniform(0.5, 1.5, 128).astype(np.float32))
+    ref = norm.rmsnorm(storage_rows(q.reshape(-1, 128)), gamma.numpy().astype(np.float64), 1e-6)
+    out = torch.empty_like(q).cuda()
+    qd = q.cuda()
+    api.rmsnorm_heads(qd, out, gamma=gamma.cuda(), eps=1e-6)
+    torch.cuda.synchronize()
+    compress_tol_check(storage_rows(out.cpu().reshape(-1, 128)), ref, dtype, "rmsnorm_heads")
+    assert torch.all(out[3, 5] == 0)
+    api.rmsnorm_heads(qd, gamma=gamma.cuda(), eps=1e-6)  # in place
+    torch.cuda.synchronize()
+    assert torch.equal(qd, out)

@@ -169,3 +169,22 @@ def test_selection_stable_beside_hca_layer(name, reps):
         torch.cuda.synchronize()
         assert int(step2.status.item()) == 0
         assert torch.equal(step2.idx, ref), f"graph replay {rep} selects differently"
+
+
+def test_step_pools_its_entries_keys():
+    # per-token indexer keys: the CSA compression of the step also pools its entries' keys
+    # (fused), the indexer reads them; the codes are checked against the exact fp64 pooling
+    # (band rule) and the selection and outputs against the oracle's step with pooled keys
+    from helpers import check_pooled_keys
+    spec = spec_by_name("b8_ctx64k").replace(batch=4, seq_len=(65536, 30001, 4097, 4100), heads=64, pool_keys=True)
+    w = Workload(spec)
+    step, dev = _run_gpu(w, two_streams=True)
+    m, a = w.meta, np_arrays(w)
+    codes, scales = dev["k_idx"].cpu().numpy(), dev["k_scale"].cpu().numpy()
+    for b in range(m["B"]):
+        ents, _, _ = ostep.pooled_step_keys(m, a, b)
+        o = m["csa_x_off"][b]
+        tok = storage_rows(w.arrays["k_tok"][o + 4 * ents[0] - m["csa_t0"][b]: o + m["n"][b] - m["csa_t0"][b]])
+        rows = m["csa_off"][b] + ents
+        check_pooled_keys(codes[rows], scales[rows], tok, 4, what=f"seq {b}")
+    _check(w, step, dev, list(range(m["T"])))
