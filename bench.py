@@ -6,14 +6,19 @@ A step = every row of the hot path on one batch of synthetic input: CSA
 compression of the entries the new tokens complete, the Lightning Indexer
 scan + exact top-k, CSA attention (top-k + window + sink), HCA compression,
 HCA dense attention (+ window + sink), split merges.  Inputs are resident in
-HBM; the step is replayed from a CUDA graph.  Prints one JSON line on rank 0.
+HBM.  Prints one JSON line on rank 0.
 
 L2 discipline (--l2): "rotate" (default) keeps R device replicas of the whole
-workload, each with its own captured graph, and replays them round-robin, R
-chosen so that the other replicas' step bytes exceed three L2 capacities: every
-step reads inputs that are not in L2, and L2 holds what a real model leaves
-there (mostly clean lines).  "flush" instead writes a 256 MiB buffer before
-every timed step, outside its events, which leaves L2 full of dirty lines.
+workload and runs their steps round-robin, R chosen so that the other
+replicas' step bytes exceed three L2 capacities: every step reads inputs that
+are not in L2, and L2 holds what a real model leaves there (mostly clean
+lines).  The timed steps replay CUDA graphs that each hold R consecutive steps
+(replicas 0..R-1, each step waiting for the one before), as a decode
+iteration's layers replay from one graph; the same K steps as single-step
+graph replays are reported beside it (single_step_graphs_us_per_step: every
+graph launch adds the GPU's per-graph overhead).  "flush" instead writes a
+256 MiB buffer before every timed step, outside its events, which leaves L2
+full of dirty lines, and replays one single-step graph per step.
 
 --impl reference times the CPU oracle (plain fp64 numpy) on the machine's host
 cores on a bounded sample of the same workload.
@@ -408,13 +413,45 @@ def run_cskv(args, ws, rank, local):
         if int(st.status.item()) != 0:
             raise RuntimeError(f"device status {int(st.status.item())} during warm-up")
 
-    # ---- timed region: K graph replays (replica i mod R)
+    # ---- the timed steps run from CUDA graphs of consecutive steps, one per replica in turn
+    #      (as a decode iteration's layers run from one graph): `chain_all` holds steps 0..R-1,
+    #      `chain_part` the first K mod R; K steps = (K div R) x chain_all + chain_part.  Each
+    #      step in a graph still waits for the one before (both of its streams).
+    def chain_graph(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for st in steps[:n]:
+                st.run()
+        return g
+
+    chain_all = chain_graph(R)
+    n_full, rem = divmod(args.steps, R)
+    chain_part = chain_graph(rem) if rem else None
+    for _ in range(2):
+        chain_all.replay()
+        if chain_part is not None:
+            chain_part.replay()
+    torch.cuda.synchronize()
+
+    def chained_steps():
+        for _ in range(n_full):
+            chain_all.replay()
+        if chain_part is not None:
+            chain_part.replay()
+
+    # ---- timed region: K steps
     clocks = ClockSampler(ClockSampler.selector(torch.cuda.current_device()))
     clocks.start()
     time.sleep(0.3)
     barrier(ws)
-    ms_local = timed(lambda i: steps[i % R].replay(), args.steps)
+    if flush is None:
+        ms_local = timed(lambda i: chained_steps() if i == 0 else None, 1) / args.steps
+    else:  # a flush between steps: one single-step graph per step, events around each
+        ms_local = timed(lambda i: steps[i % R].replay(), args.steps)
     barrier(ws)
+    # the same K steps as K single-step graph replays (each graph launch adds the GPU's
+    # per-graph overhead, several microseconds for a two-stream graph)
+    ms_single = timed(lambda i: steps[i % R].replay(), args.steps)
 
     # ---- dominant kernel alone (indexer scan + top-k), same L2 discipline.  (1) back to back:
     #      one graph holding one launch per replica in a row (each a dependent launch of the one
@@ -515,7 +552,11 @@ def run_cskv(args, ws, rank, local):
         spec.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": args.workload, "batch": m["B"], "context": max(m["n"]), "query_tokens_per_step": T,
                    "heads": m["H"], "topk": m["k"], "window": m["W"], "indexer": f"{m['Hi']}x{m['di']} "
-                   f"{spec.idx_dtype}", "l2": l2, "replay": "cuda graph", "streams": 1 if args.one_stream else 2},
+                   f"{spec.idx_dtype}", "l2": l2,
+                   "replay": (f"CUDA graphs of consecutive steps ({R} steps, one per replica, per graph)"
+                              if flush is None else "one single-step CUDA graph per step"),
+                   "streams": 1 if args.one_stream else 2},
+        "single_step_graphs_us_per_step": reduce_max(ms_single, ws) * 1e3,
         "step_hbm_bytes": by["total"], "step_gbs": by["total"] / (ms * 1e-3) / 1e9,
         "step_frac_of_measured_hbm": by["total"] / (ms * 1e-3) / 1e9 / hbm,
         "roofline": {"kernel": "lindex_topk_kernel (indexer scan + top-k)", "bound": "hbm", "achieved": achieved,
@@ -538,7 +579,7 @@ def run_cskv(args, ws, rank, local):
         line["cpu_baseline"] = oracle_sample(w, budget_s=args.ref_budget, max_queries=10000)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del idx_graphs, chain, steps
+    del idx_graphs, chain, chain_all, chain_part, steps
     torch.cuda.synchronize()
 
 

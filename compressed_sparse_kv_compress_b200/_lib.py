@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(_HERE, "libcskv.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_LAUNCH = 0, 1, 2, 3, 4
 F32, BF16, FP8E4M3 = 0, 1, 2
+OVERLAP_PREVIOUS = 1  # csa_compress flags (CSKV_OVERLAP_PREVIOUS)
 CSA, HCA = 0, 1
 DEV_BAD_INDEX, DEV_TAIL_MISSING, DEV_CAPACITY, DEV_TIMEOUT = 1, 2, 4, 8
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -31,7 +32,7 @@ SIGNATURES = {
     "cskv_launch_count": (ctypes.c_ulonglong, []),
     "cskv_copy_segments": (_i32, [_p, _p, _p, _p, _i32, _p]),
     "csa_compress": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p,
-                            _i32, _p, _f, _p, _i32, _i32, _p, _p, _p, _p]),
+                            _i32, _p, _f, _p, _i32, _i32, _p, _p, _i32, _p, _p]),
     "hca_compress": (_i32, [_p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p, _i32, _p, _f, _p, _p]),
     "rmsnorm_heads": (_i32, [_p, _i32, _i64, _i32, _p, _f, _p, _p]),
     "lindex_pool_keys": (_i32, [_p, _i32, _i32, _p, _p, _i32, _p, _p, _p, _i64, _p, _p, _p, _p]),

@@ -12,7 +12,7 @@ import math
 import torch
 
 from . import _lib
-from ._lib import BF16, CSA, F32, FP8E4M3, HCA  # noqa: F401
+from ._lib import BF16, CSA, F32, FP8E4M3, HCA, OVERLAP_PREVIOUS  # noqa: F401
 
 _DT = {torch.float32: F32, torch.bfloat16: BF16, torch.uint8: FP8E4M3, torch.float8_e4m3fn: FP8E4M3}
 
@@ -39,18 +39,20 @@ def _stream(stream) -> int:
 
 def csa_compress(x_a, z_a, x_b, z_b, tok_off, ent_off, out, *, max_blocks, bias_a=None, bias_b=None, tok0=None,
                  first_block=None, num_blocks=None, rmsnorm=False, norm_gamma=None, norm_eps=1e-6, k_tok=None,
-                 k_codes=None, k_scale=None, dev_status=None, stream=None):
+                 k_codes=None, k_scale=None, overlap_previous=False, dev_status=None, stream=None):
     """rmsnorm: normalise each entry's K and V halves (norm_gamma [256] fp32, K then V; None =
     ones).  k_tok [rows, Di] (rows indexed like x_a): also pool the per-token indexer keys of
-    the same entries into k_codes [*, Di] uint8 (E4M3) and k_scale [*] fp32."""
+    the same entries into k_codes [*, Di] uint8 (E4M3) and k_scale [*] fp32.
+    overlap_previous: CSKV_OVERLAP_PREVIOUS (the kernel issued just before this call on the
+    stream neither writes its inputs nor reads its outputs; see the C header)."""
     lib = _lib.load()
     k_dt = _dt(k_tok) if k_tok is not None else F32
     Di = int(k_tok.shape[-1]) if k_tok is not None else 0
     st = lib.csa_compress(_ptr(x_a), _ptr(z_a), _ptr(x_b), _ptr(z_b), _ptr(bias_a), _ptr(bias_b), _ptr(tok_off),
                           _ptr(tok0), tok_off.numel() - 1, _ptr(ent_off), _ptr(first_block), _ptr(num_blocks),
                           int(max_blocks), _dt(x_a), _dt(out), _ptr(out), int(bool(rmsnorm)), _ptr(norm_gamma),
-                          float(norm_eps), _ptr(k_tok), k_dt, Di, _ptr(k_codes), _ptr(k_scale), _ptr(dev_status),
-                          _stream(stream))
+                          float(norm_eps), _ptr(k_tok), k_dt, Di, _ptr(k_codes), _ptr(k_scale),
+                          OVERLAP_PREVIOUS if overlap_previous else 0, _ptr(dev_status), _stream(stream))
     _lib.check("csa_compress", st)
     return out
 

@@ -4,6 +4,7 @@
 
 #include "launch.cuh"
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -104,9 +105,10 @@ int csa_compress(const void* x_a, const void* z_a, const void* x_b, const void* 
                  const int64_t* ent_off, const int64_t* first_block, const int64_t* num_blocks,
                  int64_t max_blocks, int in_dtype, int out_dtype, void* out, int rmsnorm, const float* norm_gamma,
                  float norm_eps, const void* k_tok, int k_dtype, int Di, uint8_t* k_codes, float* k_scale,
-                 int* dev_status, cskv_stream_t stream) {
+                 int flags, int* dev_status, cskv_stream_t stream) {
   int rc = check_compress_common(x_a, z_a, tok_off, batch, ent_off, max_blocks, in_dtype, out_dtype, out);
   if (rc) return rc;
+  if (flags & ~CSKV_OVERLAP_PREVIOUS) return CSKV_ERR_INVALID_ARG;
   if ((x_b == nullptr) != (z_b == nullptr)) return CSKV_ERR_INVALID_ARG;
   if (x_b && (!aligned16(x_b) || !aligned16(z_b))) return CSKV_ERR_INVALID_ARG;
   if ((bias_a && !aligned16(bias_a)) || (bias_b && !aligned16(bias_b))) return CSKV_ERR_INVALID_ARG;
@@ -124,7 +126,7 @@ int csa_compress(const void* x_a, const void* z_a, const void* x_b, const void* 
   return launch_status(launch_csa_compress(x_a, z_a, x_b, z_b, bias_a, bias_b, tok_off, tok0, batch, ent_off,
                                            first_block, num_blocks, max_blocks, in_dtype, out_dtype, out, rmsnorm,
                                            norm_gamma, norm_eps, k_tok, k_dtype, k_tok ? Di : 0, k_codes, k_scale,
-                                           dev_status, (cudaStream_t)stream));
+                                           flags, dev_status, (cudaStream_t)stream));
 }
 
 int lindex_pool_keys(const void* k_tok, int in_dtype, int Di, const int64_t* tok_off, const int64_t* tok0,
@@ -286,15 +288,35 @@ int lindex_topk_from_scores(const float* scores, int64_t ld_scores, const int64_
   return launch_status(launch_lindex(p, CSKV_F32, T, (cudaStream_t)stream));
 }
 
-// Split plan of hybrid_decode_attn: rows per split R and the split count S for the
-// tensor-core kernel (bf16) or the CUDA-core kernel (fp32).
-static int attn_plan(int mode, int T, int k, int window, int64_t max_entries, bool tc, int* R, int* S) {
+// Split plan of hybrid_decode_attn for the tensor-core kernel (bf16) or the CUDA-core kernel
+// (fp32): rows per split R and split count S; ws_splits = the split count the workspace of
+// partials is sized for (the larger of the two plans below).  A tensor-core plan of at most
+// kClusterMaxSplits splits instead merges inside a thread-block cluster (cluster = S, a power
+// of two <= 16, rows spread evenly over it) when such a cluster fits on the device.
+constexpr int kClusterMaxSplits = 18;
+struct AttnPlan {
+  int R, S, ws_splits, cluster;
+};
+static int attn_plan(int mode, int T, int k, int window, int64_t max_entries, bool tc, AttnPlan* pl) {
   int sms = 0;
   int rc = device_sms(&sms);
   if (rc) return rc;
-  *R = tc ? attn_tc_rows_per_split(mode, T, k, window, max_entries, sms)
-          : attn_rows_per_split(mode, T, k, window, max_entries, sms);
-  *S = attn_max_splits(mode, k, window, max_entries, *R);
+  pl->R = tc ? attn_tc_rows_per_split(mode, T, k, window, max_entries, sms)
+             : attn_rows_per_split(mode, T, k, window, max_entries, sms);
+  pl->S = attn_max_splits(mode, k, window, max_entries, pl->R);
+  pl->ws_splits = pl->S;
+  pl->cluster = 0;
+  if (tc && pl->S <= kClusterMaxSplits) {
+    int want = 1;
+    while (want < pl->S && want < 16) want <<= 1;
+    if (attn_tc_cluster_fit(want) == want) {
+      const int64_t rows_max = (mode == CSKV_CSA ? (int64_t)k : max_entries) + window;
+      pl->R = (int)std::max<int64_t>(1, (rows_max + want - 1) / want);
+      pl->S = want;
+      pl->cluster = want;
+      pl->ws_splits = std::max(pl->ws_splits, want);
+    }
+  }
   return CSKV_OK;
 }
 
@@ -302,9 +324,9 @@ size_t hybrid_attn_workspace_size(int mode, int T, int H, int d, int k, int wind
   if (T < 1 || H < 1 || d != kHeadDim || window < 0) return 0;
   size_t best = 0;
   for (int tc = 0; tc < 2; ++tc) {
-    int R = 0, S = 0;
-    if (attn_plan(mode, T, k, window, max_entries, tc != 0, &R, &S)) return 0;
-    const size_t need = (size_t)T * S * H * (kHeadDim + 2) * sizeof(float);
+    AttnPlan pl;
+    if (attn_plan(mode, T, k, window, max_entries, tc != 0, &pl)) return 0;
+    const size_t need = (size_t)T * pl.ws_splits * H * (kHeadDim + 2) * sizeof(float);
     if (need > best) best = need;
   }
   return best;
@@ -344,10 +366,10 @@ int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_
                             T, H, d, dtype, max_entries, out);
   if (arc != CSKV_OK || T == 0) return arc;
   const bool tc = dtype == CSKV_BF16;
-  int R = 0, S = 0;
-  int rc = attn_plan(mode, T, mode == CSKV_CSA ? k : 0, window, max_entries, tc, &R, &S);
+  AttnPlan pl;
+  int rc = attn_plan(mode, T, mode == CSKV_CSA ? k : 0, window, max_entries, tc, &pl);
   if (rc) return rc;
-  const size_t need = (size_t)T * S * H * (kHeadDim + 2) * sizeof(float);
+  const size_t need = (size_t)T * pl.ws_splits * H * (kHeadDim + 2) * sizeof(float);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSKV_ERR_WORKSPACE;
   AttnParams p = {};
   p.mode = mode;
@@ -367,10 +389,11 @@ int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_
   p.batch = batch;
   p.T = T;
   p.H = H;
-  p.rows_per_split = R;
-  p.max_splits = S;
+  p.rows_per_split = pl.R;
+  p.max_splits = pl.S;
+  p.cluster = pl.cluster;
   p.part_acc = (float*)workspace;
-  p.part_ml = p.part_acc + (size_t)T * S * H * kHeadDim;
+  p.part_ml = p.part_acc + (size_t)T * pl.S * H * kHeadDim;
   p.out = out;
   p.lse = lse;
   p.st = dev_status;

@@ -19,8 +19,18 @@
 //      P = 2^(s - m) as bf16 into shared memory;
 //   4. one thread issues O[128 x 128] (+)= P[128 x nc] V[nc x 128] (V read MN-major).
 // Q, K and P are K-major operands, V is MN-major; all four use the same swizzled layout.
-// The split's (m, l, O) go to the workspace; attn_combine_kernel merges the splits and the
-// sink.  Heads beyond H are zero rows of Q (M is always 128).
+// Heads beyond H are zero rows of Q (M is always 128).
+//
+// Merging the splits of a query ([TR] §3.1; the sink joins once, [SW] §十二):
+//  * cluster mode (p.cluster = the split count, at most 16): the query's splits are the CTAs
+//    of one thread-block cluster.  Each writes its partial (unnormalised O rows, (m, l)) to
+//    the workspace, a cluster barrier publishes them, and each CTA merges 128 / p.cluster of
+//    the heads from L2 -- no second kernel and no launch gap.  (Reading the partials from the
+//    other CTAs' shared memory instead was slower: every remote load a round trip over the
+//    SM-to-SM network.)
+//  * otherwise the split's (m, l, O) go to the workspace and attn_combine_kernel merges.
+#include <mutex>
+
 #include "attn_rows.cuh"
 #include "sm100.cuh"
 
@@ -43,6 +53,82 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c) {
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Cluster mode: merges the query's splits (the CTAs of this cluster, rank = split) once every
+// split has written its partial to the workspace -- the unnormalised O as float4 groups of
+// dimensions, [split][group 0..31][h] (a warp's write of one group is 512 contiguous bytes),
+// and (m, l) per head -- and writes the output and lse.  Called by all threads of every CTA of
+// the cluster.  The cluster barrier (release / acquire at cluster scope) makes the partials of
+// all splits visible; they stay in L2.  CTA r then merges heads r * 128 / CS ..
+// (r + 1) * 128 / CS - 1 (HPC heads): thread (g, hh) = (tid / HPC, tid % HPC) takes head
+// r * HPC + hh and the dimension groups g, g + CS, ..., so a warp's loads are runs of HPC
+// consecutive heads.  For its head a thread folds every split's (m, l) with the sink,
+//   M = max(max_s m_s, sink),  L = sum_s 2^(m_s - M) l_s + 2^(sink - M),
+// and sums the splits' values scaled by 2^(m_s - M) / L.  A thread's loads go in two rounds:
+// the CS (m, l) pairs with the first 16 groups of values, then the other 16 (all 32 at once
+// would take the kernel past 250 registers, and then it no longer fits on an SM beside the
+// kernels that share one during a decode step).
+template <int CS>
+__device__ __forceinline__ void cluster_merge(const AttnParams& p, int t) {
+  cluster_sync();
+  const int tid = threadIdx.x, H = p.H;
+  const uint32_t rank = cluster_rank();
+  constexpr int HPC = 128 / CS;  // heads merged by this CTA
+  constexpr int NG = 32 / CS;    // dimension groups per thread: NG x CS = 32 loads
+  constexpr int NG1 = NG / 2;    // groups of the first round (the second round: the rest)
+  const int h = (int)rank * HPC + tid % HPC, g0 = tid / HPC;
+  if (h >= H) return;  // no barrier follows: a thread without a head is done
+  const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)t * CS * H + h;
+  const float4* po = reinterpret_cast<const float4*>(p.part_acc) + (size_t)t * CS * 32 * H + h;
+  float2 mls[CS];
+  float4 v[NG1][CS];
+#pragma unroll
+  for (int s = 0; s < CS; ++s) mls[s] = __ldcg(ml + (size_t)s * H);
+#pragma unroll
+  for (int k = 0; k < NG1; ++k)
+#pragma unroll
+    for (int s = 0; s < CS; ++s) v[k][s] = __ldcg(po + ((size_t)s * 32 + g0 + CS * k) * H);
+  const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+  float M = sk;
+#pragma unroll
+  for (int s = 0; s < CS; ++s) M = fmaxf(M, mls[s].x);
+  float f[CS], L = 0.f;
+#pragma unroll
+  for (int s = 0; s < CS; ++s) {
+    f[s] = mls[s].x == -INFINITY ? 0.f : exp2f(mls[s].x - M);  // a split without rows wrote no O
+    L = fmaf(mls[s].y, f[s], L);
+  }
+  if (M != -INFINITY && p.sink) L += exp2f(sk - M);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  float* dst = p.out + ((size_t)t * H + h) * kHeadDim;
+#pragma unroll
+  for (int round = 0; round < 2; ++round) {
+    if (round == 1) {
+#pragma unroll
+      for (int k = 0; k < NG1; ++k)
+#pragma unroll
+        for (int s = 0; s < CS; ++s) v[k][s] = __ldcg(po + ((size_t)s * 32 + g0 + CS * (NG1 + k)) * H);
+    }
+#pragma unroll
+    for (int k = 0; k < NG1; ++k) {
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s = 0; s < CS; ++s)
+        if (f[s] != 0.f) {
+          a.x = fmaf(v[k][s].x, f[s], a.x);
+          a.y = fmaf(v[k][s].y, f[s], a.y);
+          a.z = fmaf(v[k][s].z, f[s], a.z);
+          a.w = fmaf(v[k][s].w, f[s], a.w);
+        }
+      const int grp = g0 + CS * (round * NG1 + k);
+      dst[4 * grp] = a.x * inv;
+      dst[4 * grp + 1] = a.y * inv;
+      dst[4 * grp + 2] = a.z * inv;
+      dst[4 * grp + 3] = a.w * inv;
+    }
+  }
+  if (g0 == 0 && p.lse) p.lse[(size_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
@@ -69,13 +155,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     mbar_init(&bar_o, 1);
     fence_mbar_init();
   }
+  // warm L2 with the query's metadata and the selected indices of this split's first rows
+  // (prefetches only move lines into L2, which stays coherent with the writes being waited for)
+  const int64_t r0 = (int64_t)split * p.rows_per_split;
+  if (tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_seq + t));
+  if (tid == 1) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_pos + t));
+  if (p.mode == CSKV_CSA && tid >= 32 && tid < 32 + kTcChunk / 32 && r0 + (tid - 32) * 32 < p.k)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p.idx + (size_t)t * p.k + r0 + (tid - 32) * 32));
   pdl_wait();
+  // the first chunk's selected indices load beside the query's metadata
+  const int64_t r_pre = r0 + tid;
+  const int64_t e_pre = (p.mode == CSKV_CSA && r_pre < p.k && tid < min((int64_t)kTcChunk, (int64_t)p.rows_per_split))
+                            ? (int64_t)__ldg(p.idx + (size_t)t * p.k + r_pre)
+                            : (int64_t)-2;
   const QueryRows q = query_rows(p, t);
   if (q.s < 0 && split == 0 && tid == 0) flag(p.st, CSKV_DEV_BAD_INDEX);
-  const int64_t r0 = (int64_t)split * p.rows_per_split;
   // a CTA without rows (bad query, or a split past the query's rows) runs no chunk and
   // only releases its TMEM at the end
   const int64_t r1 = q.s < 0 ? r0 : max(r0, min(q.n_rows, r0 + p.rows_per_split));
+  // cluster mode has no merge kernel to notice rows beyond the last split: flag them here
+  if (p.cluster && q.s >= 0 && split == p.max_splits - 1 && tid == 0 && q.n_rows > r0 + p.rows_per_split)
+    flag(p.st, CSKV_DEV_CAPACITY);
   const int H = p.H;
   const __nv_bfloat16* cmp = reinterpret_cast<const __nv_bfloat16*>(p.kv_cmp);
   const __nv_bfloat16* raw = reinterpret_cast<const __nv_bfloat16*>(p.kv_raw);
@@ -104,7 +204,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     {
       int64_t off = -1;
       bool is_raw = false;
-      if (tid < rows) off = resolve_row(p, q, t, a + tid, &is_raw);
+      if (tid < rows) off = resolve_row(p, q, t, a + tid, &is_raw, a == r0 ? e_pre : (int64_t)-2);
       row_src[tid] = off >= 0 ? (is_raw ? raw : cmp) + off : nullptr;
       const uint32_t bal = __ballot_sync(0xffffffffu, off >= 0);
       if (lane == 0) row_mask[warp] = bal;
@@ -223,10 +323,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     alive = !__syncthreads_or(timed_out);  // block-uniform, so every thread leaves the loop together
     tc_fence_after();
   }
-  // ---- partial of this split: O row (unnormalised, relative to m_run), m_run, l_run.
-  //      Every lane takes part in the warp-collective TMEM loads; only real heads store.
-  //      Partials are stored dimension-major ([split][j][h]), so a warp's stores are contiguous.
-  if (c > 0) {
+  if (p.cluster) {
+    // ---- partial of this split (float4 groups of dimensions, head-minor), then the merge
+    const size_t sb = (size_t)t * p.max_splits + split;
+    if (c > 0) {
+      const uint32_t tO = tmem_base + 128;
+      float4* og = reinterpret_cast<float4*>(p.part_acc) + sb * 32 * H + tid;  // group j at og[j * H]
+      for (int cc = 0; cc < 128; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(tO + lane_base + cc, v);
+        tmem_ld_wait();
+        if (tid < H) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            og[(size_t)((cc >> 2) + i) * H] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                          __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+    }
+    if (tid < H)
+      reinterpret_cast<float2*>(p.part_ml)[sb * H + tid] = c > 0 ? make_float2(m_run, l_run) : make_float2(-INFINITY, 0.f);
+    switch (p.cluster) {
+      case 1: cluster_merge<1>(p, t); break;
+      case 2: cluster_merge<2>(p, t); break;
+      case 4: cluster_merge<4>(p, t); break;
+      case 8: cluster_merge<8>(p, t); break;
+      default: cluster_merge<16>(p, t); break;
+    }
+  } else if (c > 0) {
+    // ---- partial of this split: O row (unnormalised, relative to m_run), m_run, l_run.
+    //      Every lane takes part in the warp-collective TMEM loads; only real heads store.
+    //      Partials are stored dimension-major ([split][j][h]), so a warp's stores are contiguous.
     const uint32_t tO = tmem_base + 128;
     const size_t sb = (size_t)t * p.max_splits + split;
     float* dst = p.part_acc + sb * kHeadDim * H + tid;
@@ -244,8 +371,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
       p.part_ml[(sb * 2 + 1) * H + tid] = l_run;
     }
   }
-  // the merge kernel may launch now; it waits for this grid to finish before it reads
-  // (launching it earlier would park its CTAs on SMs that other kernels of the step need)
+  // the next kernel (the merge kernel, without a cluster) may launch now; it waits for this
+  // grid to finish before it reads (launching it earlier would park its CTAs on SMs that
+  // other kernels of the step need)
   pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
@@ -255,15 +383,68 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   }
 }
 
+// Largest cluster size (a power of two, at most `want` and 16) at which one cluster of
+// attn_tc_kernel CTAs fits on the current device, 0 if none; cached per device.
+int attn_tc_cluster_fit(int want) {
+  static std::mutex mu;
+  static int fit[64][5];  // [device][log2 size]: 0 unknown, 1 fits, -1 does not
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (ensure_smem(attn_tc_kernel, kTcSmem) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  int best = 0;
+  for (int lg = 0; lg < 5 && (1 << lg) <= want; ++lg) {
+    if (fit[dev][lg] == 0) {
+      const int cs = 1 << lg;
+      bool ok = true;
+      if (cs > 8)
+        ok = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+      int n = 0;
+      if (ok) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(cs, 1);
+        cfg.blockDim = dim3(kTcThreads);
+        cfg.dynamicSmemBytes = kTcSmem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        ok = cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) == cudaSuccess && n > 0;
+      }
+      cudaGetLastError();  // a refused query leaves no sticky error
+      fit[dev][lg] = ok ? 1 : -1;
+    }
+    if (fit[dev][lg] > 0) best = 1 << lg;
+  }
+  return best;
+}
+
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
   auto kern = attn_tc_kernel;
   cudaError_t e = ensure_smem(kern, kTcSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.max_splits, p.T);
-  kern<<<grid, kTcThreads, kTcSmem, stream>>>(p);
+  // a dependent launch: the CTAs may start (TMEM, barriers) while the previous kernel -- the
+  // indexer, or the compression after it -- finishes, and wait for it before reading
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.max_splits, p.T);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = kTcSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = p.cluster ? p.cluster : 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.cluster ? 2 : 1;
+  e = cudaLaunchKernelEx(&cfg, kern, p);
   note_launch();
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || p.cluster) return e;
   return launch_attn_combine(p, stream);
 }
 

@@ -43,14 +43,15 @@ __device__ __forceinline__ QueryRows query_rows(const AttnParams& p, int t) {
 }
 
 // Row pointer (element offset into kv_cmp or kv_raw) of virtual row r, or -1 when the
-// row is skipped.  *raw tells which array.
+// row is skipped.  *raw tells which array.  e_pre >= -1: idx[t, r], already loaded (CSA rows
+// r < k only; the caller issues that load beside the query's other loads).
 __device__ __forceinline__ int64_t resolve_row(const AttnParams& p, const QueryRows& q, int t, int64_t r,
-                                               bool* raw) {
+                                               bool* raw, int64_t e_pre = -2) {
   if (r < q.n_cmp) {
     *raw = false;
     int64_t e = r;
     if (p.mode == CSKV_CSA) {
-      e = __ldg(p.idx + (size_t)t * p.k + r);
+      e = e_pre >= -1 ? e_pre : __ldg(p.idx + (size_t)t * p.k + r);
       if (e < 0) return -1;
       if (e >= q.vis_c) {
         flag(p.st, CSKV_DEV_BAD_INDEX);

@@ -100,6 +100,7 @@ struct CsaExtras {
   int Di;
   uint8_t* k_codes;
   float* k_scale;
+  int overlap;  // CSKV_OVERLAP_PREVIOUS: read before the previous kernel completes, wait at the end
 };
 
 template <typename TI, typename TO, bool kTwo>
@@ -110,10 +111,13 @@ __global__ void __maxnreg__(144) csa_compress_kernel(
     const int64_t* __restrict__ ent_off, const int64_t* __restrict__ first_block,
     const int64_t* __restrict__ num_blocks, int64_t max_blocks, TO* __restrict__ out, CsaExtras ex, int* st) {
   constexpr int kC = kTwo ? 8 : 4;  // candidates: 4 path-A (+ 4 path-B)
-  // A few small CTAs: the next kernel (the indexer in a decode step) may launch at once and
-  // sit beside them; it waits for this grid before reading anything.
+  // A few small CTAs: the next kernel may launch at once and sit beside them; it waits for
+  // this grid before reading anything.  With ex.overlap the caller guarantees that the kernel
+  // before this one neither writes this call's inputs nor reads its outputs: the entries are
+  // computed while it runs (in a decode step: beside the indexer), and the wait moves to the
+  // end, so this grid still completes after it and a kernel that waits for this grid sees both.
   pdl_launch_dependents();
-  pdl_wait();
+  if (!ex.overlap) pdl_wait();
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SeqRange s = seq_range(b, 4, tok_off, tok0, ent_off, first_block, num_blocks);
@@ -221,6 +225,7 @@ __global__ void __maxnreg__(144) csa_compress_kernel(
       if (lane == 0) ex.k_scale[s.ent0 + i] = scale;
     }
   }
+  if (ex.overlap) pdl_wait();
 }
 
 // ------------------------------------------------------------------ HCA
@@ -250,6 +255,9 @@ __global__ void __launch_bounds__(kHcaThreads, 8) hca_compress_kernel(
     const int64_t* __restrict__ ent_off, const int64_t* __restrict__ first_block,
     const int64_t* __restrict__ num_blocks, int64_t max_blocks, TO* __restrict__ out, int* st) {
   __shared__ float sm_max[4][16], sm_sum[4][16], sm_acc[4][16];
+  // the next kernel (the HCA attention in a decode step) may start its set-up at once; it
+  // waits for this grid before reading anything
+  pdl_launch_dependents();
   pdl_wait();
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, half = lane & 1;
@@ -463,13 +471,14 @@ cudaError_t launch_csa_compress(const void* xa, const void* za, const void* xb, 
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
                                 int in_dt, int out_dt, void* out, int norm, const float* gamma, float eps,
-                                const void* k_tok, int k_dt, int Di, uint8_t* k_codes, float* k_scale, int* st,
-                                cudaStream_t stream) {
-  // many entries: the TMA-ring kernel (one CTA per SM); a few (a decode step): warp per entry
+                                const void* k_tok, int k_dt, int Di, uint8_t* k_codes, float* k_scale, int flags,
+                                int* st, cudaStream_t stream) {
+  // many entries: the TMA-ring kernel (one CTA per SM); a few (a decode step): warp per entry.
+  // (The overlap flag is a permission: the TMA-ring kernel does not use it.)
   if (max_blocks >= kCsaBulkMinEntries)
     return launch_csa_bulk(xa, za, xb, zb, ba, bb, tok_off, tok0, batch, ent_off, first, num, max_blocks, in_dt,
                            out_dt, out, gamma, eps, norm, k_tok, k_dt, Di, k_codes, k_scale, st, stream);
-  CsaExtras ex{norm, gamma, eps, k_tok, k_dt == CSKV_F32, Di, k_codes, k_scale};
+  CsaExtras ex{norm, gamma, eps, k_tok, k_dt == CSKV_F32, Di, k_codes, k_scale, (flags & CSKV_OVERLAP_PREVIOUS) ? 1 : 0};
   if (in_dt == CSKV_BF16 && out_dt == CSKV_BF16)
     return launch_csa_t<__nv_bfloat16, __nv_bfloat16>(xa, za, xb, zb, ba, bb, tok_off, tok0, batch,
                                                       ent_off, first, num, max_blocks, out, ex, st, stream);

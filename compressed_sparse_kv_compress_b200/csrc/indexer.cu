@@ -1224,7 +1224,6 @@ template <int SRC, int KS, int NTILE>
 __global__ void __maxnreg__(88) lindex_topk_kernel(IdxParams p) {
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ IdxShared S;
-  pdl_launch_dependents();  // the kernel after the indexer may start its set-up now
   // While the previous kernel finishes: warm L2 with the lines the plan and the first tile
   // need (the query's position, sequence and offsets, its indexer vectors).  Prefetches only
   // move lines into L2, which stays coherent with the writes of the kernel being waited for.
@@ -1241,6 +1240,10 @@ __global__ void __maxnreg__(88) lindex_topk_kernel(IdxParams p) {
   }
   if (threadIdx.x == 0) S.scan_err = 0;  // read only after later block barriers
   pdl_wait();
+  // The kernel after the indexer may start now.  Only now: every kernel before the indexer has
+  // completed, so a dependent that reads nothing the indexer writes (a compression issued with
+  // CSKV_OVERLAP_PREVIOUS) may start reading at once.
+  pdl_launch_dependents();
   uint8_t* un = dsm;                                              // ring / histogram / candidates
   float* sc = reinterpret_cast<float*>(dsm + p.un_bytes);  // segment scores
   if (p.split && p.T == 1) {
@@ -1330,10 +1333,11 @@ static size_t idx_dyn_smem(int Di, int64_t seg_cap, int stages) {
   return idx_union_bytes(Di, stages) + (size_t)seg_cap * 4;
 }
 
-// Shared memory an indexer CTA of a split-mode launch may take when choosing a deeper ring: a
-// tensor-core attention CTA (~97 KB) of a decode step must still fit on the same SM (228 KB,
-// 1 KB of it reserved per CTA).
-constexpr size_t kIdxDeepRingSmem = 127 * 1024;
+// Dynamic shared memory an indexer CTA of a split-mode launch may take when choosing a deeper
+// ring: a tensor-core attention CTA of a decode step (97 KB dynamic + 3 KB static) must still
+// fit on the same SM beside it (228 KB per SM, 1 KB of it reserved per CTA; the indexer's own
+// static shared memory is 2 KB): 228 - 101 - 1 - 2 - 1 = 123 KB, rounded down.
+constexpr size_t kIdxDeepRingSmem = 123 * 1024;
 
 // Ring stages of a launch: the minimum (64 KiB), deepened towards the whole segment (every
 // fill issued at once) while the CTA stays within kIdxDeepRingSmem.

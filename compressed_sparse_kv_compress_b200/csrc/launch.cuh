@@ -46,8 +46,8 @@ cudaError_t launch_csa_compress(const void* xa, const void* za, const void* xb, 
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
                                 int in_dt, int out_dt, void* out, int norm, const float* gamma, float eps,
-                                const void* k_tok, int k_dt, int Di, uint8_t* k_codes, float* k_scale, int* st,
-                                cudaStream_t stream);
+                                const void* k_tok, int k_dt, int Di, uint8_t* k_codes, float* k_scale, int flags,
+                                int* st, cudaStream_t stream);
 cudaError_t launch_hca_compress(const void* x, const void* z, const float* bias, const int64_t* tok_off,
                                 const int64_t* tok0, int batch, const int64_t* ent_off,
                                 const int64_t* first, const int64_t* num, int64_t max_blocks,
@@ -123,6 +123,7 @@ struct AttnParams {
   int batch, T, H;
   int rows_per_split;
   int max_splits;
+  int cluster;  // tensor-core kernel: the splits of a query form a cluster of this size (0: merge kernel)
   float* part_acc;
   float* part_ml;
   float* out;
@@ -132,6 +133,7 @@ struct AttnParams {
 cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t stream);
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream);
 int attn_tc_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms);
+int attn_tc_cluster_fit(int want);
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
 int attn_rows_per_split(int mode, int T, int k, int window, int64_t max_entries, int sms);
 int attn_max_splits(int mode, int k, int window, int64_t max_entries, int R);

@@ -8,11 +8,13 @@ as cited in the C header):
              -> lindex_score_topk -> hybrid_decode_attn(CSA)
   HCA layer: hca_compress -> hybrid_decode_attn(HCA)
 
-The HCA layer does not depend on the CSA layer, so with ``two_streams`` it
-runs on a side stream that forks from and joins the caller's stream; the
-CSA compression runs on a second side stream beside the indexer (which reads
-the entry keys, not the compressed cache), and the CSA attention waits for
-both.  The whole step can be captured into a CUDA graph and replayed.
+Inside the CSA layer the indexer reads the entry keys, not the compressed
+cache, so it is issued first and the compression of the newest entries runs
+beside it as a dependent launch (CSKV_OVERLAP_PREVIOUS); the attention waits
+for both.  The HCA layer does not depend on the CSA layer, so with
+``two_streams`` it runs on a side stream that forks from and joins the
+caller's stream.  The whole step can be captured into a CUDA graph and
+replayed.
 
 Tensor names (all device tensors, int64 offsets unless noted):
   CSA rows  x_a z_a x_b z_b [rows, 256], csa_x_off [B+1], csa_t0 [B],
@@ -56,8 +58,6 @@ class DecodeStep:
         self.ws_h = api.attn_workspace(api.HCA, T, H, 0, self.W, self.max_hca_visible, dev)
         self.two_streams = two_streams
         self.side = torch.cuda.Stream(device=dev) if two_streams else None
-        self.side_c = torch.cuda.Stream(device=dev) if two_streams else None
-        self.ev_c = torch.cuda.Event() if two_streams else None
         self.graph = None
 
     # ------------------------------------------------------------------
@@ -73,16 +73,19 @@ class DecodeStep:
                          max_blocks=max_hca_entries, bias=t.get("bias_h"), tok0=t["hca_t0"],
                          dev_status=self.status, stream=stream)
 
-    def csa_compress(self, stream=None):
+    def csa_compress(self, stream=None, after_select=False):
         """The CSA entries the new tokens complete; with per-token indexer keys (k_tok) the
-        same kernel also pools those entries' indexer keys into k_idx / k_scale."""
+        same kernel also pools those entries' indexer keys into k_idx / k_scale.
+        after_select: issued right after csa_select on the same stream, which writes none of its
+        inputs and reads none of its outputs (no key pooling): it then runs beside the indexer."""
         t = self.t
         pool = t.get("k_tok") is not None
         api.csa_compress(t["x_a"], t["z_a"], t["x_b"], t["z_b"], t["csa_x_off"], t["csa_off"], t["cmp_c"],
                          max_blocks=self.max_csa_blocks, bias_a=t.get("bias_a"), bias_b=t.get("bias_b"),
                          tok0=t["csa_t0"], first_block=t["csa_first"], num_blocks=t["csa_num"],
                          k_tok=t["k_tok"] if pool else None, k_codes=t["k_idx"] if pool else None,
-                         k_scale=t["k_scale"] if pool else None, dev_status=self.status, stream=stream)
+                         k_scale=t["k_scale"] if pool else None, overlap_previous=after_select and not pool,
+                         dev_status=self.status, stream=stream)
 
     def csa_select(self, stream=None):
         t = self.t
@@ -99,8 +102,17 @@ class DecodeStep:
                                stream=stream)
 
     def csa_layer(self, stream=None):
-        self.csa_compress(stream)
-        self.csa_select(stream)
+        """Compression, indexer and attention of the CSA layer on one stream.  The indexer reads
+        the entry keys, not the compressed cache, so it goes first and the compression of the
+        newest entries runs beside it (a dependent launch that waits for the indexer only at its
+        end); the attention waits for both.  With per-token keys (k_tok) the compression pools
+        the keys the indexer reads, so it goes first."""
+        if self.t.get("k_tok") is not None:
+            self.csa_compress(stream)
+            self.csa_select(stream)
+        else:
+            self.csa_select(stream)
+            self.csa_compress(stream, after_select=True)
         self.csa_attend(stream)
 
     def hca_layer(self, stream=None):
@@ -121,23 +133,13 @@ class DecodeStep:
             self.csa_layer(main)
             self.hca_layer(main)
             return
-        # The HCA layer runs beside the CSA layer, which it does not depend on.  Inside the CSA
-        # layer the indexer reads the entry keys, not the compressed cache, so it starts at
-        # once on the main stream while the compression of the newest entries runs on a
-        # second side stream; the CSA attention (a dependent launch of the indexer) also waits
-        # for that compression.
+        # The HCA layer runs on a side stream beside the CSA layer, which it does not depend on.
+        # The CSA layer is issued first, so that in a captured graph the indexer (the longest
+        # kernel) is the first node to launch; its kernels chain by dependent launches alone.
         self.side.wait_stream(main)
-        self.side_c.wait_stream(main)
+        self.csa_layer(main)
         self.hca_layer(self.side)
-        self.csa_compress(self.side_c)
-        self.ev_c.record(self.side_c)
-        if self.t.get("k_tok") is not None:
-            main.wait_event(self.ev_c)  # the indexer reads the keys the compression pools
-        self.csa_select(main)
-        main.wait_event(self.ev_c)
-        self.csa_attend(main)
         main.wait_stream(self.side)
-        main.wait_stream(self.side_c)
 
     # ------------------------------------------------------------------
     def capture(self):

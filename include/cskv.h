@@ -113,10 +113,22 @@ CSKV_API unsigned long long cskv_launch_count(void);
  *                      aligned), Di 64 or 128; entry i of sequence b writes
  *                      k_codes[ent_off[b] + i, :] (E4M3, 16-byte aligned) and
  *                      k_scale[ent_off[b] + i] (fp32).
+ * flags              : 0, or CSKV_OVERLAP_PREVIOUS: the caller guarantees that the
+ *                      kernel issued just before this call on `stream` neither
+ *                      writes any of its inputs nor reads its outputs, and that
+ *                      every kernel before that one has completed by the time that
+ *                      one starts its dependents (true right after lindex_score_topk,
+ *                      which starts them only after its own wait).  The entries are
+ *                      then computed while that kernel still runs (in a decode
+ *                      step: beside the indexer), and this call still completes
+ *                      after it, so a later kernel that waits for this call sees
+ *                      both.  A permission, not a request: the many-entry kernel
+ *                      ignores it.  Other bits: CSKV_ERR_INVALID_ARG.
  * Many entries (max_blocks >= 512) run a TMA-ring kernel, one CTA per SM; a few
  * (a decode step) run a warp per entry.  Both give the same results up to fp32
  * rounding order.
  * ------------------------------------------------------------------------ */
+#define CSKV_OVERLAP_PREVIOUS 1
 CSKV_API int csa_compress(const void* x_a, const void* z_a, const void* x_b, const void* z_b,
                  const float* bias_a, const float* bias_b,
                  const int64_t* tok_off, const int64_t* tok0, int batch,
@@ -124,7 +136,7 @@ CSKV_API int csa_compress(const void* x_a, const void* z_a, const void* x_b, con
                  int64_t max_blocks, int in_dtype, int out_dtype, void* out,
                  int rmsnorm, const float* norm_gamma, float norm_eps,
                  const void* k_tok, int k_dtype, int Di, uint8_t* k_codes, float* k_scale,
-                 int* dev_status, cskv_stream_t stream);
+                 int flags, int* dev_status, cskv_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * hca_compress -- HCA compression, 128 tokens -> 1 entry, one stream.

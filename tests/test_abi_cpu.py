@@ -58,9 +58,9 @@ def test_compress_validation(lib):
     nul = None
 
     def csa(x=_p(), z=_p(), xb=nul, zb=nul, out=_p(), in_dt=1, out_dt=1, max_blocks=4, norm=0, gamma=nul, eps=1e-6,
-            k_tok=nul, k_dt=1, Di=64, codes=_p(), scale=_p()):
+            k_tok=nul, k_dt=1, Di=64, codes=_p(), scale=_p(), flags=0):
         return lib.csa_compress(x, z, xb, zb, nul, nul, _p(), nul, 1, _p(), nul, nul, max_blocks, in_dt, out_dt, out,
-                                norm, gamma, eps, k_tok, k_dt, Di, codes, scale, nul, nul)
+                                norm, gamma, eps, k_tok, k_dt, Di, codes, scale, flags, nul, nul)
 
     def hca(batch=1, in_dt=1, max_blocks=4, norm=0, gamma=nul, eps=1e-6):
         return lib.hca_compress(_p(), _p(), nul, _p(), nul, batch, _p(), nul, nul, max_blocks, in_dt, 1, _p(), norm,
@@ -69,6 +69,8 @@ def test_compress_validation(lib):
     assert csa(x=nul) == _lib.ERR_INVALID_ARG               # null rows
     assert csa(xb=_p()) == _lib.ERR_INVALID_ARG             # x_b without z_b
     assert csa(out=_p(0x1004)) == _lib.ERR_INVALID_ARG      # misaligned output
+    assert csa(flags=2) == _lib.ERR_INVALID_ARG             # unknown flag bit
+    assert csa(flags=1, max_blocks=0) == _lib.OK            # the overlap permission alone is valid
     assert hca(in_dt=2) == _lib.ERR_UNSUPPORTED             # fp8 rows are not a compression input
     assert hca(batch=0) == _lib.ERR_INVALID_ARG             # bad batch / bad enum
     assert hca(in_dt=7) == _lib.ERR_INVALID_ARG
