@@ -42,6 +42,7 @@ SIGNATURES = {
                                        _p, _p, _p, _i64, _p, _sz, _p, _p]),
     "lindex_topk_from_scores": (_i32, [_p, _i64, _p, _i32, _i32, _i64, _p, _p, _p, _sz, _p, _p]),
     "lindex_workspace_size": (_sz, [_i32, _i32, _i64]),
+    "lindex_workspace_size_scan": (_sz, [_i32, _i64]),
     "hybrid_decode_attn": (_i32, [_i32, _p, _p, _p, _p, _i32, _p, _p, _p, _i32, _p, _f, _p, _p, _i32, _i32,
                                   _i32, _i32, _i32, _i64, _p, _p, _p, _sz, _p, _p]),
     "hybrid_attn_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i64]),

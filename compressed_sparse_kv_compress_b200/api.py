@@ -96,9 +96,15 @@ def lindex_workspace_size(T: int, k: int, max_entries: int) -> int:
     return int(_lib.load().lindex_workspace_size(int(T), int(k), int(max_entries)))
 
 
-def lindex_workspace(T: int, k: int, max_entries: int, device="cuda") -> torch.Tensor:
-    """A zero-filled workspace; calls hand it back zero-filled."""
-    return torch.zeros(max(16, lindex_workspace_size(T, k, max_entries)), dtype=torch.uint8, device=device)
+def lindex_workspace_size_scan(T: int, max_entries: int) -> int:
+    return int(_lib.load().lindex_workspace_size_scan(int(T), int(max_entries)))
+
+
+def lindex_workspace(T: int, k: int, max_entries: int, device="cuda", scan_only=False) -> torch.Tensor:
+    """A zero-filled workspace; calls hand it back zero-filled.  scan_only: the per-query scan's
+    size (many-query calls then skip the tensor-core path)."""
+    n = lindex_workspace_size_scan(T, max_entries) if scan_only else lindex_workspace_size(T, k, max_entries)
+    return torch.zeros(max(16, n), dtype=torch.uint8, device=device)
 
 
 def lindex_score_topk(q_idx, k_idx, q_seq, q_pos, ent_off, out_idx, workspace, *, max_entries, q_scale=None,

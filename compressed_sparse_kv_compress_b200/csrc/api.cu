@@ -172,10 +172,25 @@ int rmsnorm_heads(const void* x, int dtype, int64_t rows, int d, const float* ga
   return launch_status(launch_rmsnorm_rows(x, dtype, rows, gamma, eps, out, (cudaStream_t)stream));
 }
 
-size_t lindex_workspace_size(int T, int k, int64_t max_entries) {
-  (void)k;
+// Workspace of the tensor-core path (many queries): the candidate lists, then the workspace of
+// the exact top-k over them.
+static size_t tc_area(size_t b) { return (b + 255) / 256 * 256; }
+static size_t lindex_tc_ws_bytes(int T, int k, int64_t max_entries) {
+  const int64_t cap = lindex_tc_cap(k, max_entries);
+  return tc_area((size_t)T * cap * sizeof(float)) + tc_area((size_t)T * cap * sizeof(int32_t)) +
+         tc_area((size_t)T * sizeof(int64_t)) + lindex_ws_bytes(T, cap);
+}
+
+size_t lindex_workspace_size_scan(int T, int64_t max_entries) {
   if (T < 1) return 0;
   return lindex_ws_bytes(T, max_entries);
+}
+
+size_t lindex_workspace_size(int T, int k, int64_t max_entries) {
+  if (T < 1) return 0;
+  size_t b = lindex_ws_bytes(T, max_entries);
+  if (T >= kLindexTcMinQueries && k >= 1) b = std::max(b, lindex_tc_ws_bytes(T, k, max_entries));
+  return b;
 }
 
 static int check_topk_common(int T, int k, int64_t max_entries, const int32_t* out_idx, const void* ws,
@@ -221,6 +236,38 @@ int lindex_score_topk(const void* q_idx, const float* q_scale, const void* k_idx
   p.pf_row_bytes = prefetch_rows ? prefetch_row_bytes : 0;
   p.ws = (QueryWS*)workspace;
   p.st = dev_status;
+  if (T >= kLindexTcMinQueries && lindex_tc_shape(dtype, Hi, Di) && ws_bytes >= lindex_tc_ws_bytes(T, k, max_entries)) {
+    // many queries: tensor-core scores -> candidate lists -> exact top-k over the lists ->
+    // candidate positions mapped back to entry indices
+    const int64_t cap = lindex_tc_cap(k, max_entries);
+    uint8_t* w = (uint8_t*)workspace;
+    float* cand_score = (float*)w;
+    w += tc_area((size_t)T * cap * sizeof(float));
+    int32_t* cand_idx = (int32_t*)w;
+    w += tc_area((size_t)T * cap * sizeof(int32_t));
+    int64_t* cand_n = (int64_t*)w;
+    w += tc_area((size_t)T * sizeof(int64_t));
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = launch_lindex_tc_candidates(p.q_idx, q_scale, p.k_idx, k_scale, head_w, q_seq, q_pos, ent_off,
+                                                batch, T, Hi, Di, k, cap, cand_score, cand_idx, cand_n, dev_status, s);
+    if (e != cudaSuccess) return launch_status(e);
+    IdxParams ps = {};
+    ps.scores = cand_score;
+    ps.ld_scores = cap;
+    ps.n_valid = cand_n;
+    ps.Hi = 1;
+    ps.Di = 64;
+    ps.k = k;
+    ps.max_entries = cap;
+    ps.out_idx = out_idx;
+    ps.out_score = out_score;
+    ps.ws = (QueryWS*)w;
+    ps.st = dev_status;
+    e = launch_lindex(ps, CSKV_F32, T, s);
+    if (e != cudaSuccess) return launch_status(e);
+    return launch_status(launch_map_candidates(out_idx, cand_idx, cap, T, k, ent_off, q_seq, p.pf_rows,
+                                               p.pf_row_bytes, s));
+  }
   return launch_status(launch_lindex(p, dtype, T, (cudaStream_t)stream));
 }
 

@@ -103,6 +103,18 @@ cudaError_t launch_lindex(const IdxParams& p, int dtype, int T, cudaStream_t str
 size_t lindex_ws_bytes(int T, int64_t max_entries);
 bool lindex_shape_supported(int dtype, int Hi, int Di);
 bool lindex_capacity_ok(int64_t max_entries, int T);
+// indexer_tc.cu: many queries (a prefill chunk) on the tensor cores -> per-query candidate lists
+constexpr int kLindexTcMinQueries = 256;
+bool lindex_tc_shape(int dtype, int Hi, int Di);
+int64_t lindex_tc_cap(int k, int64_t max_entries);
+cudaError_t launch_lindex_tc_candidates(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                        const float* k_scale, const float* head_w, const int32_t* q_seq,
+                                        const int64_t* q_pos, const int64_t* ent_off, int batch, int T, int Hi,
+                                        int Di, int k, int64_t cap, float* cand_score, int32_t* cand_idx,
+                                        int64_t* cand_n, int* st, cudaStream_t stream);
+cudaError_t launch_map_candidates(int32_t* out_idx, const int32_t* cand_idx, int64_t cap, int T, int k,
+                                  const int64_t* ent_off, const int32_t* q_seq, const uint8_t* pf_rows,
+                                  int64_t pf_row_bytes, cudaStream_t stream);
 
 // attention.cu
 struct AttnParams {

@@ -1,7 +1,7 @@
 // Thin inline-PTX wrappers for sm_100a features used by the cskv kernels:
 // mbarriers with bounded waits, TMA bulk copies (global -> shared, no multicast),
 // the fp8 (E4M3) warp-level MMA used by the indexer scan, tcgen05 / TMEM, and the
-// cluster barrier and distributed shared memory (DSMEM) loads.
+// thread-block cluster barrier.
 #pragma once
 
 #include <stdint.h>
@@ -206,6 +206,13 @@ __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src, unsi
                : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Groups of cp.async copies: close the group of the copies issued since the last commit; wait
+// until at most N groups are still in flight.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // ---------------------------------------------------------------- thread-block clusters
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -218,26 +225,6 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Address, in the cluster's shared window, of this CTA's shared location `local` in CTA `rank`.
-__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float2 dsmem_ld2(uint32_t a) {
-  float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a) : "memory");
-  return v;
-}
-__device__ __forceinline__ float4 dsmem_ld4(uint32_t a) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(a)
-               : "memory");
-  return v;
-}
-
 // 2^x with the hardware approximation (relative error ~2^-22; flushes subnormal results to 0).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

@@ -275,7 +275,17 @@ CSKV_API int lindex_topk_from_scores(const float* scores, int64_t ld_scores, con
                             int T, int k, int64_t max_entries, int32_t* out_idx, float* out_score,
                             void* workspace, size_t ws_bytes, int* dev_status, cskv_stream_t stream);
 
+/* Workspace bytes of lindex_score_topk / lindex_topk_from_scores for T queries.
+ * Many queries (T >= 256) of E4M3 vectors with Hi in {8, 16} and Di in {64, 128} (a
+ * prefill chunk) run on the tensor cores: tcgen05 kind::f8f6f4 products of 16 (or 8)
+ * queries' heads with 128-entry key tiles, two passes (a per-query histogram of the
+ * scores, then every entry that can be among the k best appended to the query's
+ * candidate list in index order), and the exact top-k over the lists.  That path needs
+ * lindex_workspace_size bytes (about T * 8 * max(8192, 2k) for the lists); with less,
+ * but at least lindex_workspace_size_scan(T, max_entries), such calls take the
+ * per-query scan instead.  Both give the same selection up to fp32 rounding order. */
 CSKV_API size_t lindex_workspace_size(int T, int k, int64_t max_entries);
+CSKV_API size_t lindex_workspace_size_scan(int T, int64_t max_entries);
 
 /* ------------------------------------------------------------------------
  * hybrid_decode_attn -- MQA attention over compressed entries + raw window + sink.

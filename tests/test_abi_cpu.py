@@ -192,3 +192,15 @@ def test_pool_keys_validation(lib):
     assert call(a5=0) == _lib.ERR_INVALID_ARG                # empty batch
     assert call(a9=-1) == _lib.ERR_INVALID_ARG
     assert call(a9=0) == _lib.OK                             # nothing to do, nothing launched
+
+
+def test_indexer_workspace_sizes(lib):
+    # many queries: the tensor-core path's candidate lists on top of the scan's workspace;
+    # few queries: the scan's alone
+    scan = lib.lindex_workspace_size_scan(4096, 33792)  # (0 without a GPU: sized from the device)
+    full = lib.lindex_workspace_size(4096, 1024, 33792)
+    assert 0 <= scan < full
+    assert full >= 4096 * 8192 * 8  # two [T, cap] lists, cap = max(8192, 2k) capped by the entries
+    assert lib.lindex_workspace_size(255, 1024, 33792) == lib.lindex_workspace_size_scan(255, 33792)
+    # a short cache caps the lists at its entry count
+    assert lib.lindex_workspace_size(300, 1024, 2000) < lib.lindex_workspace_size(300, 1024, 20000)
