@@ -572,6 +572,29 @@ def run_cskv(args, ws, rank, local):
         "gpu_launches": int(launches_per_step) * args.steps,
         "clocks": clk,
     }
+    if T >= 256 and spec.idx_dtype == "fp8" and m["Hi"] in (8, 16) and m["di"] in (64, 128):
+        # many queries: the indexer runs on the tensor cores (E4M3 products, two passes over the
+        # keys); its work against the E4M3 tensor peak (2 x the measured sustained bf16 peak) and
+        # against the FP32 pipe (the epilogue's ReLU + weighted head sum: 2 ops per (query,
+        # head, entry) and pass)
+        tf_bf16 = 1375.3
+        try:
+            with open(PEAKS_FILE) as f:
+                tf_bf16 = float(json.load(f)["bf16_tflops_sustained"])
+        except Exception:
+            pass
+        qhe = sum(m["Hi"] * ((p + 1) // 4) for p in m["q_pos"])  # (query, head, visible entry)
+        flops = 2.0 * m["di"] * qhe
+        sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        alu_peak = sm * 128 * 1.965e9  # FP32 lanes x the part's maximum SM clock: ops/s
+        t_s = idx_us * 1e-6
+        line["prefill_indexer_roofline"] = {
+            "bound": "alu", "kernel": "lindex_tc_kernel + exact top-k over the candidate lists",
+            "us_per_call": idx_us, "tensor_tflops": flops / t_s / 1e12, "tensor_peak_tflops": 2 * tf_bf16,
+            "tensor_frac": flops / t_s / 1e12 / (2 * tf_bf16),
+            "alu_ops_per_s": 2 * 2 * qhe / t_s, "alu_peak_ops_per_s": alu_peak,
+            "alu_frac": 2 * 2 * qhe / t_s / alu_peak,
+            "note": "tensor peak: E4M3 = 2 x measured sustained bf16; alu: FP32 pipe at 1965 MHz"}
     if rank == 0 and ws == 1 and not args.no_bulk:
         line["bulk_compress"] = bulk_compress_rate()
         line["bulk_compress"]["combined_with_one_step"] = combined_rate(line["bulk_compress"], by["total"], ms, hbm)

@@ -121,9 +121,14 @@ def test_ragged_b64_full_sampled():
 
 
 def test_prefill_chunk_full_sampled():
+    # 4096 queries: the indexer takes its tensor-core path (16-query tiles) and the attention its
+    # many-query plan; the first and last query of every 128-query block, and a few between
     w = Workload(spec_by_name("prefill_4k_at_128k"))
     step, dev = _run_gpu(w)
-    _check(w, step, dev, [0, 1, 2, 3, 1001, 2048, 4094, 4095])
+    T = w.meta["T"]
+    queries = sorted({q for b in range(0, T, 128) for q in (b, b + 127)} | {1, 2, 3, 15, 16, 1001, 2048, 4094})
+    assert len(queries) >= 64
+    _check(w, step, dev, queries)
 
 
 def _issue_layers(step, order):
