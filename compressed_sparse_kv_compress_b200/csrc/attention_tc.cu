@@ -24,8 +24,9 @@
 // Merging the splits of a query ([TR] §3.1; the sink joins once, [SW] §十二):
 //  * cluster mode (p.cluster = the split count, at most 16): the query's splits are the CTAs
 //    of one thread-block cluster.  Each writes its partial (unnormalised O rows, (m, l)) to
-//    the workspace, a cluster barrier publishes them, and each CTA merges 128 / p.cluster of
-//    the heads from L2 -- no second kernel and no launch gap.  (Reading the partials from the
+//    the workspace, a cluster barrier publishes them, and each CTA fetches its heads' slices
+//    of every split with TMA bulk copies and merges 128 / p.cluster of the heads -- no second
+//    kernel and no launch gap.  (Reading the partials from the
 //    other CTAs' shared memory instead was slower: every remote load a round trip over the
 //    SM-to-SM network.)
 //  * otherwise the split's (m, l, O) go to the workspace and attn_combine_kernel merges.
@@ -56,40 +57,44 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 
 // Cluster mode: merges the query's splits (the CTAs of this cluster, rank = split) once every
-// split has written its partial to the workspace -- the unnormalised O as float4 groups of
-// dimensions, [split][group 0..31][h] (a warp's write of one group is 512 contiguous bytes),
-// and (m, l) per head -- and writes the output and lse.  Called by all threads of every CTA of
-// the cluster.  The cluster barrier (release / acquire at cluster scope) makes the partials of
-// all splits visible; they stay in L2.  CTA r then merges heads r * 128 / CS ..
-// (r + 1) * 128 / CS - 1 (HPC heads): thread (g, hh) = (tid / HPC, tid % HPC) takes head
-// r * HPC + hh and the dimension groups g, g + CS, ..., so a warp's loads are runs of HPC
-// consecutive heads.  For its head a thread folds every split's (m, l) with the sink,
+// split has written its partial to the workspace, and writes the output and lse.  Called by
+// all threads of every CTA of the cluster.  Partial layout, per (query, split): the
+// unnormalised O as float4 groups of 4 dimensions, grouped by merging CTA -- CTA r merges the
+// heads r HPC .. r HPC + nh_r - 1 (HPC = 128 / CS, nh_r = min(HPC, H - r HPC)), and its slice
+// [group 0..31][head] of nh_r * 512 contiguous bytes sits at offset r HPC * 512 -- and (m, l)
+// per head.  After the cluster barrier (release / acquire at cluster scope; the writers'
+// proxy fence lets the TMA see their stores) one thread fetches the CS slices of its heads
+// with TMA bulk copies into the dead K||V tile (all in flight at once: one round trip), the
+// threads load their heads' (m, l) meanwhile, and each thread (head hh, groups g0, g0 + CS,
+// ...) folds every split's (m, l) with the sink,
 //   M = max(max_s m_s, sink),  L = sum_s 2^(m_s - M) l_s + 2^(sink - M),
-// and sums the splits' values scaled by 2^(m_s - M) / L.  A thread's loads go in two rounds:
-// the CS (m, l) pairs with the first 16 groups of values, then the other 16 (all 32 at once
-// would take the kernel past 250 registers, and then it no longer fits on an SM beside the
-// kernels that share one during a decode step).
+// and sums the splits' values, scaled by 2^(m_s - M) / L, from shared memory.
 template <int CS>
-__device__ __forceinline__ void cluster_merge(const AttnParams& p, int t) {
+__device__ __forceinline__ void cluster_merge(const AttnParams& p, int t, float4* stage, uint64_t* bar_m) {
   cluster_sync();
+  fence_proxy_async_global();
   const int tid = threadIdx.x, H = p.H;
   const uint32_t rank = cluster_rank();
-  constexpr int HPC = 128 / CS;  // heads merged by this CTA
-  constexpr int NG = 32 / CS;    // dimension groups per thread: NG x CS = 32 loads
-  constexpr int NG1 = NG / 2;    // groups of the first round (the second round: the rest)
-  const int h = (int)rank * HPC + tid % HPC, g0 = tid / HPC;
-  if (h >= H) return;  // no barrier follows: a thread without a head is done
-  const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)t * CS * H + h;
-  const float4* po = reinterpret_cast<const float4*>(p.part_acc) + (size_t)t * CS * 32 * H + h;
+  constexpr int HPC = 128 / CS;  // heads merged by a CTA
+  constexpr int NG = 32 / CS;    // dimension groups per thread
+  const int h0 = (int)rank * HPC;
+  const int nh = max(0, min(HPC, H - h0));
+  if (nh == 0) return;  // no barrier follows: a CTA without heads is done
+  const float4* po = reinterpret_cast<const float4*>(p.part_acc) + (size_t)t * CS * H * 32 + (size_t)h0 * 32;
+  const uint32_t slice = (uint32_t)nh * 512u;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_m, CS * slice);
+#pragma unroll
+    for (int s = 0; s < CS; ++s) tma_bulk_g2s(stage + (size_t)s * nh * 32, po + (size_t)s * H * 32, slice, bar_m);
+  }
+  const int hh = tid % HPC, g0 = tid / HPC;
+  const int h = h0 + hh;
+  const bool mine = hh < nh;
   float2 mls[CS];
-  float4 v[NG1][CS];
+  const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)t * CS * H + (mine ? h : h0);
 #pragma unroll
   for (int s = 0; s < CS; ++s) mls[s] = __ldcg(ml + (size_t)s * H);
-#pragma unroll
-  for (int k = 0; k < NG1; ++k)
-#pragma unroll
-    for (int s = 0; s < CS; ++s) v[k][s] = __ldcg(po + ((size_t)s * 32 + g0 + CS * k) * H);
-  const float sk = p.sink ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+  const float sk = (p.sink && mine) ? __ldg(p.sink + h) * kLog2e : -INFINITY;
   float M = sk;
 #pragma unroll
   for (int s = 0; s < CS; ++s) M = fmaxf(M, mls[s].x);
@@ -101,37 +106,33 @@ __device__ __forceinline__ void cluster_merge(const AttnParams& p, int t) {
   }
   if (M != -INFINITY && p.sink) L += exp2f(sk - M);
   const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (!mbar_wait_bounded(bar_m, 0)) flag(p.st, CSKV_DEV_TIMEOUT);
+  if (!mine) return;
   float* dst = p.out + ((size_t)t * H + h) * kHeadDim;
 #pragma unroll
-  for (int round = 0; round < 2; ++round) {
-    if (round == 1) {
+  for (int k = 0; k < NG; ++k) {
+    const int g = g0 + CS * k;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int k = 0; k < NG1; ++k)
-#pragma unroll
-        for (int s = 0; s < CS; ++s) v[k][s] = __ldcg(po + ((size_t)s * 32 + g0 + CS * (NG1 + k)) * H);
-    }
-#pragma unroll
-    for (int k = 0; k < NG1; ++k) {
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int s = 0; s < CS; ++s)
-        if (f[s] != 0.f) {
-          a.x = fmaf(v[k][s].x, f[s], a.x);
-          a.y = fmaf(v[k][s].y, f[s], a.y);
-          a.z = fmaf(v[k][s].z, f[s], a.z);
-          a.w = fmaf(v[k][s].w, f[s], a.w);
-        }
-      const int grp = g0 + CS * (round * NG1 + k);
-      dst[4 * grp] = a.x * inv;
-      dst[4 * grp + 1] = a.y * inv;
-      dst[4 * grp + 2] = a.z * inv;
-      dst[4 * grp + 3] = a.w * inv;
-    }
+    for (int s = 0; s < CS; ++s)
+      if (f[s] != 0.f) {
+        const float4 v = stage[(size_t)s * nh * 32 + g * nh + hh];
+        a.x = fmaf(v.x, f[s], a.x);
+        a.y = fmaf(v.y, f[s], a.y);
+        a.z = fmaf(v.z, f[s], a.z);
+        a.w = fmaf(v.w, f[s], a.w);
+      }
+    dst[4 * g] = a.x * inv;
+    dst[4 * g + 1] = a.y * inv;
+    dst[4 * g + 2] = a.z * inv;
+    dst[4 * g + 3] = a.w * inv;
   }
   if (g0 == 0 && p.lse) p.lse[(size_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
+// At most 160 registers a thread: 4 warps x 32 x 160 = 20,480, what an SM has left beside the
+// indexer (16 warps x 32 x 88), so the HCA attention and a parked CSA attention fit beside it.
+__global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smraw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~(uintptr_t)1023);
   uint8_t* Qs = sm;                   // A of S = Q K^T   [128 heads x 128 d], K-major
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
                                       // V: B of O = P V [128 rows (K) x 128 d (N)], MN-major (2-3)
   uint8_t* Ps = KVs;                  // A of O = P V     [128 heads x 128 rows], K-major: K's regions,
                                       // written only after the S MMA has read K (bar_s)
-  __shared__ uint64_t bar_s, bar_o;
+  __shared__ uint64_t bar_s, bar_o, bar_m;
   __shared__ uint32_t tmem_base;
   __shared__ const __nv_bfloat16* row_src[kTcChunk];  // address of each chunk row, null = skipped
   __shared__ uint32_t row_mask[kTcChunk / 32];  // bit r: chunk row r is attended
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
   if (tid == 0) {
     mbar_init(&bar_s, 1);
     mbar_init(&bar_o, 1);
+    mbar_init(&bar_m, 1);
     fence_mbar_init();
   }
   // warm L2 with the query's metadata and the selected indices of this split's first rows
@@ -324,11 +326,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
     tc_fence_after();
   }
   if (p.cluster) {
-    // ---- partial of this split (float4 groups of dimensions, head-minor), then the merge
+    // ---- partial of this split (float4 groups of dimensions, sliced by merging CTA), then the
+    //      merge.  Head tid's group j: slice r = tid / HPC (nh_r heads) at r HPC * 32 + j nh_r + hh.
     const size_t sb = (size_t)t * p.max_splits + split;
     if (c > 0) {
+      const int hpc = 128 / p.cluster;
+      const int r = tid / hpc, hh = tid % hpc;
+      const int nh = min(hpc, H - r * hpc);
       const uint32_t tO = tmem_base + 128;
-      float4* og = reinterpret_cast<float4*>(p.part_acc) + sb * 32 * H + tid;  // group j at og[j * H]
+      float4* og = reinterpret_cast<float4*>(p.part_acc) + sb * 32 * H + (size_t)r * hpc * 32 + hh;
       for (int cc = 0; cc < 128; cc += 32) {
         uint32_t v[32];
         tmem_ld32(tO + lane_base + cc, v);
@@ -336,19 +342,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnParams p) {
         if (tid < H) {
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            og[(size_t)((cc >> 2) + i) * H] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                          __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            og[(size_t)((cc >> 2) + i) * nh] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                           __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
         }
       }
     }
     if (tid < H)
       reinterpret_cast<float2*>(p.part_ml)[sb * H + tid] = c > 0 ? make_float2(m_run, l_run) : make_float2(-INFINITY, 0.f);
+    fence_proxy_async_global();  // the other CTAs' TMA reads these stores after the cluster barrier
+    float4* stage = reinterpret_cast<float4*>(KVs);  // the dead K||V tile: 64 KiB
     switch (p.cluster) {
-      case 1: cluster_merge<1>(p, t); break;
-      case 2: cluster_merge<2>(p, t); break;
-      case 4: cluster_merge<4>(p, t); break;
-      case 8: cluster_merge<8>(p, t); break;
-      default: cluster_merge<16>(p, t); break;
+      case 1: cluster_merge<1>(p, t, stage, &bar_m); break;
+      case 2: cluster_merge<2>(p, t, stage, &bar_m); break;
+      case 4: cluster_merge<4>(p, t, stage, &bar_m); break;
+      case 8: cluster_merge<8>(p, t, stage, &bar_m); break;
+      default: cluster_merge<16>(p, t, stage, &bar_m); break;
     }
   } else if (c > 0) {
     // ---- partial of this split: O row (unnormalised, relative to m_run), m_run, l_run.
