@@ -369,7 +369,10 @@ def run_cskv(args, ws, rank, local):
               max_hca_visible=max((p + 1) // 128 for p in m["q_pos"]))
     steps = []
     for dev in devs:
-        st = DecodeStep(dev, k=m["k"], window=m["W"], scale=m["scale"], two_streams=not args.one_stream, **bd)
+        # a prefill chunk's queries are one sequence's consecutive positions (an even count per
+        # sequence): the HCA attention takes them in pairs
+        st = DecodeStep(dev, k=m["k"], window=m["W"], scale=m["scale"], two_streams=not args.one_stream,
+                        adjacent_pairs=m["Q"] >= 2 and m["Q"] % 2 == 0, **bd)
         if spec.cache == "compress":
             st.bulk_compress(max(m["ncsa"]), max(m["nhca"]))
         torch.cuda.synchronize()

@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libcskv.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_LAUNCH = 0, 1, 2, 3, 4
 F32, BF16, FP8E4M3 = 0, 1, 2
 OVERLAP_PREVIOUS = 1  # csa_compress flags (CSKV_OVERLAP_PREVIOUS)
+ATTN_PAIRS = 0x100  # OR-ed into hybrid_decode_attn's mode (CSKV_ATTN_PAIRS)
 CSA, HCA = 0, 1
 DEV_BAD_INDEX, DEV_TAIL_MISSING, DEV_CAPACITY, DEV_TIMEOUT = 1, 2, 4, 8
 NOALLOC_SCRATCH_BYTES = 16 << 20

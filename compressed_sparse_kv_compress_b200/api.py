@@ -12,7 +12,7 @@ import math
 import torch
 
 from . import _lib
-from ._lib import BF16, CSA, F32, FP8E4M3, HCA, OVERLAP_PREVIOUS  # noqa: F401
+from ._lib import ATTN_PAIRS, BF16, CSA, F32, FP8E4M3, HCA, OVERLAP_PREVIOUS  # noqa: F401
 
 _DT = {torch.float32: F32, torch.bfloat16: BF16, torch.uint8: FP8E4M3, torch.float8_e4m3fn: FP8E4M3}
 
@@ -164,9 +164,13 @@ def attn_workspace(mode, T, H, k, window, max_entries, device="cuda") -> torch.T
 
 
 def hybrid_decode_attn(mode, q, kv_cmp, cmp_off, kv_raw, raw_off, q_seq, q_pos, out, workspace, *, window,
-                       idx=None, raw_tok0=None, sink=None, scale=None, lse=None, max_entries=0, dev_status=None,
-                       stream=None):
+                       idx=None, raw_tok0=None, sink=None, scale=None, lse=None, max_entries=0, adjacent_pairs=False,
+                       dev_status=None, stream=None):
+    """adjacent_pairs: CSKV_ATTN_PAIRS (queries 2j, 2j + 1 are one sequence's consecutive
+    positions; see the C header)."""
     T, H, d = q.shape
+    if adjacent_pairs:
+        mode = int(mode) | ATTN_PAIRS
     k = idx.shape[1] if idx is not None else 0
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lib = _lib.load()

@@ -367,13 +367,25 @@ static int attn_plan(int mode, int T, int k, int window, int64_t max_entries, bo
   return CSKV_OK;
 }
 
+// Adjacent-query pairs (CSKV_ATTN_PAIRS) for the tensor-core HCA kernel: H == 64 heads, so a
+// pair's two queries fill the 128 rows of the tile.
+constexpr int kPairHeads = 64;
+
 size_t hybrid_attn_workspace_size(int mode, int T, int H, int d, int k, int window, int64_t max_entries) {
+  mode &= ~CSKV_ATTN_PAIRS;
   if (T < 1 || H < 1 || d != kHeadDim || window < 0) return 0;
   size_t best = 0;
   for (int tc = 0; tc < 2; ++tc) {
     AttnPlan pl;
     if (attn_plan(mode, T, k, window, max_entries, tc != 0, &pl)) return 0;
     const size_t need = (size_t)T * pl.ws_splits * H * (kHeadDim + 2) * sizeof(float);
+    if (need > best) best = need;
+  }
+  if (mode == CSKV_HCA && H == kPairHeads && T >= 2) {  // the pair plan: (T + 1) / 2 units of 2H heads
+    AttnPlan pl;
+    const int Tp = (T + 1) / 2;
+    if (attn_plan(mode, Tp, 0, window + 1, max_entries, true, &pl)) return 0;
+    const size_t need = (size_t)Tp * pl.ws_splits * 2 * H * (kHeadDim + 2) * sizeof(float);
     if (need > best) best = need;
   }
   return best;
@@ -387,7 +399,8 @@ int cskv::check_attn_args(int mode, const void* q, const void* kv_cmp, const int
                           int k, const void* kv_raw, const int64_t* raw_off, int window, float scale,
                           const int32_t* q_seq, const int64_t* q_pos, int batch, int T, int H, int d, int dtype,
                           int64_t max_entries, const float* out) {
-  if (mode != CSKV_CSA && mode != CSKV_HCA) return CSKV_ERR_INVALID_ARG;
+  if ((mode & ~CSKV_ATTN_PAIRS) != CSKV_CSA && (mode & ~CSKV_ATTN_PAIRS) != CSKV_HCA) return CSKV_ERR_INVALID_ARG;
+  mode &= ~CSKV_ATTN_PAIRS;
   if (dtype != CSKV_F32 && dtype != CSKV_BF16) return dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
   if (d != kHeadDim) return CSKV_ERR_UNSUPPORTED;
   if (H < 1 || H > 128 || T < 0 || window < 0 || window > (1 << 20) || batch < 1) return CSKV_ERR_INVALID_ARG;
@@ -412,11 +425,26 @@ int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_
   int arc = check_attn_args(mode, q, kv_cmp, cmp_off, idx, k, kv_raw, raw_off, window, scale, q_seq, q_pos, batch,
                             T, H, d, dtype, max_entries, out);
   if (arc != CSKV_OK || T == 0) return arc;
+  const bool want_pairs = (mode & CSKV_ATTN_PAIRS) != 0;
+  mode &= ~CSKV_ATTN_PAIRS;
   const bool tc = dtype == CSKV_BF16;
   AttnPlan pl;
   int rc = attn_plan(mode, T, mode == CSKV_CSA ? k : 0, window, max_entries, tc, &pl);
   if (rc) return rc;
-  const size_t need = (size_t)T * pl.ws_splits * H * (kHeadDim + 2) * sizeof(float);
+  // adjacent-query pairs: the HCA tensor-core kernel with 64 heads, when the pairs' plan merges
+  // inside a cluster (a unit of two queries is one 128-head "query" of the plan)
+  int units = T, Hv = H;
+  if (want_pairs && tc && mode == CSKV_HCA && H == kPairHeads && T >= 2) {
+    AttnPlan pp;
+    rc = attn_plan(mode, (T + 1) / 2, 0, window + 1, max_entries, tc, &pp);
+    if (rc) return rc;
+    if (pp.cluster) {
+      pl = pp;
+      units = (T + 1) / 2;
+      Hv = 2 * H;
+    }
+  }
+  const size_t need = (size_t)units * pl.ws_splits * Hv * (kHeadDim + 2) * sizeof(float);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return CSKV_ERR_WORKSPACE;
   AttnParams p = {};
   p.mode = mode;
@@ -439,8 +467,10 @@ int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_
   p.rows_per_split = pl.R;
   p.max_splits = pl.S;
   p.cluster = pl.cluster;
+  p.pairs = Hv != H ? 1 : 0;
+  p.Hv = Hv;
   p.part_acc = (float*)workspace;
-  p.part_ml = p.part_acc + (size_t)T * pl.S * H * kHeadDim;
+  p.part_ml = p.part_acc + (size_t)units * pl.S * Hv * kHeadDim;
   p.out = out;
   p.lse = lse;
   p.st = dev_status;

@@ -73,7 +73,7 @@ template <int CS>
 __device__ __forceinline__ void cluster_merge(const AttnParams& p, int t, float4* stage, uint64_t* bar_m) {
   cluster_sync();
   fence_proxy_async_global();
-  const int tid = threadIdx.x, H = p.H;
+  const int tid = threadIdx.x, H = p.Hv;  // a pair: 2 p.H heads, its queries' outputs adjacent in memory
   const uint32_t rank = cluster_rank();
   constexpr int HPC = 128 / CS;  // heads merged by a CTA
   constexpr int NG = 32 / CS;    // dimension groups per thread
@@ -89,12 +89,13 @@ __device__ __forceinline__ void cluster_merge(const AttnParams& p, int t, float4
   }
   const int hh = tid % HPC, g0 = tid / HPC;
   const int h = h0 + hh;
-  const bool mine = hh < nh;
+  // a pair's second query may not exist (an odd T): its heads write nothing
+  const bool mine = hh < nh && (!p.pairs || 2 * t + (h >= p.H ? 1 : 0) < p.T);
   float2 mls[CS];
   const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)t * CS * H + (mine ? h : h0);
 #pragma unroll
   for (int s = 0; s < CS; ++s) mls[s] = __ldcg(ml + (size_t)s * H);
-  const float sk = (p.sink && mine) ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+  const float sk = (p.sink && mine) ? __ldg(p.sink + h % p.H) * kLog2e : -INFINITY;
   float M = sk;
 #pragma unroll
   for (int s = 0; s < CS; ++s) M = fmaxf(M, mls[s].x);
@@ -143,9 +144,12 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
   __shared__ uint64_t bar_s, bar_o, bar_m;
   __shared__ uint32_t tmem_base;
   __shared__ const __nv_bfloat16* row_src[kTcChunk];  // address of each chunk row, null = skipped
-  __shared__ uint32_t row_mask[kTcChunk / 32];  // bit r: chunk row r is attended
+  __shared__ uint32_t row_mask[2][kTcChunk / 32];  // bit r: chunk row r is attended (by the pair's
+                                                   // first / second query; one query: [0])
 
+  // t: the unit of work -- a query, or (pairs) the pair of queries 2t, 2t + 1
   const int t = blockIdx.y, split = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tq0 = p.pairs ? 2 * t : t;
   // ---- set-up that reads no input overlaps the previous kernel (dependent launch)
   if (warp == 0) {
     tmem_alloc(&tmem_base, 256);  // S: columns 0..127, O: columns 128..255
@@ -160,8 +164,8 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
   // warm L2 with the query's metadata and the selected indices of this split's first rows
   // (prefetches only move lines into L2, which stays coherent with the writes being waited for)
   const int64_t r0 = (int64_t)split * p.rows_per_split;
-  if (tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_seq + t));
-  if (tid == 1) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_pos + t));
+  if (tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_seq + tq0));
+  if (tid == 1) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_pos + tq0));
   if (p.mode == CSKV_CSA && tid >= 32 && tid < 32 + kTcChunk / 32 && r0 + (tid - 32) * 32 < p.k)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p.idx + (size_t)t * p.k + r0 + (tid - 32) * 32));
   pdl_wait();
@@ -170,27 +174,44 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
   const int64_t e_pre = (p.mode == CSKV_CSA && r_pre < p.k && tid < min((int64_t)kTcChunk, (int64_t)p.rows_per_split))
                             ? (int64_t)__ldg(p.idx + (size_t)t * p.k + r_pre)
                             : (int64_t)-2;
-  const QueryRows q = query_rows(p, t);
+  const QueryRows q = query_rows(p, tq0);
   if (q.s < 0 && split == 0 && tid == 0) flag(p.st, CSKV_DEV_BAD_INDEX);
+  // a pair: its second query must be the next position of the same sequence (else flagged and
+  // left out: its rows then attend to nothing); the union of the two row lists
+  QueryRows q1 = q;
+  bool q1v = false;
+  int64_t nu = 0, n_rows = q.n_rows;
+  if (p.pairs) {
+    if (tq0 + 1 < p.T) {
+      q1 = query_rows(p, tq0 + 1);
+      q1v = q.s >= 0 && q1.s == q.s && q1.pos == q.pos + 1;
+      if (!q1v && split == 0 && tid == 0) flag(p.st, CSKV_DEV_BAD_INDEX);
+    }
+    nu = max(q.n_cmp, q1v ? q1.n_cmp : (int64_t)0);
+    n_rows = nu + p.window + (q1v ? 1 : 0);
+  }
   // a CTA without rows (bad query, or a split past the query's rows) runs no chunk and
   // only releases its TMEM at the end
-  const int64_t r1 = q.s < 0 ? r0 : max(r0, min(q.n_rows, r0 + p.rows_per_split));
+  const int64_t r1 = q.s < 0 ? r0 : max(r0, min(n_rows, r0 + p.rows_per_split));
   // cluster mode has no merge kernel to notice rows beyond the last split: flag them here
-  if (p.cluster && q.s >= 0 && split == p.max_splits - 1 && tid == 0 && q.n_rows > r0 + p.rows_per_split)
+  if (p.cluster && q.s >= 0 && split == p.max_splits - 1 && tid == 0 && n_rows > r0 + p.rows_per_split)
     flag(p.st, CSKV_DEV_CAPACITY);
-  const int H = p.H;
+  const int H = p.Hv;  // heads of the unit: the partials and the merge count in these
   const __nv_bfloat16* cmp = reinterpret_cast<const __nv_bfloat16*>(p.kv_cmp);
   const __nv_bfloat16* raw = reinterpret_cast<const __nv_bfloat16*>(p.kv_raw);
-  const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(p.q) + (size_t)t * H * kHeadDim;
+  const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(p.q) + (size_t)tq0 * p.H * kHeadDim;
+  // rows of the Q tile that hold a head: h < H for one query; a pair's second query (rows
+  // p.H .. 2 p.H - 1) only when it is there
+  const int hq = p.pairs ? (q1v ? H : p.H) : H;
 
-  // Q tile: a warp instruction copies two 256-byte head rows (zero rows beyond H); the copies
-  // complete together with the first chunk's gather, and the barriers of that chunk publish
-  // the TMEM address.
+  // Q tile: a warp instruction copies two 256-byte head rows (zero rows beyond the heads); the
+  // copies complete together with the first chunk's gather, and the barriers of that chunk
+  // publish the TMEM address.  A pair's second query follows the first in memory.
   if (r0 < r1)
     for (int it = 0; it < 16; ++it) {
       const int h = warp * 32 + it * 2 + (lane >> 4), c = lane & 15;
-      cp_async16(Qs + sw_off(h, c), h < H ? (const void*)(qg + (size_t)h * kHeadDim + 8 * c) : (const void*)qg,
-                 h < H ? 16u : 0u);
+      cp_async16(Qs + sw_off(h, c), h < hq ? (const void*)(qg + (size_t)h * kHeadDim + 8 * c) : (const void*)qg,
+                 h < hq ? 16u : 0u);
     }
   tc_fence_before();
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -205,11 +226,19 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
     // ---- resolve the chunk's rows
     {
       int64_t off = -1;
-      bool is_raw = false;
-      if (tid < rows) off = resolve_row(p, q, t, a + tid, &is_raw, a == r0 ? e_pre : (int64_t)-2);
+      bool is_raw = false, ok0 = false, ok1 = false;
+      if (p.pairs) {
+        if (tid < rows) off = resolve_pair_row(p, q, q1, q1v, nu, a + tid, &is_raw, &ok0, &ok1);
+      } else {
+        if (tid < rows) off = resolve_row(p, q, tq0, a + tid, &is_raw, a == r0 ? e_pre : (int64_t)-2);
+        ok0 = off >= 0;
+      }
       row_src[tid] = off >= 0 ? (is_raw ? raw : cmp) + off : nullptr;
-      const uint32_t bal = __ballot_sync(0xffffffffu, off >= 0);
-      if (lane == 0) row_mask[warp] = bal;
+      const uint32_t b0 = __ballot_sync(0xffffffffu, ok0), b1 = __ballot_sync(0xffffffffu, ok1);
+      if (lane == 0) {
+        row_mask[0][warp] = b0;
+        row_mask[1][warp] = b1;
+      }
     }
     __syncthreads();
     // ---- gather: one whole 512-byte K||V row per warp instruction (lane j copies its
@@ -240,14 +269,16 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
     }
     if (!mbar_wait_bounded(&bar_s, c & 1)) flag(p.st, CSKV_DEV_TIMEOUT);
     tc_fence_after();
-    // ---- online softmax of row tid over the nc columns (log2 units)
+    // ---- online softmax of row tid over the nc columns (log2 units); a pair's rows take the
+    //      mask of their query
+    const int mhalf = (p.pairs && tid >= p.H) ? 1 : 0;
     const float sl2 = p.scale_log2;
     // pass 1: row max of the raw logits over the attended columns (the scale is positive, so
     // it is applied once, to the max); four independent max chains.  Blocks of 32 columns
     // that are all attended (the common case) skip the mask.
     float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     for (int cc = 0; cc < nc; cc += 32) {
-      const uint32_t vm = row_mask[cc >> 5];
+      const uint32_t vm = row_mask[mhalf][cc >> 5];
       uint32_t v[32];
       tmem_ld32(tS + lane_base + cc, v);
       tmem_ld_wait();
@@ -267,7 +298,7 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
     // pass 2: P = 2^(s * scale - m) as bf16 into the P tile; four independent partial sums
     float ls4[4] = {0.f, 0.f, 0.f, 0.f};
     for (int cc = 0; cc < nc; cc += 32) {
-      const uint32_t vm = row_mask[cc >> 5];
+      const uint32_t vm = row_mask[mhalf][cc >> 5];
       uint32_t v[32];
       tmem_ld32(tS + lane_base + cc, v);
       tmem_ld_wait();
@@ -437,7 +468,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t stream) {
   // a dependent launch: the CTAs may start (TMEM, barriers) while the previous kernel -- the
   // indexer, or the compression after it -- finishes, and wait for it before reading
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.max_splits, p.T);
+  cfg.gridDim = dim3(p.max_splits, p.pairs ? (p.T + 1) / 2 : p.T);
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = kTcSmem;
   cfg.stream = stream;

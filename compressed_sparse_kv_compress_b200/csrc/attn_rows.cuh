@@ -75,4 +75,31 @@ __device__ __forceinline__ int64_t resolve_row(const AttnParams& p, const QueryR
   return (q.raw0 + row) * kRow;
 }
 
+// A pair of adjacent queries (HCA mode, a prefill chunk): q0 at p, q1 at p + 1 of the same
+// sequence (q1v false: q0 alone).  Their union row list: the HCA entries [0, nu), nu the larger
+// visible count, then the window tokens p - W + 1 .. p + 1.  Returns the row's element offset
+// (-1: skipped for both) and whether each query attends to it.
+__device__ __forceinline__ int64_t resolve_pair_row(const AttnParams& p, const QueryRows& q0, const QueryRows& q1,
+                                                    bool q1v, int64_t nu, int64_t r, bool* raw, bool* ok0,
+                                                    bool* ok1) {
+  if (r < nu) {
+    *raw = false;
+    *ok0 = r < q0.n_cmp;
+    *ok1 = q1v && r < q1.n_cmp;
+    return (*ok0 || *ok1) ? (q0.cmp0 + r) * kRow : -1;
+  }
+  *raw = true;
+  const int64_t tok = q0.pos - p.window + 1 + (r - nu);
+  *ok0 = tok >= 0 && tok <= q0.pos;
+  *ok1 = q1v && tok >= 0 && tok >= q1.pos - p.window + 1 && tok <= q1.pos;
+  if (!*ok0 && !*ok1) return -1;
+  const int64_t row = tok - q0.tok0;
+  if (row < 0 || row >= q0.raw_rows) {
+    flag(p.st, row < 0 ? CSKV_DEV_TAIL_MISSING : CSKV_DEV_BAD_INDEX);
+    *ok0 = *ok1 = false;
+    return -1;
+  }
+  return (q0.raw0 + row) * kRow;
+}
+
 }  // namespace cskv

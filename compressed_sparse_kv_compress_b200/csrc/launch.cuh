@@ -136,6 +136,8 @@ struct AttnParams {
   int rows_per_split;
   int max_splits;
   int cluster;  // tensor-core kernel: the splits of a query form a cluster of this size (0: merge kernel)
+  int pairs;    // tensor-core HCA kernel: CTA row y takes queries 2y, 2y + 1 (adjacent positions)
+  int Hv;       // heads of a unit of work: H, or 2H for a pair (its rows 0..H-1, then H..2H-1)
   float* part_acc;
   float* part_ml;
   float* out;

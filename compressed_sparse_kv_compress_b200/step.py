@@ -37,8 +37,12 @@ from . import api
 
 class DecodeStep:
     def __init__(self, t: dict, *, k: int, window: int, scale: float, max_csa_blocks: int, max_hca_blocks: int,
-                 max_csa_visible: int, max_hca_visible: int, two_streams: bool = False):
+                 max_csa_visible: int, max_hca_visible: int, two_streams: bool = False,
+                 adjacent_pairs: bool = False):
+        """adjacent_pairs: queries 2j and 2j + 1 are one sequence's consecutive positions (a
+        prefill chunk): the HCA attention takes them in pairs (CSKV_ATTN_PAIRS)."""
         self.t = t
+        self.adjacent_pairs = bool(adjacent_pairs)
         self.k, self.W, self.scale = int(k), int(window), float(scale)
         self.max_csa_blocks, self.max_hca_blocks = int(max_csa_blocks), int(max_hca_blocks)
         self.max_csa_visible, self.max_hca_visible = int(max_csa_visible), int(max_hca_visible)
@@ -124,7 +128,8 @@ class DecodeStep:
         api.hybrid_decode_attn(api.HCA, t["q_h"], t["cmp_h"], t["hca_off"], t["raw_h"], t["raw_off"], t["q_seq"],
                                t["q_pos"], self.o_h, self.ws_h, window=self.W, raw_tok0=t["raw_t0"],
                                sink=t.get("sink_h"), scale=self.scale, lse=self.lse_h,
-                               max_entries=self.max_hca_visible, dev_status=self.status, stream=stream)
+                               max_entries=self.max_hca_visible, adjacent_pairs=self.adjacent_pairs,
+                               dev_status=self.status, stream=stream)
 
     def run(self, stream=None):
         """Issue the whole step on `stream` (default: the current stream)."""

@@ -56,6 +56,8 @@ enum cskv_status {
 
 enum cskv_dtype { CSKV_F32 = 0, CSKV_BF16 = 1, CSKV_FP8E4M3 = 2 };
 enum cskv_mode { CSKV_CSA = 0, CSKV_HCA = 1 };
+/* OR-ed into hybrid_decode_attn's mode (see there): queries 2j and 2j + 1 are adjacent. */
+#define CSKV_ATTN_PAIRS 0x100
 
 /* Bits OR-ed into *dev_status by device-side checks. */
 enum cskv_dev_status {
@@ -313,6 +315,16 @@ CSKV_API size_t lindex_workspace_size_scan(int T, int64_t max_entries);
  * max_entries : host; mode HCA: >= every visible HCA entry count; mode CSA: unused.
  * out     : [T, H, d] fp32;  lse: [T, H] fp32 or NULL.
  * workspace : hybrid_attn_workspace_size(...) bytes (no zero-fill needed).
+ * mode | CSKV_ATTN_PAIRS : the caller states that queries 2j and 2j + 1 (j < T/2) are the
+ *           same sequence's consecutive positions p, p + 1 (a prefill chunk; with an odd T the
+ *           last query is alone).  With bf16 and H == 64 the HCA kernel then gives each pair
+ *           one pass over the union of the two row lists (the visible entries, then the
+ *           window tokens p - window + 1 .. p + 1, each masked for the query that does not
+ *           see it): the rows are gathered once and the pair's 128 heads fill the tensor-core
+ *           tile.  Results are those of the queries taken one by one.  A pair that is not
+ *           adjacent is flagged CSKV_DEV_BAD_INDEX and its second query attends to nothing
+ *           (output 0).  Elsewhere (CSA, fp32, other H, or a plan whose splits do not fit
+ *           one cluster) the bit is ignored.
  * ------------------------------------------------------------------------ */
 CSKV_API int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off,
                        const int32_t* idx, int k, const void* kv_raw, const int64_t* raw_off,

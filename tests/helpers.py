@@ -32,11 +32,19 @@ def bounds(w: Workload) -> dict:
     )
 
 
+def adjacent_pairs(w: Workload) -> bool:
+    """Queries 2j, 2j + 1 are one sequence's consecutive positions (every sequence has an even
+    number of queries, at its last positions)."""
+    Q = w.meta["Q"]
+    return Q >= 2 and Q % 2 == 0
+
+
 def decode_step(w: Workload, dev=None, two_streams=False):
     from compressed_sparse_kv_compress_b200 import DecodeStep
     dev = dev if dev is not None else w.device("cuda")
     m = w.meta
-    step = DecodeStep(dev, k=m["k"], window=m["W"], scale=m["scale"], two_streams=two_streams, **bounds(w))
+    step = DecodeStep(dev, k=m["k"], window=m["W"], scale=m["scale"], two_streams=two_streams,
+                      adjacent_pairs=adjacent_pairs(w), **bounds(w))
     return step, dev
 
 

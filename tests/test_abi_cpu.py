@@ -144,6 +144,9 @@ def test_attention_validation(lib):
 
     for na in (False, True):  # both entry points report the same error for the same mistake
         assert call(mode=5, noalloc=na) == _lib.ERR_INVALID_ARG
+        assert call(mode=0x200 | 1, noalloc=na) == _lib.ERR_INVALID_ARG  # an unknown flag bit
+        assert call(mode=_lib.ATTN_PAIRS | 7, noalloc=na) == _lib.ERR_INVALID_ARG
+        assert call(mode=_lib.ATTN_PAIRS | 1, T=0, noalloc=na) == _lib.OK  # HCA with pairs: valid
         assert call(d=64, noalloc=na) == _lib.ERR_UNSUPPORTED
         assert call(dtype=_lib.FP8E4M3, noalloc=na) == _lib.ERR_UNSUPPORTED
         assert call(H=0, noalloc=na) == _lib.ERR_INVALID_ARG

@@ -24,7 +24,7 @@ def _oracle_rows(w, a):
     return rows
 
 
-def _attn(w, dev, mode, idx=None, sink=True):
+def _attn(w, dev, mode, idx=None, sink=True, pairs=False):
     m = w.meta
     b = bounds(w)
     T, H = m["T"], m["H"]
@@ -37,15 +37,15 @@ def _attn(w, dev, mode, idx=None, sink=True):
     api.hybrid_decode_attn(mode, dev["q_" + layer], dev["cmp_" + layer], off, dev["raw_" + layer], dev["raw_off"],
                            dev["q_seq"], dev["q_pos"], out, ws, window=m["W"], idx=idx, raw_tok0=dev["raw_t0"],
                            sink=dev["sink_" + layer] if sink else None, scale=m["scale"], lse=lse,
-                           max_entries=b["max_hca_visible"], dev_status=st)
+                           max_entries=b["max_hca_visible"], adjacent_pairs=pairs, dev_status=st)
     torch.cuda.synchronize()
     return to_f64(out), to_f64(lse), int(st.item())
 
 
-def _compare(w, dev, a, mode, rows=None, sink=True, extra_rel=None, queries=None):
+def _compare(w, dev, a, mode, rows=None, sink=True, extra_rel=None, queries=None, pairs=False):
     m = w.meta
     idx = None if rows is None else torch.from_numpy(rows.astype(np.int32)).cuda()
-    o, lse, st = _attn(w, dev, mode, idx, sink)
+    o, lse, st = _attn(w, dev, mode, idx, sink, pairs)
     layer = "c" if mode == api.CSA else "h"
     arr = a if sink else {**a, "sink_" + layer: None}
     for t in (queries if queries is not None else range(m["T"])):
@@ -101,3 +101,32 @@ def test_invisible_index_is_flagged_and_skipped():
     rows[0, 5] = -1
     st = _compare(w, dev, a, api.CSA, rows)
     assert st & 1
+
+
+@pytest.mark.parametrize("Q,sink", [(34, True), (33, True), (8, False)])
+def test_hca_adjacent_query_pairs(Q, sink):
+    # a prefill-like run of consecutive positions, 64 heads: the HCA kernel takes the queries in
+    # pairs (one pass over the union of the two row lists); an odd count leaves the last alone.
+    # Positions straddle 128-token block boundaries, so the two queries of a pair can see a
+    # different number of entries.
+    spec = spec_by_name("prefill_4k_at_128k").replace(seq_len=(20096 + 10,), queries_per_seq=Q, heads=64)
+    w = Workload(spec)
+    dev = w.device("cuda")
+    a = np_arrays(w)
+    assert _compare(w, dev, a, api.HCA, sink=sink, pairs=True) == 0
+    # and the per-query path agrees to the kernels' rounding (P is rounded to bf16 relative to a
+    # running maximum, and the pair's chunks cut the rows elsewhere)
+    o1, l1, _ = _attn(w, dev, api.HCA, sink=sink, pairs=True)
+    o2, l2, _ = _attn(w, dev, api.HCA, sink=sink, pairs=False)
+    assert np.abs(o1 - o2).max() <= 1e-3 * max(1.0, np.abs(o2).max())
+
+
+def test_hca_pairs_not_adjacent_are_flagged():
+    # two sequences of 5 queries: the pair (4, 5) straddles them, which the caller promised not
+    # to happen: flagged, and every other query still matches the oracle
+    spec = spec_by_name("prefill_4k_at_128k").replace(batch=2, seq_len=(9000, 12000), queries_per_seq=5, heads=64)
+    w = Workload(spec)
+    dev = w.device("cuda")
+    a = np_arrays(w)
+    st = _compare(w, dev, a, api.HCA, pairs=True, queries=[0, 1, 2, 3, 4, 6, 7, 8, 9])
+    assert st & 1  # CSKV_DEV_BAD_INDEX
