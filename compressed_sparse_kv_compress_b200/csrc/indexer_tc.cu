@@ -76,6 +76,13 @@ __device__ __forceinline__ int score_bin(float f) {
   return min(max(k12 - (127 - 30) * 16 + 1, 0), kTcIdxBins - 1);
 }
 
+// The lowest score of bin b (b >= 1; bin 0: -inf): score_bin(f) >= b  <=>  f >= bin_floor(b).
+__device__ __forceinline__ float bin_floor(int b) {
+  if (b <= 0) return -INFINITY;
+  if (b >= kTcIdxBins) return INFINITY;
+  return __uint_as_float((uint32_t)(b - 1 + (127 - 30) * 16) << 19);
+}
+
 __device__ __forceinline__ uint32_t sw_off_idx(int r, int c) {
   return (uint32_t)r * kTcIdxRow + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
 }
@@ -242,11 +249,13 @@ __global__ void __launch_bounds__(kTcIdxThreads, 1) lindex_tc_kernel(TcIdxParams
         if (tid < QT) q_floor[tid] = 0;
       }
       int64_t run[QPW];  // pass 2: candidates appended so far for each of the warp's queries
-      int thr[QPW];
+      float thr_lo[QPW], thr_hi[QPW];  // pass 2: the scores of bin b* are thr_lo <= s < thr_hi
 #pragma unroll
       for (int j = 0; j < QPW; ++j) {
         run[j] = 0;
-        thr[j] = pass == 1 ? q_thr[q0 + j] : 0;
+        const int thr = pass == 1 ? q_thr[q0 + j] : 0;
+        thr_lo[j] = bin_floor(thr);
+        thr_hi[j] = bin_floor(thr + 1);
       }
       if (tid < kTcIdxStages + 1) tile_np[tid] = -1;
       __syncthreads();
@@ -304,7 +313,7 @@ __global__ void __launch_bounds__(kTcIdxThreads, 1) lindex_tc_kernel(TcIdxParams
         }
         // both 128-entry halves of the tile: TMEM columns buf * 256 + half * 128 + (t, h)
         float sc[2][QPW];
-        int bin[2][QPW];
+        bool vis[2][QPW];
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t v[32];
@@ -330,28 +339,33 @@ __global__ void __launch_bounds__(kTcIdxThreads, 1) lindex_tc_kernel(TcIdxParams
               }
             }
             sc[hf][j] = a;
-            bin[hf][j] = (mine[j] && e < V[j]) ? score_bin(a) : -1;  // -1: not visible to the query
+            vis[hf][j] = mine[j] && e < V[j];
           }
         }
         if (pass == 0) {
+          // only scores at or above the query's floor are binned (a comparison first: most fail)
 #pragma unroll
           for (int j = 0; j < QPW; ++j) {
-            const int fl = *(volatile int*)&q_floor[q0 + j];
+            const float flv = bin_floor(*(volatile int*)&q_floor[q0 + j]);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf)
-              if (bin[hf][j] >= 0 && bin[hf][j] >= fl)
-                atomicAdd(&hist[(q0 + j) * HB + bin[hf][j] + (bin[hf][j] >> 5)], 1u);
+              if (vis[hf][j] && sc[hf][j] >= flv) {
+                const int b = score_bin(sc[hf][j]);
+                atomicAdd(&hist[(q0 + j) * HB + b + (b >> 5)], 1u);
+              }
           }
           return;
         }
         // pass 2: each query's kept entries of this thread's two 32-entry segments (half, lane
         // quarter) in lane order (ballot), after the segments before them in the tile
         unsigned mask[2][QPW];
+        bool keep[2][QPW];
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
           for (int j = 0; j < QPW; ++j) {
-            mask[hf][j] = __ballot_sync(0xffffffffu, bin[hf][j] >= thr[j]);
+            keep[hf][j] = vis[hf][j] && sc[hf][j] >= thr_lo[j];
+            mask[hf][j] = __ballot_sync(0xffffffffu, keep[hf][j]);
             if (lane == 0) q_cnt[hf * 4 + lq][q0 + j] = __popc(mask[hf][j]);
           }
         __syncthreads();
@@ -367,7 +381,7 @@ __global__ void __launch_bounds__(kTcIdxThreads, 1) lindex_tc_kernel(TcIdxParams
           const int tq = t0 + q0 + j;
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            if (bin[hf][j] >= thr[j]) {
+            if (keep[hf][j]) {
               int before = 0;
 #pragma unroll
               for (int c = 0; c < 8; ++c) before += c < hf * 4 + lq ? cnt[c] : 0;
@@ -378,7 +392,7 @@ __global__ void __launch_bounds__(kTcIdxThreads, 1) lindex_tc_kernel(TcIdxParams
               } else {
                 q_over[q0 + j] = 1;
               }
-              if (bin[hf][j] == thr[j]) {
+              if (sc[hf][j] < thr_hi[j]) {  // in bin b*
                 atomicMin(&q_bin_lo[q0 + j], ord_key(sc[hf][j]));
                 atomicMax(&q_bin_hi[q0 + j], ord_key(sc[hf][j]));
               }
