@@ -314,6 +314,13 @@ def barrier(ws: int):
 
 
 # ---------------------------------------------------------------------- arms
+def workload_config(name: str, w: Workload) -> dict:
+    """The workload part of the line's config (the same in both arms)."""
+    m, spec = w.meta, w.spec
+    return {"workload": name, "batch": m["B"], "context": max(m["n"]), "query_tokens_per_step": m["T"],
+            "heads": m["H"], "topk": m["k"], "window": m["W"], "indexer": f"{m['Hi']}x{m['di']} {spec.idx_dtype}"}
+
+
 def run_reference(args, ws, rank):
     if rank != 0:
         return
@@ -335,7 +342,9 @@ def run_reference(args, ws, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(per),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload}, "cpu_baseline": cb,
+            "data": "synthetic",
+            "config": {**workload_config(args.workload, w), "l2": "not applicable (the oracle on host cores)"},
+            "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -553,9 +562,7 @@ def run_cskv(args, ws, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if
         spec.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": args.workload, "batch": m["B"], "context": max(m["n"]), "query_tokens_per_step": T,
-                   "heads": m["H"], "topk": m["k"], "window": m["W"], "indexer": f"{m['Hi']}x{m['di']} "
-                   f"{spec.idx_dtype}", "l2": l2,
+        "config": {**workload_config(args.workload, w), "l2": l2,
                    "replay": (f"CUDA graphs of consecutive steps ({R} steps, one per replica, per graph)"
                               if flush is None else "one single-step CUDA graph per step"),
                    "streams": 1 if args.one_stream else 2},
