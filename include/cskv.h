@@ -233,6 +233,12 @@ CSKV_API int lindex_pool_keys(const void* k_tok, int in_dtype, int Di, const int
  *           the rest scratch), so it can be reused as is, unless the call flagged
  *           CSKV_DEV_TIMEOUT (zero-fill it again then).
  *           Calls sharing a workspace must be ordered on one stream.
+ * Many queries (T >= 256, E4M3, Hi in {8, 16}, Di in {64, 128}) with that full
+ * workspace run on the tensor cores (see lindex_workspace_size): the scores are
+ * the same up to fp32 rounding order (the positive scales are applied after the
+ * ReLU and head weights, where exact algebra allows it), the selection the same
+ * exact top-k of them; an entry list that overflows inside one score bin of
+ * unequal scores flags CSKV_DEV_CAPACITY.
  * ------------------------------------------------------------------------ */
 CSKV_API int lindex_score_topk(const void* q_idx, const float* q_scale, const void* k_idx, const float* k_scale,
                       const float* head_w, const int32_t* q_seq, const int64_t* q_pos,
