@@ -11,19 +11,20 @@
 //
 // Across the queries of a chunk the <q_{t,h}, k_i> form a dense product.  A CTA takes QT =
 // 128 / Hi consecutive queries -- their (t, h) rows are the N = 128 columns of tcgen05.mma
-// kind::f8f6f4 (E4M3 x E4M3 -> fp32 in TMEM) -- and streams its sequence's keys in tiles of 256
-// entries, two MMAs of M = 128 entries (the TMEM lanes): D[i, (t, h)] = K_half Q^T.  Two TMEM
-// accumulators of 256 columns let the MMAs of one tile run while the epilogue reads the other.  Operands are K-major in the 128-byte
-// swizzle layout (row r at r * 128 bytes, 16-byte chunk c at chunk c ^ (r & 7)); key tiles are
-// gathered with 16-byte cp.async copies into a ring of four stages (three tiles in flight while
-// one is multiplied) and their scales ride along.
+// kind::f8f6f4 (E4M3 x E4M3 -> fp32 in TMEM) -- and streams its sequence's keys in tiles of
+// 256 entries, two MMAs of M = 128 entries (the TMEM lanes): D[i, (t, h)] = K_half Q^T.  Two
+// TMEM accumulators of 256 columns let the MMAs of one tile run while the epilogue reads the
+// other.  Operands are K-major in the 128-byte swizzle layout (row r at r * 128 bytes, 16-byte
+// chunk c at chunk c ^ (r & 7)); key tiles are gathered with 16-byte cp.async copies into a
+// ring of four stages (three tiles in flight while one is multiplied), their scales alongside.
 //
 // Epilogue (16 warps: warp w reads the TMEM lane quarter w % 4 -- 32 entries of each half, one
-// per lane -- and the 32 columns 32 (w / 4) .. -- 32 / Hi queries): a lane sums, in registers, its entry's
-// score for each of those queries, s = sk_i * sum_h (w_h sq_{t,h}) max(0, acc) -- factoring
-// the scales out of the ReLU needs sq > 0 and sk > 0 (quantisation scales are); a tile or a
-// CTA with a non-positive scale takes the unfactored form sum_h w_h max(0, (sq sk) acc).
-
+// per lane -- and the 32 columns 32 (w / 4) .. -- 32 / Hi queries): a lane sums, in
+// registers, its entry's score for each of those queries, s = sk_i * sum_h (w_h sq_{t,h})
+// max(0, acc) -- factoring the scales out of the ReLU needs sq > 0 and sk > 0 (quantisation
+// scales are); a tile or a CTA with a non-positive scale takes the unfactored form
+// sum_h w_h max(0, (sq sk) acc).
+//
 // The k-th best score of a query is not known before all of its entries are scored, so the
 // kernel makes two passes over the keys:
 //   1. every visible entry's score goes into a per-query histogram (1024 bins, 16 per octave
@@ -32,7 +33,7 @@
 //   2. the scores are computed again (the same instructions on the same data: the same values)
 //      and every visible entry with bin > b*, and the entries of bin b* while the list has
 //      room, are appended to the query's candidate list in ascending entry order (a ballot
-//      orders the 32 entries of a lane quarter, shared counts the four quarters of a tile).
+//      orders the 32 entries of a lane quarter, shared counts the tile's eight segments).
 // In pass 1 a per-query floor (raised every 4 tiles to the lowest bin of the 32-bin block in
 // which the count from the top reaches k_eff) lets entries far below the k-th score skip the
 // histogram: b* is never below the floor, and every bin at or above it is counted exactly.
@@ -48,7 +49,7 @@
 
 namespace cskv {
 
-constexpr int kTcIdxThreads = 512;   // 16 warps: warp w reads TMEM lanes 32 (w % 4) .. (entries), columns 32 (w / 4) ..
+constexpr int kTcIdxThreads = 512;   // 16 warps: TMEM lanes 32 (w % 4) .. (entries), columns 32 (w / 4) ..
 constexpr int kTcIdxN = 256;         // entries per key tile: two MMAs of M = 128 entries
 constexpr int kTcIdxBins = 1024;     // histogram bins per query
 constexpr uint32_t kTcIdxRow = 128;  // bytes per operand row in the swizzled layout (Di <= 128)
@@ -56,8 +57,8 @@ constexpr uint32_t kTcIdxTile = kTcIdxN * kTcIdxRow;  // 32 KiB: one key tile
 constexpr int kTcIdxStages = 4;      // key tiles in flight (cp.async groups)
 
 struct TcIdxSmem {
-  static constexpr size_t a = 0;                                     // A: 128 rows x 128 B
-  static constexpr size_t b = a + 128 * kTcIdxRow;                               // B: key tile ring
+  static constexpr size_t a = 0;                                     // the Q tile: 128 rows x 128 B
+  static constexpr size_t b = a + 128 * kTcIdxRow;                   // the key tile ring
   static constexpr size_t ks = b + kTcIdxStages * (size_t)kTcIdxTile;            // key scales
   static constexpr size_t hist = ks + (kTcIdxStages + 1) * kTcIdxN * sizeof(float);  // QT x padded bins
   static size_t bytes(int QT) { return hist + (size_t)QT * (kTcIdxBins + kTcIdxBins / 32) * sizeof(unsigned) + 1024; }
