@@ -170,6 +170,16 @@ class DecodeStep:
         the buffer and one cskv_copy_segments launch that spreads it to the device tensors
         (which must be contiguous).  d2h: (device, host pinned) pairs copied back after the
         step.  A replay costs one launch on the host, whatever the number of tensors."""
+        views = self.prepare_io(h2d, d2h)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run_io()
+        self.graph_io = g
+        return views
+
+    def prepare_io(self, h2d=(), d2h=()):
+        """The pinned staging buffer and scatter tables of capture_io (returns the host views);
+        run_io() then issues upload, step and read-back on the current stream."""
         if self.graph is None:
             self.capture()  # sets kernel attributes and warms up outside capture
         dev = self.o_c.device
@@ -188,18 +198,18 @@ class DecodeStep:
             views.append(v)
         self._io = (stage_h, stage_d, torch.tensor(offs, dtype=torch.int64, device=dev),
                     torch.tensor([d.data_ptr() for _, d in h2d], dtype=torch.int64, device=dev),
-                    torch.tensor(sizes, dtype=torch.int64, device=dev))
-        _, _, src_off, dst_ptrs, lens = self._io
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            if h2d:
-                stage_d.copy_(stage_h, non_blocking=True)
-                api.copy_segments(stage_d, src_off, dst_ptrs, lens)
-            self.run()
-            for d, h in d2h:
-                h.copy_(d, non_blocking=True)
-        self.graph_io = g
+                    torch.tensor(sizes, dtype=torch.int64, device=dev), len(h2d) > 0, list(d2h))
         return views
+
+    def run_io(self):
+        """Upload (one copy + one scatter launch), the step, the read-back (prepare_io first)."""
+        stage_h, stage_d, src_off, dst_ptrs, lens, up, d2h = self._io
+        if up:
+            stage_d.copy_(stage_h, non_blocking=True)
+            api.copy_segments(stage_d, src_off, dst_ptrs, lens)
+        self.run()
+        for d, h in d2h:
+            h.copy_(d, non_blocking=True)
 
     def replay_io(self):
         self.graph_io.replay()
