@@ -166,6 +166,9 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
   const int64_t r0 = (int64_t)split * p.rows_per_split;
   if (tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_seq + tq0));
   if (tid == 1) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.q_pos + tq0));
+  if (tid == 2) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.cmp_off));
+  if (tid == 3) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.raw_off));
+  if (tid == 4 && p.raw_tok0) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.raw_tok0));
   if (p.mode == CSKV_CSA && tid >= 32 && tid < 32 + kTcChunk / 32 && r0 + (tid - 32) * 32 < p.k)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p.idx + (size_t)t * p.k + r0 + (tid - 32) * 32));
   pdl_wait();

@@ -22,18 +22,24 @@ struct QueryRows {
 
 __device__ __forceinline__ QueryRows query_rows(const AttnParams& p, int t) {
   QueryRows q;
+  // the query's sequence and position load together with sequence 0's offsets (speculatively:
+  // one round trip instead of two dependent ones when the query is in sequence 0)
   q.s = __ldg(p.q_seq + t);
+  q.pos = __ldg(p.q_pos + t);
+  const int64_t c0 = __ldg(p.cmp_off), c1 = __ldg(p.cmp_off + 1);
+  const int64_t w0 = __ldg(p.raw_off), w1 = __ldg(p.raw_off + 1);
+  const int64_t k0 = p.raw_tok0 ? __ldg(p.raw_tok0) : 0;
   if (q.s < 0 || q.s >= p.batch) {
     q.s = -1;
     q.n_rows = 0;
     return q;
   }
-  q.pos = __ldg(p.q_pos + t);
-  q.cmp0 = __ldg(p.cmp_off + q.s);
-  q.cmp_cap = __ldg(p.cmp_off + q.s + 1) - q.cmp0;
-  q.raw0 = __ldg(p.raw_off + q.s);
-  q.raw_rows = __ldg(p.raw_off + q.s + 1) - q.raw0;
-  q.tok0 = p.raw_tok0 ? __ldg(p.raw_tok0 + q.s) : 0;
+  const bool s0 = q.s == 0;
+  q.cmp0 = s0 ? c0 : __ldg(p.cmp_off + q.s);
+  q.cmp_cap = (s0 ? c1 : __ldg(p.cmp_off + q.s + 1)) - q.cmp0;
+  q.raw0 = s0 ? w0 : __ldg(p.raw_off + q.s);
+  q.raw_rows = (s0 ? w1 : __ldg(p.raw_off + q.s + 1)) - q.raw0;
+  q.tok0 = p.raw_tok0 ? (s0 ? k0 : __ldg(p.raw_tok0 + q.s)) : 0;
   const int64_t ratio = p.mode == CSKV_CSA ? 4 : 128;
   const int64_t vis = q.pos >= 0 ? (q.pos + 1) / ratio : 0;
   q.vis_c = vis < q.cmp_cap ? vis : q.cmp_cap;
