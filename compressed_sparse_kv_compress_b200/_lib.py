@@ -32,6 +32,7 @@ SIGNATURES = {
     "cskv_version": (_i32, []),
     "cskv_launch_count": (ctypes.c_ulonglong, []),
     "cskv_copy_segments": (_i32, [_p, _p, _p, _p, _i32, _p]),
+    "cskv_mapped_pointer": (_i32, [_p, _p]),
     "csa_compress": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p,
                             _i32, _p, _f, _p, _i32, _i32, _p, _p, _i32, _p, _p]),
     "hca_compress": (_i32, [_p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p, _i32, _p, _f, _p, _p]),

@@ -7,6 +7,7 @@ one given).  All computation happens in the CUDA library.
 
 from __future__ import annotations
 
+import ctypes
 import math
 
 import torch
@@ -184,10 +185,24 @@ def hybrid_decode_attn(mode, q, kv_cmp, cmp_off, kv_raw, raw_off, q_seq, q_pos, 
 
 
 def copy_segments(src, src_off, dst_ptrs, lens, stream=None):
-    """Scatter segments of the device byte buffer `src` (int64 device arrays src_off, lens and
+    """Scatter segments of the byte buffer `src` (int64 device arrays src_off, lens and
     dst_ptrs = destination addresses) with one kernel: the unpacking half of a staged
-    host-to-device copy of a step's new inputs."""
+    host-to-device copy of a step's new inputs, or a read-back into host memory.  `src` is a
+    device tensor or an address from mapped_pointer(); host destinations in dst_ptrs must be
+    mapped_pointer() addresses too."""
     lib = _lib.load()
-    st = lib.cskv_copy_segments(_ptr(src), _ptr(src_off), _ptr(dst_ptrs), _ptr(lens), int(src_off.numel()),
+    src_p = src if isinstance(src, int) else _ptr(src)
+    st = lib.cskv_copy_segments(src_p, _ptr(src_off), _ptr(dst_ptrs), _ptr(lens), int(src_off.numel()),
                                 _stream(stream))
     _lib.check("cskv_copy_segments", st)
+
+
+def mapped_pointer(t) -> int:
+    """The address at which the current device reaches tensor `t`'s data: its own address for
+    device memory, the mapped address for page-locked host memory.  Raises for pageable host
+    memory, which the device cannot address."""
+    lib = _lib.load()
+    out = ctypes.c_void_p()
+    st = lib.cskv_mapped_pointer(_ptr(t), ctypes.byref(out))
+    _lib.check("cskv_mapped_pointer", st)
+    return int(out.value)

@@ -79,6 +79,28 @@ int cskv_copy_segments(const void* src, const int64_t* src_off, void* const* dst
   return launch_status(launch_copy_segments(src, src_off, dst, len, n, (cudaStream_t)stream));
 }
 
+int cskv_mapped_pointer(const void* p, void** out) {
+  if (!out) return CSKV_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!p) return CSKV_ERR_INVALID_ARG;
+  cudaPointerAttributes at;
+  const cudaError_t e = cudaPointerGetAttributes(&at, p);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();  // a failed query leaves no error behind for the next launch
+    return launch_status(e);
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
+    *out = const_cast<void*>(p);
+    return CSKV_OK;
+  }
+  // page-locked host memory: the address this device reads it at (none: not mapped here)
+  if (at.type == cudaMemoryTypeHost && at.devicePointer) {
+    *out = at.devicePointer;
+    return CSKV_OK;
+  }
+  return CSKV_ERR_INVALID_ARG;  // pageable host memory: the device cannot address it
+}
+
 unsigned long long cskv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 static int check_compress_common(const void* x, const void* z, const int64_t* tok_off, int batch,

@@ -160,56 +160,82 @@ class DecodeStep:
         self.graph = g
         return g
 
-    def capture_io(self, h2d=(), d2h=()):
+    def capture_io(self, h2d=(), d2h=(), zero_copy=True):
         """Capture, into one CUDA graph, the upload of this step's new inputs, the step, and the
         read-back of its results; replay with replay_io().
 
         h2d: (host, device) pairs.  The host sides are packed into one pinned staging buffer:
         the returned host tensors (views into it, initialised from the given ones) are where
-        the caller writes each step's new inputs.  A replay makes one host-to-device copy of
-        the buffer and one cskv_copy_segments launch that spreads it to the device tensors
-        (which must be contiguous).  d2h: (device, host pinned) pairs copied back after the
-        step.  A replay costs one launch on the host, whatever the number of tensors."""
-        views = self.prepare_io(h2d, d2h)
+        the caller writes each step's new inputs.  d2h: (device, host pinned) pairs copied back
+        after the step.  With zero_copy (the default) one cskv_copy_segments launch reads the
+        staging buffer over the bus and spreads it to the device tensors (which must be
+        contiguous), and one more writes the results straight into the host tensors; without
+        it, a host-to-device copy of the buffer precedes the spreading launch and each result
+        comes back by a device-to-host copy.  A replay costs one launch on the host, whatever
+        the number of tensors."""
+        views = self.prepare_io(h2d, d2h, zero_copy)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             self.run_io()
         self.graph_io = g
         return views
 
-    def prepare_io(self, h2d=(), d2h=()):
-        """The pinned staging buffer and scatter tables of capture_io (returns the host views);
+    def prepare_io(self, h2d=(), d2h=(), zero_copy=True):
+        """The pinned staging buffer and copy tables of capture_io (returns the host views);
         run_io() then issues upload, step and read-back on the current stream."""
         if self.graph is None:
             self.capture()  # sets kernel attributes and warms up outside capture
         dev = self.o_c.device
+
+        def i64(vals):
+            return torch.tensor(list(vals), dtype=torch.int64, device=dev)
+
         sizes = [d.numel() * d.element_size() for _, d in h2d]
         offs, total = [], 0
         for nb in sizes:
             offs.append(total)
             total += (nb + 15) // 16 * 16
         stage_h = torch.empty(max(total, 16), dtype=torch.uint8, pin_memory=True)
-        stage_d = torch.empty(max(total, 16), dtype=torch.uint8, device=dev)
         views = []
         for (h, d), o, nb in zip(h2d, offs, sizes):
             assert d.is_contiguous()
             v = stage_h[o:o + nb].view(d.dtype).view(d.shape)
             v.copy_(h)
             views.append(v)
-        self._io = (stage_h, stage_d, torch.tensor(offs, dtype=torch.int64, device=dev),
-                    torch.tensor([d.data_ptr() for _, d in h2d], dtype=torch.int64, device=dev),
-                    torch.tensor(sizes, dtype=torch.int64, device=dev), len(h2d) > 0, list(d2h))
+        up = None
+        if h2d:
+            dst = i64(d.data_ptr() for _, d in h2d)
+            if zero_copy:
+                up = (api.mapped_pointer(stage_h), i64(offs), dst, i64(sizes))
+            else:
+                stage_d = torch.empty(stage_h.shape, dtype=torch.uint8, device=dev)
+                up = (stage_d, i64(offs), dst, i64(sizes))
+        down = None
+        if d2h and zero_copy:
+            for d, h in d2h:
+                assert d.is_contiguous() and h.is_contiguous() and h.is_pinned()
+                assert d.numel() * d.element_size() == h.numel() * h.element_size()
+            base = min(d.data_ptr() for d, _ in d2h)
+            down = (base, i64(d.data_ptr() - base for d, _ in d2h), i64(api.mapped_pointer(h) for _, h in d2h),
+                    i64(d.numel() * d.element_size() for d, _ in d2h))
+        # the host tensors stay referenced for as long as the captured graph may touch them
+        self._io = (zero_copy, stage_h, up, down, list(d2h))
         return views
 
     def run_io(self):
-        """Upload (one copy + one scatter launch), the step, the read-back (prepare_io first)."""
-        stage_h, stage_d, src_off, dst_ptrs, lens, up, d2h = self._io
-        if up:
-            stage_d.copy_(stage_h, non_blocking=True)
-            api.copy_segments(stage_d, src_off, dst_ptrs, lens)
+        """Upload, the step, the read-back (prepare_io first)."""
+        zero_copy, stage_h, up, down, d2h = self._io
+        if up is not None:
+            if not zero_copy:
+                up[0].copy_(stage_h, non_blocking=True)
+            api.copy_segments(*up)
         self.run()
-        for d, h in d2h:
-            h.copy_(d, non_blocking=True)
+        if zero_copy:
+            if down is not None:
+                api.copy_segments(*down)
+        else:
+            for d, h in d2h:
+                h.copy_(d, non_blocking=True)
 
     def replay_io(self):
         self.graph_io.replay()

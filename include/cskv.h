@@ -377,17 +377,36 @@ CSKV_API int hybrid_decode_attn_noalloc(int mode, const void* q, const void* kv_
  * cskv_copy_segments -- device-side scatter of byte segments (input staging).
  *
  * Not a step of the method: plumbing for callers that move a decode step's new
- * inputs (queries, the newest token rows, the newest indexer keys) to the GPU in
- * one host->device copy of a packed staging buffer and then spread them to their
- * places.  Segment i copies len[i] bytes from src + src_off[i] to dst[i].
- * src     : device buffer holding the packed segments.
- * src_off, len : [n] int64 device arrays; dst : [n] device array of device
- *           pointers.  Segments must not overlap their destinations.
+ * inputs (queries, the newest token rows, the newest indexer keys) to the GPU from
+ * one packed staging buffer and spread them to their places, or read results back.
+ * Segment i copies len[i] bytes from src + src_off[i] to dst[i].
+ * src     : buffer holding the packed segments: device memory, or page-locked host
+ *           memory through the address cskv_mapped_pointer() gives for it (the
+ *           kernel then reads the host buffer over the bus: no separate copy).
+ * src_off, len : [n] int64 device arrays; dst : [n] device array of pointers the
+ *           device can write: device memory, or mapped page-locked host memory
+ *           (cskv_mapped_pointer() addresses).  Segments must not overlap their
+ *           destinations.  The caller keeps host buffers alive and unchanged until
+ *           the stream has passed the copy.
  * n       : number of segments (0 launches nothing).
- * Errors: CSKV_ERR_INVALID_ARG for a null pointer with n > 0 or n < 0.
+ * Errors: CSKV_ERR_INVALID_ARG for a null pointer with n > 0 or n < 0.  The
+ * pointers inside the arrays are not checked: take host addresses from
+ * cskv_mapped_pointer(), never a plain host pointer.
  * ------------------------------------------------------------------------ */
 CSKV_API int cskv_copy_segments(const void* src, const int64_t* src_off, void* const* dst, const int64_t* len, int n,
                                 cskv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * cskv_mapped_pointer -- the address at which the current device reaches p.
+ *
+ * Plumbing for zero-copy staging (cskv_copy_segments).  Device or managed memory:
+ * *out = p.  Page-locked host memory mapped into the device's address space:
+ * *out = the device-side address of p (under unified addressing, p itself).
+ * Pageable host memory, or a null p / out: CSKV_ERR_INVALID_ARG with *out = NULL
+ * (when out is not null).  A failed CUDA query: CSKV_ERR_LAUNCH.  Host-side query
+ * only: launches nothing, allocates nothing.
+ * ------------------------------------------------------------------------ */
+CSKV_API int cskv_mapped_pointer(const void* p, void** out);
 
 #ifdef __cplusplus
 }

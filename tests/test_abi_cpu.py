@@ -171,6 +171,14 @@ def test_copy_segments_validation(lib):
     assert lib.cskv_copy_segments(nul, nul, nul, nul, 0, nul) == _lib.OK
 
 
+def test_mapped_pointer_validation(lib):
+    # null arguments are refused before any CUDA query; the out-pointer is cleared
+    out = ctypes.c_void_p(1)
+    assert lib.cskv_mapped_pointer(None, ctypes.byref(out)) == _lib.ERR_INVALID_ARG
+    assert out.value is None
+    assert lib.cskv_mapped_pointer(_p(), None) == _lib.ERR_INVALID_ARG
+
+
 def test_pool_keys_validation(lib):
     nul = None
     # (k_tok, in_dtype, Di, tok_off, tok0, batch, ent_off, first, num, max_blocks, codes, scale, st, stream)

@@ -76,9 +76,11 @@ def test_small_bf16_two_streams_graph_equal_eager():
     assert torch.equal(s1.o_c, s2.o_c) and torch.equal(s1.o_h, s2.o_h)
 
 
-def test_graph_with_host_copies_equals_eager():
+@pytest.mark.parametrize("zero_copy", [True, False])
+def test_graph_with_host_copies_equals_eager(zero_copy):
     # capture_io: new queries copied from pinned host memory and both outputs read back, all
-    # inside the step's graph; replayed twice with different queries
+    # inside the step's graph (zero copy: the kernels read and write the host buffers over the
+    # bus; otherwise through copies); replayed twice with different queries
     spec = spec_by_name("ragged_b64").replace(batch=3, len_range=(3000, 20000), heads=64)
     w = Workload(spec)
     step, dev = decode_step(w, two_streams=True)
@@ -86,7 +88,7 @@ def test_graph_with_host_copies_equals_eager():
     h_q = torch.empty(dev["q_c"].shape, dtype=dev["q_c"].dtype, pin_memory=True)
     h_oc = torch.empty(step.o_c.shape, dtype=step.o_c.dtype, pin_memory=True)
     h_oh = torch.empty(step.o_h.shape, dtype=step.o_h.dtype, pin_memory=True)
-    views = step.capture_io([(h_q, dev["q_c"])], [(step.o_c, h_oc), (step.o_h, h_oh)])
+    views = step.capture_io([(h_q, dev["q_c"])], [(step.o_c, h_oc), (step.o_h, h_oh)], zero_copy=zero_copy)
     for q in qs:
         views[0].copy_(q.cpu())
         step.replay_io()
