@@ -499,7 +499,7 @@ def run_cskv(args, ws, rank, local):
 
     # ---- end to end through the public API with host buffers: per step, the step's new
     #      inputs go host -> device from pinned memory and both outputs come back, all in the
-    #      step's graph (DecodeStep.capture_io)
+    #      step's graph (DecodeStep.capture_io; small transfers zero-copy, large ones by copies)
     def host_pairs(st):
         t = st.t
         pairs = []  # (pinned host tensor, device destination view)
@@ -578,7 +578,9 @@ def run_cskv(args, ws, rank, local):
                      "traffic": profiled_traffic(args.workload)},
         "e2e": {"value": whole_job_rate(T, ws, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "device_us_per_step": ms_e2e * 1e3,
-                "host_wall_us_per_step": wall_us},
+                "host_wall_us_per_step": wall_us,
+                "transfer": {"upload": "zero copy" if steps[0].io_zero_copy[0] else "copy + scatter",
+                             "read_back": "zero copy" if steps[0].io_zero_copy[1] else "copy"}},
         "gpu_launches": int(launches_per_step) * args.steps,
         "clocks": clk,
     }

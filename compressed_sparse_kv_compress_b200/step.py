@@ -160,19 +160,29 @@ class DecodeStep:
         self.graph = g
         return g
 
-    def capture_io(self, h2d=(), d2h=(), zero_copy=True):
+    # transfers up to this size per direction go zero-copy by default: the pieces' CTAs reach
+    # the pinned host buffer in one bus round trip each, where a copy node costs a fixed few
+    # microseconds more (measured at 0.07-6.6 MB a step); larger ones, a prefill chunk's queries
+    # and outputs, go through the copy engines
+    ZERO_COPY_MAX_BYTES = 8 << 20
+    # a segment is split into pieces of at most this size, one CTA each: 256 threads x 8 loads
+    # of 16 bytes, so a piece costs one round trip over the bus
+    PIECE_BYTES = 32 << 10
+
+    def capture_io(self, h2d=(), d2h=(), zero_copy=None):
         """Capture, into one CUDA graph, the upload of this step's new inputs, the step, and the
         read-back of its results; replay with replay_io().
 
         h2d: (host, device) pairs.  The host sides are packed into one pinned staging buffer:
         the returned host tensors (views into it, initialised from the given ones) are where
         the caller writes each step's new inputs.  d2h: (device, host pinned) pairs copied back
-        after the step.  With zero_copy (the default) one cskv_copy_segments launch reads the
-        staging buffer over the bus and spreads it to the device tensors (which must be
-        contiguous), and one more writes the results straight into the host tensors; without
-        it, a host-to-device copy of the buffer precedes the spreading launch and each result
-        comes back by a device-to-host copy.  A replay costs one launch on the host, whatever
-        the number of tensors."""
+        after the step.  Zero copy: one cskv_copy_segments launch reads the staging buffer over
+        the bus and spreads it to the device tensors (which must be contiguous), and one more
+        writes the results straight into the host tensors.  Otherwise a host-to-device copy of
+        the buffer precedes the spreading launch and each result comes back by a
+        device-to-host copy.  zero_copy: True / False for both directions; None (default)
+        chooses zero copy for a direction whose bytes are at most ZERO_COPY_MAX_BYTES.  A
+        replay costs one launch on the host, whatever the number of tensors."""
         views = self.prepare_io(h2d, d2h, zero_copy)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
@@ -180,7 +190,7 @@ class DecodeStep:
         self.graph_io = g
         return views
 
-    def prepare_io(self, h2d=(), d2h=(), zero_copy=True):
+    def prepare_io(self, h2d=(), d2h=(), zero_copy=None):
         """The pinned staging buffer and copy tables of capture_io (returns the host views);
         run_io() then issues upload, step and read-back on the current stream."""
         if self.graph is None:
@@ -190,7 +200,10 @@ class DecodeStep:
         def i64(vals):
             return torch.tensor(list(vals), dtype=torch.int64, device=dev)
 
-        sizes = [d.numel() * d.element_size() for _, d in h2d]
+        def nbytes(t):
+            return t.numel() * t.element_size()
+
+        sizes = [nbytes(d) for _, d in h2d]
         offs, total = [], 0
         for nb in sizes:
             offs.append(total)
@@ -202,37 +215,52 @@ class DecodeStep:
             v = stage_h[o:o + nb].view(d.dtype).view(d.shape)
             v.copy_(h)
             views.append(v)
-        up = None
+        down_bytes = sum(nbytes(d) for d, _ in d2h)
+        up_zc = zero_copy if zero_copy is not None else total <= self.ZERO_COPY_MAX_BYTES
+        down_zc = zero_copy if zero_copy is not None else down_bytes <= self.ZERO_COPY_MAX_BYTES
+
+        def pieces(segs):
+            """(src_off, dst, len) segments cut into PIECE_BYTES pieces (16-byte boundaries
+            inside a segment stay 16-byte boundaries), as three int64 device arrays."""
+            so, da, ln = [], [], []
+            for o, d, n in segs:
+                for c in range(0, n, self.PIECE_BYTES):
+                    so.append(o + c)
+                    da.append(d + c)
+                    ln.append(min(self.PIECE_BYTES, n - c))
+            return i64(so), i64(da), i64(ln)
+
+        up = None  # (staging buffer to fill first or None, copy_segments arguments)
         if h2d:
-            dst = i64(d.data_ptr() for _, d in h2d)
-            if zero_copy:
-                up = (api.mapped_pointer(stage_h), i64(offs), dst, i64(sizes))
+            segs = [(o, d.data_ptr(), nb) for o, (_, d), nb in zip(offs, h2d, sizes)]
+            if up_zc:
+                up = (None, (api.mapped_pointer(stage_h), *pieces(segs)))
             else:
                 stage_d = torch.empty(stage_h.shape, dtype=torch.uint8, device=dev)
-                up = (stage_d, i64(offs), dst, i64(sizes))
+                up = (stage_d, (stage_d, *pieces(segs)))
         down = None
-        if d2h and zero_copy:
+        if d2h and down_zc:
             for d, h in d2h:
                 assert d.is_contiguous() and h.is_contiguous() and h.is_pinned()
-                assert d.numel() * d.element_size() == h.numel() * h.element_size()
+                assert nbytes(d) == nbytes(h)
             base = min(d.data_ptr() for d, _ in d2h)
-            down = (base, i64(d.data_ptr() - base for d, _ in d2h), i64(api.mapped_pointer(h) for _, h in d2h),
-                    i64(d.numel() * d.element_size() for d, _ in d2h))
+            down = (base, *pieces([(d.data_ptr() - base, api.mapped_pointer(h), nbytes(d)) for d, h in d2h]))
         # the host tensors stay referenced for as long as the captured graph may touch them
-        self._io = (zero_copy, stage_h, up, down, list(d2h))
+        self._io = (stage_h, up, down, list(d2h))
+        self.io_zero_copy = (up_zc if h2d else None, down_zc if d2h else None)
         return views
 
     def run_io(self):
         """Upload, the step, the read-back (prepare_io first)."""
-        zero_copy, stage_h, up, down, d2h = self._io
+        stage_h, up, down, d2h = self._io
         if up is not None:
-            if not zero_copy:
-                up[0].copy_(stage_h, non_blocking=True)
-            api.copy_segments(*up)
+            stage_d, args = up
+            if stage_d is not None:
+                stage_d.copy_(stage_h, non_blocking=True)
+            api.copy_segments(*args)
         self.run()
-        if zero_copy:
-            if down is not None:
-                api.copy_segments(*down)
+        if down is not None:
+            api.copy_segments(*down)
         else:
             for d, h in d2h:
                 h.copy_(d, non_blocking=True)

@@ -76,7 +76,7 @@ def test_small_bf16_two_streams_graph_equal_eager():
     assert torch.equal(s1.o_c, s2.o_c) and torch.equal(s1.o_h, s2.o_h)
 
 
-@pytest.mark.parametrize("zero_copy", [True, False])
+@pytest.mark.parametrize("zero_copy", [True, False, None])
 def test_graph_with_host_copies_equals_eager(zero_copy):
     # capture_io: new queries copied from pinned host memory and both outputs read back, all
     # inside the step's graph (zero copy: the kernels read and write the host buffers over the
