@@ -29,13 +29,15 @@ def _run_indexer(w, dev=None):
                           head_w=dev["head_w"], out_score=sc, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    first = idx.clone()
-    # a second call on the same workspace gives the same selection
+    first, first_sc = idx.clone(), sc.clone()
+    # a second call on the same workspace gives the same selection; it also asks for the L2
+    # prefetch of the kept rows of the compressed cache, a hint that changes no result
     api.lindex_score_topk(dev["q_idx"], dev["k_idx"], dev["q_seq"], dev["q_pos"], dev["csa_off"], idx, ws,
                           max_entries=b["max_csa_visible"], q_scale=dev["q_scale"], k_scale=dev["k_scale"],
-                          head_w=dev["head_w"], out_score=sc, dev_status=st)
+                          head_w=dev["head_w"], out_score=sc, prefetch_rows=dev["cmp_c"], dev_status=st)
     torch.cuda.synchronize()
-    assert torch.equal(first, idx)
+    assert int(st.item()) == 0
+    assert torch.equal(first, idx) and torch.equal(first_sc, sc)
     return idx.cpu().numpy(), sc.cpu().numpy()
 
 
