@@ -227,6 +227,8 @@ CSKV_API int lindex_pool_keys(const void* k_tok, int in_dtype, int Di, const int
  *           multiple of 16, 16-byte aligned) -- e.g. the compressed CSA cache that
  *           the attention call gathers next.  The rows of the kept entries are
  *           prefetched into L2 as they are emitted; a hint with no effect on results.
+ *           Issuing the prefetches lengthens the call's tail; on the decode shapes
+ *           measured (1-64 queries, k = 1024) it cost more than the gather saved.
  * workspace : lindex_workspace_size(T, k, max_entries) bytes, zero-filled before
  *           its first use; every call leaves it ready for the next (arrival
  *           counters and histograms back at zero, barrier generations advanced,
