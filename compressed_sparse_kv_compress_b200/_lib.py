@@ -16,6 +16,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_LAUNCH = 0, 1, 2, 3, 4
 F32, BF16, FP8E4M3 = 0, 1, 2
 OVERLAP_PREVIOUS = 1  # csa_compress flags (CSKV_OVERLAP_PREVIOUS)
 ATTN_PAIRS = 0x100  # OR-ed into hybrid_decode_attn's mode (CSKV_ATTN_PAIRS)
+ATTN_KV_FP8 = 0x200  # OR-ed into hybrid_decode_attn's mode (CSKV_ATTN_KV_FP8)
+KV8_ROW_BYTES = 336  # CSKV_KV8_ROW_BYTES
 CSA, HCA = 0, 1
 DEV_BAD_INDEX, DEV_TAIL_MISSING, DEV_CAPACITY, DEV_TIMEOUT = 1, 2, 4, 8
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -37,6 +39,7 @@ SIGNATURES = {
                             _i32, _p, _f, _p, _i32, _i32, _p, _p, _i32, _p, _p]),
     "hca_compress": (_i32, [_p, _p, _p, _p, _p, _i32, _p, _p, _p, _i64, _i32, _i32, _p, _i32, _p, _f, _p, _p]),
     "rmsnorm_heads": (_i32, [_p, _i32, _i64, _i32, _p, _f, _p, _p]),
+    "kv_quantize_fp8": (_i32, [_p, _i32, _i64, _p, _p]),
     "lindex_pool_keys": (_i32, [_p, _i32, _i32, _p, _p, _i32, _p, _p, _p, _i64, _p, _p, _p, _p]),
     "lindex_score_topk": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _i32, _i32, _i32, _i32, _i32, _i64,
                                  _p, _p, _p, _i64, _p, _sz, _p, _p]),

@@ -13,7 +13,7 @@ import math
 import torch
 
 from . import _lib
-from ._lib import ATTN_PAIRS, BF16, CSA, F32, FP8E4M3, HCA, OVERLAP_PREVIOUS  # noqa: F401
+from ._lib import ATTN_KV_FP8, ATTN_PAIRS, BF16, CSA, F32, FP8E4M3, HCA, KV8_ROW_BYTES, OVERLAP_PREVIOUS  # noqa: F401
 
 _DT = {torch.float32: F32, torch.bfloat16: BF16, torch.uint8: FP8E4M3, torch.float8_e4m3fn: FP8E4M3}
 
@@ -166,12 +166,15 @@ def attn_workspace(mode, T, H, k, window, max_entries, device="cuda") -> torch.T
 
 def hybrid_decode_attn(mode, q, kv_cmp, cmp_off, kv_raw, raw_off, q_seq, q_pos, out, workspace, *, window,
                        idx=None, raw_tok0=None, sink=None, scale=None, lse=None, max_entries=0, adjacent_pairs=False,
-                       dev_status=None, stream=None):
+                       kv_fp8=False, dev_status=None, stream=None):
     """adjacent_pairs: CSKV_ATTN_PAIRS (queries 2j, 2j + 1 are one sequence's consecutive
-    positions; see the C header)."""
+    positions; see the C header).  kv_fp8: CSKV_ATTN_KV_FP8, kv_cmp holds FP8 main-KV rows
+    ([entries, 336] uint8, from kv_quantize_fp8)."""
     T, H, d = q.shape
     if adjacent_pairs:
         mode = int(mode) | ATTN_PAIRS
+    if kv_fp8:
+        mode = int(mode) | ATTN_KV_FP8
     k = idx.shape[1] if idx is not None else 0
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lib = _lib.load()
@@ -195,6 +198,18 @@ def copy_segments(src, src_off, dst_ptrs, lens, stream=None):
     st = lib.cskv_copy_segments(src_p, _ptr(src_off), _ptr(dst_ptrs), _ptr(lens), int(src_off.numel()),
                                 _stream(stream))
     _lib.check("cskv_copy_segments", st)
+
+
+def kv_quantize_fp8(rows, out=None, stream=None):
+    """FP8 main-KV rows ([n, 336] uint8) from K||V rows [n, 256] (fp32 or bf16, device)."""
+    assert rows.dim() == 2 and rows.shape[1] == 256
+    n = rows.shape[0]
+    if out is None:
+        out = torch.empty(n, KV8_ROW_BYTES, dtype=torch.uint8, device=rows.device)
+    lib = _lib.load()
+    st = lib.kv_quantize_fp8(_ptr(rows), _dt(rows), n, _ptr(out), _stream(stream))
+    _lib.check("kv_quantize_fp8", st)
+    return out
 
 
 def mapped_pointer(t) -> int:

@@ -183,6 +183,14 @@ int hca_compress(const void* x, const void* z, const float* bias, const int64_t*
                                            dev_status, (cudaStream_t)stream));
 }
 
+int kv_quantize_fp8(const void* rows, int dtype, int64_t n, void* out, cskv_stream_t stream) {
+  if (n < 0 || n > (int64_t)0x7FFFFFFF * 8) return CSKV_ERR_INVALID_ARG;  // grid.x: 8 rows a CTA
+  if (dtype != CSKV_F32 && dtype != CSKV_BF16) return dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
+  if (n == 0) return CSKV_OK;
+  if (!rows || !out || !aligned16(rows) || !aligned16(out)) return CSKV_ERR_INVALID_ARG;
+  return launch_status(cskv::launch_kv_quantize_fp8(rows, dtype, n, (uint8_t*)out, (cudaStream_t)stream));
+}
+
 int rmsnorm_heads(const void* x, int dtype, int64_t rows, int d, const float* gamma, float eps, void* out,
                   cskv_stream_t stream) {
   if (dtype != CSKV_F32 && dtype != CSKV_BF16) return dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
@@ -394,7 +402,7 @@ static int attn_plan(int mode, int T, int k, int window, int64_t max_entries, bo
 constexpr int kPairHeads = 64;
 
 size_t hybrid_attn_workspace_size(int mode, int T, int H, int d, int k, int window, int64_t max_entries) {
-  mode &= ~CSKV_ATTN_PAIRS;
+  mode &= ~(CSKV_ATTN_PAIRS | CSKV_ATTN_KV_FP8);
   if (T < 1 || H < 1 || d != kHeadDim || window < 0) return 0;
   size_t best = 0;
   for (int tc = 0; tc < 2; ++tc) {
@@ -421,8 +429,9 @@ int cskv::check_attn_args(int mode, const void* q, const void* kv_cmp, const int
                           int k, const void* kv_raw, const int64_t* raw_off, int window, float scale,
                           const int32_t* q_seq, const int64_t* q_pos, int batch, int T, int H, int d, int dtype,
                           int64_t max_entries, const float* out) {
-  if ((mode & ~CSKV_ATTN_PAIRS) != CSKV_CSA && (mode & ~CSKV_ATTN_PAIRS) != CSKV_HCA) return CSKV_ERR_INVALID_ARG;
-  mode &= ~CSKV_ATTN_PAIRS;
+  constexpr int kFlags = CSKV_ATTN_PAIRS | CSKV_ATTN_KV_FP8;
+  if ((mode & ~kFlags) != CSKV_CSA && (mode & ~kFlags) != CSKV_HCA) return CSKV_ERR_INVALID_ARG;
+  mode &= ~kFlags;
   if (dtype != CSKV_F32 && dtype != CSKV_BF16) return dtype == CSKV_FP8E4M3 ? CSKV_ERR_UNSUPPORTED : CSKV_ERR_INVALID_ARG;
   if (d != kHeadDim) return CSKV_ERR_UNSUPPORTED;
   if (H < 1 || H > 128 || T < 0 || window < 0 || window > (1 << 20) || batch < 1) return CSKV_ERR_INVALID_ARG;
@@ -448,8 +457,9 @@ int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_
                             T, H, d, dtype, max_entries, out);
   if (arc != CSKV_OK || T == 0) return arc;
   const bool want_pairs = (mode & CSKV_ATTN_PAIRS) != 0;
-  mode &= ~CSKV_ATTN_PAIRS;
-  const bool tc = dtype == CSKV_BF16;
+  const bool kv8 = (mode & CSKV_ATTN_KV_FP8) != 0;  // FP8 main-KV rows: the CUDA-core kernel
+  mode &= ~(CSKV_ATTN_PAIRS | CSKV_ATTN_KV_FP8);
+  const bool tc = dtype == CSKV_BF16 && !kv8;
   AttnPlan pl;
   int rc = attn_plan(mode, T, mode == CSKV_CSA ? k : 0, window, max_entries, tc, &pl);
   if (rc) return rc;
@@ -491,6 +501,7 @@ int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_
   p.cluster = pl.cluster;
   p.pairs = Hv != H ? 1 : 0;
   p.Hv = Hv;
+  p.kv8 = kv8 ? 1 : 0;
   p.part_acc = (float*)workspace;
   p.part_ml = p.part_acc + (size_t)units * pl.S * Hv * kHeadDim;
   p.out = out;

@@ -13,9 +13,11 @@
 //   [n_cmp, +W)      window token p - W + 1 + (r - n_cmp) (skipped when < 0)
 // CTA (split s, query t) runs an online softmax over rows [s*R, (s+1)*R) in tiles of 32
 // and writes (m, l, acc) in the log2 domain; attn_combine merges the splits of a query
-// and folds the sink logit in once.  This generic kernel serves fp32 and any head count;
-// bf16 with many heads goes to the tensor-core kernel.
+// and folds the sink logit in once.  This generic kernel serves fp32 and any head count, and
+// FP8 main-KV rows (KV8: kv_cmp rows in the kv8.cuh layout, dequantised as they are loaded;
+// the window's raw rows stay bf16 / fp32); bf16 with many heads goes to the tensor-core kernel.
 #include "attn_rows.cuh"
+#include "kv8.cuh"
 
 namespace cskv {
 
@@ -24,7 +26,7 @@ constexpr int kAttnThreads = 256;
 constexpr int kAttnTile = 32;
 constexpr int kPsStride = kAttnTile + 1;  // padded row of the probability tile
 
-template <typename T, int HP>
+template <typename T, int HP, bool KV8>
 __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) {
   constexpr int d = kHeadDim;
   constexpr int TPH = kAttnThreads / HP;  // threads per head in the PV update
@@ -74,19 +76,26 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(AttnParams p) 
       if (r < r1) off = resolve_row(p, q, t, r, &is_raw);
       if (part == 0) valid[rr] = off >= 0;
       if (off >= 0) {
-        const T* src = (is_raw ? raw : cmp) + off + part * 32;
+        float f[32];
+        if (KV8 && !is_raw) {
+          kv8_load_part(reinterpret_cast<const uint8_t*>(p.kv_cmp) + (size_t)(off / kRow) * kKv8RowBytes, part, f);
+        } else {
+          const T* src = (is_raw ? raw : cmp) + off + part * 32;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          float f[8];
-          Vec8<T>::load(src + 8 * v, f);
+          for (int v = 0; v < 4; ++v) {
+            float g[8];
+            Vec8<T>::load(src + 8 * v, g);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int col = part * 32 + 8 * v + u;
-            if (col < d)
-              ks[rr * (d + 1) + col] = f[u];
-            else
-              vs[rr * d + col - d] = f[u];
+            for (int u = 0; u < 8; ++u) f[8 * v + u] = g[u];
           }
+        }
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const int col = part * 32 + u;
+          if (col < d)
+            ks[rr * (d + 1) + col] = f[u];
+          else
+            vs[rr * d + col - d] = f[u];
         }
       }
     }
@@ -345,16 +354,21 @@ int attn_max_splits(int mode, int k, int window, int64_t max_entries, int R) {
   return (int)(s > 0 ? s : 1);
 }
 
-template <typename T, int HP>
-static cudaError_t launch_split(const AttnParams& p, cudaStream_t stream) {
+template <typename T, int HP, bool KV8>
+static cudaError_t launch_split_as(const AttnParams& p, cudaStream_t stream) {
   const size_t smem = attn_smem(HP);
-  auto kern = attn_split_kernel<T, HP>;
+  auto kern = attn_split_kernel<T, HP, KV8>;
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.max_splits, p.T);
   e = launch_dependent(kern, grid, dim3(kAttnThreads), smem, stream, p);
   note_launch();
   return e;
+}
+
+template <typename T, int HP>
+static cudaError_t launch_split(const AttnParams& p, cudaStream_t stream) {
+  return p.kv8 ? launch_split_as<T, HP, true>(p, stream) : launch_split_as<T, HP, false>(p, stream);
 }
 
 cudaError_t launch_attn_generic(const AttnParams& p, int dtype, cudaStream_t stream) {

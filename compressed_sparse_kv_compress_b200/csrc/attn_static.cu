@@ -66,7 +66,7 @@ extern "C" int hybrid_decode_attn_noalloc(int mode, const void* q, const void* k
   const int arc = cskv::check_attn_args(mode, q, kv_cmp, cmp_off, idx, k, kv_raw, raw_off, window, scale, q_seq,
                                         q_pos, batch, T, H, d, dtype, max_entries, out);
   if (arc != CSKV_OK || T == 0) return arc;
-  const size_t need = hybrid_attn_workspace_size(mode, T, H, d, (mode & ~CSKV_ATTN_PAIRS) == CSKV_CSA ? k : 0, window,
+  const size_t need = hybrid_attn_workspace_size(mode, T, H, d, (mode & ~(CSKV_ATTN_PAIRS | CSKV_ATTN_KV_FP8)) == CSKV_CSA ? k : 0, window,
                                                  max_entries);
   if (need > CSKV_NOALLOC_SCRATCH_BYTES) return CSKV_ERR_WORKSPACE;
   float* scratch = nullptr;

@@ -138,6 +138,7 @@ struct AttnParams {
   int cluster;  // tensor-core kernel: the splits of a query form a cluster of this size (0: merge kernel)
   int pairs;    // tensor-core HCA kernel: CTA row y takes queries 2y, 2y + 1 (adjacent positions)
   int Hv;       // heads of a unit of work: H, or 2H for a pair (its rows 0..H-1, then H..2H-1)
+  int kv8;      // CUDA-core kernel: kv_cmp rows are FP8 main-KV rows (kv8.cuh), kv_raw rows plain
   float* part_acc;
   float* part_ml;
   float* out;
@@ -156,6 +157,8 @@ int check_attn_args(int mode, const void* q, const void* kv_cmp, const int64_t* 
                     const void* kv_raw, const int64_t* raw_off, int window, float scale, const int32_t* q_seq,
                     const int64_t* q_pos, int batch, int T, int H, int d, int dtype, int64_t max_entries,
                     const float* out);
+// kv8.cu
+cudaError_t launch_kv_quantize_fp8(const void* rows, int dtype, int64_t n, uint8_t* out, cudaStream_t stream);
 // staging.cu
 cudaError_t launch_copy_segments(const void* src, const int64_t* src_off, void* const* dst, const int64_t* len, int n,
                                  cudaStream_t stream);

@@ -58,6 +58,8 @@ enum cskv_dtype { CSKV_F32 = 0, CSKV_BF16 = 1, CSKV_FP8E4M3 = 2 };
 enum cskv_mode { CSKV_CSA = 0, CSKV_HCA = 1 };
 /* OR-ed into hybrid_decode_attn's mode (see there): queries 2j and 2j + 1 are adjacent. */
 #define CSKV_ATTN_PAIRS 0x100
+#define CSKV_ATTN_KV_FP8 0x200  /* hybrid_decode_attn: kv_cmp rows are FP8 main-KV rows */
+#define CSKV_KV8_ROW_BYTES 336  /* bytes of one FP8 main-KV row (kv_quantize_fp8) */
 
 /* Bits OR-ed into *dev_status by device-side checks. */
 enum cskv_dev_status {
@@ -155,6 +157,24 @@ CSKV_API int hca_compress(const void* x, const void* z, const float* bias,
                  int64_t max_blocks, int in_dtype, int out_dtype, void* out,
                  int rmsnorm, const float* norm_gamma, float norm_eps,
                  int* dev_status, cskv_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * kv_quantize_fp8 -- FP8 main-KV rows from K||V rows.
+ *
+ * [SW] shareware.cn/news/167317 §十三.4: the main KV may be stored in FP8 while the
+ * dimensions most sensitive to position information keep a higher precision.  A
+ * compressed row (K dims 0..127 then V dims 0..127) becomes CSKV_KV8_ROW_BYTES (336)
+ * bytes: K dims 0..63 as OCP E4M3 codes (64 B) | K dims 64..127, the RoPE dims, as
+ * bf16 (128 B) | V dims 0..127 as E4M3 codes (128 B) | scale_k, scale_v fp32 | 8 zero
+ * bytes.  A group's scale is amax / 448 over the group (1 when it is all zero); a
+ * code is E4M3(value / scale), round to nearest even, saturating; a value is decoded
+ * as code x scale.  hybrid_decode_attn reads such rows with CSKV_ATTN_KV_FP8.
+ * rows : [n, 256] dtype (CSKV_F32 or CSKV_BF16), 16-byte aligned, device.
+ * out  : [n, 336] bytes, 16-byte aligned, device.
+ * n == 0 launches nothing.  Errors: CSKV_ERR_INVALID_ARG (null or misaligned pointer
+ * with n > 0, n < 0 or n > 8 (2^31 - 1), bad dtype), CSKV_ERR_UNSUPPORTED (FP8 input).
+ * ------------------------------------------------------------------------ */
+CSKV_API int kv_quantize_fp8(const void* rows, int dtype, int64_t n, void* out, cskv_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * rmsnorm_heads -- RMSNorm of head vectors (the query-side pass).
@@ -333,6 +353,10 @@ CSKV_API size_t lindex_workspace_size_scan(int T, int64_t max_entries);
  *           adjacent is flagged CSKV_DEV_BAD_INDEX and its second query attends to nothing
  *           (output 0).  Elsewhere (CSA, fp32, other H, or a plan whose splits do not fit
  *           one cluster) the bit is ignored.
+ * mode | CSKV_ATTN_KV_FP8 : kv_cmp holds FP8 main-KV rows (kv_quantize_fp8: 336 bytes a
+ *           row, indexed by cmp_off like the plain rows); kv_raw stays in dtype.  The rows
+ *           are decoded as they are loaded, on the CUDA cores (the tensor-core kernel takes
+ *           plain rows only; ignores CSKV_ATTN_PAIRS).  The workspace size is the same.
  * ------------------------------------------------------------------------ */
 CSKV_API int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_t* cmp_off,
                        const int32_t* idx, int k, const void* kv_raw, const int64_t* raw_off,

@@ -100,13 +100,20 @@ def query_scores(meta, arrays, dtypes, t):
     return indexer.index_scores(q_idx, k_idx, q_scale, k_scale, arrays.get("head_w"))
 
 
-def query_attention(meta, arrays, dtypes, cmp, t, layer, entries):
-    """(o [H, d], lse [H], p_sink [H]) of query t in layer 'c' (CSA) or 'h' (HCA)."""
+def query_attention(meta, arrays, dtypes, cmp, t, layer, entries, cmp_decoded=False):
+    """(o [H, d], lse [H], p_sink [H]) of query t in layer 'c' (CSA) or 'h' (HCA).
+    cmp_decoded: `cmp` already holds float64 values (e.g. FP8 main-KV rows decoded by
+    kv8.decode_rows) instead of rows in the workload's storage dtype."""
     kv, d = dtypes["kv"], meta["d"]
     b, p = meta["q_seq"][t], meta["q_pos"][t]
     off = meta["csa_off"][b] if layer == "c" else meta["hca_off"][b]
     ent = np.asarray(entries, dtype=np.int64)
-    cmp_rows = codecs.decode(cmp[off + ent], kv) if len(ent) else np.zeros((0, 2 * d))
+    if not len(ent):
+        cmp_rows = np.zeros((0, 2 * d))
+    elif cmp_decoded:
+        cmp_rows = np.asarray(cmp[off + ent], dtype=np.float64)
+    else:
+        cmp_rows = codecs.decode(cmp[off + ent], kv)
     ro, r1 = meta["raw_off"][b], meta["raw_off"][b + 1]
     raw = codecs.decode(arrays["raw_" + layer][ro:r1], kv)
     keys, values = attention.gather_rows(cmp_rows, np.arange(len(ent)), raw, meta["raw_t0"][b], p,

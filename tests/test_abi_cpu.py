@@ -144,7 +144,9 @@ def test_attention_validation(lib):
 
     for na in (False, True):  # both entry points report the same error for the same mistake
         assert call(mode=5, noalloc=na) == _lib.ERR_INVALID_ARG
-        assert call(mode=0x200 | 1, noalloc=na) == _lib.ERR_INVALID_ARG  # an unknown flag bit
+        assert call(mode=0x400 | 1, noalloc=na) == _lib.ERR_INVALID_ARG  # an unknown flag bit
+        assert call(mode=0x800 | _lib.ATTN_KV_FP8, noalloc=na) == _lib.ERR_INVALID_ARG
+        assert call(mode=_lib.ATTN_KV_FP8 | 1, T=0, noalloc=na) == _lib.OK  # HCA over FP8 rows: valid
         assert call(mode=_lib.ATTN_PAIRS | 7, noalloc=na) == _lib.ERR_INVALID_ARG
         assert call(mode=_lib.ATTN_PAIRS | 1, T=0, noalloc=na) == _lib.OK  # HCA with pairs: valid
         assert call(d=64, noalloc=na) == _lib.ERR_UNSUPPORTED
@@ -169,6 +171,19 @@ def test_copy_segments_validation(lib):
     assert lib.cskv_copy_segments(_p(), _p(), nul, _p(), 3, nul) == _lib.ERR_INVALID_ARG
     assert lib.cskv_copy_segments(_p(), _p(), _p(), nul, 3, nul) == _lib.ERR_INVALID_ARG
     assert lib.cskv_copy_segments(nul, nul, nul, nul, 0, nul) == _lib.OK
+
+
+def test_kv_quantize_fp8_validation(lib):
+    # refused on the host before any launch (no GPU needed); n == 0 is a no-op
+    nul = None
+    assert lib.kv_quantize_fp8(_p(), _lib.F32, -1, _p(), nul) == _lib.ERR_INVALID_ARG
+    assert lib.kv_quantize_fp8(_p(), _lib.F32, 8 * (2 ** 31 - 1) + 1, _p(), nul) == _lib.ERR_INVALID_ARG
+    assert lib.kv_quantize_fp8(_p(), 7, 4, _p(), nul) == _lib.ERR_INVALID_ARG
+    assert lib.kv_quantize_fp8(_p(), _lib.FP8E4M3, 4, _p(), nul) == _lib.ERR_UNSUPPORTED
+    assert lib.kv_quantize_fp8(nul, _lib.BF16, 4, _p(), nul) == _lib.ERR_INVALID_ARG
+    assert lib.kv_quantize_fp8(_p(), _lib.BF16, 4, nul, nul) == _lib.ERR_INVALID_ARG
+    assert lib.kv_quantize_fp8(_p(0x1008), _lib.BF16, 4, _p(), nul) == _lib.ERR_INVALID_ARG  # misaligned
+    assert lib.kv_quantize_fp8(nul, _lib.F32, 0, nul, nul) == _lib.OK
 
 
 def test_mapped_pointer_validation(lib):
