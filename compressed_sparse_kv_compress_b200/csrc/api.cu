@@ -457,9 +457,9 @@ int hybrid_decode_attn(int mode, const void* q, const void* kv_cmp, const int64_
                             T, H, d, dtype, max_entries, out);
   if (arc != CSKV_OK || T == 0) return arc;
   const bool want_pairs = (mode & CSKV_ATTN_PAIRS) != 0;
-  const bool kv8 = (mode & CSKV_ATTN_KV_FP8) != 0;  // FP8 main-KV rows: the CUDA-core kernel
+  const bool kv8 = (mode & CSKV_ATTN_KV_FP8) != 0;  // FP8 main-KV rows, decoded as gathered
   mode &= ~(CSKV_ATTN_PAIRS | CSKV_ATTN_KV_FP8);
-  const bool tc = dtype == CSKV_BF16 && !kv8;
+  const bool tc = dtype == CSKV_BF16;
   AttnPlan pl;
   int rc = attn_plan(mode, T, mode == CSKV_CSA ? k : 0, window, max_entries, tc, &pl);
   if (rc) return rc;

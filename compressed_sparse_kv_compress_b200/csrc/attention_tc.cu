@@ -33,6 +33,7 @@
 #include <mutex>
 
 #include "attn_rows.cuh"
+#include "kv8.cuh"
 #include "sm100.cuh"
 
 namespace cskv {
@@ -236,7 +237,12 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
         if (tid < rows) off = resolve_row(p, q, tq0, a + tid, &is_raw, a == r0 ? e_pre : (int64_t)-2);
         ok0 = off >= 0;
       }
-      row_src[tid] = off >= 0 ? (is_raw ? raw : cmp) + off : nullptr;
+      // an FP8 main-KV row (kv8.cuh) is marked by bit 0 of its address (rows are 16-byte aligned)
+      row_src[tid] = off < 0   ? nullptr
+                     : is_raw ? raw + off
+                     : p.kv8  ? reinterpret_cast<const __nv_bfloat16*>(
+                                   reinterpret_cast<uintptr_t>(p.kv_cmp) + (uintptr_t)(off / kRow) * kKv8RowBytes + 1u)
+                              : cmp + off;
       const uint32_t b0 = __ballot_sync(0xffffffffu, ok0), b1 = __ballot_sync(0xffffffffu, ok1);
       if (lane == 0) {
         row_mask[0][warp] = b0;
@@ -246,11 +252,16 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
     __syncthreads();
     // ---- gather: one whole 512-byte K||V row per warp instruction (lane j copies its
     //      16-byte piece j), eight rows in flight per warp; skipped rows up to nc are
-    //      zero-filled
+    //      zero-filled; an FP8 main-KV row is decoded to bf16 by the lanes and stored
 #pragma unroll 8
     for (int r = warp; r < nc; r += 4) {
       const __nv_bfloat16* row = row_src[r];
-      cp_async16(KVs + sw_off(r, lane), row ? (const void*)(row + 8 * lane) : (const void*)qg, row ? 16u : 0u);
+      const uintptr_t ra = reinterpret_cast<uintptr_t>(row);
+      if (ra & 1u)
+        *reinterpret_cast<uint4*>(KVs + sw_off(r, lane)) =
+            kv8_lane_bf16x8(reinterpret_cast<const uint8_t*>(ra - 1u), lane);
+      else
+        cp_async16(KVs + sw_off(r, lane), row ? (const void*)(row + 8 * lane) : (const void*)qg, row ? 16u : 0u);
     }
     cp_async_wait_all();
     fence_proxy_async_smem();

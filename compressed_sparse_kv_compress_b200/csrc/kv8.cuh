@@ -56,4 +56,25 @@ __device__ __forceinline__ void kv8_load_part(const uint8_t* row, int part, floa
   }
 }
 
+// The 16 bytes of bf16 values 8 * lane .. 8 * lane + 7 (lane 0..31 over the 256 K||V values)
+// of an FP8 row, as the tensor-core kernel's gather stores them: lanes 0..7 decode 8 K codes,
+// 8..15 copy the RoPE dims, 16..31 decode 8 V codes; a decoded value code x scale is rounded
+// to bf16 (nearest even).
+__device__ __forceinline__ uint4 kv8_lane_bf16x8(const uint8_t* row, int lane) {
+  if (lane >= 8 && lane < 16) return __ldg(reinterpret_cast<const uint4*>(row + 64 + 16 * (lane - 8)));
+  const bool is_v = lane >= 16;
+  const float s = __ldg(reinterpret_cast<const float*>(row + 320) + (is_v ? 1 : 0));
+  const uint2 w = __ldg(reinterpret_cast<const uint2*>(row + (is_v ? 192 + 8 * (lane - 16) : 8 * lane)));
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t x = i < 2 ? w.x : w.y;
+    const int b = (i & 1) * 16;
+    const __nv_bfloat162 h = __floats2bfloat162_rn(e4m3_to_float((x >> b) & 0xFFu) * s,
+                                                   e4m3_to_float((x >> (b + 8)) & 0xFFu) * s);
+    o[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 }  // namespace cskv

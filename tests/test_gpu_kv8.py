@@ -2,7 +2,8 @@
 oracle/kv8.py (codes equal outside the fp32 error band around an E4M3 rounding boundary, the
 neighbouring code allowed inside it; scales within one fp32 rounding; the bf16 RoPE dims and
 the padding bit-exact), and hybrid_decode_attn over such rows (CSKV_ATTN_KV_FP8) against the
-oracle's attention over the same rows decoded exactly."""
+oracle's attention over the same rows decoded exactly (bf16 queries on the tensor-core
+kernel, which decodes the rows to bf16 as it gathers them; fp32 on the CUDA cores)."""
 
 import numpy as np
 import pytest
@@ -91,7 +92,7 @@ def _oracle_rows(w, a):
     return rows
 
 
-def _attend_fp8(w, dev, mode, cache8, idx=None):
+def _attend_fp8(w, dev, mode, cache8, idx=None, pairs=False):
     m = w.meta
     b = bounds(w)
     T, H = m["T"], m["H"]
@@ -104,7 +105,7 @@ def _attend_fp8(w, dev, mode, cache8, idx=None):
     api.hybrid_decode_attn(mode, dev["q_" + layer], cache8, off, dev["raw_" + layer], dev["raw_off"], dev["q_seq"],
                            dev["q_pos"], out, ws, window=m["W"], idx=idx, raw_tok0=dev["raw_t0"],
                            sink=dev["sink_" + layer], scale=m["scale"], lse=lse, max_entries=b["max_hca_visible"],
-                           kv_fp8=True, dev_status=st)
+                           adjacent_pairs=pairs, kv_fp8=True, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     return to_f64(out), to_f64(lse)
@@ -143,5 +144,24 @@ def test_attention_over_fp8_rows(case, mode, quantiser):
             ent = np.arange(indexer.visible_entries(m["q_pos"][t], 128))
         ro, rl, _ = ostep.query_attention(m, a, dtypes(w), dec, t, layer, ent, cmp_decoded=True)
         check_attention(o[t], ro, 1e-4 if case == "tiny_f32" else None, f"{case} {mode} query {t}")
+        fin = np.isfinite(rl)
+        assert np.allclose(lse[t][fin], rl[fin], rtol=1e-5, atol=1e-5)
+
+
+def test_hca_adjacent_pairs_over_fp8_rows():
+    # the tensor-core HCA kernel taking adjacent queries in pairs (one pass over the union of
+    # their rows) over an FP8 cache; positions straddle 128-token block boundaries
+    spec = spec_by_name("prefill_4k_at_128k").replace(seq_len=(20096 + 10,), queries_per_seq=34, heads=64)
+    w = Workload(spec)
+    a = np_arrays(w)
+    dev = w.device("cuda")
+    m = w.meta
+    cache8 = api.kv_quantize_fp8(dev["cmp_h"])
+    dec = kv8.decode_rows(cache8.cpu().numpy())
+    o, lse = _attend_fp8(w, dev, api.HCA, cache8, pairs=True)
+    for t in range(m["T"]):
+        ent = np.arange(indexer.visible_entries(m["q_pos"][t], 128))
+        ro, rl, _ = ostep.query_attention(m, a, dtypes(w), dec, t, "h", ent, cmp_decoded=True)
+        check_attention(o[t], ro, None, f"pairs query {t}")
         fin = np.isfinite(rl)
         assert np.allclose(lse[t][fin], rl[fin], rtol=1e-5, atol=1e-5)
