@@ -253,15 +253,23 @@ __global__ void __maxnreg__(160) attn_tc_kernel(AttnParams p) {
     // ---- gather: one whole 512-byte K||V row per warp instruction (lane j copies its
     //      16-byte piece j), eight rows in flight per warp; skipped rows up to nc are
     //      zero-filled; an FP8 main-KV row is decoded to bf16 by the lanes and stored
+    if (p.kv8) {
 #pragma unroll 8
-    for (int r = warp; r < nc; r += 4) {
-      const __nv_bfloat16* row = row_src[r];
-      const uintptr_t ra = reinterpret_cast<uintptr_t>(row);
-      if (ra & 1u)
-        *reinterpret_cast<uint4*>(KVs + sw_off(r, lane)) =
-            kv8_lane_bf16x8(reinterpret_cast<const uint8_t*>(ra - 1u), lane);
-      else
+      for (int r = warp; r < nc; r += 4) {
+        const __nv_bfloat16* row = row_src[r];
+        const uintptr_t ra = reinterpret_cast<uintptr_t>(row);
+        if (ra & 1u)
+          *reinterpret_cast<uint4*>(KVs + sw_off(r, lane)) =
+              kv8_lane_bf16x8(reinterpret_cast<const uint8_t*>(ra - 1u), lane);
+        else
+          cp_async16(KVs + sw_off(r, lane), row ? (const void*)(row + 8 * lane) : (const void*)qg, row ? 16u : 0u);
+      }
+    } else {
+#pragma unroll 8
+      for (int r = warp; r < nc; r += 4) {
+        const __nv_bfloat16* row = row_src[r];
         cp_async16(KVs + sw_off(r, lane), row ? (const void*)(row + 8 * lane) : (const void*)qg, row ? 16u : 0u);
+      }
     }
     cp_async_wait_all();
     fence_proxy_async_smem();
