@@ -18,8 +18,9 @@ it (cited by page and section in each function):
 
 All arithmetic is float64 on values decoded exactly from their storage form
 (bf16, fp32, OCP E4M3).  Where floating point decides an integer -- the E4M3 codes
-of pooled indexer keys -- the definition is exact (indexer.pool_keys_f64,
-quantize_keys_f64) and indexer.quotient_error_bound says where an fp32 evaluation
+of pooled indexer keys and of FP8 main-KV rows -- the definition is exact
+(indexer.pool_keys_f64, quantize_keys_f64; kv8.quantize_rows_f64) and
+indexer.quotient_error_bound / kv8.quotient_error_bound say where an fp32 evaluation
 may round to the neighbouring code; indexer.pool_keys / quantize_keys restate the
 same steps in fp32 (the kernel's precision) as a second, labelled check.
 Loops are vectorised with numpy but follow each definition term by term; nothing
